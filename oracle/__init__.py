@@ -1,0 +1,169 @@
+"""CPU oracle for the fine-grained FP8 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  The product path (the CUDA library and its Python
+binding) never imports, loads or calls it, and it shares no code with them.
+
+The arithmetic lives in ``fg8_oracle.cpp`` (plain C++, float32 scales and
+quotients, double accumulation); this module only marshals numpy arrays.
+bf16 data is passed as ``uint16`` bit patterns, e4m3fn and UE8M0 as ``uint8``.
+
+Sources: [zh] "Transformers 中的细粒度 FP8 量化：配置、DeepGEMM 加速路径与 UE8M0
+缩放格式完全指南" and [pt] "FP8 de granularidade fina".  The quantizers follow
+[zh] §一 (1x128 per-token activation groups, 128x128 weight blocks,
+weight_scale_inv shaped (ceil(out/128), ceil(in/128))) and [zh] §七 (UE8M0
+scales); the GEMM follows [zh] §八 step 6 (FP8Linear.forward -> fp8_linear).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+FMT_FLOAT = 0
+FMT_UE8M0 = 1
+GROUP = 128
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        c_u8p = ctypes.POINTER(ctypes.c_uint8)
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e8m0_value.restype = ctypes.c_float
+        L.orc_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_ceil_byte.restype = ctypes.c_uint8
+        L.orc_e8m0_ceil_byte.argtypes = [ctypes.c_float]
+        L.orc_group_scale.restype = ctypes.c_float
+        L.orc_group_scale.argtypes = [ctypes.c_float]
+        L.orc_bf16_from_double.restype = ctypes.c_uint16
+        L.orc_bf16_from_double.argtypes = [ctypes.c_double]
+        L.orc_e4m3_encode_many.restype = None
+        L.orc_e4m3_encode_many.argtypes = [ctypes.c_void_p, ctypes.c_int64, c_u8p]
+        for name in ("orc_quantize_act", "orc_quantize_weight"):
+            f = getattr(L, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                          ctypes.c_void_p, ctypes.c_void_p]
+        L.orc_linear_dequant.restype = ctypes.c_int
+        L.orc_linear_dequant.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _kb(k):
+    return (k + GROUP - 1) // GROUP
+
+
+def _scale_dtype(fmt):
+    return np.float32 if fmt == FMT_FLOAT else np.uint8
+
+
+# ---------------------------------------------------------------- scalars --
+def e4m3_value(code: int) -> float:
+    return lib().orc_e4m3_value(int(code))
+
+
+def e4m3_encode(f: float) -> int:
+    return int(lib().orc_e4m3_encode(float(np.float32(f))))
+
+
+def e4m3_encode_many(f: np.ndarray) -> np.ndarray:
+    f = np.ascontiguousarray(f, dtype=np.float32).ravel()
+    out = np.empty(f.size, dtype=np.uint8)
+    lib().orc_e4m3_encode_many(_ptr(f), f.size, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
+
+
+def e8m0_value(b: int) -> float:
+    return float(lib().orc_e8m0_value(int(b)))
+
+
+def e8m0_ceil_byte(s: float) -> int:
+    return int(lib().orc_e8m0_ceil_byte(float(np.float32(s))))
+
+
+def group_scale(amax: float) -> float:
+    return float(np.float32(lib().orc_group_scale(float(np.float32(amax)))))
+
+
+def bf16_from_double(v: float) -> int:
+    return int(lib().orc_bf16_from_double(float(v)))
+
+
+# ------------------------------------------------------------- quantizers --
+def quantize_act(x_bf16: np.ndarray, fmt: int):
+    """x bf16 bits [M, K] -> (xq e4m3 [M, K], x_scale [M, ceil(K/128)] float32|uint8)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    xq = np.empty((M, K), dtype=np.uint8)
+    xs = np.empty((M, _kb(K)), dtype=_scale_dtype(fmt))
+    rc = lib().orc_quantize_act(_ptr(x), M, K, K, fmt, _ptr(xq), _ptr(xs))
+    if rc != 0:
+        raise ValueError("orc_quantize_act: bad argument")
+    return xq, xs
+
+
+def quantize_weight(w_bf16: np.ndarray, fmt: int):
+    """W bf16 bits [N, K] -> (wq e4m3 [N, K], w_scale_inv [ceil(N/128), ceil(K/128)])."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    N, K = w.shape
+    wq = np.empty((N, K), dtype=np.uint8)
+    ws = np.empty((_kb(N), _kb(K)), dtype=_scale_dtype(fmt))
+    rc = lib().orc_quantize_weight(_ptr(w), N, K, K, fmt, _ptr(wq), _ptr(ws))
+    if rc != 0:
+        raise ValueError("orc_quantize_weight: bad argument")
+    return wq, ws
+
+
+def linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows=None):
+    """Reference y for quantized operands.
+
+    Returns (y64 [R, N] float64, bound [R, N] float64, y_bf16 [R, N] uint16),
+    R = len(rows) (or M when rows is None).
+    """
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    xs = np.ascontiguousarray(xs, dtype=_scale_dtype(fmt))
+    ws = np.ascontiguousarray(ws, dtype=_scale_dtype(fmt))
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K2 != K:
+        raise ValueError("K mismatch")
+    if xs.shape != (M, _kb(K)) or ws.shape != (_kb(N), _kb(K)):
+        raise ValueError("scale shape mismatch")
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    if b is not None and b.shape != (N,):
+        raise ValueError("bias shape mismatch")
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    R = M if r is None else r.size
+    y64 = np.empty((R, N), dtype=np.float64)
+    bound = np.empty((R, N), dtype=np.float64)
+    ybf = np.empty((R, N), dtype=np.uint16)
+    rc = lib().orc_linear_dequant(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(b), M, N, K, fmt,
+                                  _ptr(r), 0 if r is None else r.size, _ptr(y64), _ptr(bound), _ptr(ybf))
+    if rc != 0:
+        raise ValueError("orc_linear_dequant: bad argument")
+    return y64, bound, ybf
+
+
+def linear(x_bf16, wq, ws, bias_bf16, fmt, rows=None):
+    """Whole layer: quantize x per token, then linear_dequant."""
+    xq, xs = quantize_act(x_bf16, fmt)
+    return linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows)
+
