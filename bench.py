@@ -1,0 +1,451 @@
+"""Benchmark of the fine-grained FP8 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl fg8|reference]
+
+One step is one pass of the whole layer path over one batch: for every
+linear of the workload, dynamic per-token activation quantization (1x128
+groups) followed by the block-scaled FP8 GEMM with the bf16 epilogue.  The
+default workload is the ESM-2 35M-shaped FFN (8 x 1022 = 8176 tokens,
+hidden 480 -> FFN 1920 -> 480, float scales, both GEMMs back to back, no
+activation function between them), on synthetic seeded inputs.
+
+Rank 0 prints ONE JSON line.  `value` is whole-job TFLOP/s (2*M*N*K summed
+over the step's GEMMs, all ranks, / the max-over-ranks device time); weak
+scaling: every rank runs its own batch with replicated weights and there is
+no collective on the data path (token rows are independent).
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (rows of the batch), reporting the same metric.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "block-scaled FP8 linear TFLOP/s and % of B200 dense FP8 peak; act-quant GB/s"
+L2_FLUSH_BYTES = 256 << 20
+FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+
+
+# ------------------------------------------------------------ workloads ----
+def workload_layers(name):
+    """[(cfg, Gemm, stage)] of one step."""
+    if name == "esm2_ffn":
+        return [("esm2", W.ESM_W1, 1), ("esm2", W.ESM_W2, 2)]
+    if name.startswith("llama_"):        # llama_m4096: gate/up then down
+        M = int(name.split("_m")[1])
+        return [("llama", W.llama(M, "gate_up"), 1), ("llama", W.llama(M, "down"), 2)]
+    if name == "dsv3_mlp":
+        return [("dsv3", W.DSV3_UP, 1), ("dsv3", W.DSV3_DOWN, 2)]
+    if name.startswith("square_"):       # square_m8192_float / square_m8192_ue8m0
+        _, m, f = name.split("_")
+        return [("square", W.square(int(m[1:]), 1 if f == "ue8m0" else 0), 1)]
+    raise SystemExit(f"unknown workload {name}")
+
+
+def workload_config(name, layers):
+    g0 = layers[0][1]
+    cfg = {"workload": name, "tokens": g0.M, "layers": [[g.K, g.N] for _, g, _ in layers],
+           "scale_fmt": "ue8m0" if g0.fmt else "float", "block": [128, 128], "act_group": 128,
+           "l2": "flushed between steps (256 MiB write outside the step events)"}
+    if name == "esm2_ffn":
+        cfg.update({"model": "ESM-2 35M FFN shape (hidden 480, ffn 1920, 8 x 1022 tokens)"})
+    return cfg
+
+
+# ---------------------------------------------------------- distributed ----
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(value, world, device):
+    """Max of a float over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed loop runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], None, [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------ roofline ----
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_bytes(g):
+    """Algorithmic HBM bytes of one GEMM launch: xq + x scales + Wq + W scales + y + bias."""
+    Kb, Nb = -(-g.K // 128), -(-g.N // 128)
+    sb = 4 if g.fmt == 0 else 1
+    return g.M * g.K + g.M * Kb * sb + g.N * g.K + Nb * Kb * sb + 2 * g.M * g.N + 2 * g.N
+
+
+def quant_bytes(g):
+    """Algorithmic HBM bytes of one activation-quant launch: read bf16 x, write e4m3 + scales."""
+    Kb = -(-g.K // 128)
+    return 2 * g.M * g.K + g.M * g.K + g.M * Kb * (4 if g.fmt == 0 else 1)
+
+
+def gemm_flops(g):
+    return 2.0 * g.M * g.N * g.K
+
+
+# ------------------------------------------------------------ fg8 arm ----
+def run_fg8(args, rank, world, local):
+    import fine_grained_fp8_act_b200 as fg8
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    layers = workload_layers(args.workload)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    # weights (replicated), quantized once on the device
+    plan = []
+    x0 = None
+    for i, (cfg, g, stage) in enumerate(layers):
+        x, w, b = W.make_inputs(cfg, g, device=dev, stage=stage)
+        if i == 0:
+            # weak scaling: every rank runs its own batch of the same shape
+            x0 = x if rank == 0 else x.roll(rank, 0).contiguous()
+        wq, ws = fg8.quantize_weight(w, g.fmt)
+        del w
+        wsp = torch.zeros(fg8.fg8_linear_workspace_bytes(g.M, g.N, g.K, g.fmt), dtype=torch.uint8, device=dev)
+        y = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+        plan.append(dict(g=g, wq=wq, ws=ws, b=b, wsp=wsp, y=y))
+    for i, L in enumerate(plan):
+        L["x"] = x0 if i == 0 else plan[i - 1]["y"]
+        assert L["x"].shape == (L["g"].M, L["g"].K), "consecutive layers must chain"
+
+    def launch_layer(L, ev_mid=None):
+        g = L["g"]
+        fg8.fg8_linear_prepare(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["ws"].data_ptr(), g.fmt,
+                               L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), g.M, g.N,
+                           g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    nl = len(plan)
+    # events per step: start, then per layer (after quant, after gemm)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(1 + 2 * nl)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        for i, L in enumerate(plan):
+            launch_layer(L, None if e is None else e[1 + 2 * i])
+            if e is not None:
+                e[2 + 2 * i].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    for L in plan:
+        st = fg8.fg8_check_device_status(L["wsp"].data_ptr(), sp)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    time.sleep(0.25)
+    clk = clocks.stop()
+
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    quant_ms = [[e[2 * i].elapsed_time(e[1 + 2 * i]) for e in evs] for i in range(nl)]
+    gemm_ms = [[e[1 + 2 * i].elapsed_time(e[2 + 2 * i]) for e in evs] for i in range(nl)]
+    total_ms = sum(step_ms)
+    total_ms_max = max_over_ranks(total_ms, world, dev)
+    flops_step = sum(gemm_flops(L["g"]) for L in plan)
+    flops_all = sum_over_ranks(flops_step * args.steps, world, dev)
+    tflops = flops_all / (total_ms_max * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    # per-kernel roofline: the dominant kernel is the GEMM launch with the largest mean time
+    gm = [statistics.mean(v) for v in gemm_ms]
+    qm = [statistics.mean(v) for v in quant_ms]
+    dom = max(range(nl), key=lambda i: gm[i])
+    g = plan[dom]["g"]
+    t_s = gm[dom] * 1e-3
+    t_tensor = gemm_flops(g) / (fp8_peak * 1e12)
+    t_hbm = gemm_bytes(g) / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": gemm_flops(g) / t_s / 1e12, "peak": fp8_peak, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = f"fg8_gemm_kernel ({g.name}: M={g.M} K={g.K} N={g.N})"
+    roof["kernel_us"] = gm[dom] * 1e3
+    roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
+                           f"HBM {peaks['hbm_gbs']} GB/s")
+    per_kernel = []
+    for i, L in enumerate(plan):
+        gi = L["g"]
+        per_kernel.append({"layer": gi.name, "act_quant_us": qm[i] * 1e3,
+                           "act_quant_gbs": quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
+                           "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
+                           "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
+
+    e2e = run_e2e(fg8, plan, args, stream, dev, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+
+    launches_per_step = sum(2 + (1 if L["g"].fmt == 1 else 0) for L in plan)
+    out = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": dict(workload_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)]),
+                       parallelism=f"dp{world} (token rows, replicated weights, no collective)"),
+        "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
+        "act_quant_gbs": [k["act_quant_gbs"] for k in per_kernel],
+        "per_kernel": per_kernel,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s": wall,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_e2e(fg8, plan, args, stream, dev, world):
+    """Same metric through the public call with host buffers: pinned x -> device,
+    the layers via fg8_linear, y -> pinned host, every step inside the timed region."""
+    L0, Ln = plan[0], plan[-1]
+    x_host = L0["x"].to("cpu").pin_memory()
+    y_host = torch.empty(Ln["y"].shape, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(L0["x"])
+    sp = stream.cuda_stream
+    steps = max(3, min(args.steps, 50))
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        xin = x_dev
+        for L in plan:
+            g = L["g"]
+            fg8.fg8_linear(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
+                           L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, L["wsp"].data_ptr(),
+                           L["wsp"].numel(), sp)
+            xin = L["y"]
+        y_host.copy_(Ln["y"], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    flops = sum_over_ranks(sum(gemm_flops(L["g"]) for L in plan) * steps, world, dev)
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 2,
+            "steps": steps, "ms_per_step": ms / steps}
+
+
+# ------------------------------------------------------ oracle (CPU) arm ----
+def cpu_baseline(workload, budget_s=15.0, rows=None):
+    """The CPU oracle, as it stands, on a bounded sample of the workload: the
+    first R token rows of the batch through every layer (quantize, dequantized
+    double GEMM, bf16 out), weights quantized once outside the timing.
+    Reported in TFLOP/s of the sampled rows."""
+    import oracle
+    layers = workload_layers(workload)
+    ops = []
+    xb = None
+    for i, (cfg, g, stage) in enumerate(layers):
+        x, w, b = W.make_inputs(cfg, g, device="cpu", stage=stage)
+        if i == 0:
+            xb = W.bf16_bits(x)
+        wq, ws = oracle.quantize_weight(W.bf16_bits(w), g.fmt)
+        ops.append((g, wq, ws, W.bf16_bits(b)))
+
+    def run(R):
+        t0 = time.perf_counter()
+        a = xb[:R]
+        for g, wq, ws, bb in ops:
+            _, _, ybf = oracle.linear(a, wq, ws, bb, g.fmt)
+            a = ybf
+        return time.perf_counter() - t0
+
+    if rows is None:
+        probe = 16
+        t = run(probe)
+        rows = int(max(16, min(layers[0][1].M, probe * budget_s / max(t, 1e-6))))
+    t = run(rows)
+    flops = sum(2.0 * rows * g.N * g.K for g, _, _, _ in ops)
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(ops)} layers "
+                      f"({t:.1f} s; weights quantized outside the timing)",
+            "seconds": t}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    layers = workload_layers(args.workload)
+    # size each step so warm-up + steps stay within ~2 minutes
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    probe = cpu_baseline(args.workload, rows=16)
+    rows = int(max(1, min(layers[0][1].M, 16 * budget / max(probe["seconds"], 1e-6))))
+    for _ in range(args.warmup):
+        cpu_baseline(args.workload, rows=rows)
+    ts = []
+    for _ in range(args.steps):
+        ts.append(cpu_baseline(args.workload, rows=rows)["seconds"])
+    flops = sum(2.0 * rows * g.N * g.K for _, g, _ in layers)
+    tot = sum(ts)
+    value = flops * len(ts) / tot / 1e12
+    cpu = {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+           "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(layers)} layers per step"}
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: float32 quantization, double GEMM)",
+           "data": "synthetic", "impl": "reference",
+           "config": dict(workload_config(args.workload, layers), parallelism="cpu oracle, rank 0 only"),
+           "cpu_baseline": cpu,
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="esm2_ffn")
+    ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_fg8(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

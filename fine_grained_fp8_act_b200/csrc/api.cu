@@ -1,0 +1,368 @@
+// api.cu -- the extern "C" boundary of libfg8 (declared in include/fg8.h).
+//
+// Host-side argument checks happen before anything is launched; every
+// accepted call enqueues its kernels on the caller's stream and returns.  No
+// device memory is allocated here: fg8_linear / fg8_gemm_prequant carve their
+// scratch out of the caller's workspace.
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "fg8.h"
+#include "fg8_internal.h"
+
+namespace {
+
+using namespace fg8;
+
+constexpr int64_t kMaxDim = 2147483647LL;
+constexpr size_t kHeaderBytes = 256;  // status word + reserved
+constexpr size_t kAlign = 256;
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  bool ok = false;
+  int sms = 0;
+};
+
+// Compute capability 10.0 (B200) and SM count of the current device, cached.
+fg8_status current_device(DeviceInfo* out) {
+  static std::atomic<int> cached_cc[64];
+  static std::atomic<int> cached_sms[64];
+  static std::atomic<bool> init{false};
+  if (!init.load()) {
+    for (int i = 0; i < 64; ++i) {
+      cached_cc[i].store(-1);
+      cached_sms[i].store(0);
+    }
+    init.store(true);
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return FG8_ERR_UNSUPPORTED_DEVICE;
+  }
+  int cc = dev < 64 ? cached_cc[dev].load() : -1;
+  int sms = dev < 64 ? cached_sms[dev].load() : 0;
+  if (cc < 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FG8_ERR_UNSUPPORTED_DEVICE;
+    }
+    cc = major * 10 + minor;
+    if (dev < 64) {
+      cached_cc[dev].store(cc);
+      cached_sms[dev].store(sms);
+    }
+  }
+  if (cc != 100) return FG8_ERR_UNSUPPORTED_DEVICE;
+  out->ok = true;
+  out->sms = sms;
+  return FG8_OK;
+}
+
+bool fmt_ok(int fmt) { return fmt == FG8_SCALE_FLOAT || fmt == FG8_SCALE_UE8M0; }
+
+// Shared shape checks of the GEMM entry points.
+fg8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int fmt) {
+  if (!fmt_ok(fmt)) return FG8_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FG8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 8 != 0) return FG8_ERR_ALIGNMENT;
+  return FG8_OK;
+}
+
+// Workspace of fg8_linear: [header | xq (M*K) | x scales | W scale-factor tiles].
+struct LinearWs {
+  size_t xq_off, xs_off, sfb_off, total;
+  int64_t ld_s;
+};
+
+LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
+  LinearWs w;
+  const int Kb = ceil_div(K, kGroup);
+  const int Kq = ceil_div(Kb, 4);
+  w.xq_off = kHeaderBytes;
+  size_t off = align_up(w.xq_off + static_cast<size_t>(M) * K, kAlign);
+  w.xs_off = off;
+  w.ld_s = static_cast<int64_t>(align_up(static_cast<size_t>(M), 32));
+  if (fmt == FG8_SCALE_FLOAT) {
+    off = align_up(off + static_cast<size_t>(Kb) * w.ld_s * sizeof(float), kAlign);
+    w.sfb_off = off;
+  } else {
+    off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
+    w.sfb_off = off;
+    off = align_up(off + static_cast<size_t>(ceil_div(N, 128)) * Kq * kSfChunkBytes, kAlign);
+  }
+  w.total = off;
+  return w;
+}
+
+// Workspace of fg8_gemm_prequant: [header | A tiles | B tiles] (tiles: UE8M0 only).
+struct GemmWs {
+  size_t sfa_off, sfb_off, total;
+};
+
+GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
+  GemmWs w;
+  const int Kb = ceil_div(K, kGroup);
+  const int Kq = ceil_div(Kb, 4);
+  size_t off = kHeaderBytes;
+  w.sfa_off = off;
+  if (fmt == FG8_SCALE_UE8M0) {
+    off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
+    w.sfb_off = off;
+    off = align_up(off + static_cast<size_t>(ceil_div(N, 128)) * Kq * kSfChunkBytes, kAlign);
+  } else {
+    w.sfb_off = off;
+  }
+  w.total = off;
+  return w;
+}
+
+fg8_status check_workspace(void* ws, size_t bytes, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || bytes < need) return FG8_ERR_WORKSPACE;
+  return FG8_OK;
+}
+
+fg8_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FG8_OK;
+  cudaGetLastError();
+  return FG8_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fg8_version(void) { return 100; }
+
+const char* fg8_status_string(fg8_status st) {
+  switch (st) {
+    case FG8_OK: return "ok";
+    case FG8_ERR_INVALID_ARG: return "invalid argument (format, size, pointer or leading dimension)";
+    case FG8_ERR_ALIGNMENT: return "alignment (K % 16, N % 8, ld % 8 for bf16, 16-byte pointers)";
+    case FG8_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0, B200)";
+    case FG8_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FG8_ERR_CUDA: return "CUDA launch or runtime error";
+    case FG8_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+void fg8_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+fg8_status fg8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w, void* wq_e4m3,
+                               void* w_scale_inv, fg8_scale_fmt fmt, void* stream) {
+  if (!fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K) return FG8_ERR_INVALID_ARG;
+  if (w_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr) return FG8_ERR_INVALID_ARG;
+  if (ceil_div(N, 128) > 65535) return FG8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld_w % 8 != 0 || !aligned16(w_bf16) || !aligned16(wq_e4m3)) return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  return cuda_status(launch_weight_quant(w_bf16, ld_w, static_cast<int>(N), static_cast<int>(K),
+                                         static_cast<uint8_t*>(wq_e4m3), w_scale_inv, fmt,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+fg8_status fg8_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* xq_e4m3, void* x_scale,
+                            fg8_scale_fmt fmt, void* stream) {
+  if (!fmt_ok(fmt) || M < 0 || K <= 0 || M > kMaxDim || K > kMaxDim || ld_x < K) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || xq_e4m3 == nullptr || x_scale == nullptr) return FG8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld_x % 8 != 0 || !aligned16(x_bf16) || !aligned16(xq_e4m3)) return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  ActQuantArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.Kb = ceil_div(K, kGroup);
+  a.xq = static_cast<uint8_t*>(xq_e4m3);
+  a.xs = x_scale;
+  a.layout = kScaleRowMajor;
+  return cuda_status(launch_act_quant(a, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
+  if (check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
+  return linear_ws_layout(M, N, K, fmt).total;
+}
+
+size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
+  if (check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
+  return gemm_ws_layout(M, N, K, fmt).total;
+}
+
+fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                              const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || w_scale_inv == nullptr) return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || !aligned16(x_bf16)) return FG8_ERR_ALIGNMENT;
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
+  ActQuantArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.Kb = Kb;
+  a.xq = ws + L.xq_off;
+  a.xs = ws + L.xs_off;
+  a.layout = fmt == FG8_SCALE_FLOAT ? kScaleKMajor : kScaleSfTiles;
+  a.ld_s = L.ld_s;
+  a.Kq = Kq;
+  a.M_pad = ceil_div(M, 128) * 128;
+  if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
+  if (fmt == FG8_SCALE_UE8M0)
+    return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), 128, Kb,
+                                      ws + L.sfb_off, s));
+  return FG8_OK;
+}
+
+fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16, void* y_bf16,
+                          int64_t M, int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr) return FG8_ERR_INVALID_ARG;
+  if (ld_y % 8 != 0 || !aligned16(wq_e4m3) || !aligned16(y_bf16) || (bias_bf16 != nullptr && !aligned16(bias_bf16)) ||
+      !aligned16(w_scale_inv))
+    return FG8_ERR_ALIGNMENT;
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
+  GemmArgs g{};
+  g.xq = ws + L.xq_off;
+  g.wq = wq_e4m3;
+  g.y = y_bf16;
+  g.ld_y = ld_y;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.Kb = Kb;
+  g.Kq = Kq;
+  g.bias = bias_bf16;
+  g.status = reinterpret_cast<uint32_t*>(ws);
+  g.wait_limit_ns = g_wait_limit_ns.load();
+  if (fmt == FG8_SCALE_FLOAT) {
+    g.xs = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.xs_sm = 1;
+    g.xs_sk = L.ld_s;
+    g.ws = static_cast<const float*>(w_scale_inv);
+  } else {
+    g.sfa = ws + L.xs_off;
+    g.sfb = ws + L.sfb_off;
+  }
+  return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
+fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
+                      const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
+      (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv))
+    return FG8_ERR_ALIGNMENT;
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_ws_layout(M, N, K, fmt).total);
+      st != FG8_OK)
+    return st;
+  if (fg8_status st = fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes, stream);
+      st != FG8_OK)
+    return st;
+  return fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes,
+                        stream);
+}
+
+fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const void* wq_e4m3, const void* w_scale_inv,
+                             const void* bias_bf16, void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
+                             fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (xq_e4m3 == nullptr || x_scale == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_y % 8 != 0 || !aligned16(xq_e4m3) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
+      (bias_bf16 != nullptr && !aligned16(bias_bf16)))
+    return FG8_ERR_ALIGNMENT;
+  const GemmWs L = gemm_ws_layout(M, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
+
+  GemmArgs g{};
+  g.xq = xq_e4m3;
+  g.wq = wq_e4m3;
+  g.y = y_bf16;
+  g.ld_y = ld_y;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.Kb = Kb;
+  g.Kq = Kq;
+  g.bias = bias_bf16;
+  g.status = reinterpret_cast<uint32_t*>(ws);
+  g.wait_limit_ns = g_wait_limit_ns.load();
+  if (fmt == FG8_SCALE_FLOAT) {
+    g.xs = static_cast<const float*>(x_scale);
+    g.xs_sm = Kb;
+    g.xs_sk = 1;
+    g.ws = static_cast<const float*>(w_scale_inv);
+  } else {
+    if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(x_scale), static_cast<int>(M), 1, Kb,
+                                                   ws + L.sfa_off, s));
+        st != FG8_OK)
+      return st;
+    if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N),
+                                                   128, Kb, ws + L.sfb_off, s));
+        st != FG8_OK)
+      return st;
+    g.sfa = ws + L.sfa_off;
+    g.sfb = ws + L.sfb_off;
+  }
+  return cuda_status(launch_gemm(g, fmt, dev.sms, s));
+}
+
+fg8_status fg8_check_device_status(void* workspace, void* stream) {
+  if (workspace == nullptr) return FG8_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FG8_ERR_CUDA;
+  }
+  return word == 0 ? FG8_OK : static_cast<fg8_status>(word);
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// fg8_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace fg8 {
+
+constexpr int kGroup = 128;      // activation group width = weight block width
+constexpr int kBlockM = 128;     // GEMM tile rows (tokens)
+constexpr int kSfChunkBytes = 512;  // one scale-factor tile: 128 rows x 4 K-blocks, UE8M0
+
+enum ScaleLayout : int {
+  kScaleRowMajor = 0,   // [M, Kb] row-major (the public layout)
+  kScaleKMajor = 1,     // float32 [Kb, ld] (column m contiguous): what the float GEMM epilogue reads
+  kScaleSfTiles = 2,    // UE8M0 tensor-core scale-factor tiles (see sf_tile_offset)
+};
+
+// Byte offset of the UE8M0 scale of (row r, K-block kb) inside the tensor-core
+// scale-factor tile stream: tiles of 128 rows x 4 K-blocks, 512 bytes each,
+// tile (r/128, kb/4) at ((r/128)*Kq + kb/4)*512, inside a tile the word for
+// row 32c + i (i < 32) is at i*16 + c*4 and K-block kb%4 is byte kb%4 of it.
+// That is the shared-memory source shape of tcgen05.cp.32x128b.warpx4, which
+// lands row 32c + i in TMEM lane i (of every sub-partition), column c.
+__host__ __device__ inline size_t sf_tile_offset(int64_t r, int kb, int Kq) {
+  const int64_t tile = r / 128, rr = r % 128;
+  return static_cast<size_t>((tile * Kq + kb / 4) * kSfChunkBytes + (rr % 32) * 16 + (rr / 32) * 4 + (kb % 4));
+}
+
+struct ActQuantArgs {
+  const void* x;      // bf16 [M, K], row stride ld_x
+  int64_t ld_x;
+  int M, K, Kb;
+  uint8_t* xq;        // e4m3 [M, K], row stride K
+  void* xs;           // scales, layout below
+  int layout;         // ScaleLayout
+  int64_t ld_s;       // kScaleKMajor: column stride (>= M)
+  int Kq;             // kScaleSfTiles: ceil(Kb / 4)
+  int M_pad;          // kScaleSfTiles: rows rounded up to 128 (padding rows get scale 2^0)
+};
+
+cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s);
+
+cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
+                                cudaStream_t s);
+
+// Pack a UE8M0 [R_src, Kb] row-major scale matrix into scale-factor tiles for
+// R rows (padded to 128): row r takes src[(r / row_div) * Kb + kb]; padding
+// rows and K-blocks get byte 127 (2^0).
+cudaError_t launch_sf_pack(const uint8_t* src, int R, int row_div, int Kb, uint8_t* dst, cudaStream_t s);
+
+struct GemmArgs {
+  const void* xq;     // e4m3 [M, K] row stride K
+  const void* wq;     // e4m3 [N, K] row stride K
+  void* y;            // bf16 [M, N] row stride ld_y
+  int64_t ld_y;
+  int M, N, K, Kb;
+  // float path: xs(m, kb) = xs[m * xs_sm + kb * xs_sk]; ws [Nb, Kb] row-major float32
+  const float* xs;
+  int64_t xs_sm, xs_sk;
+  const float* ws;
+  // UE8M0 path: scale-factor tiles of x (rows M) and W (rows N)
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int Kq;
+  const void* bias;   // bf16 [N] or nullptr
+  uint32_t* status;   // device status word (0 = ok)
+  uint64_t wait_limit_ns;
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s);
+
+}  // namespace fg8

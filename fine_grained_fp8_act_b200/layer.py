@@ -1,0 +1,147 @@
+"""PyTorch-facing wrappers: tensors in, tensors out, through the C ABI.
+
+These functions allocate outputs with torch on the input's device, pass raw
+pointers and the current CUDA stream to libfg8, and return.  They do no
+arithmetic of their own.
+
+Storage follows the Transformers fine-grained FP8 page ("Transformers 中的细粒度
+FP8 量化 ... 完全指南", §一 and §七): weights as torch.float8_e4m3fn, one
+weight_scale_inv per 128x128 block shaped (ceil(out/128), ceil(in/128)),
+float32 or torch.float8_e8m0fnu for scale_fmt "ue8m0".
+"""
+from typing import Optional, Tuple
+
+import torch
+
+from . import _capi as C
+
+_SCALE_DTYPES = {C.FG8_SCALE_FLOAT: torch.float32, C.FG8_SCALE_UE8M0: torch.float8_e8m0fnu}
+
+
+def scale_fmt_code(scale_fmt) -> int:
+    """"float" -> 0, "ue8m0" -> 1 (the only two values [zh] §四 accepts)."""
+    if isinstance(scale_fmt, int) and scale_fmt in (C.FG8_SCALE_FLOAT, C.FG8_SCALE_UE8M0):
+        return scale_fmt
+    if scale_fmt == "float":
+        return C.FG8_SCALE_FLOAT
+    if scale_fmt == "ue8m0":
+        return C.FG8_SCALE_UE8M0
+    raise ValueError(f"scale_fmt must be 'float' or 'ue8m0', got {scale_fmt!r}")
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _cdiv(a: int, b: int) -> int:
+    return (a + b - 1) // b
+
+
+def _check_bf16_matrix(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_cuda:
+        raise ValueError(f"{name} must be a 2-D bf16 CUDA tensor")
+    if t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride in its last dimension")
+
+
+def quantize_weight(w: torch.Tensor, scale_fmt="float") -> Tuple[torch.Tensor, torch.Tensor]:
+    """W bf16 [N, K] -> (wq float8_e4m3fn [N, K], weight_scale_inv [ceil(N/128), ceil(K/128)])."""
+    fmt = scale_fmt_code(scale_fmt)
+    _check_bf16_matrix(w, "w")
+    N, K = w.shape
+    wq = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    ws = torch.empty((_cdiv(N, 128), _cdiv(K, 128)), dtype=_SCALE_DTYPES[fmt], device=w.device)
+    with torch.cuda.device(w.device):
+        C.fg8_quantize_weight(w.data_ptr(), N, K, w.stride(0), wq.data_ptr(), ws.data_ptr(), fmt, _stream(w))
+    return wq, ws
+
+
+def quantize_act(x: torch.Tensor, scale_fmt="float") -> Tuple[torch.Tensor, torch.Tensor]:
+    """x bf16 [M, K] -> (xq float8_e4m3fn [M, K], x_scale [M, ceil(K/128)])."""
+    fmt = scale_fmt_code(scale_fmt)
+    _check_bf16_matrix(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    xs = torch.empty((M, _cdiv(K, 128)), dtype=_SCALE_DTYPES[fmt], device=x.device)
+    with torch.cuda.device(x.device):
+        C.fg8_quantize_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), xs.data_ptr(), fmt, _stream(x))
+    return xq, xs
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return workspace
+    # zero-filled: the first bytes hold the (sticky) device status word
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: Optional[torch.Tensor] = None,
+           scale_fmt="float", out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [M, N] bf16 = dequant(quantize_act(x)) . dequant(wq)^T + bias."""
+    fmt = scale_fmt_code(scale_fmt)
+    _check_bf16_matrix(x, "x")
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape != (N, K):
+        raise ValueError("wq must be [N, K]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    nbytes = C.fg8_linear_workspace_bytes(M, N, K, fmt)
+    ws = _workspace(nbytes, x.device, workspace)
+    with torch.cuda.device(x.device):
+        C.fg8_linear(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(),
+                     0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0), fmt, ws.data_ptr(),
+                     ws.numel() * ws.element_size(), _stream(x))
+    return y
+
+
+def gemm_prequant(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor,
+                  bias: Optional[torch.Tensor] = None, scale_fmt="float", out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The GEMM on already-quantized activations (layouts of quantize_act)."""
+    fmt = scale_fmt_code(scale_fmt)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    nbytes = C.fg8_gemm_workspace_bytes(M, N, K, fmt)
+    ws = _workspace(nbytes, xq.device, workspace)
+    with torch.cuda.device(xq.device):
+        C.fg8_gemm_prequant(xq.data_ptr(), x_scale.data_ptr(), wq.data_ptr(), w_scale_inv.data_ptr(),
+                            0 if bias is None else bias.data_ptr(), y.data_ptr(), M, N, K, y.stride(0), fmt,
+                            ws.data_ptr(), ws.numel() * ws.element_size(), _stream(xq))
+    return y
+
+
+class FP8Linear(torch.nn.Module):
+    """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
+    weight float8_e4m3fn [out, in], weight_scale_inv per 128x128 block, bias
+    kept in bf16 (not quantized, [zh] §三)."""
+
+    def __init__(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None, scale_fmt="float"):
+        super().__init__()
+        self.scale_fmt = scale_fmt_code(scale_fmt)
+        wq, ws = quantize_weight(weight.to(torch.bfloat16).contiguous(), self.scale_fmt)
+        self.register_buffer("weight", wq)
+        self.register_buffer("weight_scale_inv", ws)
+        self.register_buffer("bias", None if bias is None else bias.to(torch.bfloat16).contiguous())
+        self._ws = None
+
+    @property
+    def in_features(self) -> int:
+        return self.weight.shape[1]
+
+    @property
+    def out_features(self) -> int:
+        return self.weight.shape[0]
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, x.shape[-1]).to(torch.bfloat16).contiguous()
+        M, N, K = x2.shape[0], self.out_features, self.in_features
+        need = C.fg8_linear_workspace_bytes(M, N, K, self.scale_fmt)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != x2.device:
+            self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x2.device)
+        y = linear(x2, self.weight, self.weight_scale_inv, self.bias, self.scale_fmt, workspace=self._ws)
+        return y.reshape(*lead, N)

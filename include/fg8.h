@@ -1,0 +1,162 @@
+/*
+ * fg8.h -- C ABI of the B200 (sm_100a) fine-grained FP8 linear layer.
+ *
+ * The method is the one the Transformers fine-grained FP8 pages describe:
+ *   [zh] "Transformers 中的细粒度 FP8 量化：配置、DeepGEMM 加速路径与 UE8M0 缩放格式完全指南"
+ *   [pt] "FP8 de granularidade fina" (Transformers documentation)
+ * Weights are e4m3fn with one scale per 128x128 block ([zh] §一, [pt]);
+ * activations are quantized dynamically per token in groups of 128 input
+ * channels aligned with the weight blocks ([zh] §一); scales are float32 or
+ * UE8M0 powers of two ([zh] §四 scale_fmt, §七); the layer computes
+ *   y = dequant(xq) . dequant(Wq)^T + bias   (bf16 out; bias not quantized, [zh] §三).
+ *
+ * Arithmetic (the pages print none; the readings used):
+ *   scale s = max(amax / 448, 2^-126), a float32 division, amax over the real
+ *   elements of the group/block; UE8M0 stores s rounded up to a power of two
+ *   ([zh] §七 补充: float scales are rounded *up* to UE8M0); every element is
+ *   q = e4m3(x / s) with the quotient a correctly rounded float32 and the cast
+ *   round-to-nearest-even, saturating at +-448, sign kept.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers on the current CUDA device; the
+ *     caller allocates and owns them.  The library allocates no device memory.
+ *   - `stream` is a cudaStream_t (passed as void*); work is enqueued on it and
+ *     the call returns without synchronizing (except fg8_check_device_status).
+ *   - bf16 / e4m3 / UE8M0 buffers are raw bytes (uint16 / uint8 per element).
+ *   - Matrices are row-major.  ld_* are row strides in ELEMENTS.
+ *   - Host-detectable problems return an error before anything is launched:
+ *       FG8_ERR_INVALID_ARG        bad format, non-positive size (M may be 0),
+ *                                  NULL required pointer, ld < row length,
+ *                                  size beyond 2^31-1
+ *       FG8_ERR_ALIGNMENT          K % 16 != 0, N % 8 != 0, ld % 8 != 0 for
+ *                                  bf16 operands, or a pointer not 16-byte aligned
+ *       FG8_ERR_UNSUPPORTED_DEVICE current device is not compute capability 10.0
+ *       FG8_ERR_WORKSPACE          workspace NULL, misaligned (256 B) or too small
+ *     A failed launch returns FG8_ERR_CUDA.  There is no fallback path.
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified outputs.
+ */
+#ifndef FG8_H_
+#define FG8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Symbols of the C ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define FG8_API __attribute__((visibility("default")))
+#else
+#define FG8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* [zh] §四: scale_fmt is "float" or "ue8m0". One format per call governs both
+ * the activation and the weight scales. */
+typedef enum fg8_scale_fmt {
+  FG8_SCALE_FLOAT = 0, /* float32 scales */
+  FG8_SCALE_UE8M0 = 1  /* one byte: biased exponent b, scale = 2^(b-127) */
+} fg8_scale_fmt;
+
+typedef enum fg8_status {
+  FG8_OK = 0,
+  FG8_ERR_INVALID_ARG = 1,
+  FG8_ERR_ALIGNMENT = 2,
+  FG8_ERR_UNSUPPORTED_DEVICE = 3,
+  FG8_ERR_WORKSPACE = 4,
+  FG8_ERR_CUDA = 5,
+  FG8_ERR_TIMEOUT = 6 /* a device-side bounded wait expired (see fg8_check_device_status) */
+} fg8_status;
+
+/* Quantize a weight once, on load ([zh] §八 step 4, Fp8Quantize; [zh] §一).
+ *   w_bf16      [N, K] bf16, row stride ld_w elements (nn.Linear [out, in])
+ *   wq_e4m3     [N, K] e4m3fn bytes, row stride K (output)
+ *   w_scale_inv [ceil(N/128), ceil(K/128)] row-major (output): float32 for
+ *               FG8_SCALE_FLOAT, UE8M0 bytes for FG8_SCALE_UE8M0.
+ * W ~= value(wq) * scale_inv per 128x128 block; edge blocks use their real
+ * elements only. */
+FG8_API fg8_status fg8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w,
+                               void* wq_e4m3, void* w_scale_inv, fg8_scale_fmt fmt, void* stream);
+
+/* Dynamic per-token activation quantization ([zh] §一 "激活按每个 token 一组";
+ * [pt] first list): each row is cut into groups of 128 channels (the last
+ * group holds K mod 128 real channels), one scale per group.
+ *   x_bf16  [M, K] bf16, row stride ld_x elements
+ *   xq_e4m3 [M, K] e4m3fn bytes, row stride K (output)
+ *   x_scale [M, ceil(K/128)] row-major (output): float32 or UE8M0 bytes. */
+FG8_API fg8_status fg8_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                            void* xq_e4m3, void* x_scale, fg8_scale_fmt fmt, void* stream);
+
+/* Bytes of caller-owned device workspace fg8_linear needs for this shape
+ * (quantized activations, their scales in the GEMM's layout, the scale-factor
+ * tiles of the UE8M0 path and a device status word).  0 on bad arguments. */
+FG8_API size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
+
+/* The layer ([zh] §八 step 6, FP8Linear.forward -> fp8_linear; [zh] §6.1 the
+ * block (128,128) + dynamic-activation fast path):
+ *   y[M, N] = dequant(quantize_act(x)) . dequant(wq, w_scale_inv)^T + bias
+ *   x_bf16      [M, K] bf16, row stride ld_x
+ *   wq_e4m3     [N, K] e4m3fn, row stride K; w_scale_inv as fg8_quantize_weight
+ *   bias_bf16   [N] bf16 or NULL
+ *   y_bf16      [M, N] bf16, row stride ld_y (output; written once, RNE)
+ *   workspace   >= fg8_linear_workspace_bytes(M, N, K, fmt), 256-byte aligned,
+ *               caller-owned device memory.  Its first 256 bytes hold a sticky
+ *               device status word: zero them once before first use (e.g.
+ *               allocate the workspace zero-filled); fg8_check_device_status
+ *               reads and clears it.  Calls sharing a workspace must not
+ *               overlap on the device.
+ * Float scales are applied exactly per 128-K block in float32 (never rounded
+ * to a power of two, [zh] §七 补充); UE8M0 scales go through the tensor
+ * core's block-scaled MMA.  M == 0 is a no-op. */
+FG8_API fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                      const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                      void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* fg8_linear in two halves, for callers that reuse one quantized activation
+ * for several weights (same K) or time the GEMM on its own:
+ *   fg8_linear_prepare  quantizes x into the workspace in the GEMM's layouts
+ *                       (and, for UE8M0, packs w_scale_inv's scale-factor tiles);
+ *   fg8_linear_run      runs the GEMM from that workspace.
+ * prepare followed by run on the same stream and workspace is fg8_linear.
+ * Arguments and checks are those of fg8_linear. */
+FG8_API fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                      const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+FG8_API fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                  void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
+                                  fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace fg8_gemm_prequant needs.  0 on bad arguments. */
+FG8_API size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
+
+/* The GEMM alone on already-quantized activations (the layouts
+ * fg8_quantize_act writes): same result as fg8_linear for the same xq/x_scale.
+ *   xq_e4m3 [M, K] row stride K; x_scale [M, ceil(K/128)] row-major. */
+FG8_API fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const void* wq_e4m3,
+                             const void* w_scale_inv, const void* bias_bf16, void* y_bf16,
+                             int64_t M, int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, reads and clears the status word a previous
+ * fg8_linear / fg8_gemm_prequant left in `workspace`: FG8_OK, or
+ * FG8_ERR_TIMEOUT if one of its device-side waits gave up (the kernel then
+ * returned early; y is unspecified). */
+FG8_API fg8_status fg8_check_device_status(void* workspace, void* stream);
+
+/* Upper bound, in nanoseconds, on any single device-side wait of the GEMM
+ * before it gives up with FG8_ERR_TIMEOUT (default 2e9).  Process-wide. */
+FG8_API void fg8_set_wait_limit_ns(uint64_t ns);
+
+/* Static description of a status code. */
+FG8_API const char* fg8_status_string(fg8_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+FG8_API int fg8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FG8_H_ */

@@ -1,0 +1,147 @@
+"""The C ABI without a GPU: libfg8.so loads, exports every function
+include/fg8.h declares, and rejects bad arguments on the host before any
+launch.  (No compute call runs here.)"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fg8.h")
+
+
+@pytest.fixture(scope="module")
+def fg8():
+    from fine_grained_fp8_act_b200 import build
+    build.build()
+    import fine_grained_fp8_act_b200 as m
+    m.lib()
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fg8_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fg8_quantize_weight", "fg8_quantize_act", "fg8_linear", "fg8_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(fg8):
+    names = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", fg8.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    # the Python binding binds exactly the declared set
+    assert sorted(fg8._capi.SIGNATURES) == names
+    # nothing else leaks out of the library under an fg8_ name
+    extra = [s for s in exported if s.startswith("fg8_") and s not in names]
+    assert not extra, extra
+
+
+def test_library_needs_no_driver_to_load(fg8):
+    out = subprocess.run(["ldd", fg8.library_path()], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out  # the driver is resolved at call time only
+
+
+def test_status_strings(fg8):
+    for code in range(7):
+        assert fg8.fg8_status_string(code) and "unknown" not in fg8.fg8_status_string(code)
+    assert "unknown" in fg8.fg8_status_string(99)
+    assert fg8.fg8_version() >= 100
+
+
+L = None
+
+
+def _raw(fg8):
+    return fg8.lib()
+
+
+FAKE = 0x10000  # a 16-byte-aligned non-null "device" address; never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (M, N, K, ld_x, ld_y, fmt)
+    ((16, 256, 256, 256, 256, 7), 1),      # bad format
+    ((16, 256, 256, 256, 256, -1), 1),
+    ((-1, 256, 256, 256, 256, 0), 1),      # negative M
+    ((16, 0, 256, 256, 256, 0), 1),        # N = 0
+    ((16, 256, 0, 256, 256, 0), 1),        # K = 0
+    ((16, 256, 200, 200, 256, 0), 2),      # K % 16
+    ((16, 252, 256, 256, 256, 0), 2),      # N % 8
+    ((16, 256, 256, 255, 256, 0), 1),      # ld_x < K
+    ((16, 256, 256, 256, 255, 0), 1),      # ld_y < N
+    ((16, 256, 256, 260, 256, 0), 2),      # ld_x % 8
+    ((1 << 31, 256, 256, 256, 256, 0), 1),  # M beyond int32
+])
+def test_linear_rejects_bad_shapes(fg8, args, expect):
+    M, N, K, ldx, ldy, fmt = args
+    st = _raw(fg8).fg8_linear(FAKE, M, N, K, ldx, FAKE, FAKE, None, FAKE, ldy, fmt, FAKE * 16, 1 << 40, None)
+    assert st == expect
+
+
+def test_linear_rejects_null_and_misaligned(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_linear(None, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, FAKE * 16, 1 << 40, None) == 1
+    assert raw.fg8_linear(FAKE + 8, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, FAKE * 16, 1 << 40, None) == 2
+    assert raw.fg8_linear(FAKE, 16, 256, 256, 256, FAKE, FAKE, FAKE + 2, FAKE, 256, 0, FAKE * 16, 1 << 40, None) == 2
+    # workspace: null, misaligned, too small
+    assert raw.fg8_linear(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, None, 1 << 40, None) == 4
+    assert raw.fg8_linear(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, FAKE + 16, 1 << 40, None) == 4
+    assert raw.fg8_linear(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, FAKE * 16, 100, None) == 4
+
+
+def test_empty_m_is_a_noop(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_linear(None, 0, 256, 256, 256, None, None, None, None, 256, 0, None, 0, None) == 0
+    assert raw.fg8_quantize_act(None, 0, 256, 256, None, None, 0, None) == 0
+
+
+def test_quantizers_reject_bad_args(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_quantize_act(FAKE, 4, 256, 256, FAKE, FAKE, 2, None) == 1
+    assert raw.fg8_quantize_act(FAKE, 4, 120, 128, FAKE, FAKE, 0, None) == 2
+    assert raw.fg8_quantize_act(FAKE, 4, 256, 128, FAKE, FAKE, 0, None) == 1
+    assert raw.fg8_quantize_weight(FAKE, 0, 256, 256, FAKE, FAKE, 0, None) == 1
+    assert raw.fg8_quantize_weight(FAKE, 256, 248, 248, FAKE, FAKE, 1, None) == 2
+    assert raw.fg8_quantize_weight(None, 256, 256, 256, FAKE, FAKE, 1, None) == 1
+
+
+def test_valid_call_without_gpu_reports_unsupported_device(fg8):
+    """No CPU fallback: a well-formed call on a host without a B200 returns
+    FG8_ERR_UNSUPPORTED_DEVICE instead of computing anything."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    raw = _raw(fg8)
+    assert raw.fg8_quantize_act(FAKE, 4, 256, 256, FAKE, FAKE, 0, None) == 3
+
+
+def test_workspace_sizes(fg8):
+    f = fg8.fg8_linear_workspace_bytes
+    assert f(16, 256, 256, 7) == 0
+    assert f(16, 256, 200, 0) == 0
+    a = f(8176, 1920, 480, 0)
+    assert a >= 8176 * 480 + 4 * 8176 * 4
+    b = f(8192, 18432, 7168, 1)
+    assert b >= 8192 * 7168
+    assert f(0, 256, 256, 0) > 0
+    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 0) == 256
+    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 1) > 256
+
+
+def test_scale_fmt_validation(fg8):
+    from fine_grained_fp8_act_b200 import scale_fmt_code
+    assert scale_fmt_code("float") == 0 and scale_fmt_code("ue8m0") == 1
+    for bad in ("Float", "e8m0", "fp32", 3, None):
+        with pytest.raises(ValueError):
+            scale_fmt_code(bad)
