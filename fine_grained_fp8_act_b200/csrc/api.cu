@@ -82,9 +82,11 @@ fg8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int fmt) {
   return FG8_OK;
 }
 
-// Workspace of fg8_linear: [header | xq (M*K) | x scales | W scale-factor tiles].
+// Workspace of fg8_linear: [header | xq (M*K) | x scales | W scales].
+//   float: x scales K-major [Kb][ld_s] float32, W scales [Nb][Kb] 16-byte entries
+//   UE8M0: x and W scale-factor tiles (512 bytes per 128 rows x 4 K-blocks)
 struct LinearWs {
-  size_t xq_off, xs_off, sfb_off, total;
+  size_t xq_off, xs_off, wsc_off, total;
   int64_t ld_s;
 };
 
@@ -92,39 +94,47 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   LinearWs w;
   const int Kb = ceil_div(K, kGroup);
   const int Kq = ceil_div(Kb, 4);
+  const int Nb = ceil_div(N, 128);
   w.xq_off = kHeaderBytes;
   size_t off = align_up(w.xq_off + static_cast<size_t>(M) * K, kAlign);
   w.xs_off = off;
-  w.ld_s = static_cast<int64_t>(align_up(static_cast<size_t>(M), 32));
+  w.ld_s = kmajor_ld(M);
   if (fmt == FG8_SCALE_FLOAT) {
     off = align_up(off + static_cast<size_t>(Kb) * w.ld_s * sizeof(float), kAlign);
-    w.sfb_off = off;
+    w.wsc_off = off;
+    off = align_up(off + static_cast<size_t>(Nb) * Kb * 16, kAlign);
   } else {
     off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
-    w.sfb_off = off;
-    off = align_up(off + static_cast<size_t>(ceil_div(N, 128)) * Kq * kSfChunkBytes, kAlign);
+    w.wsc_off = off;
+    off = align_up(off + static_cast<size_t>(sfb_rows(N) / 128) * Kq * kSfChunkBytes, kAlign);
   }
   w.total = off;
   return w;
 }
 
-// Workspace of fg8_gemm_prequant: [header | A tiles | B tiles] (tiles: UE8M0 only).
+// Workspace of fg8_gemm_prequant: [header | x scales | W scales] in the GEMM's
+// layouts (as fg8_linear's).
 struct GemmWs {
-  size_t sfa_off, sfb_off, total;
+  size_t xs_off, wsc_off, total;
+  int64_t ld_s;
 };
 
 GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   GemmWs w;
   const int Kb = ceil_div(K, kGroup);
   const int Kq = ceil_div(Kb, 4);
+  const int Nb = ceil_div(N, 128);
   size_t off = kHeaderBytes;
-  w.sfa_off = off;
-  if (fmt == FG8_SCALE_UE8M0) {
-    off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
-    w.sfb_off = off;
-    off = align_up(off + static_cast<size_t>(ceil_div(N, 128)) * Kq * kSfChunkBytes, kAlign);
+  w.xs_off = off;
+  w.ld_s = kmajor_ld(M);
+  if (fmt == FG8_SCALE_FLOAT) {
+    off = align_up(off + static_cast<size_t>(Kb) * w.ld_s * sizeof(float), kAlign);
+    w.wsc_off = off;
+    off = align_up(off + static_cast<size_t>(Nb) * Kb * 16, kAlign);
   } else {
-    w.sfb_off = off;
+    off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
+    w.wsc_off = off;
+    off = align_up(off + static_cast<size_t>(sfb_rows(N) / 128) * Kq * kSfChunkBytes, kAlign);
   }
   w.total = off;
   return w;
@@ -232,10 +242,15 @@ fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t 
   a.ld_s = L.ld_s;
   a.Kq = Kq;
   a.M_pad = ceil_div(M, 128) * 128;
+  if (fmt == FG8_SCALE_FLOAT) {  // the weight-scale padding rides in the same launch
+    a.ws = static_cast<const float*>(w_scale_inv);
+    a.ws_pad = reinterpret_cast<float*>(ws + L.wsc_off);
+    a.Nb = ceil_div(N, 128);
+  }
   if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
   if (fmt == FG8_SCALE_UE8M0)
-    return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), 128, Kb,
-                                      ws + L.sfb_off, s));
+    return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), sfb_rows(N),
+                                      128, Kb, ws + L.wsc_off, s));
   return FG8_OK;
 }
 
@@ -269,13 +284,12 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
   if (fmt == FG8_SCALE_FLOAT) {
-    g.xs = reinterpret_cast<const float*>(ws + L.xs_off);
-    g.xs_sm = 1;
-    g.xs_sk = L.ld_s;
-    g.ws = static_cast<const float*>(w_scale_inv);
+    g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.ld_s = L.ld_s;
+    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
   } else {
     g.sfa = ws + L.xs_off;
-    g.sfb = ws + L.sfb_off;
+    g.sfb = ws + L.wsc_off;
   }
   return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
 }
@@ -334,21 +348,28 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
   if (fmt == FG8_SCALE_FLOAT) {
-    g.xs = static_cast<const float*>(x_scale);
-    g.xs_sm = Kb;
-    g.xs_sk = 1;
-    g.ws = static_cast<const float*>(w_scale_inv);
+    if (fg8_status st = cuda_status(launch_xs_transpose(static_cast<const float*>(x_scale), static_cast<int>(M), Kb,
+                                                        L.ld_s, reinterpret_cast<float*>(ws + L.xs_off), s));
+        st != FG8_OK)
+      return st;
+    if (fg8_status st = cuda_status(launch_ws_pad(static_cast<const float*>(w_scale_inv), ceil_div(N, 128), Kb,
+                                                  reinterpret_cast<float*>(ws + L.wsc_off), s));
+        st != FG8_OK)
+      return st;
+    g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.ld_s = L.ld_s;
+    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
   } else {
-    if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(x_scale), static_cast<int>(M), 1, Kb,
-                                                   ws + L.sfa_off, s));
+    if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(x_scale), static_cast<int>(M),
+                                                   (M + 127) / 128 * 128, 1, Kb, ws + L.xs_off, s));
         st != FG8_OK)
       return st;
     if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N),
-                                                   128, Kb, ws + L.sfb_off, s));
+                                                   sfb_rows(N), 128, Kb, ws + L.wsc_off, s));
         st != FG8_OK)
       return st;
-    g.sfa = ws + L.sfa_off;
-    g.sfb = ws + L.sfb_off;
+    g.sfa = ws + L.xs_off;
+    g.sfb = ws + L.wsc_off;
   }
   return cuda_status(launch_gemm(g, fmt, dev.sms, s));
 }

@@ -39,6 +39,10 @@ struct ActQuantArgs {
   int64_t ld_s;       // kScaleKMajor: column stride (>= M)
   int Kq;             // kScaleSfTiles: ceil(Kb / 4)
   int M_pad;          // kScaleSfTiles: rows rounded up to 128 (padding rows get scale 2^0)
+  // optional, same launch: float weight scales [Nb, Kb] -> 16-byte entries (ws_pad)
+  const float* ws;
+  float* ws_pad;
+  int Nb;
 };
 
 cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s);
@@ -47,9 +51,13 @@ cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8
                                 cudaStream_t s);
 
 // Pack a UE8M0 [R_src, Kb] row-major scale matrix into scale-factor tiles for
-// R rows (padded to 128): row r takes src[(r / row_div) * Kb + kb]; padding
-// rows and K-blocks get byte 127 (2^0).
-cudaError_t launch_sf_pack(const uint8_t* src, int R, int row_div, int Kb, uint8_t* dst, cudaStream_t s);
+// R rows, written for R_pad rows (a multiple of 128): row r takes
+// src[(r / row_div) * Kb + kb]; padding rows and K-blocks get byte 127 (2^0).
+cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, uint8_t* dst,
+                           cudaStream_t s);
+
+// Rows of weight scale-factor tiles: N rounded up to the widest GEMM tile.
+inline int64_t sfb_rows(int64_t N) { return (N + 255) / 256 * 256; }
 
 struct GemmArgs {
   const void* xq;     // e4m3 [M, K] row stride K
@@ -57,10 +65,11 @@ struct GemmArgs {
   void* y;            // bf16 [M, N] row stride ld_y
   int64_t ld_y;
   int M, N, K, Kb;
-  // float path: xs(m, kb) = xs[m * xs_sm + kb * xs_sk]; ws [Nb, Kb] row-major float32
-  const float* xs;
-  int64_t xs_sm, xs_sk;
-  const float* ws;
+  // float path: x scales K-major [Kb][ld_s] (ld_s a multiple of 128, >= M),
+  // weight scales padded to one 16-byte entry per (nb, kb) (see launch_ws_pad)
+  const float* xs_t;
+  int64_t ld_s;
+  const float* ws_pad;
   // UE8M0 path: scale-factor tiles of x (rows M) and W (rows N)
   const uint8_t* sfa;
   const uint8_t* sfb;
@@ -69,6 +78,18 @@ struct GemmArgs {
   uint32_t* status;   // device status word (0 = ok)
   uint64_t wait_limit_ns;
 };
+
+// Rows of the K-major float x-scale matrix: M rounded up to the GEMM tile.
+inline int64_t kmajor_ld(int64_t M) { return (M + 127) / 128 * 128; }
+
+// Float weight scales [Nb, Kb] -> [Nb, Kb] 16-byte entries {s, 0, 0, 0}
+// (what the GEMM's producer bulk-copies per K-block).
+cudaError_t launch_ws_pad(const float* ws, int Nb, int Kb, float* out, cudaStream_t s);
+
+// Float x scales row-major [M, Kb] -> K-major [Kb][ld_s].
+cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s);
+
+int choose_block_n(int M, int N, int num_sms);
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s);
 

@@ -6,29 +6,32 @@
 // through ("Transformers 中的细粒度 FP8 量化 ... 完全指南", §八 step 6 and the
 // block (128,128) + dynamic-activation fast path of §6.1).
 //
-// One persistent CTA per SM walks 128 x BN output tiles.  Warp roles:
-//   warp 0      TMA producer: A (128 x 128 e4m3) and B (BN x 128 e4m3) tiles
-//               per 128-wide K-block into a STAGES-deep shared-memory ring
-//               (128-byte swizzle), plus UE8M0 scale-factor tiles.
-//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32 each) per
-//               K-block into a TMEM accumulator buffer.
+// One persistent CTA per SM walks 128 x BN output tiles (BN = 128 or 256).
+// 384 threads in three warpgroups; the first gives up registers
+// (setmaxnreg 40-56) to the two epilogue warpgroups (setmaxnreg 224-232):
+//   warp 0      producer: per 128-wide K-block, TMA loads of the A tile
+//               (128 x 128 e4m3) and B tile (BN x 128 e4m3) into a STAGES-deep
+//               ring (128-byte swizzle); bulk copies of the K-block's scales
+//               (float path) into a scale ring, of UE8M0 scale-factor tiles
+//               (every 4th K-block), and of the tile's bias into a bias ring.
+//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32) per K-block.
 //   warp 2      TMEM allocator.
-//   warps 4..   epilogue warpgroups; warp w reads TMEM lanes 32*(w%4)..+31,
-//               warpgroup g owns columns [g*BN/EPI_WG, (g+1)*BN/EPI_WG).
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4)..+31; warpgroup g
+//               owns columns [g*BN/2, (g+1)*BN/2).
 //
-// Float scales (FMT 0): every K-block's partial product P_kb lands in its own
-// TMEM buffer (ring of 4); the epilogue promotes it in registers,
-// acc += P_kb * (sx * sw), so the float32 scales are applied exactly as given
-// -- they are never rounded to a power of two (§七 补充 names that hazard).
+// Float scales (FMT 0): each K-block's partial product P_kb goes to its own
+// TMEM buffer (512/BN of them); the epilogue promotes it in registers,
+// acc += P_kb * (sx * sw), applying the float32 scales exactly as given --
+// never rounded to a power of two (§七 补充 names that hazard).
 // UE8M0 scales (FMT 1): tcgen05.mma.kind::mxf8f6f4.block_scale applies the
-// power-of-two scales inside the tensor core (one scale per 32 K-elements,
-// every group of four equal), accumulating the whole K range in TMEM.
+// power-of-two scales inside the tensor core (one per 32 K-elements; four
+// equal ones per 128-block), accumulating the whole K range in TMEM.
 // Ragged edges: TMA zero-fills out-of-range rows/columns of A and B (they add
 // 0), and the bf16 TMA store clips rows >= M and columns >= N.
 //
-// Every wait is bounded (global-timer limit, shared abort flag); on expiry
-// the kernel records FG8_ERR_TIMEOUT in the status word, drains its own
-// in-flight copies and tensor-core ops, frees TMEM and returns.
+// Every wait is bounded (global-timer limit and a shared abort flag); on
+// expiry the kernel records FG8_ERR_TIMEOUT in the status word, drains its
+// own in-flight copies and tensor-core ops, frees TMEM and returns.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -39,41 +42,60 @@
 namespace fg8 {
 namespace {
 
-constexpr uint32_t kStatusTimeout = 6u;      // FG8_ERR_TIMEOUT
+constexpr uint32_t kStatusTimeout = 6u;  // FG8_ERR_TIMEOUT
 constexpr uint64_t kTeardownNs = 1000000000ull;
+constexpr int kMaxSmem = 232448;
 
 struct KParams {
-  int M, N, K, Kb, Kq;
+  int M, N, K, Kb, Kq, Nb;
   int num_m, num_n, num_tiles;
-  const float* xs;
-  int64_t xs_sm, xs_sk;
-  const float* ws;
-  const uint8_t* sfa;
+  const float* xs_t;    // float path: x scales, K-major [Kb][ld_s]
+  int64_t ld_s;
+  const float* ws_pad;  // float path: weight scales, one 16-byte entry per (nb, kb)
+  const uint8_t* sfa;   // UE8M0 path: scale-factor tiles
   const uint8_t* sfb;
   const uint16_t* bias;
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 
-template <int BN, int FMT, int STAGES, int EPI_WG>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_>
 struct Cfg {
+  static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
   static constexpr int kA = kBlockM * 128;
   static constexpr int kB = BN * 128;
-  static constexpr int kSF = FMT == 1 ? 2 * kSfChunkBytes : 0;
-  static constexpr int kStage = kA + kB + kSF;
-  static constexpr int kEpiWarps = 4 * EPI_WG;
-  static constexpr int kThreads = 128 + 32 * kEpiWarps;
-  static constexpr int kCols = BN / EPI_WG;
-  static constexpr int kNumAcc = FMT == 0 ? 512 / BN : (512 - 16) / BN;
-  static constexpr int kTmemCols = 512;
-  static constexpr int kStageOut = 32 * 32 * 2;  // one 32 x 32 bf16 box
-  static constexpr int kStagingBytes = kEpiWarps * 2 * kStageOut;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmem = 1024 + STAGES * kStage + kStagingBytes + kBarBytes;
-  static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment for the 128B swizzle");
-  static_assert(kCols % 32 == 0, "epilogue works in 32-column chunks");
-  static_assert(BN == 128, "one weight block row per tile (scale sw is per tile)");
-  static_assert(kSmem <= 232448, "shared memory budget");
+  static constexpr int kSfBytes = FMT == 1 ? kSfChunkBytes * (1 + BN / 128) : 0;
+  static constexpr int kStage = (kA + kB + kSfBytes + 1023) / 1024 * 1024;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 384;
+  static constexpr int kCols = BN / 2;  // columns per epilogue thread
+  static constexpr int kChunks = kCols / 32;
+  static constexpr int kNumAcc = FMT == 0 ? 512 / BN : (BN == 256 ? 1 : 3);
+  static constexpr int kSfaCol = kNumAcc * BN;
+  static constexpr int kSfbCol = kSfaCol + 4;
+  static constexpr int kScSlots = FMT == 0 ? 6 : 0;
+  static constexpr int kScSlot = 512 + 32;  // 128 x-scales, then two 16-byte weight-scale entries
+  static constexpr int kBiasSlot = BN * 2;
+  // register split after launch (384 x 168): the wide float epilogue holds
+  // 128 accumulators + 32 TMEM registers per thread, the others need less
+  static constexpr uint32_t kRegsLow = (FMT == 0 && BN == 256) ? 48 : (BN == 128 ? 80 : 56);
+  static constexpr uint32_t kRegsHigh = (FMT == 0 && BN == 256) ? 224 : (BN == 128 ? 208 : 224);
+  static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch allocation");
+  static constexpr int kOutBuf = 32 * 32 * 2;  // one 32 x 32 bf16 box
+  // output staging boxes per epilogue warp: with kChunks of them a warp never
+  // waits for its own TMA stores inside a tile
+  static constexpr int kOutBufs = OUTBUFS_;
+  static_assert(kOutBufs >= 1 && kOutBufs <= kChunks, "staging buffers per warp");
+  // shared memory map (offsets from the 1024-aligned base)
+  static constexpr int kOffStaging = STAGES * kStage;
+  static constexpr int kOffSc = kOffStaging + kEpiWarps * kOutBufs * kOutBuf;
+  static constexpr int kOffBias = kOffSc + kScSlots * kScSlot;
+  static constexpr int kOffBar = kOffBias + 2 * kBiasSlot;
+  static constexpr int kSmem = 1024 + kOffBar + 512;
+  static_assert(kSmem <= kMaxSmem, "shared memory budget");
+  static_assert(kStage % 1024 == 0, "stages keep 1024-byte alignment for the 128B swizzle");
+  static_assert(kOffSc % 16 == 0 && kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
+  static_assert(kNumAcc * BN + (FMT == 1 ? 4 + BN / 32 : 0) <= 512, "TMEM columns");
   // instruction descriptors (M = 128, K-major A and B, e4m3 x e4m3 -> f32)
   static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24);
   static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBlockM >> 4) << 24);
@@ -95,9 +117,31 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* 
   atomicExch(status, kStatusTimeout);
 }
 
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(r);
   tmem_ld_32x32b_x32(taddr, a);
+}
+
+// Ties 32 registers written by tcgen05.ld to the preceding tcgen05.wait::ld,
+// so no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_reg_fence(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -105,34 +149,344 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN, int FMT, int STAGES, int EPI_WG>
-__global__ void __launch_bounds__(Cfg<BN, FMT, STAGES, EPI_WG>::kThreads, 1)
+// Ring position: slot index and the parity of its current use.
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  template <int N>
+  __device__ __forceinline__ void advance() {
+    if (++slot == N) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// ---------------------------------------------------------------- roles ----
+template <class C>
+__device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
+                                         uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* scfull,
+                                         uint64_t* scempty, uint64_t* bfull, uint64_t* bempty,
+                                         volatile int* abort_flag) {
+  const uint64_t limit = p.wait_limit_ns;
+  Ring st, sc, bi;
+  // most recent issue phase per slot, for the drain at the end
+  uint32_t st_issued = 0, sc_issued = 0, bi_issued = 0;
+  uint32_t st_par[C::STAGES], sc_par[C::kScSlots > 0 ? C::kScSlots : 1], bi_par[2];
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    int mb, nb;
+    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    const int n0 = nb * C::BN;
+    // bias of the tile (clipped to N; nothing when there is no bias)
+    if (!mbar_wait(bempty + bi.slot, bi.phase ^ 1u, limit, abort_flag)) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    {
+      const int ncols = min(C::BN, p.N - n0);
+      const uint32_t bytes = p.bias != nullptr ? static_cast<uint32_t>(ncols) * 2u : 0u;
+      mbar_arrive_expect_tx(bfull + bi.slot, bytes);
+      if (bytes) bulk_load(smem + C::kOffBias + bi.slot * C::kBiasSlot, p.bias + n0, bytes, bfull + bi.slot);
+      bi_par[bi.slot] = bi.phase;
+      bi_issued |= 1u << bi.slot;
+      bi.template advance<2>();
+    }
+    for (int kb = 0; kb < p.Kb; ++kb) {
+      if (!mbar_wait(empty + st.slot, st.phase ^ 1u, limit, abort_flag)) {
+        raise_abort(abort_flag, p.status);
+        ok = false;
+        break;
+      }
+      const bool sf = C::FMT == 1 && (kb & 3) == 0;
+      uint8_t* sa = smem + st.slot * C::kStage;
+      mbar_arrive_expect_tx(full + st.slot, C::kA + C::kB + (sf ? C::kSfBytes : 0));
+      tma_load_2d(sa, tmA, full + st.slot, kb * 128, mb * kBlockM);
+      tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, n0);
+      if (sf) {
+        uint8_t* sfs = sa + C::kA + C::kB;
+        bulk_load(sfs, p.sfa + (static_cast<size_t>(mb) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
+                  full + st.slot);
+#pragma unroll
+        for (int h = 0; h < C::BN / 128; ++h)
+          bulk_load(sfs + kSfChunkBytes * (1 + h),
+                    p.sfb + (static_cast<size_t>(n0 / 128 + h) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
+                    full + st.slot);
+      }
+      st_par[st.slot] = st.phase;
+      st_issued |= 1u << st.slot;
+      st.template advance<C::STAGES>();
+      if (C::FMT == 0) {
+        if (!mbar_wait(scempty + sc.slot, sc.phase ^ 1u, limit, abort_flag)) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        const int nb0 = n0 / 128;
+        const bool second = C::BN == 256 && nb0 + 1 < p.Nb;
+        uint8_t* slot = smem + C::kOffSc + sc.slot * C::kScSlot;
+        mbar_arrive_expect_tx(scfull + sc.slot, 512u + 16u + (second ? 16u : 0u));
+        bulk_load(slot, p.xs_t + static_cast<int64_t>(kb) * p.ld_s + mb * kBlockM, 512u, scfull + sc.slot);
+        bulk_load(slot + 512, p.ws_pad + (static_cast<int64_t>(nb0) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
+        if (second)
+          bulk_load(slot + 528, p.ws_pad + (static_cast<int64_t>(nb0 + 1) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
+        sc_par[sc.slot] = sc.phase;
+        sc_issued |= 1u << sc.slot;
+        sc.template advance<(C::kScSlots > 0 ? C::kScSlots : 1)>();
+      }
+    }
+  }
+  // Every issued copy must have landed before the CTA's shared memory goes away.
+  for (int s = 0; s < C::STAGES; ++s)
+    if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
+  for (int s = 0; s < C::kScSlots; ++s)
+    if ((sc_issued >> s) & 1u) (void)mbar_wait(scfull + s, sc_par[s], kTeardownNs, nullptr);
+  for (int s = 0; s < 2; ++s)
+    if ((bi_issued >> s) & 1u) (void)mbar_wait(bfull + s, bi_par[s], kTeardownNs, nullptr);
+}
+
+template <class C>
+__device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint32_t tmem_base, uint64_t* full,
+                                           uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* teardown,
+                                           volatile int* abort_flag) {
+  const uint64_t limit = p.wait_limit_ns;
+  Ring st, ab;
+  bool ok = true;
+  const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
+  const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
+  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int kb = 0; kb < p.Kb; ++kb) {
+      if (!mbar_wait(full + st.slot, st.phase, limit, abort_flag)) {
+        raise_abort(abort_flag, p.status);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (C::FMT == 0 || kb == 0) {
+        if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      const uint32_t a_addr = smem_u32(smem + st.slot * C::kStage);
+      const uint32_t b_addr = a_addr + C::kA;
+      const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
+      if (C::FMT == 1 && (kb & 3) == 0) {
+        // UE8M0 scales of 128 rows x 4 K-blocks for A, and for B, into TMEM;
+        // issued before the MMAs that read them (tcgen05 ops of one thread
+        // execute in issue order).
+        const uint32_t sfs = b_addr + C::kB;
+        tc_cp_32x128b_warpx4(sfa_t, smem_desc(sfs, 128, 128, 0));
+#pragma unroll
+        for (int h = 0; h < C::BN / 128; ++h)
+          tc_cp_32x128b_warpx4(sfb_t + 4 * h, smem_desc(sfs + kSfChunkBytes * (1 + h), 128, 128, 0));
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
+        const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
+        if (C::FMT == 0) {
+          mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
+        } else {
+          const uint32_t j = static_cast<uint32_t>(kb & 3);
+          mma_mxf8f6f4(d, ad, bd, C::kIdescMx | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
+                       (kb > 0 || k > 0) ? 1u : 0u);
+        }
+      }
+      tc_commit(empty + st.slot);
+      if (C::FMT == 0 || kb == p.Kb - 1) {
+        tc_commit(tfull + ab.slot);
+        ab.template advance<C::kNumAcc>();
+      }
+      st.template advance<C::STAGES>();
+    }
+  }
+  // All issued tensor-core ops must finish before TMEM is released.
+  tc_commit(teardown);
+  (void)mbar_wait(teardown, 0, kTeardownNs, nullptr);
+}
+
+template <class C>
+__device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& p, uint8_t* smem, uint32_t tmem_base,
+                                         uint64_t* tfull, uint64_t* tempty, uint64_t* scfull, uint64_t* scempty,
+                                         uint64_t* bfull, uint64_t* bempty, volatile int* abort_flag, int warp,
+                                         int lane) {
+  const uint64_t limit = p.wait_limit_ns;
+  const int ew = warp - 4;
+  const int q = warp & 3;      // TMEM lane quadrant
+  const int wg = ew >> 2;      // column half of the tile
+  const int col0 = wg * C::kCols;
+  uint8_t* stg = smem + C::kOffStaging + ew * C::kOutBufs * C::kOutBuf;
+  const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+  Ring ab, sc, bi;
+  int nstore = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    int mb, nb;
+    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    const int row0 = mb * kBlockM + q * 32;
+    uint32_t acc[C::kCols];  // float bits
+    if (C::FMT == 0) {
+#pragma unroll
+      for (int j = 0; j < C::kCols; ++j) acc[j] = 0u;
+      for (int kb = 0; kb < p.Kb; ++kb) {
+        // scale of this row and K-block: sx(m, kb) * sw(block of my columns, kb)
+        if (!mbar_wait(scfull + sc.slot, sc.phase, limit, abort_flag)) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        const uint8_t* slot = smem + C::kOffSc + sc.slot * C::kScSlot;
+        const float sx = reinterpret_cast<const float*>(slot)[q * 32 + lane];
+        const float sw = *reinterpret_cast<const float*>(slot + 512 + (C::BN == 256 ? 16 * wg : 0));
+        const float s = sx * sw;
+        const float2 s2 = make_float2(s, s);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(scempty + sc.slot);
+        sc.template advance<(C::kScSlots > 0 ? C::kScSlots : 1)>();
+
+        if (!mbar_wait(tfull + ab.slot, ab.phase, limit, abort_flag)) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(ab.slot * C::BN + col0);
+        // TMEM -> registers in groups of up to 64 columns (two x32 loads, one
+        // wait), then packed f32x2 FMAs: one or two load round trips per
+        // K-block instead of one per 32 columns.
+        constexpr int GRP = C::kCols < 64 ? C::kCols : 64;
+#pragma unroll
+        for (int g0 = 0; g0 < C::kCols; g0 += GRP) {
+          uint32_t r[GRP];
+#pragma unroll
+          for (int c = 0; c < GRP / 32; ++c) tmem_ld32(taddr + g0 + c * 32, r + c * 32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < GRP / 32; ++c) tmem_reg_fence(r + c * 32);
+          if (g0 + GRP == C::kCols) {  // all of this K-block's columns are in registers: free the buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + ab.slot);
+          }
+#pragma unroll
+          for (int j = 0; j < GRP; j += 2) {  // packed f32x2 FMA: two promotions per instruction
+            const float2 r2 = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), s2,
+                                         make_float2(__uint_as_float(acc[g0 + j]), __uint_as_float(acc[g0 + j + 1])));
+            acc[g0 + j] = __float_as_uint(r2.x);
+            acc[g0 + j + 1] = __float_as_uint(r2.y);
+          }
+        }
+        ab.template advance<C::kNumAcc>();
+      }
+      if (!ok) break;
+    } else {
+      if (!mbar_wait(tfull + ab.slot, ab.phase, limit, abort_flag)) {
+        raise_abort(abort_flag, p.status);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(ab.slot * C::BN + col0);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) tmem_ld32(taddr + c * 32, acc + c * 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) tmem_reg_fence(acc + c * 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + ab.slot);
+      ab.template advance<C::kNumAcc>();
+    }
+
+    // + bias (from the bias ring), round to bf16, stage 32 x 32 boxes (64-byte
+    // swizzle) and store them with TMA.
+    if (!mbar_wait(bfull + bi.slot, bi.phase, limit, abort_flag)) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    const uint8_t* bias_s = smem + C::kOffBias + bi.slot * C::kBiasSlot;
+#pragma unroll
+    for (int c = 0; c < C::kChunks; ++c) {
+      const int nloc = col0 + c * 32;
+      const int n0 = nb * C::BN + nloc;
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+        if (p.bias != nullptr && n0 + 8 * i < p.N) bv = *reinterpret_cast<const uint4*>(bias_s + (nloc + 8 * i) * 2);
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int j = c * 32 + 8 * i + 2 * h;
+          w[4 * i + h] = pack_bf16x2(__uint_as_float(acc[j]) + __uint_as_float(bw[h] << 16),
+                                     __uint_as_float(acc[j + 1]) + __uint_as_float(bw[h] & 0xFFFF0000u));
+        }
+      }
+      uint8_t* buf = stg + (nstore % C::kOutBufs) * C::kOutBuf;
+      if (lane == 0) {  // the store that last used this buffer has read it
+        if (C::kOutBufs == 4) bulk_wait_group_read<3>();
+        else if (C::kOutBufs == 2) bulk_wait_group_read<1>();
+        else bulk_wait_group_read<0>();
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int chunk = i ^ ((lane >> 1) & 3);
+        *reinterpret_cast<uint4*>(buf + lane * 64 + chunk * 16) =
+            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (n0 < p.N && row0 < p.M) tma_store_2d(tmY, buf, n0, row0);
+        bulk_commit_group();
+      }
+      ++nstore;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bempty + bi.slot);
+    bi.template advance<2>();
+  }
+  if (lane == 0) bulk_wait_group<0>();
+}
+
+template <class C>
+__global__ void __launch_bounds__(384, 1)
     fg8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const KParams p) {
-  using C = Cfg<BN, FMT, STAGES, EPI_WG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* staging = smem + STAGES * C::kStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::kStagingBytes);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + C::kNumAcc;
-  uint64_t* teardown = tempty + C::kNumAcc;
+  uint64_t* scfull = tempty + C::kNumAcc;
+  uint64_t* scempty = scfull + C::kScSlots;
+  uint64_t* bfull = scempty + C::kScSlots;
+  uint64_t* bempty = bfull + 2;
+  uint64_t* teardown = bempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Kb = p.Kb;
-  const uint64_t limit = p.wait_limit_ns;
-
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
     for (int a = 0; a < C::kNumAcc; ++a) {
       mbar_init(tfull + a, 1);
       mbar_init(tempty + a, C::kEpiWarps);
+    }
+    for (int s = 0; s < C::kScSlots; ++s) {
+      mbar_init(scfull + s, 1);
+      mbar_init(scempty + s, C::kEpiWarps);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bfull + s, 1);
+      mbar_init(bempty + s, C::kEpiWarps);
     }
     mbar_init(teardown, 1);
     *abort_flag = 0;
@@ -144,7 +498,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT, STAGES, EPI_WG>::kThreads, 1)
     prefetch_tmap(&tmY);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -152,221 +506,21 @@ __global__ void __launch_bounds__(Cfg<BN, FMT, STAGES, EPI_WG>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer --
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, issued = 0;
-      uint32_t issued_par[STAGES];
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, p.num_m, p.num_n, mb, nb);
-        for (int kb = 0; kb < Kb; ++kb) {
-          if (!mbar_wait(empty + stage, phase ^ 1u, limit, abort_flag)) {
-            raise_abort(abort_flag, p.status);
-            ok = false;
-            break;
-          }
-          const bool sf = FMT == 1 && (kb & 3) == 0;
-          uint8_t* sa = smem + stage * C::kStage;
-          mbar_arrive_expect_tx(full + stage, C::kA + C::kB + (sf ? C::kSF : 0));
-          tma_load_2d(sa, &tmA, full + stage, kb * 128, mb * kBlockM);
-          tma_load_2d(sa + C::kA, &tmB, full + stage, kb * 128, nb * BN);
-          if (sf) {
-            bulk_load(sa + C::kA + C::kB, p.sfa + (static_cast<size_t>(mb) * p.Kq + (kb >> 2)) * kSfChunkBytes,
-                      kSfChunkBytes, full + stage);
-            bulk_load(sa + C::kA + C::kB + kSfChunkBytes,
-                      p.sfb + (static_cast<size_t>(nb) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
-                      full + stage);
-          }
-          issued_par[stage] = phase;
-          issued |= 1u << stage;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // Every issued copy must have landed before the CTA's shared memory goes away.
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) (void)mbar_wait(full + s, issued_par[s], kTeardownNs, nullptr);
-    }
-  } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
-      int stage = 0, abuf = 0;
-      uint32_t phase = 0, aphase = 0;
-      bool ok = true;
-      const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kNumAcc * BN);
-      const uint32_t sfb_t = sfa_t + 4;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        for (int kb = 0; kb < Kb; ++kb) {
-          if (!mbar_wait(full + stage, phase, limit, abort_flag)) {
-            raise_abort(abort_flag, p.status);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (FMT == 0 || kb == 0) {
-            if (!mbar_wait(tempty + abuf, aphase ^ 1u, limit, abort_flag)) {
-              raise_abort(abort_flag, p.status);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          const uint32_t a_addr = smem_u32(smem + stage * C::kStage);
-          const uint32_t b_addr = a_addr + C::kA;
-          const uint32_t d = tmem_base + static_cast<uint32_t>(abuf * BN);
-          if (FMT == 1 && (kb & 3) == 0) {
-            // 128 rows x 4 K-blocks of UE8M0 scales for A and for B into TMEM
-            // (issued before the MMAs that read them; tcgen05 ops of one
-            // thread execute in issue order).
-            tc_cp_32x128b_warpx4(sfa_t, smem_desc(b_addr + C::kB, 128, 128, 0));
-            tc_cp_32x128b_warpx4(sfb_t, smem_desc(b_addr + C::kB + kSfChunkBytes, 128, 128, 0));
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
-            if (FMT == 0) {
-              mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
-            } else {
-              const uint32_t j = static_cast<uint32_t>(kb & 3);
-              mma_mxf8f6f4(d, ad, bd, C::kIdescMx | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
-                           (kb > 0 || k > 0) ? 1u : 0u);
-            }
-          }
-          tc_commit(empty + stage);
-          if (FMT == 0 || kb == Kb - 1) {
-            tc_commit(tfull + abuf);
-            if (++abuf == C::kNumAcc) {
-              abuf = 0;
-              aphase ^= 1u;
-            }
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // All issued tensor-core ops must finish before TMEM is released.
-      tc_commit(teardown);
-      (void)mbar_wait(teardown, 0, kTeardownNs, nullptr);
-    }
-  } else if (warp >= 4) {
-    // ----------------------------------------------------------- epilogue --
-    const int ew = warp - 4;
-    const int q = warp & 3;
-    const int col0 = (ew >> 2) * C::kCols;
-    uint8_t* stg = staging + ew * 2 * C::kStageOut;
-    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int abuf = 0, nstore = 0;
-    uint32_t aphase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
-      const int row0 = mb * kBlockM + q * 32;
-      float acc[C::kCols];
-      uint32_t r[C::kCols];
-      if (FMT == 0) {
-#pragma unroll
-        for (int j = 0; j < C::kCols; ++j) acc[j] = 0.0f;
-        const int row_c = min(row0 + lane, p.M - 1);
-        const float* xs_row = p.xs + static_cast<int64_t>(row_c) * p.xs_sm;
-        const float* ws_row = p.ws + static_cast<int64_t>(nb) * Kb;
-        float sx = __ldg(xs_row), sw = __ldg(ws_row);
-        for (int kb = 0; kb < Kb; ++kb) {
-          const float sc = sx * sw;
-          if (kb + 1 < Kb) {
-            sx = __ldg(xs_row + static_cast<int64_t>(kb + 1) * p.xs_sk);
-            sw = __ldg(ws_row + kb + 1);
-          }
-          if (!mbar_wait(tfull + abuf, aphase, limit, abort_flag)) {
-            raise_abort(abort_flag, p.status);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN + col0);
-#pragma unroll
-          for (int c = 0; c < C::kCols / 32; ++c) tmem_ld32(taddr + c * 32, r + c * 32);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty + abuf);
-          if (++abuf == C::kNumAcc) {
-            abuf = 0;
-            aphase ^= 1u;
-          }
-#pragma unroll
-          for (int j = 0; j < C::kCols; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
-        }
-        if (!ok) break;
-      } else {
-        if (!mbar_wait(tfull + abuf, aphase, limit, abort_flag)) {
-          raise_abort(abort_flag, p.status);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN + col0);
-#pragma unroll
-        for (int c = 0; c < C::kCols / 32; ++c) tmem_ld32(taddr + c * 32, r + c * 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty + abuf);
-        if (++abuf == C::kNumAcc) {
-          abuf = 0;
-          aphase ^= 1u;
-        }
-#pragma unroll
-        for (int j = 0; j < C::kCols; ++j) acc[j] = __uint_as_float(r[j]);
-      }
-      // + bias, round to bf16, stage a 32 x 32 box (64-byte swizzle), TMA store.
-#pragma unroll
-      for (int c = 0; c < C::kCols / 32; ++c) {
-        const int n0 = nb * BN + col0 + c * 32;
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-          if (p.bias != nullptr && n0 + 8 * i < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * i));
-          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int j = c * 32 + 8 * i + 2 * h;
-            w[4 * i + h] = pack_bf16x2(acc[j] + __uint_as_float(bw[h] << 16), acc[j + 1] + __uint_as_float(bw[h] & 0xFFFF0000u));
-          }
-        }
-        uint8_t* buf = stg + (nstore & 1) * C::kStageOut;
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int chunk = i ^ ((lane >> 1) & 3);
-          *reinterpret_cast<uint4*>(buf + lane * 64 + chunk * 16) =
-              make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (n0 < p.N && row0 < p.M) tma_store_2d(&tmY, buf, n0, row0);
-          bulk_commit_group();
-        }
-        ++nstore;
-      }
-    }
-    if (lane == 0) bulk_wait_group<0>();
+  if (warp < 4) {
+    setmaxnreg_dec<C::kRegsLow>();
+    if (warp == 0 && lane == 0)
+      producer<C>(&tmA, &tmB, p, smem, full, empty, scfull, scempty, bfull, bempty, abort_flag);
+    else if (warp == 1 && lane == 0)
+      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, abort_flag);
+  } else {
+    setmaxnreg_inc<C::kRegsHigh>();
+    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, scfull, scempty, bfull, bempty, abort_flag, warp, lane);
   }
 
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -399,17 +553,17 @@ bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int FMT, int STAGES, int EPI_WG>
+template <class C>
 cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
-  using C = Cfg<BN, FMT, STAGES, EPI_WG>;
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K, g.M, g.K, 128, kBlockM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K, g.N, g.K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K, g.N, g.K, 128, C::BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, static_cast<uint64_t>(g.ld_y) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  auto kern = fg8_gemm_kernel<BN, FMT, STAGES, EPI_WG>;
+  auto kern = fg8_gemm_kernel<C>;
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -424,13 +578,13 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.K = g.K;
   p.Kb = g.Kb;
   p.Kq = g.Kq;
+  p.Nb = (g.N + 127) / 128;
   p.num_m = (g.M + kBlockM - 1) / kBlockM;
-  p.num_n = (g.N + BN - 1) / BN;
+  p.num_n = (g.N + C::BN - 1) / C::BN;
   p.num_tiles = p.num_m * p.num_n;
-  p.xs = g.xs;
-  p.xs_sm = g.xs_sm;
-  p.xs_sk = g.xs_sk;
-  p.ws = g.ws;
+  p.xs_t = g.xs_t;
+  p.ld_s = g.ld_s;
+  p.ws_pad = g.ws_pad;
   p.sfa = g.sfa;
   p.sfb = g.sfb;
   p.bias = static_cast<const uint16_t*>(g.bias);
@@ -444,9 +598,37 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
+int choose_block_n(int M, int N, int num_sms) {
+  // Per-CTA time ~ waves x (tile width / its throughput); the 256-wide tile
+  // moves ~1.6x more MMA work per operand byte and per epilogue instruction,
+  // so the 128-wide tile wins only when it cuts the wave count a lot.
+  const int64_t m_tiles = (M + kBlockM - 1) / kBlockM;
+  auto waves = [&](int bn) {
+    const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
+    return (tiles + num_sms - 1) / num_sms;
+  };
+  const double cost128 = static_cast<double>(waves(128)) * 128.0 / 0.6;
+  const double cost256 = static_cast<double>(waves(256)) * 256.0;
+  return cost128 < cost256 ? 128 : 256;
+}
+
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s) {
-  if (fmt == 0) return launch_cfg<128, 0, 5, 2>(g, num_sms, s);
-  return launch_cfg<128, 1, 5, 2>(g, num_sms, s);
+  const int bn = choose_block_n(g.M, g.N, num_sms);
+  // Short K: few K-blocks per tile, so the tile's output path dominates --
+  // give every output chunk its own staging box and keep one stage fewer.
+  const bool short_k = g.Kb <= 32;
+  if (fmt == 0) {
+    if (bn == 256) {
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 1>>(g, num_sms, s);
+    }
+    return launch_cfg<Cfg<128, 0, 5, 2>>(g, num_sms, s);
+  }
+  if (bn == 256) {
+    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4>>(g, num_sms, s);
+    return launch_cfg<Cfg<256, 1, 4, 1>>(g, num_sms, s);
+  }
+  return launch_cfg<Cfg<128, 1, 5, 2>>(g, num_sms, s);
 }
 
 }  // namespace fg8

@@ -47,6 +47,18 @@ __device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
   return copysignf(q, a);
 }
 
+// The same correctly rounded quotient for two values at once with packed
+// f32x2 arithmetic (each lane of FMUL2/FFMA2 rounds exactly like the scalar op).
+__device__ __forceinline__ float2 div2_rn_from_rcp(float2 a, float b, float y) {
+  const float2 Y = make_float2(y, y), nB = make_float2(-b, -b);
+  float2 q = __fmul2_rn(a, Y);
+  float2 r = __ffma2_rn(q, nB, a);
+  q = __ffma2_rn(r, Y, q);
+  r = __ffma2_rn(q, nB, a);
+  q = __ffma2_rn(r, Y, q);
+  return make_float2(copysignf(q.x, a.x), copysignf(q.y, a.y));
+}
+
 __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -60,6 +72,33 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
   const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
   return lo | (hi << 16);
+}
+
+// Quantize 16 values (two 16-byte bf16 loads) with the group's scale;
+// returns 16 packed e4m3 bytes.
+template <int FMT>
+__device__ __forceinline__ uint4 quantize16(const float (&f)[16], float s, uint32_t sbyte) {
+  float q[16];
+  if (FMT == 0) {
+    const float y = __frcp_rn(s);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 r = div2_rn_from_rcp(make_float2(f[i], f[i + 1]), s, y);
+      q[i] = r.x;
+      q[i + 1] = r.y;
+    }
+  } else {
+    const float inv = e8m0_reciprocal(sbyte);  // x * 2^-e is the correctly rounded x / 2^e
+    const float2 I = make_float2(inv, inv);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 r = __fmul2_rn(make_float2(f[i], f[i + 1]), I);
+      q[i] = r.x;
+      q[i + 1] = r.y;
+    }
+  }
+  return make_uint4(pack_e4m3x4(q[0], q[1], q[2], q[3]), pack_e4m3x4(q[4], q[5], q[6], q[7]),
+                    pack_e4m3x4(q[8], q[9], q[10], q[11]), pack_e4m3x4(q[12], q[13], q[14], q[15]));
 }
 
 // Quantize 8 values with the group's scale; returns 8 packed e4m3 bytes.
@@ -78,55 +117,99 @@ __device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s, uint32_
   return make_uint2(pack_e4m3x4(q[0], q[1], q[2], q[3]), pack_e4m3x4(q[4], q[5], q[6], q[7]));
 }
 
+// n / d and n % d for a divisor fixed per launch, by multiply-high (Granlund
+// and Montgomery, "Division by invariant integers using multiplication",
+// 1994): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// q = (t + ((n - t) >> 1)) >> (l - 1), t = umulhi(m, n), for all 32-bit n.
+struct FastDiv {
+  uint32_t d, m, l;
+};
+
+__host__ inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  while ((1ull << f.l) < d) ++f.l;
+  if (d > 1) f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << f.l) - d)) / d + 1);
+  return f;
+}
+
+__device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32_t& q, uint32_t& r) {
+  if (f.d == 1) {
+    q = n;
+  } else {
+    const uint32_t t = __umulhi(f.m, n);
+    q = (t + ((n - t) >> 1)) >> (f.l - 1);
+  }
+  r = n - q * f.d;
+}
+
 // ------------------------------------------------------------ act quant ----
-// A half-warp owns one 128-channel group: lane l loads channels [8l, 8l+8)
-// with one 16-byte load.  Each warp takes 8 groups per iteration (4 per half,
-// loads issued before any arithmetic) and strides over the grid.
+// Eight lanes own one 128-channel group: lane l loads channels [16l, 16l+16)
+// with two 16-byte loads.  A warp covers 4 groups per pass and makes 2 passes
+// per iteration (all loads issued before any arithmetic), striding over the
+// grid.  amax: per-lane max, then 3 xor-shuffles inside the 8 lanes.
 //   kScaleRowMajor: group g -> (m = g / Kb, kb = g % Kb)  (scales [M, Kb])
 //   kScaleKMajor / kScaleSfTiles: g -> (kb = g / rows, m = g % rows), so the
-//   scale writes of neighbouring half-warps are neighbouring addresses.
+//   scale writes of neighbouring lane-octets are neighbouring addresses.
 template <int FMT, int LAYOUT>
-__global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const int64_t total, const int rows,
-                                                        const int cols) {
-  const int lane = threadIdx.x & 31, half = lane >> 4, l = lane & 15;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+__global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const uint32_t total, const FastDiv div,
+                                                        const uint32_t quant_blocks) {
+  if (blockIdx.x >= quant_blocks) {
+    // trailing blocks: pad the float weight scales for the GEMM's bulk copies
+    const int64_t n = static_cast<int64_t>(a.Nb) * a.Kb;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x - quant_blocks) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x - quant_blocks) * blockDim.x)
+      reinterpret_cast<float4*>(a.ws_pad)[i] = make_float4(a.ws[i], 0.0f, 0.0f, 0.0f);
+    return;
+  }
+  constexpr int kPasses = 2;
+  const int lane = threadIdx.x & 31, oct = lane >> 3, l = lane & 7;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (quant_blocks * blockDim.x) >> 5;
   const uint16_t* x = static_cast<const uint16_t*>(a.x);
 
-  for (int64_t base = warp * 8; base < total; base += nwarps * 8) {
-    uint4 v[4];
-    int m[4], kb[4];
-    bool has[4], real[4];
+  for (uint32_t base = warp * (4 * kPasses); base < total; base += nwarps * (4 * kPasses)) {
+    uint4 v[kPasses][2];
+    int m[kPasses], kb[kPasses];
+    bool has[kPasses], real[kPasses];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t g = base + u * 2 + half;
+    for (int u = 0; u < kPasses; ++u) {
+      const uint32_t g = base + u * 4 + oct;
       has[u] = g < total;
+      uint32_t qt, r;
+      fast_divmod(div, g, qt, r);
       if (LAYOUT == kScaleRowMajor) {
-        m[u] = static_cast<int>(g / cols);
-        kb[u] = static_cast<int>(g % cols);
+        m[u] = static_cast<int>(qt);   // div = Kb
+        kb[u] = static_cast<int>(r);
       } else {
-        kb[u] = static_cast<int>(g / rows);
-        m[u] = static_cast<int>(g % rows);
+        kb[u] = static_cast<int>(qt);  // div = rows
+        m[u] = static_cast<int>(r);
       }
       real[u] = has[u] && m[u] < a.M && kb[u] < a.Kb;
-      const int k = kb[u] * kGroup + l * 8;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (real[u] && k < a.K) v[u] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m[u]) * a.ld_x + k));
+      const int k = kb[u] * kGroup + l * 16;
+      v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+      if (real[u] && k < a.K) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m[u]) * a.ld_x + k);
+        v[u][0] = __ldg(src);
+        v[u][1] = __ldg(src + 1);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float f[8];
-      unpack_bf16x8(v[u], f);
+    for (int u = 0; u < kPasses; ++u) {
+      float f[16];
+      float(&f0)[8] = *reinterpret_cast<float(*)[8]>(f);
+      float(&f1)[8] = *reinterpret_cast<float(*)[8]>(f + 8);
+      unpack_bf16x8(v[u][0], f0);
+      unpack_bf16x8(v[u][1], f1);
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+      for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
       const float s = group_scale(amax);
       const uint32_t sbyte = FMT == 1 ? e8m0_ceil_byte(s) : 0u;
-      const uint2 packed = quantize8<FMT>(f, s, sbyte);
-      const int k = kb[u] * kGroup + l * 8;
-      if (real[u] && k < a.K) *reinterpret_cast<uint2*>(a.xq + static_cast<int64_t>(m[u]) * a.K + k) = packed;
+      const uint4 packed = quantize16<FMT>(f, s, sbyte);
+      const int k = kb[u] * kGroup + l * 16;
+      if (real[u] && k < a.K) *reinterpret_cast<uint4*>(a.xq + static_cast<int64_t>(m[u]) * a.K + k) = packed;
       if (l == 0 && has[u]) {
         if (LAYOUT == kScaleRowMajor) {
           if (FMT == 0) static_cast<float*>(a.xs)[static_cast<int64_t>(m[u]) * a.Kb + kb[u]] = s;
@@ -207,7 +290,40 @@ __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict_
   }
 }
 
+__global__ void __launch_bounds__(256) ws_pad_kernel(const float* __restrict__ ws, const int64_t total,
+                                                     float4* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = make_float4(ws[i], 0.0f, 0.0f, 0.0f);
+}
+
+__global__ void __launch_bounds__(256) xs_transpose_kernel(const float* __restrict__ xs, const int M, const int Kb,
+                                                           const int64_t ld_s, float* __restrict__ out) {
+  const int64_t total = static_cast<int64_t>(M) * Kb;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t kb = i / M, m = i % M;  // consecutive threads write consecutive m
+    out[kb * ld_s + m] = xs[m * Kb + kb];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ws_pad(const float* ws, int Nb, int Kb, float* out, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(Nb) * Kb;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  ws_pad_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(ws, total, reinterpret_cast<float4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(M) * Kb;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8192) blocks = 8192;
+  xs_transpose_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(xs, M, Kb, ld_s, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s) {
   int rows, cols;
@@ -220,12 +336,21 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   }
   const int64_t total = static_cast<int64_t>(rows) * cols;
   if (total == 0) return cudaSuccess;
-  const int64_t per_block = 8 * 8;  // 8 warps x 8 groups per pass
+  if (total > 0x7FFFFFF0LL) return cudaErrorInvalidValue;  // group index is 32-bit
+  const FastDiv div = make_fastdiv(static_cast<uint32_t>(a.layout == kScaleRowMajor ? cols : rows));
+  const int64_t per_block = 8 * 8;  // 8 warps x 8 groups per iteration
   int64_t blocks = (total + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
-#define FG8_AQ(F, L) act_quant_kernel<F, L><<<grid, block, 0, s>>>(a, total, rows, cols)
+  int64_t aux_blocks = 0;
+  if (a.ws_pad != nullptr && fmt == 0) {
+    aux_blocks = (static_cast<int64_t>(a.Nb) * a.Kb + 255) / 256;
+    if (aux_blocks > 64) aux_blocks = 64;
+  }
+  const dim3 grid(static_cast<unsigned>(blocks + aux_blocks)), block(256);
+  const uint32_t t32 = static_cast<uint32_t>(total);
+  const uint32_t qb = static_cast<uint32_t>(blocks);
+#define FG8_AQ(F, L) act_quant_kernel<F, L><<<grid, block, 0, s>>>(a, t32, div, qb)
   if (fmt == 0) {
     if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor);
     else FG8_AQ(0, kScaleKMajor);
@@ -246,9 +371,10 @@ cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8
   return cudaGetLastError();
 }
 
-cudaError_t launch_sf_pack(const uint8_t* src, int R, int row_div, int Kb, uint8_t* dst, cudaStream_t s) {
+cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, uint8_t* dst,
+                           cudaStream_t s) {
   const int Kq = (Kb + 3) / 4;
-  const int64_t R_pad = (static_cast<int64_t>(R) + 127) / 128 * 128;
+  if (R_pad % 128 != 0 || R_pad < R) return cudaErrorInvalidValue;
   const int64_t total = R_pad * Kq * 4;
   int64_t blocks = (total + 255) / 256;
   if (blocks > 4096) blocks = 4096;

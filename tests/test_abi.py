@@ -135,8 +135,10 @@ def test_workspace_sizes(fg8):
     b = f(8192, 18432, 7168, 1)
     assert b >= 8192 * 7168
     assert f(0, 256, 256, 0) > 0
-    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 0) == 256
-    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 1) > 256
+    # pre-quantized GEMM: header + scales in the GEMM's layouts (x: K-major
+    # float32 over 128-row-padded M; W: 16-byte entries per 128x128 block)
+    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 0) >= 256 + 2 * 128 * 4 + 2 * 2 * 16
+    assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 1) >= 256 + 512 + 2 * 512
 
 
 def test_scale_fmt_validation(fg8):

@@ -163,6 +163,23 @@ def full_size_case(fg8, orc, cfg, gemm, stage=1):
     return check_y(_bits(y)[rows], y64, bound, gemm.name)
 
 
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(8192, 2176, 256), (8192, 384, 1040), (8192, 480, 384)])
+def test_wide_tiles_ragged_n(fg8, orc, fmt, M, N, K):
+    """Shapes whose tile choice is 256 columns wide with a ragged last tile
+    (half or fully past N), sampled rows."""
+    x = W.x_outliers(M, K, seed=M + N + K).cuda()
+    w = W.w_row_groups(N, K, 0.02, seed=N * 3 + K).cuda()
+    b = W.normal((N,), 0.1, seed=N + 1).cuda()
+    wq, ws = fg8.quantize_weight(w, fmt)
+    y = fg8.linear(x, wq, ws, b, fmt)
+    torch.cuda.synchronize()
+    owq, ows = orc.quantize_weight(_bits(w), fmt)
+    rows = _sample_rows(M, n=24, seed=N)
+    y64, bound, _ = orc.linear(_bits(x), owq, ows, _bits(b), fmt, rows=rows)
+    check_y(_bits(y)[rows], y64, bound, f"{M}x{N}x{K}")
+
+
 @pytest.mark.parametrize("stage", [1, 2])
 def test_fullsize_esm2(fg8, orc, stage):
     g = W.ESM_W1 if stage == 1 else W.ESM_W2
