@@ -27,6 +27,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_gemm_prequant,
     fg8_gemm_workspace_bytes,
     fg8_linear,
+    fg8_linear_noalloc,
     fg8_linear_prepare,
     fg8_linear_run,
     fg8_linear_workspace_bytes,

@@ -1,0 +1,81 @@
+// noalloc.cu -- fg8_linear for callers that cannot allocate device memory.
+//
+// fg8_linear needs a caller-provided device workspace.  Some callers have no
+// way to provide one: a host framework that owns every byte of device memory
+// through its own pool and forbids other allocations, or latency-critical code
+// that must never call cudaMalloc (which can synchronize the whole device).
+// fg8_linear_noalloc serves them with a fixed scratch buffer that lives in
+// this library's own device memory: a file-scope __device__ array of
+// kNoAllocScratchBytes, created when the module is loaded on a device and
+// kept until the process exits.  Nothing here calls cudaMalloc, cudaFree or
+// any allocating routine.
+
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "fg8.h"
+#include "fg8_internal.h"
+
+namespace {
+
+// 32 MiB: enough for, e.g., 8192 tokens x 3584 input channels, or the ESM-2
+// and Llama-3-8B shapes up to 2048 tokens (the workspace is M*K bytes of
+// quantized activations plus their scales and the weight scales).
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+
+// The scratch.  In host code this name is only a stand-in for the device
+// symbol; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per
+// device (this may load the module, so it must not run inside a stream
+// capture).  Returns nullptr on failure.
+void* scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                         const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                         void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* stream) {
+  if (M == 0) {  // nothing to compute; argument checks as fg8_linear
+    return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, nullptr, 0,
+                      stream);
+  }
+  const size_t need = fg8_linear_workspace_bytes(M, N, K, fmt);
+  if (need == 0) {  // bad shape or format: let fg8_linear report which
+    return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, nullptr, 0,
+                      stream);
+  }
+  if (need > kNoAllocScratchBytes) return FG8_ERR_WORKSPACE;  // shape too large for the fixed scratch
+  void* scratch = scratch_for_current_device();
+  if (scratch == nullptr) return FG8_ERR_CUDA;
+  // The scratch keeps the previous call's bytes; the only part that must
+  // start at zero is the device status word at its head.
+  if (cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FG8_ERR_CUDA;
+  }
+  return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, scratch,
+                    kNoAllocScratchBytes, stream);
+}

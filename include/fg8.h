@@ -128,6 +128,29 @@ FG8_API fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, 
                                   void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
                                   fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream);
 
+/* fg8_linear without a caller workspace, for callers that cannot allocate
+ * device memory (for example a host framework that owns all device memory
+ * through its own pool, or code that must never call cudaMalloc because it
+ * can synchronize the device).  The pages have no counterpart of this entry
+ * point; it computes exactly what fg8_linear computes, with the same
+ * arguments minus the workspace.
+ *   - Scratch: a fixed 32 MiB array in this library's device memory (a
+ *     file-scope __device__ array; every device that loads the library keeps
+ *     it until the process exits).  No call allocates or frees anything.
+ *   - Size limit: shapes whose fg8_linear_workspace_bytes(M, N, K, fmt)
+ *     exceeds 32 MiB return FG8_ERR_WORKSPACE without launching.
+ *   - The first call on each device looks up the scratch's device address
+ *     (this may load the library's device module); make that first call
+ *     before any stream capture on that device.
+ *   - All calls on a device share the one scratch, which keeps the previous
+ *     call's contents; each call clears the part that must start at zero.
+ *     Calls that overlap on the GPU (different streams, or concurrent host
+ *     threads) race on it: serialize them.
+ *   - Device-side wait timeouts are not reported through this entry point. */
+FG8_API fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                      const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                      void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* stream);
+
 /* Bytes of workspace fg8_gemm_prequant needs.  0 on bad arguments. */
 FG8_API size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
 
