@@ -65,7 +65,7 @@ struct GemmArgs {
   void* y;            // bf16 [M, N] row stride ld_y
   int64_t ld_y;
   int M, N, K, Kb;
-  // float path: x scales K-major [Kb][ld_s] (ld_s a multiple of 128, >= M),
+  // float path: x scales K-major [Kb][ld_s] (ld_s a multiple of 256, >= M),
   // weight scales padded to one 16-byte entry per (nb, kb) (see launch_ws_pad)
   const float* xs_t;
   int64_t ld_s;
@@ -79,8 +79,9 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 
-// Rows of the K-major float x-scale matrix: M rounded up to the GEMM tile.
-inline int64_t kmajor_ld(int64_t M) { return (M + 127) / 128 * 128; }
+// Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM
+// tile (256 rows for a CTA pair), so every tile's 128-row slices are in range.
+inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256 * 256; }
 
 // Float weight scales [Nb, Kb] -> [Nb, Kb] 16-byte entries {s, 0, 0, 0}
 // (what the GEMM's producer bulk-copies per K-block).

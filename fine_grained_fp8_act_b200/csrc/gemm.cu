@@ -59,11 +59,16 @@ struct KParams {
   uint64_t wait_limit_ns;
 };
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool PAIR_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
+  // PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
+  // MMAs; each CTA holds 128 rows of A and of the result, and BN/2 rows of B.
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;
   static constexpr int kA = kBlockM * 128;
-  static constexpr int kB = BN * 128;
+  static constexpr int kB = kBRows * 128;
   static constexpr int kSfBytes = FMT == 1 ? kSfChunkBytes * (1 + BN / 128) : 0;
   static constexpr int kStage = (kA + kB + kSfBytes + 1023) / 1024 * 1024;
   static constexpr int kEpiWarps = 8;
@@ -96,9 +101,14 @@ struct Cfg {
   static_assert(kStage % 1024 == 0, "stages keep 1024-byte alignment for the 128B swizzle");
   static_assert(kOffSc % 16 == 0 && kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
   static_assert(kNumAcc * BN + (FMT == 1 ? 4 + BN / 32 : 0) <= 512, "TMEM columns");
-  // instruction descriptors (M = 128, K-major A and B, e4m3 x e4m3 -> f32)
-  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24);
-  static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBlockM >> 4) << 24);
+  static_assert(!PAIR || (FMT == 0 && BN == 256), "CTA pairs: float scales, 256-wide tiles");
+  // bytes the stage's full barrier (in the pair's first CTA) waits for
+  static constexpr uint32_t kStageTx = (PAIR ? 2 : 1) * (kA + kB);
+  // arrivals that free a TMEM buffer: every epilogue warp of the pair
+  static constexpr uint32_t kTmemEmptyCount = (PAIR ? 2 : 1) * kEpiWarps;
+  // instruction descriptors (M = 128 or 256, K-major A and B, e4m3 x e4m3 -> f32)
+  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
+  static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kTileM >> 4) << 24);
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
@@ -110,6 +120,24 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb
   const int r = t - g * span;
   mb = first_m + r % gm;
   nb = r / gm;
+}
+
+// Persistent tile walk: single CTAs stride over tiles by the grid, CTA pairs
+// by the number of clusters.
+template <class C>
+__device__ __forceinline__ int tile_start() {
+  if constexpr (C::PAIR) return static_cast<int>(cluster_id_x());
+  else return static_cast<int>(blockIdx.x);
+}
+template <class C>
+__device__ __forceinline__ int tile_stride() {
+  if constexpr (C::PAIR) return static_cast<int>(nclusters_x());
+  else return static_cast<int>(gridDim.x);
+}
+template <class C>
+__device__ __forceinline__ int cta_rank() {
+  if constexpr (C::PAIR) return static_cast<int>(cluster_ctarank());
+  else return 0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
@@ -162,6 +190,17 @@ struct Ring {
   }
 };
 
+// An epilogue warp's release of a TMEM buffer: the MMA issuer waits on the
+// barrier of the pair's first CTA, so the second CTA arrives there remotely.
+template <class C>
+__device__ __forceinline__ void release_tmem(uint64_t* bar) {
+  if constexpr (C::PAIR) {
+    mbar_arrive_cluster(mapa_shared(bar, 0));
+  } else {
+    mbar_arrive(bar);
+  }
+}
+
 // ---------------------------------------------------------------- roles ----
 template <class C>
 __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
@@ -174,10 +213,12 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
   uint32_t st_issued = 0, sc_issued = 0, bi_issued = 0;
   uint32_t st_par[C::STAGES], sc_par[C::kScSlots > 0 ? C::kScSlots : 1], bi_par[2];
   bool ok = true;
-  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+  const int rank = cta_rank<C>();
+  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int n0 = nb * C::BN;
+    const int m0 = mb * C::kTileM + rank * kBlockM;  // this CTA's rows
     // bias of the tile (clipped to N; nothing when there is no bias)
     if (!mbar_wait(bempty + bi.slot, bi.phase ^ 1u, limit, abort_flag)) {
       raise_abort(abort_flag, p.status);
@@ -200,12 +241,21 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       }
       const bool sf = C::FMT == 1 && (kb & 3) == 0;
       uint8_t* sa = smem + st.slot * C::kStage;
-      mbar_arrive_expect_tx(full + st.slot, C::kA + C::kB + (sf ? C::kSfBytes : 0));
-      tma_load_2d(sa, tmA, full + st.slot, kb * 128, mb * kBlockM);
-      tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, n0);
+      if constexpr (C::PAIR) {
+        // both CTAs' tiles complete on the first CTA's full barrier, which
+        // the first CTA arms with the pair's total byte count
+        if (rank == 0) mbar_arrive_expect_tx(full + st.slot, C::kStageTx);
+        const uint32_t bar = mapa_shared(full + st.slot, 0);
+        tma_load_2d_pair(sa, tmA, bar, kb * 128, m0);
+        tma_load_2d_pair(sa + C::kA, tmB, bar, kb * 128, n0 + rank * C::kBRows);
+      } else {
+        mbar_arrive_expect_tx(full + st.slot, C::kStageTx + (sf ? C::kSfBytes : 0));
+        tma_load_2d(sa, tmA, full + st.slot, kb * 128, m0);
+        tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, n0);
+      }
       if (sf) {
         uint8_t* sfs = sa + C::kA + C::kB;
-        bulk_load(sfs, p.sfa + (static_cast<size_t>(mb) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
+        bulk_load(sfs, p.sfa + (static_cast<size_t>(m0 / kBlockM) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
                   full + st.slot);
 #pragma unroll
         for (int h = 0; h < C::BN / 128; ++h)
@@ -226,7 +276,7 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
         const bool second = C::BN == 256 && nb0 + 1 < p.Nb;
         uint8_t* slot = smem + C::kOffSc + sc.slot * C::kScSlot;
         mbar_arrive_expect_tx(scfull + sc.slot, 512u + 16u + (second ? 16u : 0u));
-        bulk_load(slot, p.xs_t + static_cast<int64_t>(kb) * p.ld_s + mb * kBlockM, 512u, scfull + sc.slot);
+        bulk_load(slot, p.xs_t + static_cast<int64_t>(kb) * p.ld_s + m0, 512u, scfull + sc.slot);
         bulk_load(slot + 512, p.ws_pad + (static_cast<int64_t>(nb0) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
         if (second)
           bulk_load(slot + 528, p.ws_pad + (static_cast<int64_t>(nb0 + 1) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
@@ -237,8 +287,12 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
     }
   }
   // Every issued copy must have landed before the CTA's shared memory goes away.
-  for (int s = 0; s < C::STAGES; ++s)
-    if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
+  // (A pair's tile loads complete on the first CTA's barriers: it waits for
+  // both CTAs' copies there; the kernel's final cluster barrier keeps the
+  // second CTA alive until then.)
+  if (rank == 0)
+    for (int s = 0; s < C::STAGES; ++s)
+      if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
   for (int s = 0; s < C::kScSlots; ++s)
     if ((sc_issued >> s) & 1u) (void)mbar_wait(scfull + s, sc_par[s], kTeardownNs, nullptr);
   for (int s = 0; s < 2; ++s)
@@ -254,7 +308,7 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   bool ok = true;
   const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
-  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     for (int kb = 0; kb < p.Kb; ++kb) {
       if (!mbar_wait(full + st.slot, st.phase, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
@@ -287,7 +341,9 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
       for (int k = 0; k < 4; ++k) {
         const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
         const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
-        if (C::FMT == 0) {
+        if (C::PAIR) {
+          mma_f8f6f4_pair(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
+        } else if (C::FMT == 0) {
           mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
         } else {
           const uint32_t j = static_cast<uint32_t>(kb & 3);
@@ -295,16 +351,28 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
                        (kb > 0 || k > 0) ? 1u : 0u);
         }
       }
-      tc_commit(empty + st.slot);
+      if constexpr (C::PAIR) {
+        tc_commit_pair(empty + st.slot, 0x3);  // frees the stage in both CTAs
+      } else {
+        tc_commit(empty + st.slot);
+      }
       if (C::FMT == 0 || kb == p.Kb - 1) {
-        tc_commit(tfull + ab.slot);
+        if constexpr (C::PAIR) {
+          tc_commit_pair(tfull + ab.slot, 0x3);
+        } else {
+          tc_commit(tfull + ab.slot);
+        }
         ab.template advance<C::kNumAcc>();
       }
       st.template advance<C::STAGES>();
     }
   }
   // All issued tensor-core ops must finish before TMEM is released.
-  tc_commit(teardown);
+  if constexpr (C::PAIR) {
+    tc_commit_pair(teardown, 0x1);
+  } else {
+    tc_commit(teardown);
+  }
   (void)mbar_wait(teardown, 0, kTeardownNs, nullptr);
 }
 
@@ -323,10 +391,11 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   Ring ab, sc, bi;
   int nstore = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+  const int rank = cta_rank<C>();
+  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
-    const int row0 = mb * kBlockM + q * 32;
+    const int row0 = mb * C::kTileM + rank * kBlockM + q * 32;
     uint32_t acc[C::kCols];  // float bits
     if (C::FMT == 0) {
 #pragma unroll
@@ -369,7 +438,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
           if (g0 + GRP == C::kCols) {  // all of this K-block's columns are in registers: free the buffer
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty + ab.slot);
+            if (lane == 0) release_tmem<C>(tempty + ab.slot);
           }
 #pragma unroll
           for (int j = 0; j < GRP; j += 2) {  // packed f32x2 FMA: two promotions per instruction
@@ -396,7 +465,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       for (int c = 0; c < C::kChunks; ++c) tmem_reg_fence(acc + c * 32);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty + ab.slot);
+      if (lane == 0) release_tmem<C>(tempty + ab.slot);
       ab.template advance<C::kNumAcc>();
     }
 
@@ -478,7 +547,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int a = 0; a < C::kNumAcc; ++a) {
       mbar_init(tfull + a, 1);
-      mbar_init(tempty + a, C::kEpiWarps);
+      mbar_init(tempty + a, C::kTmemEmptyCount);
     }
     for (int s = 0; s < C::kScSlots; ++s) {
       mbar_init(scfull + s, 1);
@@ -498,29 +567,51 @@ __global__ void __launch_bounds__(384, 1)
     prefetch_tmap(&tmY);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync();  // the peer's barriers are initialised before any use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above overlapped the preceding kernel (programmatic dependent
+  // launch); from here on its outputs (quantized activations, scales) are read.
+  grid_wait_prerequisites();
+  grid_launch_dependents();  // the next kernel may take SMs as this grid's CTAs finish
 
   if (warp < 4) {
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
       producer<C>(&tmA, &tmB, p, smem, full, empty, scfull, scempty, bfull, bempty, abort_flag);
-    else if (warp == 1 && lane == 0)
+    else if (warp == 1 && lane == 0 && cta_rank<C>() == 0)
       mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, abort_flag);
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
     epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, scfull, scempty, bfull, bempty, abort_flag, warp, lane);
   }
 
+  if (C::PAIR && *abort_flag) {
+    // after an abort the peer may still have copies in flight into this CTA:
+    // give them a bounded moment to land before the pair tears down
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 50000ull) {
+    }
+  }
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync();  // the first CTA's MMAs use this CTA's shared memory and TMEM
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    if constexpr (C::PAIR) {
+      tmem_dealloc_pair(tmem_base, 512);
+    } else {
+      tmem_dealloc(tmem_base, 512);
+    }
   }
 }
 
@@ -558,20 +649,12 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K, g.M, g.K, 128, kBlockM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K, g.N, g.K, 128, C::BN,
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K, g.N, g.K, 128, C::kBRows,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, static_cast<uint64_t>(g.ld_y) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   auto kern = fg8_gemm_kernel<C>;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
   KParams p;
   p.M = g.M;
   p.N = g.N;
@@ -579,7 +662,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.Kb = g.Kb;
   p.Kq = g.Kq;
   p.Nb = (g.N + 127) / 128;
-  p.num_m = (g.M + kBlockM - 1) / kBlockM;
+  p.num_m = (g.M + C::kTileM - 1) / C::kTileM;
   p.num_n = (g.N + C::BN - 1) / C::BN;
   p.num_tiles = p.num_m * p.num_n;
   p.xs_t = g.xs_t;
@@ -591,8 +674,52 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.status = g.status;
   p.wait_limit_ns = g.wait_limit_ns;
   if (p.num_tiles == 0) return cudaSuccess;
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  kern<<<grid, C::kThreads, C::kSmem, s>>>(tA, tB, tY, p);
+
+  static int configured_device = -1;
+  static int max_clusters = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  // start early behind the activation quantization (the kernel waits for its
+  // results before reading them)
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if constexpr (C::PAIR) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  if (configured_device != dev) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    if constexpr (C::PAIR) {
+      // how many CTA pairs fit on the device at once (SMs pair up within a GPC)
+      cfg.gridDim = dim3(2 * (num_sms / 2));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms / 2;
+      }
+      max_clusters = n;
+    }
+    configured_device = dev;
+  }
+  if constexpr (C::PAIR) {
+    const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+    cfg.gridDim = dim3(2 * clusters);
+  } else {
+    cfg.gridDim = dim3(p.num_tiles < num_sms ? p.num_tiles : num_sms);
+  }
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

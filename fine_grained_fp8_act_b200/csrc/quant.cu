@@ -15,6 +15,7 @@
 #include <cuda_fp8.h>
 
 #include "fg8_internal.h"
+#include "ptx.cuh"
 
 namespace fg8 {
 namespace {
@@ -153,6 +154,8 @@ __device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32
 template <int FMT, int LAYOUT>
 __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const uint32_t total, const FastDiv div,
                                                         const uint32_t quant_blocks) {
+  grid_wait_prerequisites();  // x may come from the preceding kernel (launched ahead of its end)
+  grid_launch_dependents();   // the GEMM may set itself up meanwhile; it waits for our results
   if (blockIdx.x >= quant_blocks) {
     // trailing blocks: pad the float weight scales for the GEMM's bulk copies
     const int64_t n = static_cast<int64_t>(a.Nb) * a.Kb;
@@ -280,6 +283,8 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const uint16_t* __res
 __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict__ src, const int R, const int row_div,
                                                       const int Kb, const int Kq, const int64_t total,
                                                       uint8_t* __restrict__ dst) {
+  grid_wait_prerequisites();
+  grid_launch_dependents();
   const int cols = Kq * 4;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -350,7 +355,16 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   const dim3 grid(static_cast<unsigned>(blocks + aux_blocks)), block(256);
   const uint32_t t32 = static_cast<uint32_t>(total);
   const uint32_t qb = static_cast<uint32_t>(blocks);
-#define FG8_AQ(F, L) act_quant_kernel<F, L><<<grid, block, 0, s>>>(a, t32, div, qb)
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start behind a GEMM's tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+#define FG8_AQ(F, L) cudaLaunchKernelEx(&cfg, act_quant_kernel<F, L>, a, t32, div, qb)
   if (fmt == 0) {
     if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor);
     else FG8_AQ(0, kScaleKMajor);
@@ -378,7 +392,17 @@ cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div
   const int64_t total = R_pad * Kq * 4;
   int64_t blocks = (total + 255) / 256;
   if (blocks > 4096) blocks = 4096;
-  sf_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(src, R, row_div, Kb, Kq, total, dst);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_pack_kernel, src, R, row_div, Kb, Kq, total, dst);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -180,6 +180,23 @@ def test_wide_tiles_ragged_n(fg8, orc, fmt, M, N, K):
     check_y(_bits(y)[rows], y64, bound, f"{M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(2176, 2304, 384), (4000, 2560, 1040), (8176, 1920, 480)])
+def test_cta_pair_tiles(fg8, orc, M, N, K):
+    """Float shapes large enough for the CTA-pair (256 x 256) tiles: a last
+    pair tile whose second CTA is entirely past M, ragged K, the ESM-2 shape."""
+    x = W.x_outliers(M, K, seed=M + 2 * K).cuda()
+    w = W.w_row_groups(N, K, 0.02, seed=N + 5 * K).cuda()
+    b = W.normal((N,), 0.1, seed=N + 7).cuda()
+    wq, ws = fg8.quantize_weight(w, FLOAT)
+    y = fg8.linear(x, wq, ws, b, FLOAT)
+    torch.cuda.synchronize()
+    owq, ows = orc.quantize_weight(_bits(w), FLOAT)
+    rows = np.unique(np.concatenate([_sample_rows(M, n=24, seed=K), [M - 129, M - 128, M - 1, 255, 256]]))
+    rows = rows[(rows >= 0) & (rows < M)].astype(np.int64)
+    y64, bound, _ = orc.linear(_bits(x), owq, ows, _bits(b), FLOAT, rows=rows)
+    check_y(_bits(y)[rows], y64, bound, f"{M}x{N}x{K}")
+
+
 @pytest.mark.parametrize("stage", [1, 2])
 def test_fullsize_esm2(fg8, orc, stage):
     g = W.ESM_W1 if stage == 1 else W.ESM_W2
