@@ -7,7 +7,10 @@ linear of the workload, dynamic per-token activation quantization (1x128
 groups) followed by the block-scaled FP8 GEMM with the bf16 epilogue.  The
 default workload is the ESM-2 35M-shaped FFN (8 x 1022 = 8176 tokens,
 hidden 480 -> FFN 1920 -> 480, float scales, both GEMMs back to back, no
-activation function between them), on synthetic seeded inputs.
+activation function between them), on synthetic seeded inputs.  By default
+the layers chain: the first GEMM's epilogue quantizes its bf16 output for
+the second layer (the same bytes a separate act-quant launch writes), so a
+step is act-quant, GEMM, GEMM; --no-chain gives each layer its own act-quant.
 
 Rank 0 prints ONE JSON line.  `value` is whole-job TFLOP/s (2*M*N*K summed
 over the step's GEMMs, all ranks, / the max-over-ranks device time); weak
@@ -214,14 +217,26 @@ def run_fg8(args, rank, world, local):
         L["x"] = x0 if i == 0 else plan[i - 1]["y"]
         assert L["x"].shape == (L["g"].M, L["g"].K), "consecutive layers must chain"
 
-    def launch_layer(L, ev_mid=None):
+    # Consecutive layers chain: the GEMM of layer i also quantizes its output
+    # for layer i+1 (fg8_linear_run_chain), so layer i+1 has no act-quant launch.
+    chain = not args.no_chain
+
+    def launch_layer(i, ev_mid=None):
+        L = plan[i]
         g = L["g"]
-        fg8.fg8_linear_prepare(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["ws"].data_ptr(), g.fmt,
-                               L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+        if i == 0 or not chain:
+            fg8.fg8_linear_prepare(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["ws"].data_ptr(), g.fmt,
+                                   L["wsp"].data_ptr(), L["wsp"].numel(), sp)
         if ev_mid is not None:
             ev_mid.record(stream)
-        fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), g.M, g.N,
-                           g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+        if chain and i + 1 < len(plan):
+            Ln = plan[i + 1]
+            fg8.fg8_linear_run_chain(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(),
+                                     g.M, g.N, g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(),
+                                     Ln["g"].N, Ln["ws"].data_ptr(), Ln["wsp"].data_ptr(), Ln["wsp"].numel(), sp)
+        else:
+            fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), g.M,
+                               g.N, g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -242,15 +257,15 @@ def run_fg8(args, rank, world, local):
     def step(e=None):
         if e is not None:
             e[0].record(stream)
-        for i, L in enumerate(plan):
-            launch_layer(L, None if e is None else e[1 + 2 * i])
+        for i in range(nl):
+            launch_layer(i, None if e is None else e[1 + 2 * i])
             if e is not None:
                 e[2 + 2 * i].record(stream)
 
     def timed_step(pair):
         pair[0].record(stream)
-        for L in plan:
-            launch_layer(L)
+        for i in range(nl):
+            launch_layer(i)
         pair[1].record(stream)
 
     for _ in range(args.warmup):
@@ -307,7 +322,8 @@ def run_fg8(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = f"fg8_gemm_kernel ({g.name}: M={g.M} K={g.K} N={g.N})"
+    roof["kernel"] = f"fg8_gemm_kernel ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+        ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
     roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
                            f"HBM {peaks['hbm_gbs']} GB/s")
@@ -316,17 +332,21 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        per_kernel.append({"layer": gi.name, "act_quant_us": qm[i] * 1e3,
-                           "act_quant_gbs": quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
+        fused = chain and i > 0  # this layer's act-quant ran in the previous GEMM's epilogue
+        per_kernel.append({"layer": gi.name, "act_quant_us": None if fused else qm[i] * 1e3,
+                           "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
+                           "act_quant": "fused into the previous GEMM" if fused else "own launch",
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
                            "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
 
-    e2e = run_e2e(fg8, plan, args, stream, dev, world)
+    e2e = run_e2e(fg8, plan, args, stream, dev, world, chain)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
 
-    launches_per_step = sum(2 + (1 if L["g"].fmt == 1 else 0) for L in plan)
+    # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM
+    prep = [1 + (1 if L["g"].fmt == 1 else 0) for L in plan]
+    launches_per_step = (prep[0] if chain else sum(prep)) + nl
     out = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
@@ -334,7 +354,8 @@ def run_fg8(args, rank, world, local):
         "config": dict(workload_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)]),
                        parallelism=f"dp{world} (token rows, replicated weights, no collective)"),
         "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
-        "act_quant_gbs": [k["act_quant_gbs"] for k in per_kernel],
+        "act_quant_gbs": [k["act_quant_gbs"] for k in per_kernel if k["act_quant_gbs"] is not None],
+        "chained": chain,
         "per_kernel": per_kernel,
         "roofline": roof,
         "cpu_baseline": cpu,
@@ -349,9 +370,10 @@ def run_fg8(args, rank, world, local):
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(fg8, plan, args, stream, dev, world):
-    """Same metric through the public call with host buffers: pinned x -> device,
-    the layers via fg8_linear, y -> pinned host, every step inside the timed region."""
+def run_e2e(fg8, plan, args, stream, dev, world, chain):
+    """Same metric through the public calls with host buffers: pinned x -> device,
+    the layers (chained as in the device-timed step, else fg8_linear per layer),
+    y -> pinned host, every step inside the timed region."""
     L0, Ln = plan[0], plan[-1]
     x_host = L0["x"].to("cpu").pin_memory()
     y_host = torch.empty(Ln["y"].shape, dtype=torch.bfloat16).pin_memory()
@@ -361,13 +383,30 @@ def run_e2e(fg8, plan, args, stream, dev, world):
 
     def one():
         x_dev.copy_(x_host, non_blocking=True)
-        xin = x_dev
-        for L in plan:
-            g = L["g"]
-            fg8.fg8_linear(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
-                           L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, L["wsp"].data_ptr(),
-                           L["wsp"].numel(), sp)
-            xin = L["y"]
+        if chain:
+            g = L0["g"]
+            fg8.fg8_linear_prepare(x_dev.data_ptr(), g.M, g.N, g.K, x_dev.stride(0), L0["ws"].data_ptr(), g.fmt,
+                                   L0["wsp"].data_ptr(), L0["wsp"].numel(), sp)
+            for i, L in enumerate(plan):
+                g = L["g"]
+                if i + 1 < len(plan):
+                    Lx = plan[i + 1]
+                    fg8.fg8_linear_run_chain(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(),
+                                             L["y"].data_ptr(), g.M, g.N, g.K, L["y"].stride(0), g.fmt,
+                                             L["wsp"].data_ptr(), L["wsp"].numel(), Lx["g"].N, Lx["ws"].data_ptr(),
+                                             Lx["wsp"].data_ptr(), Lx["wsp"].numel(), sp)
+                else:
+                    fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(),
+                                       g.M, g.N, g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(),
+                                       sp)
+        else:
+            xin = x_dev
+            for L in plan:
+                g = L["g"]
+                fg8.fg8_linear(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
+                               L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, L["wsp"].data_ptr(),
+                               L["wsp"].numel(), sp)
+                xin = L["y"]
         y_host.copy_(Ln["y"], non_blocking=True)
 
     for _ in range(3):
@@ -461,6 +500,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chain", action="store_true",
+                    help="quantize every layer's input in its own launch instead of in the previous GEMM")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -30,6 +30,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear_noalloc,
     fg8_linear_prepare,
     fg8_linear_run,
+    fg8_linear_run_chain,
     fg8_linear_workspace_bytes,
     fg8_quantize_act,
     fg8_quantize_weight,
@@ -43,6 +44,7 @@ from .layer import (  # noqa: F401
     FP8Linear,
     gemm_prequant,
     linear,
+    linear_chain,
     quantize_act,
     quantize_weight,
     scale_fmt_code,

@@ -35,6 +35,8 @@ SIGNATURES = {
     "fg8_linear": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_prepare": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
+    "fg8_linear_run_chain": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _I64, _VP, _VP, _SZ,
+                                     _VP]),
     "fg8_linear_noalloc": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP]),
     "fg8_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
     "fg8_gemm_prequant": (_INT, [_VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
@@ -117,6 +119,14 @@ def fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, works
 def fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes, stream):
     _check("fg8_linear_run", lib().fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt,
                                                   workspace, workspace_bytes, stream))
+
+
+def fg8_linear_run_chain(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes,
+                         next_N, next_w_scale_inv, next_workspace, next_workspace_bytes, stream):
+    _check("fg8_linear_run_chain", lib().fg8_linear_run_chain(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y,
+                                                              fmt, workspace, workspace_bytes, next_N,
+                                                              next_w_scale_inv, next_workspace, next_workspace_bytes,
+                                                              stream))
 
 
 def fg8_linear_noalloc(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, stream):

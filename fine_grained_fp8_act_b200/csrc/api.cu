@@ -294,6 +294,60 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
 }
 
+fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16, void* y_bf16,
+                                int64_t M, int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt, void* workspace,
+                                size_t workspace_bytes, int64_t next_N, const void* next_w_scale_inv,
+                                void* next_workspace, size_t next_workspace_bytes, void* stream) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  // the next layer: K = N (its activation is this layer's output), next_N outputs
+  if (fg8_status st = check_gemm_shape(M, next_N, N, fmt); st != FG8_OK) return st;
+  if (ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr || next_w_scale_inv == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_y % 8 != 0 || !aligned16(wq_e4m3) || !aligned16(y_bf16) || (bias_bf16 != nullptr && !aligned16(bias_bf16)) ||
+      !aligned16(w_scale_inv) || !aligned16(next_w_scale_inv))
+    return FG8_ERR_ALIGNMENT;
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  const LinearWs Ln = linear_ws_layout(M, next_N, N, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  if (fg8_status st = check_workspace(next_workspace, next_workspace_bytes, Ln.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* wn = static_cast<uint8_t*>(next_workspace);
+  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
+  GemmArgs g{};
+  g.xq = ws + L.xq_off;
+  g.wq = wq_e4m3;
+  g.y = y_bf16;
+  g.ld_y = ld_y;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.Kb = Kb;
+  g.Kq = Kq;
+  g.bias = bias_bf16;
+  g.status = reinterpret_cast<uint32_t*>(ws);
+  g.wait_limit_ns = g_wait_limit_ns.load();
+  if (fmt == FG8_SCALE_FLOAT) {
+    g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.ld_s = L.ld_s;
+    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
+  } else {
+    g.sfa = ws + L.xs_off;
+    g.sfb = ws + L.wsc_off;
+  }
+  g.nx_xq = wn + Ln.xq_off;
+  g.nx_xs = wn + Ln.xs_off;
+  g.nx_ld_s = Ln.ld_s;
+  g.nx_Kq = ceil_div(ceil_div(N, kGroup), 4);
+  g.nx_w_scale = next_w_scale_inv;
+  g.nx_w_prep = wn + Ln.wsc_off;
+  g.nx_N = static_cast<int>(next_N);
+  return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
 fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
                       const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt,
                       void* workspace, size_t workspace_bytes, void* stream) {

@@ -57,7 +57,7 @@ cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div
                            cudaStream_t s);
 
 // Rows of weight scale-factor tiles: N rounded up to the widest GEMM tile.
-inline int64_t sfb_rows(int64_t N) { return (N + 255) / 256 * 256; }
+__host__ __device__ inline int64_t sfb_rows(int64_t N) { return (N + 255) / 256 * 256; }
 
 struct GemmArgs {
   const void* xq;     // e4m3 [M, K] row stride K
@@ -77,11 +77,21 @@ struct GemmArgs {
   const void* bias;   // bf16 [N] or nullptr
   uint32_t* status;   // device status word (0 = ok)
   uint64_t wait_limit_ns;
+  // Optional: also quantize this layer's bf16 output as the activation of a
+  // next layer (K_next = N, N_next outputs) straight into that layer's
+  // workspace, exactly as its prepare step would.
+  uint8_t* nx_xq;         // e4m3 [M, N] row stride N; nullptr = off
+  void* nx_xs;            // float: K-major [N/128][nx_ld_s]; UE8M0: scale-factor tiles
+  int64_t nx_ld_s;
+  int nx_Kq;              // UE8M0: ceil(ceil(N/128) / 4)
+  const void* nx_w_scale; // next layer's weight scales [ceil(N_next/128), ceil(N/128)]
+  void* nx_w_prep;        // ... in the GEMM's layout (16-byte entries / scale-factor tiles)
+  int nx_N;               // N_next
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM
 // tile (256 rows for a CTA pair), so every tile's 128-row slices are in range.
-inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256 * 256; }
+__host__ __device__ inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256 * 256; }
 
 // Float weight scales [Nb, Kb] -> [Nb, Kb] 16-byte entries {s, 0, 0, 0}
 // (what the GEMM's producer bulk-copies per K-block).

@@ -38,6 +38,7 @@
 
 #include "fg8_internal.h"
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace fg8 {
 namespace {
@@ -57,11 +58,22 @@ struct KParams {
   const uint16_t* bias;
   uint32_t* status;
   uint64_t wait_limit_ns;
+  // output re-quantization for a next layer (REQUANT configs)
+  uint8_t* nx_xq;
+  void* nx_xs;
+  int64_t nx_ld_s;
+  int nx_Kq;
+  const void* nx_w_scale;
+  void* nx_w_prep;
+  int nx_N;
 };
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool PAIR_ = false>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool PAIR_ = false, bool REQUANT_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
+  // REQUANT: the epilogue also quantizes its bf16 output rows, one 128-column
+  // group per thread, for a next layer (needs the 256-wide tile).
+  static constexpr bool REQUANT = REQUANT_;
   // PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
   // MMAs; each CTA holds 128 rows of A and of the result, and BN/2 rows of B.
   static constexpr bool PAIR = PAIR_;
@@ -102,6 +114,7 @@ struct Cfg {
   static_assert(kOffSc % 16 == 0 && kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
   static_assert(kNumAcc * BN + (FMT == 1 ? 4 + BN / 32 : 0) <= 512, "TMEM columns");
   static_assert(!PAIR || (FMT == 0 && BN == 256), "CTA pairs: float scales, 256-wide tiles");
+  static_assert(!REQUANT || (BN == 256 && !PAIR), "output re-quantization: one 128-column group per thread");
   // bytes the stage's full barrier (in the pair's first CTA) waits for
   static constexpr uint32_t kStageTx = (PAIR ? 2 : 1) * (kA + kB);
   // arrivals that free a TMEM buffer: every epilogue warp of the pair
@@ -198,6 +211,84 @@ __device__ __forceinline__ void release_tmem(uint64_t* bar) {
     mbar_arrive_cluster(mapa_shared(bar, 0));
   } else {
     mbar_arrive(bar);
+  }
+}
+
+// Quantize one output row's 128-column group (bf16-rounded values in `v`) as
+// the next layer's activation group: the same arithmetic, hence the same bits,
+// as the stand-alone activation quantization of the stored bf16 output.
+template <class C>
+__device__ __forceinline__ void requant_group(const KParams& p, const uint32_t (&v)[C::kCols], int row, int n_first) {
+  static_assert(C::kCols == 128, "one group per thread");
+  const int valid = p.N - n_first;  // real columns of this group (may be <= 0 past N)
+  const int g = n_first / 128;      // the next layer's K-block
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 128; ++j)
+    if (j < valid) amax = fmaxf(amax, fabsf(__uint_as_float(v[j])));
+  const float s = qm::group_scale(amax);
+  const uint32_t sbyte = C::FMT == 1 ? qm::e8m0_ceil_byte(s) : 0u;
+  const bool store = row < p.M && valid > 0;
+  if (store) {
+    const float y = C::FMT == 0 ? __frcp_rn(s) : qm::e8m0_reciprocal(sbyte);
+    uint8_t* dst = p.nx_xq + static_cast<int64_t>(row) * p.N + n_first;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // 16 values -> 16 e4m3 bytes per store
+      if (c * 16 < valid) {
+        float q[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          const float2 a = make_float2(__uint_as_float(v[c * 16 + i]), __uint_as_float(v[c * 16 + i + 1]));
+          const float2 r = C::FMT == 0 ? qm::div2_rn_from_rcp(a, s, y) : __fmul2_rn(a, make_float2(y, y));
+          q[i] = r.x;
+          q[i + 1] = r.y;
+        }
+        *reinterpret_cast<uint4*>(dst + c * 16) =
+            make_uint4(qm::pack_e4m3x4(q[0], q[1], q[2], q[3]), qm::pack_e4m3x4(q[4], q[5], q[6], q[7]),
+                       qm::pack_e4m3x4(q[8], q[9], q[10], q[11]), qm::pack_e4m3x4(q[12], q[13], q[14], q[15]));
+      }
+    }
+  }
+  if constexpr (C::FMT == 0) {
+    if (store) static_cast<float*>(p.nx_xs)[static_cast<int64_t>(g) * p.nx_ld_s + row] = s;
+  } else {
+    // every (row, K-block) byte of the tiles the next GEMM reads must be a
+    // finite scale: padding rows and groups past N get 2^0
+    static_cast<uint8_t*>(p.nx_xs)[sf_tile_offset(row, g, p.nx_Kq)] =
+        store ? static_cast<uint8_t>(sbyte) : static_cast<uint8_t>(127);
+  }
+}
+
+// Idle warps of a REQUANT launch: put the next layer's weight scales in the
+// GEMM's layout, and fill the scale-factor bytes no epilogue thread owns.
+template <class C>
+__device__ __forceinline__ void prepare_next_layer(const KParams& p, int idx, int stride) {
+  const int Kb_next = (p.N + 127) / 128;
+  const int Nb_next = (p.nx_N + 127) / 128;
+  if constexpr (C::FMT == 0) {
+    const int64_t n = static_cast<int64_t>(Nb_next) * Kb_next;
+    const float* ws = static_cast<const float*>(p.nx_w_scale);
+    for (int64_t i = idx; i < n; i += stride)
+      reinterpret_cast<float4*>(p.nx_w_prep)[i] = make_float4(ws[i], 0.0f, 0.0f, 0.0f);
+  } else {
+    const int cols = p.nx_Kq * 4;
+    const int64_t rows = sfb_rows(p.nx_N);
+    const uint8_t* ws = static_cast<const uint8_t*>(p.nx_w_scale);
+    for (int64_t i = idx; i < rows * cols; i += stride) {
+      const int64_t r = i / cols;
+      const int kb = static_cast<int>(i % cols);
+      const uint8_t b = (r < p.nx_N && kb < Kb_next) ? ws[(r / 128) * Kb_next + kb] : static_cast<uint8_t>(127);
+      static_cast<uint8_t*>(p.nx_w_prep)[sf_tile_offset(r, kb, p.nx_Kq)] = b;
+    }
+    // activation scale-factor K-blocks beyond the tile grid
+    const int first_unowned = 2 * p.num_n;
+    const int64_t m_rows = static_cast<int64_t>(p.num_m) * kBlockM;
+    const int64_t extra = static_cast<int64_t>(cols > first_unowned ? cols - first_unowned : 0) * m_rows;
+    for (int64_t i = idx; i < extra; i += stride) {
+      const int64_t r = i % m_rows;
+      const int kb = first_unowned + static_cast<int>(i / m_rows);
+      static_cast<uint8_t*>(p.nx_xs)[sf_tile_offset(r, kb, p.nx_Kq)] = static_cast<uint8_t>(127);
+    }
   }
 }
 
@@ -491,6 +582,10 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
           const int j = c * 32 + 8 * i + 2 * h;
           w[4 * i + h] = pack_bf16x2(__uint_as_float(acc[j]) + __uint_as_float(bw[h] << 16),
                                      __uint_as_float(acc[j + 1]) + __uint_as_float(bw[h] & 0xFFFF0000u));
+          if constexpr (C::REQUANT) {  // keep the bf16-rounded values: they are the next layer's input
+            acc[j] = w[4 * i + h] << 16;
+            acc[j + 1] = w[4 * i + h] & 0xFFFF0000u;
+          }
         }
       }
       uint8_t* buf = stg + (nstore % C::kOutBufs) * C::kOutBuf;
@@ -517,6 +612,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
     __syncwarp();
     if (lane == 0) mbar_arrive(bempty + bi.slot);
     bi.template advance<2>();
+    if constexpr (C::REQUANT) requant_group<C>(p, acc, row0 + lane, nb * C::BN + col0);
   }
   if (lane == 0) bulk_wait_group<0>();
 }
@@ -591,6 +687,11 @@ __global__ void __launch_bounds__(384, 1)
       producer<C>(&tmA, &tmB, p, smem, full, empty, scfull, scempty, bfull, bempty, abort_flag);
     else if (warp == 1 && lane == 0 && cta_rank<C>() == 0)
       mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, abort_flag);
+    if constexpr (C::REQUANT) {
+      if (warp == 2 || warp == 3)
+        prepare_next_layer<C>(p, static_cast<int>(blockIdx.x) * 64 + (warp - 2) * 32 + lane,
+                              static_cast<int>(gridDim.x) * 64);
+    }
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
     epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, scfull, scempty, bfull, bempty, abort_flag, warp, lane);
@@ -673,6 +774,13 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.bias = static_cast<const uint16_t*>(g.bias);
   p.status = g.status;
   p.wait_limit_ns = g.wait_limit_ns;
+  p.nx_xq = g.nx_xq;
+  p.nx_xs = g.nx_xs;
+  p.nx_ld_s = g.nx_ld_s;
+  p.nx_Kq = g.nx_Kq;
+  p.nx_w_scale = g.nx_w_scale;
+  p.nx_w_prep = g.nx_w_prep;
+  p.nx_N = g.nx_N;
   if (p.num_tiles == 0) return cudaSuccess;
 
   static int configured_device = -1;
@@ -740,6 +848,15 @@ int choose_block_n(int M, int N, int num_sms) {
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s) {
+  if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
+    const bool short_k = g.Kb <= 32;
+    if (fmt == 0) {
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, false, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 1, false, true>>(g, num_sms, s);
+    }
+    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, false, true>>(g, num_sms, s);
+    return launch_cfg<Cfg<256, 1, 4, 1, false, true>>(g, num_sms, s);
+  }
   const int bn = choose_block_n(g.M, g.N, num_sms);
   // Short K: few K-blocks per tile, so the tile's output path dominates --
   // give every output chunk its own staging box and keep one stage fewer.

@@ -114,6 +114,44 @@ def gemm_prequant(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_s
     return y
 
 
+def linear_chain(x: torch.Tensor, layers, scale_fmt="float", workspaces=None):
+    """Consecutive linears y_i = linear(y_{i-1}, *layers[i]) (layers: [(wq, w_scale_inv, bias or None)]),
+    with each layer's activation quantization fused into the previous layer's GEMM epilogue: one
+    act-quant launch for the first layer, then one GEMM launch per layer.  Every y_i equals, bit for
+    bit, what `linear` gives for that layer on y_{i-1}.  Returns [y_0, ..., y_last]."""
+    fmt = scale_fmt_code(scale_fmt)
+    _check_bf16_matrix(x, "x")
+    M = x.shape[0]
+    dims = []
+    k = x.shape[1]
+    for i, (wq, _, _) in enumerate(layers):
+        if wq.dim() != 2 or wq.shape[1] != k:
+            raise ValueError(f"layer {i}: wq must be [N, {k}]")
+        dims.append((wq.shape[0], k))
+        k = wq.shape[0]
+    if workspaces is None:
+        workspaces = [None] * len(layers)
+    wss = [_workspace(C.fg8_linear_workspace_bytes(M, n, kk, fmt), x.device, w)
+           for (n, kk), w in zip(dims, workspaces)]
+    ys = [torch.empty((M, n), dtype=torch.bfloat16, device=x.device) for n, _ in dims]
+    s = _stream(x)
+    with torch.cuda.device(x.device):
+        n0, k0 = dims[0]
+        C.fg8_linear_prepare(x.data_ptr(), M, n0, k0, x.stride(0), layers[0][1].data_ptr(), fmt, wss[0].data_ptr(),
+                             wss[0].numel(), s)
+        for i, ((wq, wsc, b), (n, kk)) in enumerate(zip(layers, dims)):
+            bp = 0 if b is None else b.data_ptr()
+            if i + 1 < len(layers):
+                nn = dims[i + 1][0]
+                C.fg8_linear_run_chain(wq.data_ptr(), wsc.data_ptr(), bp, ys[i].data_ptr(), M, n, kk, n, fmt,
+                                       wss[i].data_ptr(), wss[i].numel(), nn, layers[i + 1][1].data_ptr(),
+                                       wss[i + 1].data_ptr(), wss[i + 1].numel(), s)
+            else:
+                C.fg8_linear_run(wq.data_ptr(), wsc.data_ptr(), bp, ys[i].data_ptr(), M, n, kk, n, fmt,
+                                 wss[i].data_ptr(), wss[i].numel(), s)
+    return ys
+
+
 class FP8Linear(torch.nn.Module):
     """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
     weight float8_e4m3fn [out, in], weight_scale_inv per 128x128 block, bias

@@ -128,6 +128,22 @@ FG8_API fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, 
                                   void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
                                   fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Two consecutive layers, the second fed by the first's output: runs this
+ * layer's GEMM from `workspace` (after fg8_linear_prepare) and, in the same
+ * kernel's epilogue, quantizes each bf16 output row group exactly as
+ * fg8_linear_prepare(y_bf16, M, next_N, N, ...) would, writing the result into
+ * `next_workspace` together with the next layer's weight scales
+ * (`next_w_scale_inv`, [ceil(next_N/128), ceil(N/128)]).  A following
+ * fg8_linear_run(next layer, next_workspace) then computes the second layer
+ * without its own activation-quantization pass over y.  y_bf16 is still
+ * written.  Checks as fg8_linear for both layers (N % 16 == 0, since N is the
+ * next layer's K).  Same results, bit for bit, as prepare + run per layer. */
+FG8_API fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                        void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
+                                        fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, int64_t next_N,
+                                        const void* next_w_scale_inv, void* next_workspace,
+                                        size_t next_workspace_bytes, void* stream);
+
 /* fg8_linear without a caller workspace, for callers that cannot allocate
  * device memory (for example a host framework that owns all device memory
  * through its own pool, or code that must never call cudaMalloc because it

@@ -100,6 +100,22 @@ def test_linear_rejects_null_and_misaligned(fg8):
     assert raw.fg8_linear(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, FAKE * 16, 100, None) == 4
 
 
+def test_chain_rejects_bad_next_layer(fg8):
+    raw = _raw(fg8)
+
+    def chain(M, N, K, next_N, ws=FAKE * 16, next_ws=FAKE * 32):
+        return raw.fg8_linear_run_chain(FAKE, FAKE, None, FAKE, M, N, K, N, 0, ws, 1 << 40, next_N, FAKE, next_ws,
+                                        1 << 40, None)
+
+    assert chain(16, 264, 256, 128) == 2      # the next layer's K (this N) must be a multiple of 16
+    assert chain(16, 256, 256, 0) == 1        # next_N = 0
+    assert chain(16, 256, 256, 252) == 2      # next_N % 8
+    assert chain(16, 256, 256, 256, next_ws=None) == 4
+    assert chain(0, 256, 256, 256) == 0       # empty batch
+    assert raw.fg8_linear_run_chain(FAKE, FAKE, None, FAKE, 16, 256, 256, 256, 0, FAKE * 16, 1 << 40, 256, None,
+                                    FAKE * 32, 1 << 40, None) == 1  # next layer's weight scales missing
+
+
 def test_empty_m_is_a_noop(fg8):
     raw = _raw(fg8)
     assert raw.fg8_linear(None, 0, 256, 256, 256, None, None, None, None, 256, 0, None, 0, None) == 0
