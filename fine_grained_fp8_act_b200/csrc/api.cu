@@ -83,7 +83,8 @@ fg8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int fmt) {
 }
 
 // Workspace of fg8_linear: [header | xq (M*K) | x scales | W scales].
-//   float: x scales K-major [Kb][ld_s] float32, W scales [Nb][Kb] 16-byte entries
+//   float: x scales K-major [Kb][ld_s] float32 (the GEMM reads the caller's
+//          weight scales as given: no W-scale region)
 //   UE8M0: x and W scale-factor tiles (512 bytes per 128 rows x 4 K-blocks)
 struct LinearWs {
   size_t xq_off, xs_off, wsc_off, total;
@@ -94,7 +95,6 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   LinearWs w;
   const int Kb = ceil_div(K, kGroup);
   const int Kq = ceil_div(Kb, 4);
-  const int Nb = ceil_div(N, 128);
   w.xq_off = kHeaderBytes;
   size_t off = align_up(w.xq_off + static_cast<size_t>(M) * K, kAlign);
   w.xs_off = off;
@@ -102,7 +102,6 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   if (fmt == FG8_SCALE_FLOAT) {
     off = align_up(off + static_cast<size_t>(Kb) * w.ld_s * sizeof(float), kAlign);
     w.wsc_off = off;
-    off = align_up(off + static_cast<size_t>(Nb) * Kb * 16, kAlign);
   } else {
     off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
     w.wsc_off = off;
@@ -123,14 +122,12 @@ GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   GemmWs w;
   const int Kb = ceil_div(K, kGroup);
   const int Kq = ceil_div(Kb, 4);
-  const int Nb = ceil_div(N, 128);
   size_t off = kHeaderBytes;
   w.xs_off = off;
   w.ld_s = kmajor_ld(M);
   if (fmt == FG8_SCALE_FLOAT) {
     off = align_up(off + static_cast<size_t>(Kb) * w.ld_s * sizeof(float), kAlign);
     w.wsc_off = off;
-    off = align_up(off + static_cast<size_t>(Nb) * Kb * 16, kAlign);
   } else {
     off = align_up(off + static_cast<size_t>(ceil_div(M, 128)) * Kq * kSfChunkBytes, kAlign);
     w.wsc_off = off;
@@ -242,11 +239,6 @@ fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t 
   a.ld_s = L.ld_s;
   a.Kq = Kq;
   a.M_pad = ceil_div(M, 128) * 128;
-  if (fmt == FG8_SCALE_FLOAT) {  // the weight-scale padding rides in the same launch
-    a.ws = static_cast<const float*>(w_scale_inv);
-    a.ws_pad = reinterpret_cast<float*>(ws + L.wsc_off);
-    a.Nb = ceil_div(N, 128);
-  }
   if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
   if (fmt == FG8_SCALE_UE8M0)
     return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), sfb_rows(N),
@@ -286,7 +278,7 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   if (fmt == FG8_SCALE_FLOAT) {
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
-    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
+    g.w_scale = static_cast<const float*>(w_scale_inv);
   } else {
     g.sfa = ws + L.xs_off;
     g.sfb = ws + L.wsc_off;
@@ -333,7 +325,7 @@ fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, co
   if (fmt == FG8_SCALE_FLOAT) {
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
-    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
+    g.w_scale = static_cast<const float*>(w_scale_inv);
   } else {
     g.sfa = ws + L.xs_off;
     g.sfb = ws + L.wsc_off;
@@ -406,13 +398,9 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
                                                         L.ld_s, reinterpret_cast<float*>(ws + L.xs_off), s));
         st != FG8_OK)
       return st;
-    if (fg8_status st = cuda_status(launch_ws_pad(static_cast<const float*>(w_scale_inv), ceil_div(N, 128), Kb,
-                                                  reinterpret_cast<float*>(ws + L.wsc_off), s));
-        st != FG8_OK)
-      return st;
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
-    g.ws_pad = reinterpret_cast<const float*>(ws + L.wsc_off);
+    g.w_scale = static_cast<const float*>(w_scale_inv);
   } else {
     if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(x_scale), static_cast<int>(M),
                                                    (M + 127) / 128 * 128, 1, Kb, ws + L.xs_off, s));

@@ -39,10 +39,6 @@ struct ActQuantArgs {
   int64_t ld_s;       // kScaleKMajor: column stride (>= M)
   int Kq;             // kScaleSfTiles: ceil(Kb / 4)
   int M_pad;          // kScaleSfTiles: rows rounded up to 128 (padding rows get scale 2^0)
-  // optional, same launch: float weight scales [Nb, Kb] -> 16-byte entries (ws_pad)
-  const float* ws;
-  float* ws_pad;
-  int Nb;
 };
 
 cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s);
@@ -66,10 +62,10 @@ struct GemmArgs {
   int64_t ld_y;
   int M, N, K, Kb;
   // float path: x scales K-major [Kb][ld_s] (ld_s a multiple of 256, >= M),
-  // weight scales padded to one 16-byte entry per (nb, kb) (see launch_ws_pad)
+  // weight scales as given, [ceil(N/128)][Kb] row-major
   const float* xs_t;
   int64_t ld_s;
-  const float* ws_pad;
+  const float* w_scale;
   // UE8M0 path: scale-factor tiles of x (rows M) and W (rows N)
   const uint8_t* sfa;
   const uint8_t* sfb;
@@ -85,17 +81,13 @@ struct GemmArgs {
   int64_t nx_ld_s;
   int nx_Kq;              // UE8M0: ceil(ceil(N/128) / 4)
   const void* nx_w_scale; // next layer's weight scales [ceil(N_next/128), ceil(N/128)]
-  void* nx_w_prep;        // ... in the GEMM's layout (16-byte entries / scale-factor tiles)
+  void* nx_w_prep;        // UE8M0: ... packed into scale-factor tiles (unused for float)
   int nx_N;               // N_next
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM
 // tile (256 rows for a CTA pair), so every tile's 128-row slices are in range.
 __host__ __device__ inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256 * 256; }
-
-// Float weight scales [Nb, Kb] -> [Nb, Kb] 16-byte entries {s, 0, 0, 0}
-// (what the GEMM's producer bulk-copies per K-block).
-cudaError_t launch_ws_pad(const float* ws, int Nb, int Kb, float* out, cudaStream_t s);
 
 // Float x scales row-major [M, Kb] -> K-major [Kb][ld_s].
 cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s);

@@ -11,9 +11,8 @@
 // (setmaxnreg 40-56) to the two epilogue warpgroups (setmaxnreg 224-232):
 //   warp 0      producer: per 128-wide K-block, TMA loads of the A tile
 //               (128 x 128 e4m3) and B tile (BN x 128 e4m3) into a STAGES-deep
-//               ring (128-byte swizzle); bulk copies of the K-block's scales
-//               (float path) into a scale ring, of UE8M0 scale-factor tiles
-//               (every 4th K-block), and of the tile's bias into a bias ring.
+//               ring (128-byte swizzle); bulk copies of UE8M0 scale-factor
+//               tiles (every 4th K-block) and of the tile's bias (bias ring).
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32) per K-block.
 //   warp 2      TMEM allocator.
 //   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4)..+31; warpgroup g
@@ -21,8 +20,12 @@
 //
 // Float scales (FMT 0): each K-block's partial product P_kb goes to its own
 // TMEM buffer (512/BN of them); the epilogue promotes it in registers,
-// acc += P_kb * (sx * sw), applying the float32 scales exactly as given --
-// never rounded to a power of two (§七 补充 names that hazard).
+// acc += P_kb * (sx * sw) starting from acc = bias, applying the float32
+// scales exactly as given --
+// never rounded to a power of two (§七 补充 names that hazard).  Each thread
+// loads its own sx (its row) and sw (its columns' weight block) from global
+// memory two K-blocks ahead, and reads P_kb from TMEM 32 columns at a time
+// with the next 32 in flight while it promotes the current ones.
 // UE8M0 scales (FMT 1): tcgen05.mma.kind::mxf8f6f4.block_scale applies the
 // power-of-two scales inside the tensor core (one per 32 K-elements; four
 // equal ones per 128-block), accumulating the whole K range in TMEM.
@@ -52,7 +55,7 @@ struct KParams {
   int num_m, num_n, num_tiles;
   const float* xs_t;    // float path: x scales, K-major [Kb][ld_s]
   int64_t ld_s;
-  const float* ws_pad;  // float path: weight scales, one 16-byte entry per (nb, kb)
+  const float* w_scale; // float path: weight scales [Nb][Kb] as given
   const uint8_t* sfa;   // UE8M0 path: scale-factor tiles
   const uint8_t* sfb;
   const uint16_t* bias;
@@ -90,28 +93,25 @@ struct Cfg {
   static constexpr int kNumAcc = FMT == 0 ? 512 / BN : (BN == 256 ? 1 : 3);
   static constexpr int kSfaCol = kNumAcc * BN;
   static constexpr int kSfbCol = kSfaCol + 4;
-  static constexpr int kScSlots = FMT == 0 ? 6 : 0;
-  static constexpr int kScSlot = 512 + 32;  // 128 x-scales, then two 16-byte weight-scale entries
   static constexpr int kBiasSlot = BN * 2;
   // register split after launch (384 x 168): the wide float epilogue holds
   // 128 accumulators + 32 TMEM registers per thread, the others need less
-  static constexpr uint32_t kRegsLow = (FMT == 0 && BN == 256) ? 48 : (BN == 128 ? 80 : 56);
-  static constexpr uint32_t kRegsHigh = (FMT == 0 && BN == 256) ? 224 : (BN == 128 ? 208 : 224);
+  static constexpr uint32_t kRegsLow = (FMT == 0 && BN == 256) ? 40 : (BN == 128 ? 80 : 56);
+  static constexpr uint32_t kRegsHigh = (FMT == 0 && BN == 256) ? 232 : (BN == 128 ? 208 : 224);
   static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch allocation");
   static constexpr int kOutBuf = 32 * 32 * 2;  // one 32 x 32 bf16 box
   // output staging boxes per epilogue warp: with kChunks of them a warp never
   // waits for its own TMA stores inside a tile
   static constexpr int kOutBufs = OUTBUFS_;
-  static_assert(kOutBufs >= 1 && kOutBufs <= kChunks, "staging buffers per warp");
+  static_assert(kOutBufs >= 1 && kOutBufs <= kChunks && kChunks % kOutBufs == 0, "staging buffers per warp");
   // shared memory map (offsets from the 1024-aligned base)
   static constexpr int kOffStaging = STAGES * kStage;
-  static constexpr int kOffSc = kOffStaging + kEpiWarps * kOutBufs * kOutBuf;
-  static constexpr int kOffBias = kOffSc + kScSlots * kScSlot;
+  static constexpr int kOffBias = kOffStaging + kEpiWarps * kOutBufs * kOutBuf;
   static constexpr int kOffBar = kOffBias + 2 * kBiasSlot;
   static constexpr int kSmem = 1024 + kOffBar + 512;
   static_assert(kSmem <= kMaxSmem, "shared memory budget");
   static_assert(kStage % 1024 == 0, "stages keep 1024-byte alignment for the 128B swizzle");
-  static_assert(kOffSc % 16 == 0 && kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
+  static_assert(kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
   static_assert(kNumAcc * BN + (FMT == 1 ? 4 + BN / 32 : 0) <= 512, "TMEM columns");
   static_assert(!PAIR || (FMT == 0 && BN == 256), "CTA pairs: float scales, 256-wide tiles");
   static_assert(!REQUANT || (BN == 256 && !PAIR), "output re-quantization: one 128-column group per thread");
@@ -261,16 +261,11 @@ __device__ __forceinline__ void requant_group(const KParams& p, const uint32_t (
 
 // Idle warps of a REQUANT launch: put the next layer's weight scales in the
 // GEMM's layout, and fill the scale-factor bytes no epilogue thread owns.
+// (Float: the next GEMM reads its weight scales as given; nothing to do.)
 template <class C>
 __device__ __forceinline__ void prepare_next_layer(const KParams& p, int idx, int stride) {
   const int Kb_next = (p.N + 127) / 128;
-  const int Nb_next = (p.nx_N + 127) / 128;
-  if constexpr (C::FMT == 0) {
-    const int64_t n = static_cast<int64_t>(Nb_next) * Kb_next;
-    const float* ws = static_cast<const float*>(p.nx_w_scale);
-    for (int64_t i = idx; i < n; i += stride)
-      reinterpret_cast<float4*>(p.nx_w_prep)[i] = make_float4(ws[i], 0.0f, 0.0f, 0.0f);
-  } else {
+  if constexpr (C::FMT == 1) {
     const int cols = p.nx_Kq * 4;
     const int64_t rows = sfb_rows(p.nx_N);
     const uint8_t* ws = static_cast<const uint8_t*>(p.nx_w_scale);
@@ -295,14 +290,13 @@ __device__ __forceinline__ void prepare_next_layer(const KParams& p, int idx, in
 // ---------------------------------------------------------------- roles ----
 template <class C>
 __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
-                                         uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* scfull,
-                                         uint64_t* scempty, uint64_t* bfull, uint64_t* bempty,
-                                         volatile int* abort_flag) {
+                                         uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* bfull,
+                                         uint64_t* bempty, volatile int* abort_flag) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring st, sc, bi;
+  Ring st, bi;
   // most recent issue phase per slot, for the drain at the end
-  uint32_t st_issued = 0, sc_issued = 0, bi_issued = 0;
-  uint32_t st_par[C::STAGES], sc_par[C::kScSlots > 0 ? C::kScSlots : 1], bi_par[2];
+  uint32_t st_issued = 0, bi_issued = 0;
+  uint32_t st_par[C::STAGES], bi_par[2];
   bool ok = true;
   const int rank = cta_rank<C>();
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
@@ -357,24 +351,6 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       st_par[st.slot] = st.phase;
       st_issued |= 1u << st.slot;
       st.template advance<C::STAGES>();
-      if (C::FMT == 0) {
-        if (!mbar_wait(scempty + sc.slot, sc.phase ^ 1u, limit, abort_flag)) {
-          raise_abort(abort_flag, p.status);
-          ok = false;
-          break;
-        }
-        const int nb0 = n0 / 128;
-        const bool second = C::BN == 256 && nb0 + 1 < p.Nb;
-        uint8_t* slot = smem + C::kOffSc + sc.slot * C::kScSlot;
-        mbar_arrive_expect_tx(scfull + sc.slot, 512u + 16u + (second ? 16u : 0u));
-        bulk_load(slot, p.xs_t + static_cast<int64_t>(kb) * p.ld_s + m0, 512u, scfull + sc.slot);
-        bulk_load(slot + 512, p.ws_pad + (static_cast<int64_t>(nb0) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
-        if (second)
-          bulk_load(slot + 528, p.ws_pad + (static_cast<int64_t>(nb0 + 1) * p.Kb + kb) * 4, 16u, scfull + sc.slot);
-        sc_par[sc.slot] = sc.phase;
-        sc_issued |= 1u << sc.slot;
-        sc.template advance<(C::kScSlots > 0 ? C::kScSlots : 1)>();
-      }
     }
   }
   // Every issued copy must have landed before the CTA's shared memory goes away.
@@ -384,8 +360,6 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
   if (rank == 0)
     for (int s = 0; s < C::STAGES; ++s)
       if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
-  for (int s = 0; s < C::kScSlots; ++s)
-    if ((sc_issued >> s) & 1u) (void)mbar_wait(scfull + s, sc_par[s], kTeardownNs, nullptr);
   for (int s = 0; s < 2; ++s)
     if ((bi_issued >> s) & 1u) (void)mbar_wait(bfull + s, bi_par[s], kTeardownNs, nullptr);
 }
@@ -407,6 +381,8 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
         break;
       }
       tc_fence_after();
+      const uint32_t a_addr = smem_u32(smem + st.slot * C::kStage);
+      const uint32_t b_addr = a_addr + C::kA;
       if (C::FMT == 0 || kb == 0) {
         if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
@@ -415,8 +391,6 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
         }
         tc_fence_after();
       }
-      const uint32_t a_addr = smem_u32(smem + st.slot * C::kStage);
-      const uint32_t b_addr = a_addr + C::kA;
       const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
       if (C::FMT == 1 && (kb & 3) == 0) {
         // UE8M0 scales of 128 rows x 4 K-blocks for A, and for B, into TMEM;
@@ -467,11 +441,42 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   (void)mbar_wait(teardown, 0, kTeardownNs, nullptr);
 }
 
+// The float scales one epilogue thread applies, in the order it applies them:
+// for each tile of the CTA's walk and each of its K-blocks, sx(the thread's
+// row, kb) and sw(the 128-column weight block of the thread's columns, kb).
+template <class C>
+struct ScaleStream {
+  int tile = 0, kb = 0;
+  int xoff = 0;  // row of the thread in xs_t's K-major layout
+  int woff = 0;  // offset of the weight block's row in w_scale
+  __device__ __forceinline__ void start(const KParams& p, int t, int sub_row, int col) {
+    tile = t;
+    kb = 0;
+    if (t < p.num_tiles) {
+      int mb, nb;
+      tile_coords(t, p.num_m, p.num_n, mb, nb);
+      xoff = mb * C::kTileM + sub_row;
+      // a column block past N (ragged last tile) reads the last block: its
+      // columns are never stored
+      woff = min((nb * C::BN + col) / 128, p.Nb - 1) * p.Kb;
+    }
+  }
+  // {sx, sw} of the next (tile, K-block), or zeros past the end of the walk.
+  __device__ __forceinline__ float2 next(const KParams& p, int sub_row, int col) {
+    float2 v = make_float2(0.0f, 0.0f);
+    if (tile < p.num_tiles) {
+      v.x = p.xs_t[static_cast<int64_t>(kb) * p.ld_s + xoff];
+      v.y = p.w_scale[woff + kb];
+      if (++kb == p.Kb) start(p, tile + tile_stride<C>(), sub_row, col);
+    }
+    return v;
+  }
+};
+
 template <class C>
 __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& p, uint8_t* smem, uint32_t tmem_base,
-                                         uint64_t* tfull, uint64_t* tempty, uint64_t* scfull, uint64_t* scempty,
-                                         uint64_t* bfull, uint64_t* bempty, volatile int* abort_flag, int warp,
-                                         int lane) {
+                                         uint64_t* tfull, uint64_t* tempty, uint64_t* bfull, uint64_t* bempty,
+                                         volatile int* abort_flag, int warp, int lane) {
   const uint64_t limit = p.wait_limit_ns;
   const int ew = warp - 4;
   const int q = warp & 3;      // TMEM lane quadrant
@@ -479,34 +484,51 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   const int col0 = wg * C::kCols;
   uint8_t* stg = smem + C::kOffStaging + ew * C::kOutBufs * C::kOutBuf;
   const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-  Ring ab, sc, bi;
-  int nstore = 0;
+  Ring ab, bi;
   bool ok = true;
   const int rank = cta_rank<C>();
+  const int sub_row = rank * kBlockM + q * 32 + lane;  // this thread's row inside a tile
+  // float path: scales of the current and the next K-block in registers, the
+  // one after that in flight
+  ScaleStream<C> ss;
+  float2 s_now = make_float2(0.0f, 0.0f), s_nxt = make_float2(0.0f, 0.0f);
+  if constexpr (C::FMT == 0) {
+    ss.start(p, tile_start<C>(), sub_row, col0);
+    s_now = ss.next(p, sub_row, col0);
+    s_nxt = ss.next(p, sub_row, col0);
+  }
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int row0 = mb * C::kTileM + rank * kBlockM + q * 32;
+    // the tile's bias (bias ring; zeros past N or without bias)
+    if (!mbar_wait(bfull + bi.slot, bi.phase, limit, abort_flag)) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    const uint8_t* bias_s = smem + C::kOffBias + bi.slot * C::kBiasSlot;
     uint32_t acc[C::kCols];  // float bits
-    if (C::FMT == 0) {
+    if constexpr (C::FMT == 0) {
+      // the promotion accumulates onto the bias: y = bias + sum_kb P_kb * s_kb
 #pragma unroll
-      for (int j = 0; j < C::kCols; ++j) acc[j] = 0u;
-      for (int kb = 0; kb < p.Kb; ++kb) {
-        // scale of this row and K-block: sx(m, kb) * sw(block of my columns, kb)
-        if (!mbar_wait(scfull + sc.slot, sc.phase, limit, abort_flag)) {
-          raise_abort(abort_flag, p.status);
-          ok = false;
-          break;
+      for (int i = 0; i < C::kCols / 8; ++i) {
+        uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+        if (p.bias != nullptr && nb * C::BN + col0 + 8 * i < p.N)
+          bv = *reinterpret_cast<const uint4*>(bias_s + (col0 + 8 * i) * 2);
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          acc[8 * i + 2 * h] = bw[h] << 16;
+          acc[8 * i + 2 * h + 1] = bw[h] & 0xFFFF0000u;
         }
-        const uint8_t* slot = smem + C::kOffSc + sc.slot * C::kScSlot;
-        const float sx = reinterpret_cast<const float*>(slot)[q * 32 + lane];
-        const float sw = *reinterpret_cast<const float*>(slot + 512 + (C::BN == 256 ? 16 * wg : 0));
-        const float s = sx * sw;
-        const float2 s2 = make_float2(s, s);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(scempty + sc.slot);
-        sc.template advance<(C::kScSlots > 0 ? C::kScSlots : 1)>();
-
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bempty + bi.slot);
+      bi.template advance<2>();
+      for (int kb = 0; kb < p.Kb; ++kb) {
+        const float s = s_now.x * s_now.y;  // sx(m, kb) * sw(block, kb)
+        s_now = s_nxt;
+        s_nxt = ss.next(p, sub_row, col0);
         if (!mbar_wait(tfull + ab.slot, ab.phase, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
           ok = false;
@@ -514,29 +536,27 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(ab.slot * C::BN + col0);
-        // TMEM -> registers in groups of up to 64 columns (two x32 loads, one
-        // wait), then packed f32x2 FMAs: one or two load round trips per
-        // K-block instead of one per 32 columns.
-        constexpr int GRP = C::kCols < 64 ? C::kCols : 64;
+        // 32 columns per TMEM load; group c+1 is loading while group c is
+        // promoted
+        uint32_t r[2][32];
+        tmem_ld32(taddr, r[0]);
+        tmem_wait_ld();
+        tmem_reg_fence(r[0]);
 #pragma unroll
-        for (int g0 = 0; g0 < C::kCols; g0 += GRP) {
-          uint32_t r[GRP];
-#pragma unroll
-          for (int c = 0; c < GRP / 32; ++c) tmem_ld32(taddr + g0 + c * 32, r + c * 32);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < GRP / 32; ++c) tmem_reg_fence(r + c * 32);
-          if (g0 + GRP == C::kCols) {  // all of this K-block's columns are in registers: free the buffer
+        for (int c = 0; c < C::kChunks; ++c) {
+          if (c + 1 < C::kChunks) {
+            tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
+          } else {  // every column of this K-block is in registers: hand the buffer back
             tc_fence_before();
             __syncwarp();
             if (lane == 0) release_tmem<C>(tempty + ab.slot);
           }
 #pragma unroll
-          for (int j = 0; j < GRP; j += 2) {  // packed f32x2 FMA: two promotions per instruction
-            const float2 r2 = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), s2,
-                                         make_float2(__uint_as_float(acc[g0 + j]), __uint_as_float(acc[g0 + j + 1])));
-            acc[g0 + j] = __float_as_uint(r2.x);
-            acc[g0 + j + 1] = __float_as_uint(r2.y);
+          for (int j = 0; j < 32; ++j)
+            acc[c * 32 + j] = __float_as_uint(__fmaf_rn(__uint_as_float(r[c & 1][j]), s, __uint_as_float(acc[c * 32 + j])));
+          if (c + 1 < C::kChunks) {
+            tmem_wait_ld();
+            tmem_reg_fence(r[(c + 1) & 1]);
           }
         }
         ab.template advance<C::kNumAcc>();
@@ -560,58 +580,64 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       ab.template advance<C::kNumAcc>();
     }
 
-    // + bias (from the bias ring), round to bf16, stage 32 x 32 boxes (64-byte
-    // swizzle) and store them with TMA.
-    if (!mbar_wait(bfull + bi.slot, bi.phase, limit, abort_flag)) {
-      raise_abort(abort_flag, p.status);
-      break;
-    }
-    const uint8_t* bias_s = smem + C::kOffBias + bi.slot * C::kBiasSlot;
+    // (UE8M0: + bias), round to bf16, stage 32 x 32 boxes (64-byte swizzle),
+    // store them with TMA: one proxy fence and one bulk group per batch of
+    // kOutBufs boxes.
+    if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores have read the boxes
+    __syncwarp();
 #pragma unroll
     for (int c = 0; c < C::kChunks; ++c) {
+      const int b = c % C::kOutBufs;
+      if (c >= C::kOutBufs && b == 0) {  // reusing the boxes: the previous batch must have been read
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+      }
       const int nloc = col0 + c * 32;
       const int n0 = nb * C::BN + nloc;
       uint32_t w[16];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-        if (p.bias != nullptr && n0 + 8 * i < p.N) bv = *reinterpret_cast<const uint4*>(bias_s + (nloc + 8 * i) * 2);
+        if (C::FMT == 1 && p.bias != nullptr && n0 + 8 * i < p.N)
+          bv = *reinterpret_cast<const uint4*>(bias_s + (nloc + 8 * i) * 2);
         const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const int j = c * 32 + 8 * i + 2 * h;
-          w[4 * i + h] = pack_bf16x2(__uint_as_float(acc[j]) + __uint_as_float(bw[h] << 16),
-                                     __uint_as_float(acc[j + 1]) + __uint_as_float(bw[h] & 0xFFFF0000u));
+          w[4 * i + h] = C::FMT == 0 ? pack_bf16x2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]))
+                                     : pack_bf16x2(__uint_as_float(acc[j]) + __uint_as_float(bw[h] << 16),
+                                                   __uint_as_float(acc[j + 1]) + __uint_as_float(bw[h] & 0xFFFF0000u));
           if constexpr (C::REQUANT) {  // keep the bf16-rounded values: they are the next layer's input
             acc[j] = w[4 * i + h] << 16;
             acc[j + 1] = w[4 * i + h] & 0xFFFF0000u;
           }
         }
       }
-      uint8_t* buf = stg + (nstore % C::kOutBufs) * C::kOutBuf;
-      if (lane == 0) {  // the store that last used this buffer has read it
-        if (C::kOutBufs == 4) bulk_wait_group_read<3>();
-        else if (C::kOutBufs == 2) bulk_wait_group_read<1>();
-        else bulk_wait_group_read<0>();
-      }
-      __syncwarp();
+      uint8_t* buf = stg + b * C::kOutBuf;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int chunk = i ^ ((lane >> 1) & 3);
         *reinterpret_cast<uint4*>(buf + lane * 64 + chunk * 16) =
             make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        if (n0 < p.N && row0 < p.M) tma_store_2d(tmY, buf, n0, row0);
-        bulk_commit_group();
+      if (b == C::kOutBufs - 1) {  // the batch is staged: make it visible to TMA and store it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int cc = c - b; cc <= c; ++cc) {
+            const int nn = nb * C::BN + col0 + cc * 32;
+            if (nn < p.N && row0 < p.M) tma_store_2d(tmY, stg + (cc % C::kOutBufs) * C::kOutBuf, nn, row0);
+          }
+          bulk_commit_group();
+        }
       }
-      ++nstore;
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bempty + bi.slot);
-    bi.template advance<2>();
+    if constexpr (C::FMT == 1) {  // the bias slot was read in the store phase
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bempty + bi.slot);
+      bi.template advance<2>();
+    }
     if constexpr (C::REQUANT) requant_group<C>(p, acc, row0 + lane, nb * C::BN + col0);
   }
   if (lane == 0) bulk_wait_group<0>();
@@ -627,9 +653,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + C::kNumAcc;
-  uint64_t* scfull = tempty + C::kNumAcc;
-  uint64_t* scempty = scfull + C::kScSlots;
-  uint64_t* bfull = scempty + C::kScSlots;
+  uint64_t* bfull = tempty + C::kNumAcc;
   uint64_t* bempty = bfull + 2;
   uint64_t* teardown = bempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
@@ -644,10 +668,6 @@ __global__ void __launch_bounds__(384, 1)
     for (int a = 0; a < C::kNumAcc; ++a) {
       mbar_init(tfull + a, 1);
       mbar_init(tempty + a, C::kTmemEmptyCount);
-    }
-    for (int s = 0; s < C::kScSlots; ++s) {
-      mbar_init(scfull + s, 1);
-      mbar_init(scempty + s, C::kEpiWarps);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bfull + s, 1);
@@ -684,7 +704,7 @@ __global__ void __launch_bounds__(384, 1)
   if (warp < 4) {
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
-      producer<C>(&tmA, &tmB, p, smem, full, empty, scfull, scempty, bfull, bempty, abort_flag);
+      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag);
     else if (warp == 1 && lane == 0 && cta_rank<C>() == 0)
       mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, abort_flag);
     if constexpr (C::REQUANT) {
@@ -694,7 +714,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
-    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, scfull, scempty, bfull, bempty, abort_flag, warp, lane);
+    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, abort_flag, warp, lane);
   }
 
   if (C::PAIR && *abort_flag) {
@@ -768,7 +788,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.num_tiles = p.num_m * p.num_n;
   p.xs_t = g.xs_t;
   p.ld_s = g.ld_s;
-  p.ws_pad = g.ws_pad;
+  p.w_scale = g.w_scale;
   p.sfa = g.sfa;
   p.sfb = g.sfb;
   p.bias = static_cast<const uint16_t*>(g.bias);
@@ -852,7 +872,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
     const bool short_k = g.Kb <= 32;
     if (fmt == 0) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, false, true>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 1, false, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 2, false, true>>(g, num_sms, s);
     }
     if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, false, true>>(g, num_sms, s);
     return launch_cfg<Cfg<256, 1, 4, 1, false, true>>(g, num_sms, s);
@@ -864,7 +884,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   if (fmt == 0) {
     if (bn == 256) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 1>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 2>>(g, num_sms, s);
     }
     return launch_cfg<Cfg<128, 0, 5, 2>>(g, num_sms, s);
   }

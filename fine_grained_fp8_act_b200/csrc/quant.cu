@@ -109,22 +109,13 @@ __device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32
 //   kScaleKMajor / kScaleSfTiles: g -> (kb = g / rows, m = g % rows), so the
 //   scale writes of neighbouring lane-octets are neighbouring addresses.
 template <int FMT, int LAYOUT>
-__global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const uint32_t total, const FastDiv div,
-                                                        const uint32_t quant_blocks) {
+__global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const uint32_t total, const FastDiv div) {
   grid_wait_prerequisites();  // x may come from the preceding kernel (launched ahead of its end)
   grid_launch_dependents();   // the GEMM may set itself up meanwhile; it waits for our results
-  if (blockIdx.x >= quant_blocks) {
-    // trailing blocks: pad the float weight scales for the GEMM's bulk copies
-    const int64_t n = static_cast<int64_t>(a.Nb) * a.Kb;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x - quant_blocks) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x - quant_blocks) * blockDim.x)
-      reinterpret_cast<float4*>(a.ws_pad)[i] = make_float4(a.ws[i], 0.0f, 0.0f, 0.0f);
-    return;
-  }
   constexpr int kPasses = 2;
   const int lane = threadIdx.x & 31, oct = lane >> 3, l = lane & 7;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (quant_blocks * blockDim.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const uint16_t* x = static_cast<const uint16_t*>(a.x);
 
   for (uint32_t base = warp * (4 * kPasses); base < total; base += nwarps * (4 * kPasses)) {
@@ -252,13 +243,6 @@ __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict_
   }
 }
 
-__global__ void __launch_bounds__(256) ws_pad_kernel(const float* __restrict__ ws, const int64_t total,
-                                                     float4* __restrict__ out) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    out[i] = make_float4(ws[i], 0.0f, 0.0f, 0.0f);
-}
-
 __global__ void __launch_bounds__(256) xs_transpose_kernel(const float* __restrict__ xs, const int M, const int Kb,
                                                            const int64_t ld_s, float* __restrict__ out) {
   const int64_t total = static_cast<int64_t>(M) * Kb;
@@ -270,14 +254,6 @@ __global__ void __launch_bounds__(256) xs_transpose_kernel(const float* __restri
 }
 
 }  // namespace
-
-cudaError_t launch_ws_pad(const float* ws, int Nb, int Kb, float* out, cudaStream_t s) {
-  const int64_t total = static_cast<int64_t>(Nb) * Kb;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > 4096) blocks = 4096;
-  ws_pad_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(ws, total, reinterpret_cast<float4*>(out));
-  return cudaGetLastError();
-}
 
 cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(M) * Kb;
@@ -304,14 +280,8 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   int64_t blocks = (total + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  int64_t aux_blocks = 0;
-  if (a.ws_pad != nullptr && fmt == 0) {
-    aux_blocks = (static_cast<int64_t>(a.Nb) * a.Kb + 255) / 256;
-    if (aux_blocks > 64) aux_blocks = 64;
-  }
-  const dim3 grid(static_cast<unsigned>(blocks + aux_blocks)), block(256);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
   const uint32_t t32 = static_cast<uint32_t>(total);
-  const uint32_t qb = static_cast<uint32_t>(blocks);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start behind a GEMM's tail
@@ -321,7 +291,7 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-#define FG8_AQ(F, L) cudaLaunchKernelEx(&cfg, act_quant_kernel<F, L>, a, t32, div, qb)
+#define FG8_AQ(F, L) cudaLaunchKernelEx(&cfg, act_quant_kernel<F, L>, a, t32, div)
   if (fmt == 0) {
     if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor);
     else FG8_AQ(0, kScaleKMajor);
