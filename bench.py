@@ -39,6 +39,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "block-scaled FP8 linear TFLOP/s and % of B200 dense FP8 peak; act-quant GB/s"
 L2_FLUSH_BYTES = 256 << 20
+SMALL_M_MAX = 32  # fg8_linear's fused few-token path
 FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 
 
@@ -217,13 +218,23 @@ def run_fg8(args, rank, world, local):
         L["x"] = x0 if i == 0 else plan[i - 1]["y"]
         assert L["x"].shape == (L["g"].M, L["g"].K), "consecutive layers must chain"
 
-    # Consecutive layers chain: the GEMM of layer i also quantizes its output
-    # for layer i+1 (fg8_linear_run_chain), so layer i+1 has no act-quant launch.
-    chain = not args.no_chain
+    # Few tokens (M <= 128): fg8_linear runs one fused kernel per layer
+    # (quantize, swap-AB split-K GEMM, reduce).  Otherwise consecutive layers
+    # chain: the GEMM of layer i also quantizes its output for layer i+1
+    # (fg8_linear_run_chain), so layer i+1 has no act-quant launch.
+    small = plan[0]["g"].M <= SMALL_M_MAX
+    chain = not args.no_chain and not small
 
     def launch_layer(i, ev_mid=None):
         L = plan[i]
         g = L["g"]
+        if small:
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            fg8.fg8_linear(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
+                           L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, L["wsp"].data_ptr(),
+                           L["wsp"].numel(), sp)
+            return
         if i == 0 or not chain:
             fg8.fg8_linear_prepare(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["ws"].data_ptr(), g.fmt,
                                    L["wsp"].data_ptr(), L["wsp"].numel(), sp)
@@ -322,7 +333,7 @@ def run_fg8(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = f"fg8_gemm_kernel ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+    roof["kernel"] = ("fg8_small_m_kernel" if small else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
     roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
@@ -332,10 +343,11 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        fused = chain and i > 0  # this layer's act-quant ran in the previous GEMM's epilogue
+        fused = small or (chain and i > 0)  # act-quant inside a GEMM kernel
         per_kernel.append({"layer": gi.name, "act_quant_us": None if fused else qm[i] * 1e3,
                            "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
-                           "act_quant": "fused into the previous GEMM" if fused else "own launch",
+                           "act_quant": ("fused into the few-token kernel" if small else
+                                         "fused into the previous GEMM" if fused else "own launch"),
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
                            "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
 
@@ -344,9 +356,10 @@ def run_fg8(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
 
-    # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM
+    # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM;
+    # few tokens: one kernel per layer
     prep = [1 + (1 if L["g"].fmt == 1 else 0) for L in plan]
-    launches_per_step = (prep[0] if chain else sum(prep)) + nl
+    launches_per_step = nl if small else (prep[0] if chain else sum(prep)) + nl
     out = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,

@@ -137,6 +137,17 @@ GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   return w;
 }
 
+// fg8_linear's workspace: the prepare/run layout, and for few tokens also
+// the small-M path's [header | counters | partials] (the same bytes reused).
+size_t linear_workspace_need(int64_t M, int64_t N, int64_t K, int fmt) {
+  size_t need = linear_ws_layout(M, N, K, fmt).total;
+  if (M <= kSmallMMax) {
+    const size_t small = kHeaderBytes + small_m_scratch_bytes(M, N, K);
+    if (small > need) need = small;
+  }
+  return need;
+}
+
 fg8_status check_workspace(void* ws, size_t bytes, size_t need) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || bytes < need) return FG8_ERR_WORKSPACE;
   return FG8_OK;
@@ -204,7 +215,7 @@ fg8_status fg8_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld
 
 size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
   if (check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
-  return linear_ws_layout(M, N, K, fmt).total;
+  return linear_workspace_need(M, N, K, fmt);
 }
 
 size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
@@ -351,9 +362,30 @@ fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64
   if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
       (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv))
     return FG8_ERR_ALIGNMENT;
-  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_ws_layout(M, N, K, fmt).total);
-      st != FG8_OK)
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
     return st;
+  if (M <= kSmallMMax) {  // few tokens: one fused kernel (quantize, swap-AB split-K GEMM, reduce)
+    DeviceInfo dev;
+    if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    SmallMArgs a{};
+    a.x = x_bf16;
+    a.ld_x = ld_x;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.wq = wq_e4m3;
+    a.w_scale = w_scale_inv;
+    a.bias = bias_bf16;
+    a.y = y_bf16;
+    a.ld_y = ld_y;
+    a.splits = small_m_splits(static_cast<int>(N), static_cast<int>(K));
+    a.counters = reinterpret_cast<uint32_t*>(ws + kHeaderBytes);
+    a.part = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(static_cast<size_t>(ceil_div(N, 128)) * 4, kAlign));
+    a.status = reinterpret_cast<uint32_t*>(ws);
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
+  }
   if (fg8_status st = fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes, stream);
       st != FG8_OK)
     return st;

@@ -92,6 +92,32 @@ __host__ __device__ inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256
 // Float x scales row-major [M, Kb] -> K-major [Kb][ld_s].
 cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s);
 
+// Few tokens (M <= kSmallMMax): one kernel quantizes x, runs the swap-AB
+// split-K GEMM and reduces (small_m.cu).
+constexpr int kSmallMMax = 32;
+
+struct SmallMArgs {
+  const void* x;          // bf16 [M, K], row stride ld_x
+  int64_t ld_x;
+  int M, N, K;
+  const void* wq;         // e4m3 [N, K]
+  const void* w_scale;    // [ceil(N/128), ceil(K/128)] float32 or UE8M0 bytes
+  const void* bias;       // bf16 [N] or nullptr
+  void* y;                // bf16 [M, N], row stride ld_y
+  int64_t ld_y;
+  int splits;             // small_m_splits(N, K)
+  uint32_t* counters;     // [ceil(N/128)] (zeroed by the launch)
+  float* part;            // [splits][M][N] fp32 when splits > 1
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+int small_m_splits(int N, int K);
+// Workspace bytes of the small-M path after the status header: the
+// arrival counters (256-byte padded), then the split-K partials.
+size_t small_m_scratch_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s);
+
 int choose_block_n(int M, int N, int num_sms);
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s);

@@ -172,19 +172,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   tmem_ld_32x32b_x32(taddr, a);
 }
 
-// Ties 32 registers written by tcgen05.ld to the preceding tcgen05.wait::ld,
-// so no use of them can be scheduled above the wait.
-__device__ __forceinline__ void tmem_reg_fence(uint32_t* r) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-               :
-               : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -502,7 +489,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int row0 = mb * C::kTileM + rank * kBlockM + q * 32;
     // the tile's bias (bias ring; zeros past N or without bias)
-    if (!mbar_wait(bfull + bi.slot, bi.phase, limit, abort_flag)) {
+    if (!mbar_wait_warp(bfull + bi.slot, bi.phase, limit, abort_flag)) {
       raise_abort(abort_flag, p.status);
       break;
     }
@@ -529,7 +516,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
         const float s = s_now.x * s_now.y;  // sx(m, kb) * sw(block, kb)
         s_now = s_nxt;
         s_nxt = ss.next(p, sub_row, col0);
-        if (!mbar_wait(tfull + ab.slot, ab.phase, limit, abort_flag)) {
+        if (!mbar_wait_warp(tfull + ab.slot, ab.phase, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
           ok = false;
           break;
@@ -563,7 +550,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       }
       if (!ok) break;
     } else {
-      if (!mbar_wait(tfull + ab.slot, ab.phase, limit, abort_flag)) {
+      if (!mbar_wait_warp(tfull + ab.slot, ab.phase, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
         break;
       }

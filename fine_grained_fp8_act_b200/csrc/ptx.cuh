@@ -66,6 +66,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// mbar_wait by every lane of a warp, with a warp-uniform result: a lane that
+// gave up takes the whole warp out of the warp-collective operations
+// (tcgen05.ld, shuffles) that follow the wait.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               const volatile int* abort) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, limit_ns, abort));
+}
+
 // ------------------------------------------ programmatic dependent launch ----
 // Lets the next kernel in the stream (launched with programmatic stream
 // serialization) start its prologue once every CTA of this grid got here.
@@ -194,6 +202,37 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
       : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Ties 16 / 32 registers written by tcgen05.ld to the preceding
+// tcgen05.wait::ld, so no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_reg_fence16(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_reg_fence(uint32_t* r) {
+  tmem_reg_fence16(r);
+  tmem_reg_fence16(r + 16);
+}
+
+// Barrier `id` (1..15) over the first `count` threads that reach it (a
+// multiple of 32): synchronizes a subset of the CTA's warps.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ------------------------------------------------- CTA pairs (clusters) ----

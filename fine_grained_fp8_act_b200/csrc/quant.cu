@@ -23,42 +23,6 @@ namespace {
 
 using namespace qm;
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-// Quantize 16 values (two 16-byte bf16 loads) with the group's scale;
-// returns 16 packed e4m3 bytes.
-template <int FMT>
-__device__ __forceinline__ uint4 quantize16(const float (&f)[16], float s, uint32_t sbyte) {
-  float q[16];
-  if (FMT == 0) {
-    const float y = __frcp_rn(s);
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const float2 r = div2_rn_from_rcp(make_float2(f[i], f[i + 1]), s, y);
-      q[i] = r.x;
-      q[i + 1] = r.y;
-    }
-  } else {
-    const float inv = e8m0_reciprocal(sbyte);  // x * 2^-e is the correctly rounded x / 2^e
-    const float2 I = make_float2(inv, inv);
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const float2 r = __fmul2_rn(make_float2(f[i], f[i + 1]), I);
-      q[i] = r.x;
-      q[i + 1] = r.y;
-    }
-  }
-  return make_uint4(pack_e4m3x4(q[0], q[1], q[2], q[3]), pack_e4m3x4(q[4], q[5], q[6], q[7]),
-                    pack_e4m3x4(q[8], q[9], q[10], q[11]), pack_e4m3x4(q[12], q[13], q[14], q[15]));
-}
-
 // Quantize 8 values with the group's scale; returns 8 packed e4m3 bytes.
 template <int FMT>
 __device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s, uint32_t sbyte) {

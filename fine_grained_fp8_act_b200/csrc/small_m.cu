@@ -1,0 +1,599 @@
+// small_m.cu -- the fine-grained FP8 linear for few tokens (M <= 128) as one
+// kernel (M <= 32): activation quantization, block-scaled GEMM, split-K
+// reduction, bias and bf16 output ("Transformers 中的细粒度 FP8 量化 ... 完全指南",
+// §八 step 6 with the dynamic per-token activation groups of §6.1).
+//
+// With few tokens the layer is bound by reading the weights once (N x K
+// e4m3 bytes).  The tile-per-output GEMM would give one 128-token row of
+// tiles, N/256 CTAs, most SMs idle.  Here the operands swap roles: the
+// weights are the tensor core's M side.  A CTA owns 128 weight rows -- one
+// weight block, so one weight scale per K-block -- and a range of K-blocks;
+// the MMA is M = 128 weight rows x N = MP tokens (padded to 16 or 32) x K = 32,
+// and the K-ranges of a weight tile are spread over several CTAs (split-K)
+// so that every SM streams weights.
+//
+// Roles (320 threads):
+//   warp 0      producer: per K-block, TMA loads of the weight box (128 x 128
+//               e4m3, 128-byte swizzle) and of the bf16 activation block
+//               (MP x 128, rows past M zero-filled) into one stage of a ring
+//   warp 1      MMA issuer (one thread)
+//   warps 2-5   quantizers, one K-block per warp (two or four in flight): the staged
+//               bf16 activation block (8 lanes per token, 16 channels each),
+//               amax by shuffles, the
+//               scale and e4m3 codes of quant_math.cuh -- the same bits as
+//               the stand-alone activation quantization -- written as the
+//               MMA's B operand (128-byte swizzle) in the same ring slot;
+//               float scales to a token-scale ring, UE8M0 bytes (and the
+//               weight block's byte) to the scale-factor chunks the MMA
+//               copies into TMEM
+//   warps 6-9   epilogue: thread = weight row.  Float: each K-block's
+//               partial P lands in its own TMEM buffer (4 of them) and is
+//               promoted, acc[m] += P[m] * (sx[m] * sw) (the quantizers
+//               leave the product sx[m] * sw in the token-scale ring).  UE8M0: the
+//               block-scaled MMA accumulates the whole K-range.  With one
+//               split the thread writes y[m, n] = bf16(acc[m] + bias[n]);
+//               with several, fp32 partials go to the workspace and the last
+//               CTA of the weight tile to finish sums them in split order,
+//               adds the bias and writes y.
+//
+// Every wait is bounded; on expiry the kernel records FG8_ERR_TIMEOUT in the
+// status word, drains its copies and tensor-core ops, frees TMEM and returns.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "fg8_internal.h"
+#include "ptx.cuh"
+#include "quant_math.cuh"
+
+namespace fg8 {
+namespace {
+
+constexpr uint32_t kTimeoutStatus = 6u;  // FG8_ERR_TIMEOUT
+constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr int kQuantWarp0 = 2, kQuantWarps = 4;
+constexpr int kEpiWarp0 = 6;
+
+struct SmParams {
+  const uint16_t* x;  // bf16 [M, K], row stride ld_x
+  int64_t ld_x;
+  int M, N, K, Kb, S;
+  const float* ws_f;    // float weight scales [Nb][Kb]
+  const uint8_t* ws_b;  // UE8M0 weight scales [Nb][Kb]
+  const uint16_t* bias;
+  uint16_t* y;
+  int64_t ld_y;
+  float* part;          // split-K partials [S][M][N]
+  uint32_t* counters;   // [Nb], zero at launch
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+template <int FMT_, int MP_>
+struct SmCfg {
+  static constexpr int FMT = FMT_, MP = MP_;
+  // one ring stage: weight box | bf16 activation block | its e4m3 codes (the
+  // MMA's B operand) | UE8M0: scale-factor chunks of the tokens and the weight rows
+  static constexpr int kW = 128 * 128;
+  static constexpr int kXb = MP * 256;
+  static constexpr int kX = MP * 128;
+  static constexpr int kOffXb = kW, kOffXq = kW + kXb, kOffSf = kOffXq + kX;
+  static constexpr int kStage = (kOffSf + (FMT == 1 ? 2 * kSfChunkBytes : 0) + 1023) / 1024 * 1024;
+  static constexpr int kScSlots = FMT == 0 ? 8 : 1;
+  static constexpr int kStagesFit = (220 * 1024 - kScSlots * MP * 4) / kStage;
+  // kQ quantizer warps work on K-blocks i = w (mod kQ); the ring depth is a
+  // multiple of kQ (and divides the 8 scale slots' period) so that each ring
+  // slot and scale slot is only ever waited on by one quantizer warp, in order
+  static constexpr int kQ = kStagesFit >= 8 ? 4 : 2;
+  static constexpr int STAGES = kQ == 4 ? 8 : (kStagesFit >= 6 ? 6 : 4);
+  static constexpr int kNumAcc = FMT == 0 ? 4 : 1;
+  static constexpr int kCols = MP;
+  static constexpr int kChunk = MP < 32 ? MP : 32;  // TMEM columns per load
+  static constexpr int kEpiThreads = 128;
+  static constexpr int kThreads = kEpiWarp0 * 32 + kEpiThreads;
+  static constexpr int kSfCol = 256;  // UE8M0: scale factors in TMEM, two sets of 8 columns
+  static constexpr int kOffSc = STAGES * kStage;
+  static constexpr int kOffBar = kOffSc + kScSlots * MP * 4;
+  static constexpr int kSmemUsed = 1024 + kOffBar + 512;
+  // at least 120 KB so that one CTA holds an SM (and its 512 TMEM columns)
+  static constexpr int kSmem = kSmemUsed < 120 * 1024 ? 120 * 1024 : kSmemUsed;
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(STAGES >= 4 && STAGES % kQ == 0 && 8 % kQ == 0, "ring depth");
+  static_assert(MP % 16 == 0 && MP >= 16 && MP <= 32, "token padding");
+  static_assert(kOffXq % 1024 == 0, "the swizzled B operand starts on a 1024-byte boundary");
+  static_assert(kNumAcc * MP <= 256, "TMEM columns");
+  // M = 128 (weight rows), N = MP (tokens), K-major e4m3 operands, f32 accumulate
+  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(MP >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t kIdescMx = (uint32_t(MP >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24);
+};
+
+__device__ __forceinline__ void sm_raise(volatile int* abort_flag, uint32_t* status) {
+  *abort_flag = 1;
+  atomicExch(status, kTimeoutStatus);
+}
+
+struct SmRing {
+  int slot = 0;
+  uint32_t phase = 0;
+  template <int N>
+  __device__ __forceinline__ void advance() {
+    if (++slot == N) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// W (16 or 32) consecutive TMEM columns of the warp's 32 lanes into registers, waited for.
+template <int W>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[W]) {
+  if constexpr (W == 16) {
+    tmem_ld_32x32b_x16(taddr, r);
+    tmem_wait_ld();
+    tmem_reg_fence16(r);
+  } else {
+    tmem_ld_32x32b_x32(taddr, r);
+    tmem_wait_ld();
+    tmem_reg_fence(r);
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void sm_producer(const CUtensorMap* tmW, const CUtensorMap* tmX, const SmParams& p,
+                                            uint8_t* smem, uint64_t* wfull, uint64_t* sempty, int nt, int kb0, int kb1,
+                                            volatile int* abort_flag) {
+  SmRing st;
+  uint32_t issued = 0, par[C::STAGES];
+  for (int kb = kb0; kb < kb1; ++kb) {
+    if (!mbar_wait(sempty + st.slot, st.phase ^ 1u, p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      break;
+    }
+    uint8_t* stage = smem + st.slot * C::kStage;
+    mbar_arrive_expect_tx(wfull + st.slot, C::kW + C::kXb);
+    tma_load_2d(stage, tmW, wfull + st.slot, kb * 128, nt * 128);
+    tma_load_2d(stage + C::kOffXb, tmX, wfull + st.slot, kb * 128, 0);
+    par[st.slot] = st.phase;
+    issued |= 1u << st.slot;
+    st.template advance<C::STAGES>();
+  }
+  for (int s = 0; s < C::STAGES; ++s)  // every issued copy lands before shared memory goes away
+    if ((issued >> s) & 1u) (void)mbar_wait(wfull + s, par[s], kDrainNs, nullptr);
+}
+
+// The quantizer warps: warp w < kQ quantizes K-blocks kb0 + w, kb0 + w + kQ,
+// ... (kQ K-blocks in flight at once), 8 lanes per token, 4 tokens per pass.
+template <class C>
+__device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, uint64_t* wfull, uint64_t* xfull,
+                                             uint64_t* scfull, uint64_t* scempty, int nt, int kb0, int kb1,
+                                             volatile int* abort_flag) {
+  const int qw = (static_cast<int>(threadIdx.x) >> 5) - kQuantWarp0;
+  const int lane = static_cast<int>(threadIdx.x) & 31, l = lane & 7, r_in = lane >> 3;
+  if (qw >= C::kQ) return;
+  for (int i = qw; kb0 + i < kb1; i += C::kQ) {
+    const int kb = kb0 + i;
+    const int slot = i % C::STAGES;
+    const uint32_t phase = static_cast<uint32_t>((i / C::STAGES) & 1);
+    const int sslot = i % C::kScSlots;
+    const uint32_t sphase = static_cast<uint32_t>((i / C::kScSlots) & 1);
+    // the stage's activation block has landed (and the MMA that last used
+    // the stage, hence its B operand, is done: the producer refilled it after)
+    if (!mbar_wait_warp(wfull + slot, phase, p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      break;
+    }
+    if (C::FMT == 0 && !mbar_wait_warp(scempty + sslot, sphase ^ 1u, p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      break;
+    }
+    uint8_t* stage = smem + slot * C::kStage;
+    uint8_t* xs = stage + C::kOffXq;
+    const uint8_t* xb = stage + C::kOffXb;
+    float* scs = reinterpret_cast<float*>(smem + C::kOffSc + sslot * C::MP * 4);
+    // float: the scale ring holds sx(m, kb) * sw(tile, kb), the factor the promotion applies
+    const float sw = C::FMT == 0 ? p.ws_f[static_cast<int64_t>(nt) * p.Kb + kb] : 0.0f;
+    constexpr int kPasses = C::MP / 4;
+    constexpr int kBatch = kPasses < 4 ? kPasses : 4;
+#pragma unroll
+    for (int u0 = 0; u0 < kPasses; u0 += kBatch) {
+      uint4 v[kBatch][2];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {  // channels 16 l .. 16 l + 15 of the row (zeros past M and K)
+        const int row = (u0 + u) * 4 + r_in;
+        const uint4* src = reinterpret_cast<const uint4*>(xb + row * 256 + l * 32);
+        v[u][0] = src[0];
+        v[u][1] = src[1];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int row = (u0 + u) * 4 + r_in;
+        float f[16];
+        {
+          float f0[8], f1[8];
+          qm::unpack_bf16x8(v[u][0], f0);
+          qm::unpack_bf16x8(v[u][1], f1);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            f[k] = f0[k];
+            f[8 + k] = f1[k];
+          }
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(f[k]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+        const float s = qm::group_scale(amax);
+        const uint32_t sb = C::FMT == 1 ? qm::e8m0_ceil_byte(s) : 0u;
+        const uint4 q = qm::quantize16<C::FMT>(f, s, sb);
+        // row `row`, 16-byte chunk l of the 128-byte row, 128-byte swizzle (8-row atoms)
+        *reinterpret_cast<uint4*>(xs + (row >> 3) * 1024 + (row & 7) * 128 + ((l ^ (row & 7)) << 4)) = q;
+        if (l == 0) {
+          if constexpr (C::FMT == 0) {
+            scs[row] = row < p.M ? s * sw : 0.0f;
+          } else {  // tcgen05.cp source: token row r -> word (r % 32) * 16 + (r / 32) * 4, byte 0
+            *reinterpret_cast<uint32_t*>(xs + C::kX + (row & 31) * 16 + (row >> 5) * 4) = row < p.M ? sb : 127u;
+          }
+        }
+      }
+    }
+    if constexpr (C::FMT == 1) {
+      // every weight row of the tile has the block's scale; token rows past
+      // MP get a finite scale the MMA never uses
+      const uint32_t wb = p.ws_b[static_cast<int64_t>(nt) * p.Kb + kb];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = k * 32 + lane;
+        *reinterpret_cast<uint32_t*>(xs + C::kX + kSfChunkBytes + (r & 31) * 16 + (r >> 5) * 4) = wb;
+        if (r >= C::MP) *reinterpret_cast<uint32_t*>(xs + C::kX + (r & 31) * 16 + (r >> 5) * 4) = 127u;
+      }
+    }
+    fence_proxy_async_smem();  // the tensor core reads what these threads wrote
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(xfull + slot);
+      if (C::FMT == 0) mbar_arrive(scfull + sslot);
+    }
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void sm_mma(const SmParams& p, uint8_t* smem, uint32_t tmem, uint64_t* wfull,
+                                       uint64_t* xfull, uint64_t* sempty, uint64_t* tfull, uint64_t* tempty,
+                                       uint64_t* teardown, int kb0, int kb1, volatile int* abort_flag) {
+  SmRing st, ab;
+  for (int kb = kb0; kb < kb1; ++kb) {
+    if (!mbar_wait(wfull + st.slot, st.phase, p.wait_limit_ns, abort_flag) ||
+        !mbar_wait(xfull + st.slot, st.phase, p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      break;
+    }
+    tc_fence_after();
+    if (C::FMT == 0) {
+      if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, p.wait_limit_ns, abort_flag)) {
+        sm_raise(abort_flag, p.status);
+        break;
+      }
+      tc_fence_after();
+    }
+    const uint32_t a = smem_u32(smem + st.slot * C::kStage);
+    const uint32_t b = a + C::kOffXq;
+    // UE8M0: this K-block's scale factors into one of two TMEM column sets
+    // (alternating, so a copy never lands under an MMA still reading the last one)
+    const uint32_t sf = tmem + static_cast<uint32_t>(C::kSfCol + ((kb - kb0) & 1) * 8);
+    if (C::FMT == 1) {
+      tc_cp_32x128b_warpx4(sf, smem_desc(b + C::kX, 128, 128, 0));                      // tokens (B)
+      tc_cp_32x128b_warpx4(sf + 4, smem_desc(b + C::kX + kSfChunkBytes, 128, 128, 0));  // weight rows (A)
+    }
+    const uint32_t d = tmem + static_cast<uint32_t>(C::FMT == 0 ? ab.slot * C::MP : 0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint64_t ad = smem_desc(a + k * 32, 16, 1024, 2);
+      const uint64_t bd = smem_desc(b + k * 32, 16, 1024, 2);
+      if (C::FMT == 0) mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
+      else mma_mxf8f6f4(d, ad, bd, C::kIdescMx, sf + 4, sf, (kb > kb0 || k > 0) ? 1u : 0u);
+    }
+    tc_commit(sempty + st.slot);  // frees the weight box and the activation block
+    if (C::FMT == 0) {
+      tc_commit(tfull + ab.slot);
+      ab.template advance<C::kNumAcc>();
+    }
+    st.template advance<C::STAGES>();
+  }
+  if (C::FMT == 1) tc_commit(tfull);
+  tc_commit(teardown);  // all tensor-core ops done before TMEM is released
+  (void)mbar_wait(teardown, 0, kDrainNs, nullptr);
+}
+
+template <class C>
+__device__ __forceinline__ void sm_epilogue(const SmParams& p, uint8_t* smem, uint32_t tmem, uint64_t* tfull,
+                                            uint64_t* tempty, uint64_t* scfull, uint64_t* scempty, int nt, int sp,
+                                            int kb0, int kb1, volatile int* abort_flag, volatile int* last_flag) {
+  const int warp = static_cast<int>(threadIdx.x) >> 5, lane = static_cast<int>(threadIdx.x) & 31;
+  const int q = warp & 3;  // TMEM lane quadrant
+  const int t = q * 32 + lane;
+  const int n = nt * 128 + t;
+  const int m0 = 0;  // first token of this thread's columns
+  const int et = static_cast<int>(threadIdx.x) - kEpiWarp0 * 32;
+  const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+  float acc[C::kCols];
+#pragma unroll
+  for (int j = 0; j < C::kCols; ++j) acc[j] = 0.0f;
+  bool ok = true;
+  if constexpr (C::FMT == 0) {
+    SmRing ab, sc;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait_warp(scfull + sc.slot, sc.phase, p.wait_limit_ns, abort_flag) ||
+          !mbar_wait_warp(tfull + ab.slot, ab.phase, p.wait_limit_ns, abort_flag)) {
+        sm_raise(abort_flag, p.status);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + lane_base + static_cast<uint32_t>(ab.slot * C::MP + m0);
+      const float* scs = reinterpret_cast<const float*>(smem + C::kOffSc + sc.slot * C::MP * 4) + m0;
+#pragma unroll
+      for (int c = 0; c < C::kCols / C::kChunk; ++c) {
+        uint32_t r[C::kChunk];
+        tmem_ld_chunk<C::kChunk>(taddr + c * C::kChunk, r);
+        if (c + 1 == C::kCols / C::kChunk) {  // the K-block's columns are all read: hand the buffer back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty + ab.slot);
+        }
+#pragma unroll
+        for (int j = 0; j < C::kChunk; ++j)
+          acc[c * C::kChunk + j] = __fmaf_rn(__uint_as_float(r[j]), scs[c * C::kChunk + j], acc[c * C::kChunk + j]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(scempty + sc.slot);
+      ab.template advance<C::kNumAcc>();
+      sc.template advance<C::kScSlots>();
+    }
+  } else {
+    if (!mbar_wait_warp(tfull, 0, p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      ok = false;
+    } else {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < C::kCols / C::kChunk; ++c) {
+        uint32_t r[C::kChunk];
+        tmem_ld_chunk<C::kChunk>(tmem + lane_base + static_cast<uint32_t>(m0 + c * C::kChunk), r);
+#pragma unroll
+        for (int j = 0; j < C::kChunk; ++j) acc[c * C::kChunk + j] = __uint_as_float(r[j]);
+      }
+    }
+  }
+  tc_fence_before();
+  // Every epilogue warp takes the same path from here on (the named barriers
+  // below count all of them): a warp that timed out joins them, writing nothing.
+  const float bias_n = (p.bias != nullptr && n < p.N) ? __uint_as_float(static_cast<uint32_t>(p.bias[n]) << 16) : 0.0f;
+  if (p.S == 1) {
+    if (ok && n < p.N) {
+#pragma unroll
+      for (int j = 0; j < C::kCols; ++j)
+        if (m0 + j < p.M)
+          p.y[static_cast<int64_t>(m0 + j) * p.ld_y + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j] + bias_n));
+    }
+    return;
+  }
+  if (ok && n < p.N) {
+#pragma unroll
+    for (int j = 0; j < C::kCols; ++j)
+      if (m0 + j < p.M) p.part[(static_cast<int64_t>(sp) * p.M + m0 + j) * p.N + n] = acc[j];
+  }
+  __threadfence();  // the partials are visible device-wide before the arrival is counted
+  named_barrier_sync(1, C::kEpiThreads);
+  if (et == 0) {
+    const uint32_t done = ok && !*abort_flag ? atomicAdd(p.counters + nt, 1u) + 1u : 0u;
+    *last_flag = done == static_cast<uint32_t>(p.S) ? 1 : 0;
+  }
+  named_barrier_sync(1, C::kEpiThreads);
+  if (*last_flag && n < p.N) {
+    __threadfence();
+#pragma unroll
+    for (int j = 0; j < C::kCols; ++j) {
+      if (m0 + j < p.M) {
+        float v = 0.0f;
+        for (int s = 0; s < p.S; ++s)  // split order: the same sum whichever CTA is last
+          v += s == sp ? acc[j] : __ldcg(p.part + (static_cast<int64_t>(s) * p.M + m0 + j) * p.N + n);
+        p.y[static_cast<int64_t>(m0 + j) * p.ld_y + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v + bias_n));
+      }
+    }
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    fg8_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                       const SmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* xfull = wfull + C::STAGES;
+  uint64_t* sempty = xfull + C::STAGES;
+  uint64_t* tfull = sempty + C::STAGES;
+  uint64_t* tempty = tfull + C::kNumAcc;
+  uint64_t* scfull = tempty + C::kNumAcc;
+  uint64_t* scempty = scfull + C::kScSlots;
+  uint64_t* teardown = scempty + C::kScSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = static_cast<int>(threadIdx.x) >> 5, lane = static_cast<int>(threadIdx.x) & 31;
+  const int nt = static_cast<int>(blockIdx.x) / p.S, sp = static_cast<int>(blockIdx.x) % p.S;
+  const int kb0 = static_cast<int>(static_cast<int64_t>(sp) * p.Kb / p.S);
+  const int kb1 = static_cast<int>(static_cast<int64_t>(sp + 1) * p.Kb / p.S);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(wfull + s, 1);
+      mbar_init(xfull + s, 1);
+      mbar_init(sempty + s, 1);
+    }
+    for (int a = 0; a < C::kNumAcc; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, C::kEpiThreads / 32);
+    }
+    for (int s = 0; s < C::kScSlots; ++s) {
+      mbar_init(scfull + s, 1);
+      mbar_init(scempty + s, C::kEpiThreads / 32);
+    }
+    mbar_init(teardown, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_wait_prerequisites();  // x may come from the preceding kernel
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) sm_producer<C>(&tmW, &tmX, p, smem, wfull, sempty, nt, kb0, kb1, abort_flag);
+  } else if (warp == 1) {
+    if (lane == 0) sm_mma<C>(p, smem, tmem, wfull, xfull, sempty, tfull, tempty, teardown, kb0, kb1, abort_flag);
+  } else if (warp < kEpiWarp0) {
+    sm_quantizer<C>(p, smem, wfull, xfull, scfull, scempty, nt, kb0, kb1, abort_flag);
+  } else {
+    sm_epilogue<C>(p, smem, tmem, tfull, tempty, scfull, scempty, nt, sp, kb0, kb1, abort_flag, last_flag);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFnSm)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnSm encode_fn_sm() {
+  static EncodeTiledFnSm fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnSm>(ptr);
+  }
+  return fn;
+}
+
+template <class C>
+cudaError_t launch_small_m_cfg(const SmallMArgs& a, cudaStream_t s) {
+  EncodeTiledFnSm fn = encode_fn_sm();
+  if (fn == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap tmW, tmX;
+  const cuuint32_t estr[2] = {1, 1};
+  {  // weights e4m3 [N, K]: 128 x 128 boxes, 128-byte swizzle
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K)};
+    const cuuint32_t box[2] = {128, 128};
+    if (fn(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.wq), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {  // activations bf16 [M, K] (row stride ld_x): MP x 128 boxes, rows past M zero-filled
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ld_x) * 2};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(C::MP)};
+    if (fn(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  SmParams p;
+  p.x = static_cast<const uint16_t*>(a.x);
+  p.ld_x = a.ld_x;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.Kb = (a.K + 127) / 128;
+  p.S = a.splits;
+  p.ws_f = static_cast<const float*>(a.w_scale);
+  p.ws_b = static_cast<const uint8_t*>(a.w_scale);
+  p.bias = static_cast<const uint16_t*>(a.bias);
+  p.y = static_cast<uint16_t*>(a.y);
+  p.ld_y = a.ld_y;
+  p.part = a.part;
+  p.counters = a.counters;
+  p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns;
+  const int nt = (a.N + 127) / 128;
+  auto kern = fg8_small_m_kernel<C>;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  if (a.splits > 1) {  // arrival counters of the split-K reduction start at zero
+    const cudaError_t e = cudaMemsetAsync(a.counters, 0, static_cast<size_t>(nt) * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(nt * a.splits));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmW, tmX, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int small_m_splits(int N, int K) {
+  // Work units (weight tile, K-range) over the SMs: fewest waves x K-blocks
+  // per unit, plus a K-block's worth per unit for its fixed costs and one for
+  // the reduction when the K-range is split.  Depends on the shape only (148
+  // SMs assumed), so the workspace size never depends on the device.
+  constexpr int kSms = 148;
+  const int nt = (N + 127) / 128, kb = (K + 127) / 128;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= kb && s <= 64; ++s) {
+    const int units = nt * s;
+    const int waves = (units + kSms - 1) / kSms;
+    const double cost = static_cast<double>(waves) * ((kb + s - 1) / s + 1) + (s > 1 ? 1.0 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+size_t small_m_scratch_bytes(int64_t M, int64_t N, int64_t K) {
+  const int s = small_m_splits(static_cast<int>(N), static_cast<int>(K));
+  const size_t counters = (static_cast<size_t>((N + 127) / 128) * 4 + 255) / 256 * 256;
+  return counters + (s > 1 ? static_cast<size_t>(s) * M * N * 4 : 0);
+}
+
+cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s) {
+  if (a.M < 1 || a.M > kSmallMMax) return cudaErrorInvalidValue;
+  if (fmt == 0) return a.M <= 16 ? launch_small_m_cfg<SmCfg<0, 16>>(a, s) : launch_small_m_cfg<SmCfg<0, 32>>(a, s);
+  return a.M <= 16 ? launch_small_m_cfg<SmCfg<1, 16>>(a, s) : launch_small_m_cfg<SmCfg<1, 32>>(a, s);
+}
+
+}  // namespace fg8
