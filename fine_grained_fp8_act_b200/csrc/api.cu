@@ -19,7 +19,7 @@ namespace {
 using namespace fg8;
 
 constexpr int64_t kMaxDim = 2147483647LL;
-constexpr size_t kHeaderBytes = 256;  // status word + reserved
+constexpr size_t kHeaderBytes = kWorkspaceHeaderBytes;  // status word, split-K counters
 constexpr size_t kAlign = 256;
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
@@ -137,12 +137,19 @@ GemmWs gemm_ws_layout(int64_t M, int64_t N, int64_t K, int fmt) {
   return w;
 }
 
+// Split-K counters of the few-token path that do not fit in the header
+// (more than kHeaderCounters weight tiles) go after it, cleared per call.
+size_t small_counter_bytes(int64_t N) {
+  const int64_t nt = (N + 127) / 128;
+  return nt > kHeaderCounters ? align_up(static_cast<size_t>(nt) * 4, kAlign) : 0;
+}
+
 // fg8_linear's workspace: the prepare/run layout, and for few tokens also
-// the small-M path's [header | counters | partials] (the same bytes reused).
+// the small-M path's [header | (counters) | partials] (the same bytes reused).
 size_t linear_workspace_need(int64_t M, int64_t N, int64_t K, int fmt) {
   size_t need = linear_ws_layout(M, N, K, fmt).total;
   if (M <= kSmallMMax) {
-    const size_t small = kHeaderBytes + small_m_scratch_bytes(M, N, K);
+    const size_t small = kHeaderBytes + small_counter_bytes(N) + small_m_partial_bytes(M, N, K);
     if (small > need) need = small;
   }
   return need;
@@ -380,8 +387,10 @@ fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64
     a.y = y_bf16;
     a.ld_y = ld_y;
     a.splits = small_m_splits(static_cast<int>(N), static_cast<int>(K));
-    a.counters = reinterpret_cast<uint32_t*>(ws + kHeaderBytes);
-    a.part = reinterpret_cast<float*>(ws + kHeaderBytes + align_up(static_cast<size_t>(ceil_div(N, 128)) * 4, kAlign));
+    const size_t extra = small_counter_bytes(N);
+    a.zero_counters = extra > 0;
+    a.counters = reinterpret_cast<uint32_t*>(ws + (extra > 0 ? kHeaderBytes : kHeaderCounterOffset));
+    a.part = reinterpret_cast<float*>(ws + kHeaderBytes + extra);
     a.status = reinterpret_cast<uint32_t*>(ws);
     a.wait_limit_ns = g_wait_limit_ns.load();
     return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
@@ -456,6 +465,14 @@ fg8_status fg8_check_device_status(void* workspace, void* stream) {
       cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return FG8_ERR_CUDA;
+  }
+  if (word != 0) {
+    // a kernel gave up mid-way: its split-K counters may be left counting,
+    // so the whole header starts from zero again
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return FG8_ERR_CUDA;
+    }
   }
   return word == 0 ? FG8_OK : static_cast<fg8_status>(word);
 }

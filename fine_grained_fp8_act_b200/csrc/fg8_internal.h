@@ -92,6 +92,14 @@ __host__ __device__ inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256
 // Float x scales row-major [M, Kb] -> K-major [Kb][ld_s].
 cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s);
 
+// Workspace header: the sticky device status word at byte 0 and, from byte
+// kHeaderCounterOffset, the few-token path's split-K arrival counters (one
+// per 128-row weight tile, zero at rest: the last CTA of a tile resets its
+// counter).  Zeroed by the caller before first use.
+constexpr size_t kWorkspaceHeaderBytes = 1024;
+constexpr size_t kHeaderCounterOffset = 64;
+constexpr int kHeaderCounters = static_cast<int>((kWorkspaceHeaderBytes - kHeaderCounterOffset) / 4);
+
 // Few tokens (M <= kSmallMMax): one kernel quantizes x, runs the swap-AB
 // split-K GEMM and reduces (small_m.cu).
 constexpr int kSmallMMax = 32;
@@ -106,16 +114,16 @@ struct SmallMArgs {
   void* y;                // bf16 [M, N], row stride ld_y
   int64_t ld_y;
   int splits;             // small_m_splits(N, K)
-  uint32_t* counters;     // [ceil(N/128)] (zeroed by the launch)
+  uint32_t* counters;     // [ceil(N/128)], zero at rest (or zeroed by the launch, below)
+  bool zero_counters;     // counters outside the header: clear them before the kernel
   float* part;            // [splits][M][N] fp32 when splits > 1
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 
 int small_m_splits(int N, int K);
-// Workspace bytes of the small-M path after the status header: the
-// arrival counters (256-byte padded), then the split-K partials.
-size_t small_m_scratch_bytes(int64_t M, int64_t N, int64_t K);
+// Bytes of fp32 split-K partials the small-M path needs (0 with one split).
+size_t small_m_partial_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s);
 
 int choose_block_n(int M, int N, int num_sms);

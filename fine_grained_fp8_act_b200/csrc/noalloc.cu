@@ -71,8 +71,8 @@ extern "C" fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t 
   void* scratch = scratch_for_current_device();
   if (scratch == nullptr) return FG8_ERR_CUDA;
   // The scratch keeps the previous call's bytes; the only part that must
-  // start at zero is the device status word at its head.
-  if (cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+  // start at zero is the header at its head (status word, split-K counters).
+  if (cudaMemsetAsync(scratch, 0, fg8::kWorkspaceHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return FG8_ERR_CUDA;
   }

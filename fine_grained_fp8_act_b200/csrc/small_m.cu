@@ -64,7 +64,7 @@ struct SmParams {
   uint16_t* y;
   int64_t ld_y;
   float* part;          // split-K partials [S][M][N]
-  uint32_t* counters;   // [Nb], zero at launch
+  uint32_t* counters;   // [Nb], zero at launch; the last CTA of a tile resets its own
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
@@ -389,6 +389,8 @@ __device__ __forceinline__ void sm_epilogue(const SmParams& p, uint8_t* smem, ui
   if (et == 0) {
     const uint32_t done = ok && !*abort_flag ? atomicAdd(p.counters + nt, 1u) + 1u : 0u;
     *last_flag = done == static_cast<uint32_t>(p.S) ? 1 : 0;
+    // every CTA of the tile has arrived: zero the counter for the next call
+    if (done == static_cast<uint32_t>(p.S)) p.counters[nt] = 0u;
   }
   named_barrier_sync(1, C::kEpiThreads);
   if (*last_flag && n < p.N) {
@@ -542,7 +544,7 @@ cudaError_t launch_small_m_cfg(const SmallMArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  if (a.splits > 1) {  // arrival counters of the split-K reduction start at zero
+  if (a.splits > 1 && a.zero_counters) {  // arrival counters outside the header start at zero
     const cudaError_t e = cudaMemsetAsync(a.counters, 0, static_cast<size_t>(nt) * sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
   }
@@ -564,30 +566,22 @@ cudaError_t launch_small_m_cfg(const SmallMArgs& a, cudaStream_t s) {
 }  // namespace
 
 int small_m_splits(int N, int K) {
-  // Work units (weight tile, K-range) over the SMs: fewest waves x K-blocks
-  // per unit, plus a K-block's worth per unit for its fixed costs and one for
-  // the reduction when the K-range is split.  Depends on the shape only (148
-  // SMs assumed), so the workspace size never depends on the device.
+  // One wave of work units (weight tile, K-range): as many K-splits as fit
+  // next to the other tiles on the 148 SMs (about 100 streaming SMs already
+  // reach the HBM bandwidth; a second wave would only add its ramp).
+  // Depends on the shape only, so the workspace size never depends on the
+  // device.
   constexpr int kSms = 148;
   const int nt = (N + 127) / 128, kb = (K + 127) / 128;
-  int best = 1;
-  double best_cost = 1e30;
-  for (int s = 1; s <= kb && s <= 64; ++s) {
-    const int units = nt * s;
-    const int waves = (units + kSms - 1) / kSms;
-    const double cost = static_cast<double>(waves) * ((kb + s - 1) / s + 1) + (s > 1 ? 1.0 : 0.0);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
+  int s = kSms / nt;
+  if (s > kb) s = kb;
+  if (s > 64) s = 64;
+  return s < 1 ? 1 : s;
 }
 
-size_t small_m_scratch_bytes(int64_t M, int64_t N, int64_t K) {
+size_t small_m_partial_bytes(int64_t M, int64_t N, int64_t K) {
   const int s = small_m_splits(static_cast<int>(N), static_cast<int>(K));
-  const size_t counters = (static_cast<size_t>((N + 127) / 128) * 4 + 255) / 256 * 256;
-  return counters + (s > 1 ? static_cast<size_t>(s) * M * N * 4 : 0);
+  return s > 1 ? static_cast<size_t>(s) * M * N * 4 : 0;
 }
 
 cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s) {

@@ -101,11 +101,18 @@ FG8_API size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_s
  *   bias_bf16   [N] bf16 or NULL
  *   y_bf16      [M, N] bf16, row stride ld_y (output; written once, RNE)
  *   workspace   >= fg8_linear_workspace_bytes(M, N, K, fmt), 256-byte aligned,
- *               caller-owned device memory.  Its first 256 bytes hold a sticky
- *               device status word: zero them once before first use (e.g.
- *               allocate the workspace zero-filled); fg8_check_device_status
- *               reads and clears it.  Calls sharing a workspace must not
- *               overlap on the device.
+ *               caller-owned device memory.  Its first 1024 bytes are a
+ *               header: a sticky device status word and the few-token path's
+ *               split-K arrival counters, which the kernels leave at zero.
+ *               Zero the header once before first use (e.g. allocate the
+ *               workspace zero-filled); fg8_check_device_status reads and
+ *               clears the status word, and after a failed call the whole
+ *               header.  Calls sharing a workspace must not overlap on the
+ *               device.
+ * M <= 32 runs one kernel that quantizes x, streams the weights as the
+ * tensor core's M side (128 weight rows per CTA, split over K) and reduces;
+ * larger M quantizes x (fg8_linear_prepare) and runs the tiled GEMM
+ * (fg8_linear_run).
  * Float scales are applied exactly per 128-K block in float32 (never rounded
  * to a power of two, [zh] §七 补充); UE8M0 scales go through the tensor
  * core's block-scaled MMA.  M == 0 is a no-op. */
@@ -119,7 +126,9 @@ FG8_API fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t 
  *   fg8_linear_prepare  quantizes x into the workspace in the GEMM's layouts
  *                       (and, for UE8M0, packs w_scale_inv's scale-factor tiles);
  *   fg8_linear_run      runs the GEMM from that workspace.
- * prepare followed by run on the same stream and workspace is fg8_linear.
+ * prepare followed by run on the same stream and workspace is fg8_linear for
+ * M > 32 (for M <= 32 fg8_linear runs its fused few-token kernel, whose
+ * split-K sums may round differently within the stated tolerance).
  * Arguments and checks are those of fg8_linear. */
 FG8_API fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                                       const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,
