@@ -162,6 +162,75 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ roofline ----
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "fine_grained_fp8_act_b200", "csrc")
+
+
+def source_hash():
+    """sha256 of the kernel sources: DRAM traffic recorded from ncu holds only
+    for the kernels it was taken from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload, launch):
+    """DRAM bytes (read + write) of the workload's `launch`-th GEMM launch of a
+    step, from profiles/traffic.json, or None when absent or stale."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != source_hash():
+        return None
+    v = rec.get("workloads", {}).get(workload, {}).get("gemm_dram_bytes", [])
+    return v[launch] if launch < len(v) else None
+
+
+def record_traffic(csv_path, workload):
+    """Stores, per GEMM launch of one step (in launch order), the
+    dram__bytes_read.sum + dram__bytes_write.sum of an ncu raw CSV export
+    (`ncu -i report --page raw --csv`) of that step's GEMM launches."""
+    import csv
+    with open(csv_path) as f:
+        rows = list(csv.reader(f))
+    head = rows[0]
+    body = [r for r in rows[1:] if len(r) == len(head) and r[0].strip() and r[0].strip()[0].isdigit()]
+    col = {h: i for i, h in enumerate(head)}
+
+    def val(r, name):
+        txt = r[col[name]].replace(",", "")
+        return float(txt)
+    unit_row = rows[1]
+
+    def scale(name):
+        u = unit_row[col[name]].strip().lower()
+        return {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9}.get(u, 1)
+    out = []
+    for r in body:
+        if "fg8_gemm_kernel" not in r[col["Kernel Name"]] and "fg8_small_m_kernel" not in r[col["Kernel Name"]]:
+            continue
+        out.append(val(r, "dram__bytes_read.sum") * scale("dram__bytes_read.sum") +
+                   val(r, "dram__bytes_write.sum") * scale("dram__bytes_write.sum"))
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        rec = {}
+    if rec.get("source_hash") != source_hash():
+        rec = {"source_hash": source_hash(), "workloads": {}}
+    rec["workloads"][workload] = {"gemm_dram_bytes": out, "from": os.path.basename(csv_path)}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(rec, f, indent=1)
+    print(json.dumps(rec["workloads"][workload]))
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -332,7 +401,7 @@ def run_fg8(args, rank, world, local):
     else:
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = recorded_traffic(args.workload, dom)  # ncu DRAM bytes per launch, None if stale
     roof["kernel"] = ("fg8_small_m_kernel" if small else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
@@ -515,7 +584,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true",
                     help="quantize every layer's input in its own launch instead of in the previous GEMM")
+    ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
+                    help="store the DRAM bytes of the GEMM launches in an ncu raw CSV export for --workload, then exit")
     args = ap.parse_args(argv)
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.workload)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_env()
