@@ -54,6 +54,11 @@ def lib():
             f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                           ctypes.c_void_p, ctypes.c_void_p]
         L.orc_linear_dequant.restype = ctypes.c_int
+        L.orc_dequantize_weight.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                            ctypes.c_int, ctypes.c_void_p, ctypes.c_int64]
+        L.orc_dequantize_weight.restype = ctypes.c_int
+        L.orc_scale_to_e8m0.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+        L.orc_scale_to_e8m0.restype = ctypes.c_int64
         L.orc_linear_dequant.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
@@ -167,3 +172,24 @@ def linear(x_bf16, wq, ws, bias_bf16, fmt, rows=None):
     xq, xs = quantize_act(x_bf16, fmt)
     return linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows)
 
+
+# ------------------------------------------------ checkpoint conversions --
+def dequantize_weight(wq, ws, fmt: int) -> np.ndarray:
+    """Fp8Dequantize: e4m3 [N, K] and its block scales -> bf16 bits [N, K]."""
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(ws, dtype=_scale_dtype(fmt))
+    N, K = wq.shape
+    if ws.shape != (_kb(N), _kb(K)):
+        raise ValueError("scale shape mismatch")
+    w = np.empty((N, K), dtype=np.uint16)
+    if lib().orc_dequantize_weight(_ptr(wq), N, K, _ptr(ws), fmt, _ptr(w), K) != 0:
+        raise ValueError("orc_dequantize_weight: bad argument")
+    return w
+
+
+def scale_to_e8m0(s) -> tuple:
+    """float32 power-of-two scales -> (UE8M0 bytes, number of inputs that were no UE8M0 value)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    out = np.empty(s.shape, dtype=np.uint8)
+    bad = lib().orc_scale_to_e8m0(_ptr(s), s.size, _ptr(out))
+    return out, int(bad)

@@ -305,4 +305,49 @@ int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq
   return 0;
 }
 
+// Fp8Dequantize ([zh] §五 and §八 step 4: a pre-quantized checkpoint loaded
+// with dequantize=True folds each 128x128 block's scale back into the
+// weight): w[n,k] = value(wq[n,k]) * scale_inv(n/128, k/128), the product
+// formed exactly in double and rounded once to bf16 (RNE).
+//   wq: e4m3fn [N, K] row-major; w_scale_inv as orc_quantize_weight writes;
+//   w: bf16 bits, row n at w + n*ld_w.
+int orc_dequantize_weight(const uint8_t* wq, int64_t N, int64_t K, const void* w_scale_inv, int fmt, uint16_t* w,
+                          int64_t ld_w) {
+  if (N <= 0 || K <= 0 || ld_w < K || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
+  const int Kb = ceil_div(K, kBlock);
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      const int64_t blk = (n / kBlock) * Kb + k / kBlock;
+      const double s = fmt == ORC_FMT_FLOAT ? static_cast<double>(static_cast<const float*>(w_scale_inv)[blk])
+                                            : static_cast<double>(e8m0_value(static_cast<const uint8_t*>(w_scale_inv)[blk]));
+      w[n * ld_w + k] = bf16_from_double(e4m3_signed(wq[n * K + k]) * s);
+    }
+  }
+  return 0;
+}
+
+// The checkpoint scale conversion ([zh] §七: some checkpoints keep
+// power-of-two UE8M0 scales in float32 containers under the key ".scale";
+// after loading they are converted exactly to the UE8M0 dtype).  A UE8M0
+// byte b is 2^(b-127), so s = 2^e with -127 <= e <= 127 becomes e + 127.
+// Any other input is no UE8M0 value: it becomes 255 (the UE8M0 NaN) and is
+// counted.  Returns the count.
+int64_t orc_scale_to_e8m0(const float* s, int64_t n, uint8_t* out) {
+  int64_t bad = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    const float v = s[i];
+    uint8_t b = 255;
+    if (std::isfinite(v) && v > 0.0f) {
+      int e2;
+      const double f = std::frexp(static_cast<double>(v), &e2);  // v = f * 2^e2, f in [0.5, 1)
+      const int e = e2 - 1;
+      if (f == 0.5 && e >= -127 && e <= 127) b = static_cast<uint8_t>(e + 127);
+    }
+    if (b == 255) ++bad;
+    out[i] = b;
+  }
+  return bad;
+}
+
 }  // extern "C"

@@ -433,3 +433,80 @@ def test_linear_row_subset_matches_full(orc):
     part = orc.linear_dequant(xq, xs, wq, ws, bb, FLOAT, rows=rows)
     for a, b in zip(full, part):
         assert np.array_equal(a[rows], b)
+
+
+# ------------------------------------------- checkpoint conversions ([zh] §五, §七) --
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+def test_dequantize_lossless_blocks(orc, fmt):
+    """Blocks whose largest magnitude is 448 * 2^j and whose values are e4m3
+    values times 2^j quantize losslessly (scale 2^j): Fp8Dequantize must give
+    the original weights back, bit for bit."""
+    N, K = 200, 272
+    g = torch.Generator().manual_seed(31)
+    finite = torch.from_numpy(torch_e4m3_table()[:0x7F].copy())
+    w = finite[torch.randint(0, 0x7F, (N, K), generator=g)] * torch.where(torch.rand(N, K, generator=g) < 0.5, -1.0, 1.0)
+    for nb in range(2):
+        for kb in range(3):
+            w[128 * nb, 128 * kb] = 448.0
+            w[128 * nb:128 * nb + 128, 128 * kb:128 * kb + 128] *= 2.0 ** (-9 + 2 * nb - kb)
+    wb = _bf16_bits(w.to(torch.bfloat16))
+    assert np.array_equal(w.to(torch.bfloat16).double().numpy(), w.numpy())
+    wq, ws = orc.quantize_weight(wb, fmt)
+    assert np.array_equal(orc.dequantize_weight(wq, ws, fmt), wb)
+
+
+def test_dequantize_vs_exact_rationals(orc):
+    """Non-power-of-two float scales: every dequantized element is the exact
+    rational value(q) * scale rounded once to bf16 (nearest, ties to even);
+    decode by PyTorch's e4m3 table, products in fractions.Fraction."""
+    N, K = 130, 144
+    g = torch.Generator().manual_seed(32)
+    w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    wq, ws = orc.quantize_weight(_bf16_bits(w), FLOAT)
+    out = orc.dequantize_weight(wq, ws, FLOAT)
+    table = torch_e4m3_table()
+    for n in range(0, N, 3):
+        for k in range(0, K, 5):
+            s = Fraction(float(ws[n // 128, k // 128]))
+            want = frac_bf16_rne(Fraction(float(table[wq[n, k]])) * s)
+            assert out[n, k] == want, (n, k)
+
+
+def test_dequantize_within_half_step(orc):
+    """|w - dequant(quant(w))| <= half an e4m3 step at the block's scale plus
+    the bf16 rounding of the result."""
+    N, K = 256, 384
+    g = torch.Generator().manual_seed(33)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    for fmt in (FLOAT, UE8M0):
+        wq, ws = orc.quantize_weight(_bf16_bits(w), fmt)
+        back = torch.from_numpy(orc.dequantize_weight(wq, ws, fmt).astype(np.int16)).view(torch.bfloat16).double()
+        s = torch.from_numpy(np.asarray(ws).astype(np.float64) if fmt == FLOAT else
+                             np.ldexp(1.0, np.asarray(ws).astype(np.int64) - 127))
+        s_full = s.repeat_interleave(128, 0)[:N].repeat_interleave(128, 1)[:, :K]
+        a = (w.double() / s_full).abs()
+        step = torch.where(a >= 2.0 ** -6, 2.0 ** (torch.floor(torch.log2(a.clamp(min=2.0 ** -6))) - 3), torch.full_like(a, 2.0 ** -9))
+        bound = 0.5 * step * s_full + back.abs() * 2.0 ** -8
+        assert bool(((w.double() - back).abs() <= bound).all())
+
+
+def test_scale_to_e8m0_powers_of_two(orc):
+    """s = 2^e, -127 <= e <= 127, converts to the UE8M0 byte e + 127, which
+    PyTorch's float8_e8m0fnu decodes back to s."""
+    e = np.arange(-127, 128)
+    s = np.ldexp(np.float32(1.0), e).astype(np.float32)
+    out, bad = orc.scale_to_e8m0(s)
+    assert bad == 0
+    assert np.array_equal(out.astype(np.int64), e + 127)
+    back = torch.from_numpy(out.copy()).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    assert np.array_equal(back, s.astype(np.float64))
+
+
+def test_scale_to_e8m0_rejects_non_ue8m0_values(orc):
+    """Values that are no UE8M0 scale (not a power of two, not positive,
+    not finite, below 2^-127) become the UE8M0 NaN byte and are counted."""
+    s = np.array([3.0, 1.5, 0.75 * 2.0 ** -100, 0.0, -0.0, -2.0, np.inf, -np.inf, np.nan, 2.0 ** -128, 2.0 ** -149,
+                  np.float32(2.0 ** 127) * np.float32(1.0000001)], dtype=np.float32)
+    out, bad = orc.scale_to_e8m0(s)
+    assert bad == s.size
+    assert (out == 255).all()
