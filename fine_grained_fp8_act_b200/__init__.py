@@ -24,6 +24,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     FG8_SCALE_UE8M0,
     FG8Error,
     fg8_check_device_status,
+    fg8_dequantize_weight,
     fg8_gemm_prequant,
     fg8_gemm_workspace_bytes,
     fg8_linear,
@@ -34,6 +35,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear_workspace_bytes,
     fg8_quantize_act,
     fg8_quantize_weight,
+    fg8_scale_to_ue8m0,
     fg8_set_wait_limit_ns,
     fg8_status_string,
     fg8_version,
@@ -42,10 +44,12 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
 )
 from .layer import (  # noqa: F401
     FP8Linear,
+    dequantize_weight,
     gemm_prequant,
     linear,
     linear_chain,
     quantize_act,
     quantize_weight,
     scale_fmt_code,
+    scale_to_ue8m0,
 )

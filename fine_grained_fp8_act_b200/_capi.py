@@ -40,6 +40,8 @@ SIGNATURES = {
     "fg8_linear_noalloc": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP]),
     "fg8_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
     "fg8_gemm_prequant": (_INT, [_VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
+    "fg8_dequantize_weight": (_INT, [_VP, _I64, _I64, _VP, _INT, _VP, _I64, _VP]),
+    "fg8_scale_to_ue8m0": (_INT, [_VP, _I64, _VP, _VP, _VP]),
     "fg8_check_device_status": (_INT, [_VP, _VP]),
     "fg8_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fg8_status_string": (ctypes.c_char_p, [_INT]),
@@ -139,6 +141,14 @@ def fg8_gemm_prequant(xq_e4m3, x_scale, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
                       workspace_bytes, stream):
     _check("fg8_gemm_prequant", lib().fg8_gemm_prequant(xq_e4m3, x_scale, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M,
                                                         N, K, ld_y, fmt, workspace, workspace_bytes, stream))
+
+
+def fg8_dequantize_weight(wq_e4m3, N, K, w_scale_inv, fmt, w_bf16, ld_w, stream):
+    _check("fg8_dequantize_weight", lib().fg8_dequantize_weight(wq_e4m3, N, K, w_scale_inv, fmt, w_bf16, ld_w, stream))
+
+
+def fg8_scale_to_ue8m0(scale_f32, n, scale_e8m0, invalid_count, stream):
+    _check("fg8_scale_to_ue8m0", lib().fg8_scale_to_ue8m0(scale_f32, n, scale_e8m0, invalid_count, stream))
 
 
 def fg8_check_device_status(workspace, stream) -> int:

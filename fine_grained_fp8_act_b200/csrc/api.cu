@@ -457,6 +457,32 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
   return cuda_status(launch_gemm(g, fmt, dev.sms, s));
 }
 
+fg8_status fg8_dequantize_weight(const void* wq_e4m3, int64_t N, int64_t K, const void* w_scale_inv,
+                                 fg8_scale_fmt fmt, void* w_bf16, int64_t ld_w, void* stream) {
+  if (!fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K) return FG8_ERR_INVALID_ARG;
+  if (N * K > (int64_t(1) << 40)) return FG8_ERR_INVALID_ARG;
+  if (wq_e4m3 == nullptr || w_scale_inv == nullptr || w_bf16 == nullptr) return FG8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld_w % 8 != 0 || !aligned16(wq_e4m3) || !aligned16(w_bf16)) return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  return cuda_status(launch_dequant_weight(static_cast<const uint8_t*>(wq_e4m3), static_cast<int>(N),
+                                           static_cast<int>(K), w_scale_inv, fmt, static_cast<uint16_t*>(w_bf16),
+                                           ld_w, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
+fg8_status fg8_scale_to_ue8m0(const void* scale_f32, int64_t n, void* scale_e8m0, uint32_t* invalid_count,
+                              void* stream) {
+  if (n < 0) return FG8_ERR_INVALID_ARG;
+  if (n == 0) return FG8_OK;
+  if (scale_f32 == nullptr || scale_e8m0 == nullptr) return FG8_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scale_f32) & 3u) != 0 || (reinterpret_cast<uintptr_t>(invalid_count) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  return cuda_status(launch_scale_to_e8m0(static_cast<const float*>(scale_f32), n, static_cast<uint8_t*>(scale_e8m0),
+                                          invalid_count, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
 fg8_status fg8_check_device_status(void* workspace, void* stream) {
   if (workspace == nullptr) return FG8_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -126,6 +126,11 @@ int small_m_splits(int N, int K);
 size_t small_m_partial_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s);
 
+// Checkpoint conversions (convert.cu).
+cudaError_t launch_dequant_weight(const uint8_t* wq, int N, int K, const void* ws, int fmt, uint16_t* w, int64_t ld_w,
+                                  int num_sms, cudaStream_t s);
+cudaError_t launch_scale_to_e8m0(const float* s, int64_t n, uint8_t* out, uint32_t* bad, int num_sms, cudaStream_t st);
+
 int choose_block_n(int M, int N, int num_sms);
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s);

@@ -51,7 +51,7 @@ namespace {
 
 constexpr uint32_t kTimeoutStatus = 6u;  // FG8_ERR_TIMEOUT
 constexpr uint64_t kDrainNs = 1000000000ull;
-constexpr int kQuantWarp0 = 2, kQuantWarps = 4;
+constexpr int kQuantWarp0 = 2;
 constexpr int kEpiWarp0 = 6;
 
 struct SmParams {

@@ -152,6 +152,31 @@ def linear_chain(x: torch.Tensor, layers, scale_fmt="float", workspaces=None):
     return ys
 
 
+def dequantize_weight(wq: torch.Tensor, w_scale_inv: torch.Tensor, scale_fmt="float") -> torch.Tensor:
+    """Fp8Dequantize: (e4m3 [N, K], block scales) -> bf16 [N, K] with each block's scale folded in."""
+    fmt = scale_fmt_code(scale_fmt)
+    N, K = wq.shape
+    if w_scale_inv.shape != (_cdiv(N, 128), _cdiv(K, 128)) or w_scale_inv.dtype != _SCALE_DTYPES[fmt]:
+        raise ValueError("w_scale_inv must be [ceil(N/128), ceil(K/128)] of the format's dtype")
+    w = torch.empty((N, K), dtype=torch.bfloat16, device=wq.device)
+    with torch.cuda.device(wq.device):
+        C.fg8_dequantize_weight(wq.data_ptr(), N, K, w_scale_inv.data_ptr(), fmt, w.data_ptr(), K, _stream(wq))
+    return w
+
+
+def scale_to_ue8m0(scale: torch.Tensor) -> Tuple[torch.Tensor, int]:
+    """float32 power-of-two scales (a checkpoint's ".scale" key) -> (float8_e8m0fnu scales of the same
+    shape, number of inputs that were no UE8M0 value; those become NaN).  Synchronizes for the count."""
+    s = scale.contiguous()
+    if s.dtype != torch.float32 or not s.is_cuda:
+        raise ValueError("scale must be a float32 CUDA tensor")
+    out = torch.empty(s.shape, dtype=torch.uint8, device=s.device)
+    bad = torch.zeros(1, dtype=torch.int32, device=s.device)
+    with torch.cuda.device(s.device):
+        C.fg8_scale_to_ue8m0(s.data_ptr(), s.numel(), out.data_ptr(), bad.data_ptr(), _stream(s))
+    return out.view(torch.float8_e8m0fnu), int(bad.item())
+
+
 class FP8Linear(torch.nn.Module):
     """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
     weight float8_e4m3fn [out, in], weight_scale_inv per 128x128 block, bias

@@ -187,6 +187,27 @@ FG8_API fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, c
                              int64_t M, int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Fp8Dequantize ([zh] §五 and §八 step 4: a pre-quantized checkpoint loaded
+ * with dequantize=True folds each block's scale back into the weight):
+ *   w[n, k] = bf16(value(wq[n, k]) * w_scale_inv[n / 128][k / 128]),
+ * the product exact, rounded once to nearest even.
+ *   wq_e4m3      [N, K] e4m3fn, row stride K (16-byte aligned)
+ *   w_scale_inv  [ceil(N/128), ceil(K/128)] float32 (FLOAT) or UE8M0 bytes
+ *   w_bf16       [N, K] bf16 output, row stride ld_w (16-byte aligned)
+ * K % 16 == 0 and ld_w % 8 == 0 (FG8_ERR_ALIGNMENT otherwise).  Caller owns
+ * all buffers; nothing is allocated. */
+FG8_API fg8_status fg8_dequantize_weight(const void* wq_e4m3, int64_t N, int64_t K, const void* w_scale_inv,
+                                         fg8_scale_fmt fmt, void* w_bf16, int64_t ld_w, void* stream);
+
+/* The checkpoint scale conversion of [zh] §七: power-of-two UE8M0 scales
+ * kept in float32 containers (key ".scale") become UE8M0 bytes exactly,
+ * s = 2^e with -127 <= e <= 127 -> byte e + 127.  Any other value is no
+ * UE8M0 scale: its byte is 255 (the UE8M0 NaN) and it is added to
+ * *invalid_count (a device uint32; may be NULL).
+ *   scale_f32 [n] float32 (4-byte aligned), scale_e8m0 [n] bytes. */
+FG8_API fg8_status fg8_scale_to_ue8m0(const void* scale_f32, int64_t n, void* scale_e8m0, uint32_t* invalid_count,
+                                      void* stream);
+
 /* Synchronizes `stream`, reads and clears the status word a previous
  * fg8_linear / fg8_gemm_prequant left in `workspace`: FG8_OK, or
  * FG8_ERR_TIMEOUT if one of its device-side waits gave up (the kernel then

@@ -116,6 +116,19 @@ def test_chain_rejects_bad_next_layer(fg8):
                                     FAKE * 32, 1 << 40, None) == 1  # next layer's weight scales missing
 
 
+def test_conversions_reject_bad_args(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_dequantize_weight(FAKE, 0, 256, FAKE, 0, FAKE, 256, None) == 1
+    assert raw.fg8_dequantize_weight(FAKE, 256, 256, FAKE, 3, FAKE, 256, None) == 1
+    assert raw.fg8_dequantize_weight(FAKE, 256, 256, FAKE, 0, FAKE, 255, None) == 1   # ld_w < K
+    assert raw.fg8_dequantize_weight(FAKE, 256, 200, FAKE, 0, FAKE, 200, None) == 2   # K % 16
+    assert raw.fg8_dequantize_weight(FAKE, 256, 256, FAKE, 0, FAKE, 260, None) == 2   # ld_w % 8
+    assert raw.fg8_dequantize_weight(None, 256, 256, FAKE, 0, FAKE, 256, None) == 1
+    assert raw.fg8_scale_to_ue8m0(FAKE, -1, FAKE, None, None) == 1
+    assert raw.fg8_scale_to_ue8m0(None, 0, None, None, None) == 0          # empty: no-op
+    assert raw.fg8_scale_to_ue8m0(FAKE + 2, 8, FAKE, None, None) == 2
+
+
 def test_empty_m_is_a_noop(fg8):
     raw = _raw(fg8)
     assert raw.fg8_linear(None, 0, 256, 256, 256, None, None, None, None, 256, 0, None, 0, None) == 0
