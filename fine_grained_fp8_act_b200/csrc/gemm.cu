@@ -523,27 +523,36 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(ab.slot * C::BN + col0);
-        // 32 columns per TMEM load; group c+1 is loading while group c is
-        // promoted
+        // two 32-column TMEM loads per wait: chunks c, c+1 are promoted while
+        // c+2, c+3 load into the same registers; the buffer goes back after
+        // the last wait
+        static_assert(C::kChunks % 2 == 0, "chunk pairs");
         uint32_t r[2][32];
         tmem_ld32(taddr, r[0]);
+        tmem_ld32(taddr + 32, r[1]);
         tmem_wait_ld();
         tmem_reg_fence(r[0]);
+        tmem_reg_fence(r[1]);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-          if (c + 1 < C::kChunks) {
-            tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
-          } else {  // every column of this K-block is in registers: hand the buffer back
+        for (int c = 0; c < C::kChunks; c += 2) {
+          const bool more = c + 2 < C::kChunks;
+          if (!more) {  // every column of this K-block is in registers: hand the buffer back
             tc_fence_before();
             __syncwarp();
             if (lane == 0) release_tmem<C>(tempty + ab.slot);
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[c * 32 + j] = __float_as_uint(__fmaf_rn(__uint_as_float(r[c & 1][j]), s, __uint_as_float(acc[c * 32 + j])));
-          if (c + 1 < C::kChunks) {
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              acc[(c + h) * 32 + j] =
+                  __float_as_uint(__fmaf_rn(__uint_as_float(r[h][j]), s, __uint_as_float(acc[(c + h) * 32 + j])));
+            if (more) tmem_ld32(taddr + (c + 2 + h) * 32, r[h]);
+          }
+          if (more) {
             tmem_wait_ld();
-            tmem_reg_fence(r[(c + 1) & 1]);
+            tmem_reg_fence(r[0]);
+            tmem_reg_fence(r[1]);
           }
         }
         ab.template advance<C::kNumAcc>();
