@@ -57,6 +57,9 @@ def lib():
         L.orc_dequantize_weight.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_int, ctypes.c_void_p, ctypes.c_int64]
         L.orc_dequantize_weight.restype = ctypes.c_int
+        L.orc_quantize_act_static.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_float, ctypes.c_void_p]
+        L.orc_quantize_act_static.restype = ctypes.c_int
         L.orc_scale_to_e8m0.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         L.orc_scale_to_e8m0.restype = ctypes.c_int64
         L.orc_linear_dequant.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -122,6 +125,17 @@ def quantize_act(x_bf16: np.ndarray, fmt: int):
     if rc != 0:
         raise ValueError("orc_quantize_act: bad argument")
     return xq, xs
+
+
+def quantize_act_static(x_bf16: np.ndarray, scale: float):
+    """Static scheme: x bf16 bits [M, K] and one float32 scale -> (xq e4m3 [M, K],
+    x_scale [M, ceil(K/128)] float32 all equal to the scale, the GEMM's view)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    xq = np.empty((M, K), dtype=np.uint8)
+    if lib().orc_quantize_act_static(_ptr(x), M, K, K, float(np.float32(scale)), _ptr(xq)) != 0:
+        raise ValueError("orc_quantize_act_static: bad argument")
+    return xq, np.full((M, _kb(K)), np.float32(scale), dtype=np.float32)
 
 
 def quantize_weight(w_bf16: np.ndarray, fmt: int):

@@ -350,4 +350,17 @@ int64_t orc_scale_to_e8m0(const float* s, int64_t n, uint8_t* out) {
   return bad;
 }
 
+// Static activation scheme ([zh] §四: activation_scheme is "dynamic" or
+// "static"; §6.3: static activation quantization).  The pages print no
+// formula; the reading here: one precomputed float32 scale s > 0 for the
+// whole tensor, q = e4m3_rn_satfinite(RN_f32(x / s)) -- the dynamic rule with
+// the group scale replaced by s (values beyond 448 s saturate).
+int orc_quantize_act_static(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, float s, uint8_t* xq) {
+  if (M < 0 || K <= 0 || ld_x < K || !(s > 0.0f) || !std::isfinite(s)) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) / s);
+  return 0;
+}
+
 }  // extern "C"

@@ -510,3 +510,46 @@ def test_scale_to_e8m0_rejects_non_ue8m0_values(orc):
     out, bad = orc.scale_to_e8m0(s)
     assert bad == s.size
     assert (out == 255).all()
+
+
+# ------------------------------------------------ static activation scheme --
+def test_quantize_act_static_vs_brute_force(orc):
+    """One float32 scale for the whole tensor: every code is the brute-force
+    nearest e4m3 code of the numpy float32 quotient x / s (IEEE division),
+    values beyond 448 s saturating."""
+    M, K = 5, 272
+    g = torch.Generator().manual_seed(41)
+    x = (torch.randn(M, K, generator=g) * 3.0).to(torch.bfloat16)
+    x[0, 0], x[1, 5], x[2, 7] = 3000.0, -5000.0, 0.0
+    x[3, 9] = -0.0
+    xb = _bf16_bits(x)
+    for s in (np.float32(0.0123), np.float32(1.0), np.float32(2.0 ** -7), np.float32(3.7)):
+        xq, xs = orc.quantize_act_static(xb, float(s))
+        quot = x.float().numpy() / s
+        assert np.array_equal(xq.ravel(), brute_encode(quot.ravel()))
+        assert xs.shape == (M, 3) and (xs == s).all()
+
+
+def test_quantize_act_static_lossless_and_linear(orc):
+    """x = e4m3 value * 2^j with s = 2^j quantizes losslessly, and the linear
+    layer on it equals the exact product (exact rationals)."""
+    M, N, K = 3, 5, 144
+    g = torch.Generator().manual_seed(42)
+    finite = torch.from_numpy(torch_e4m3_table()[:0x7F].copy())
+    codes = torch.randint(0, 0x7F, (M, K), generator=g)
+    sign = torch.where(torch.rand(M, K, generator=g) < 0.5, -1.0, 1.0)
+    x = finite[codes] * sign * 2.0 ** -3
+    xb = _bf16_bits(x.to(torch.bfloat16))
+    xq, xs = orc.quantize_act_static(xb, 2.0 ** -3)
+    want = (codes.numpy().astype(np.uint8) | np.where(sign.numpy() < 0, 0x80, 0).astype(np.uint8))
+    want[(codes.numpy() == 0) & (sign.numpy() < 0)] = 0x80
+    assert np.array_equal(xq, want)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    wq, ws = orc.quantize_weight(_bf16_bits(w), FLOAT)
+    y64, _, _ = orc.linear_dequant(xq, xs, wq, ws, None, FLOAT)
+    table = torch_e4m3_table()
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(x[m, k])) * Fraction(float(table[wq[n, k]])) * Fraction(float(ws[n // 128, k // 128]))
+                        for k in range(K))
+            assert abs(Fraction(y64[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
