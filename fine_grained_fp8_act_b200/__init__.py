@@ -32,8 +32,10 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear_prepare,
     fg8_linear_run,
     fg8_linear_run_chain,
+    fg8_linear_static,
     fg8_linear_workspace_bytes,
     fg8_quantize_act,
+    fg8_quantize_act_static,
     fg8_quantize_weight,
     fg8_scale_to_ue8m0,
     fg8_set_wait_limit_ns,
@@ -48,7 +50,9 @@ from .layer import (  # noqa: F401
     gemm_prequant,
     linear,
     linear_chain,
+    linear_static,
     quantize_act,
+    quantize_act_static,
     quantize_weight,
     scale_fmt_code,
     scale_to_ue8m0,

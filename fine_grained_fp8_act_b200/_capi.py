@@ -40,6 +40,8 @@ SIGNATURES = {
     "fg8_linear_noalloc": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP]),
     "fg8_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
     "fg8_gemm_prequant": (_INT, [_VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
+    "fg8_quantize_act_static": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),
+    "fg8_linear_static": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _I64, _VP, _SZ, _VP]),
     "fg8_dequantize_weight": (_INT, [_VP, _I64, _I64, _VP, _INT, _VP, _I64, _VP]),
     "fg8_scale_to_ue8m0": (_INT, [_VP, _I64, _VP, _VP, _VP]),
     "fg8_check_device_status": (_INT, [_VP, _VP]),
@@ -141,6 +143,17 @@ def fg8_gemm_prequant(xq_e4m3, x_scale, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
                       workspace_bytes, stream):
     _check("fg8_gemm_prequant", lib().fg8_gemm_prequant(xq_e4m3, x_scale, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M,
                                                         N, K, ld_y, fmt, workspace, workspace_bytes, stream))
+
+
+def fg8_quantize_act_static(x_bf16, M, K, ld_x, act_scale, xq_e4m3, x_scale, stream):
+    _check("fg8_quantize_act_static", lib().fg8_quantize_act_static(x_bf16, M, K, ld_x, act_scale, xq_e4m3, x_scale,
+                                                                    stream))
+
+
+def fg8_linear_static(x_bf16, M, N, K, ld_x, act_scale, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, workspace,
+                      workspace_bytes, stream):
+    _check("fg8_linear_static", lib().fg8_linear_static(x_bf16, M, N, K, ld_x, act_scale, wq_e4m3, w_scale_inv,
+                                                        bias_bf16, y_bf16, ld_y, workspace, workspace_bytes, stream))
 
 
 def fg8_dequantize_weight(wq_e4m3, N, K, w_scale_inv, fmt, w_bf16, ld_w, stream):

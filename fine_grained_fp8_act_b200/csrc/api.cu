@@ -457,6 +457,64 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
   return cuda_status(launch_gemm(g, fmt, dev.sms, s));
 }
 
+fg8_status fg8_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, const float* act_scale,
+                                   void* xq_e4m3, void* x_scale, void* stream) {
+  if (M < 0 || K <= 0 || M > kMaxDim || K > kMaxDim || ld_x < K) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || act_scale == nullptr || xq_e4m3 == nullptr || x_scale == nullptr) return FG8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld_x % 8 != 0 || !aligned16(x_bf16) || !aligned16(xq_e4m3) ||
+      (reinterpret_cast<uintptr_t>(act_scale) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  ActQuantArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.Kb = ceil_div(K, kGroup);
+  a.xq = static_cast<uint8_t*>(xq_e4m3);
+  a.xs = x_scale;
+  a.layout = kScaleRowMajor;
+  a.static_scale = act_scale;
+  return cuda_status(launch_act_quant(a, FG8_SCALE_FLOAT, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
+fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const float* act_scale,
+                             const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16, void* y_bf16,
+                             int64_t ld_y, void* workspace, size_t workspace_bytes, void* stream) {
+  const fg8_scale_fmt fmt = FG8_SCALE_FLOAT;
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || act_scale == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
+      (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv) ||
+      (reinterpret_cast<uintptr_t>(act_scale) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ActQuantArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.Kb = ceil_div(K, kGroup);
+  a.xq = ws + L.xq_off;
+  a.xs = ws + L.xs_off;
+  a.layout = kScaleKMajor;
+  a.ld_s = L.ld_s;
+  a.static_scale = act_scale;
+  if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, static_cast<cudaStream_t>(stream))); st != FG8_OK)
+    return st;
+  return fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes,
+                        stream);
+}
+
 fg8_status fg8_dequantize_weight(const void* wq_e4m3, int64_t N, int64_t K, const void* w_scale_inv,
                                  fg8_scale_fmt fmt, void* w_bf16, int64_t ld_w, void* stream) {
   if (!fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K) return FG8_ERR_INVALID_ARG;

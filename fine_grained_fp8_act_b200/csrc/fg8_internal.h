@@ -39,6 +39,9 @@ struct ActQuantArgs {
   int64_t ld_s;       // kScaleKMajor: column stride (>= M)
   int Kq;             // kScaleSfTiles: ceil(Kb / 4)
   int M_pad;          // kScaleSfTiles: rows rounded up to 128 (padding rows get scale 2^0)
+  // static activation scheme (float scales only): one precomputed scale for
+  // the whole tensor, read from device memory; nullptr = dynamic groups
+  const float* static_scale;
 };
 
 cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s);

@@ -65,6 +65,11 @@ __device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32
 }
 
 // ------------------------------------------------------------ act quant ----
+// Static activation scheme (float scales): the same arithmetic with the
+// group scale replaced by one scale for the tensor (values beyond 448 times it
+// saturate); the scale is still written per group, so the GEMM reads it
+// exactly as it reads dynamic scales.
+//
 // Eight lanes own one 128-channel group: lane l loads channels [16l, 16l+16)
 // with two 16-byte loads.  A warp covers 4 groups per pass and makes 2 passes
 // per iteration (all loads issued before any arithmetic), striding over the
@@ -120,7 +125,8 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, co
       for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-      const float s = group_scale(amax);
+      // dynamic: the group's scale; static (float only): the tensor's one scale
+      const float s = (FMT == 0 && a.static_scale != nullptr) ? *a.static_scale : group_scale(amax);
       const uint32_t sbyte = FMT == 1 ? e8m0_ceil_byte(s) : 0u;
       const uint4 packed = quantize16<FMT>(f, s, sbyte);
       const int k = kb[u] * kGroup + l * 16;

@@ -68,6 +68,21 @@ def quantize_act(x: torch.Tensor, scale_fmt="float") -> Tuple[torch.Tensor, torc
     return xq, xs
 
 
+def quantize_act_static(x: torch.Tensor, act_scale: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Static scheme: x bf16 [M, K] with one float32 scale (a 1-element CUDA tensor) ->
+    (xq float8_e4m3fn [M, K], x_scale [M, ceil(K/128)] float32, all equal to the scale)."""
+    _check_bf16_matrix(x, "x")
+    if act_scale.dtype != torch.float32 or act_scale.numel() != 1 or act_scale.device != x.device:
+        raise ValueError("act_scale must be one float32 on x's device")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    xs = torch.empty((M, _cdiv(K, 128)), dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        C.fg8_quantize_act_static(x.data_ptr(), M, K, x.stride(0), act_scale.data_ptr(), xq.data_ptr(), xs.data_ptr(),
+                                  _stream(x))
+    return xq, xs
+
+
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
     if workspace is not None:
         if workspace.numel() * workspace.element_size() < nbytes:
@@ -94,6 +109,24 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: O
         C.fg8_linear(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(),
                      0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0), fmt, ws.data_ptr(),
                      ws.numel() * ws.element_size(), _stream(x))
+    return y
+
+
+def linear_static(x: torch.Tensor, act_scale: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor,
+                  bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [M, N] bf16 with x quantized by one precomputed scale (float weight scales)."""
+    _check_bf16_matrix(x, "x")
+    if act_scale.dtype != torch.float32 or act_scale.numel() != 1 or act_scale.device != x.device:
+        raise ValueError("act_scale must be one float32 on x's device")
+    M, K = x.shape
+    N = wq.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(C.fg8_linear_workspace_bytes(M, N, K, C.FG8_SCALE_FLOAT), x.device, workspace)
+    with torch.cuda.device(x.device):
+        C.fg8_linear_static(x.data_ptr(), M, N, K, x.stride(0), act_scale.data_ptr(), wq.data_ptr(),
+                            w_scale_inv.data_ptr(), 0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0),
+                            ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
     return y
 
 

@@ -187,6 +187,24 @@ FG8_API fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, c
                              int64_t M, int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Static activation scheme ([zh] §四 activation_scheme "static", §6.3; float
+ * scales only): x is quantized with one precomputed scale for the whole
+ * tensor, q = e4m3_rn_satfinite(RN_f32(x / *act_scale)) (values beyond 448
+ * times the scale saturate), instead of per-group dynamic scales.
+ *   act_scale   one float32 in device memory, > 0 and finite (4-byte aligned)
+ *   fg8_quantize_act_static: xq_e4m3 [M, K] and x_scale [M, ceil(K/128)]
+ *               float32, every entry set to the scale (the layout
+ *               fg8_gemm_prequant reads)
+ *   fg8_linear_static: as fg8_linear with scale_fmt FLOAT (the same
+ *               workspace, fg8_linear_workspace_bytes(M, N, K, FLOAT)).
+ * Checks and errors as fg8_quantize_act / fg8_linear. */
+FG8_API fg8_status fg8_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                                           const float* act_scale, void* xq_e4m3, void* x_scale, void* stream);
+FG8_API fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                     const float* act_scale, const void* wq_e4m3, const void* w_scale_inv,
+                                     const void* bias_bf16, void* y_bf16, int64_t ld_y, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /* Fp8Dequantize ([zh] §五 and §八 step 4: a pre-quantized checkpoint loaded
  * with dequantize=True folds each block's scale back into the weight):
  *   w[n, k] = bf16(value(wq[n, k]) * w_scale_inv[n / 128][k / 128]),

@@ -129,6 +129,18 @@ def test_conversions_reject_bad_args(fg8):
     assert raw.fg8_scale_to_ue8m0(FAKE + 2, 8, FAKE, None, None) == 2
 
 
+def test_static_scheme_rejects_bad_args(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_quantize_act_static(FAKE, 4, 256, 256, None, FAKE, FAKE, None) == 1      # no scale
+    assert raw.fg8_quantize_act_static(FAKE, 4, 200, 200, FAKE, FAKE, FAKE, None) == 2      # K % 16
+    assert raw.fg8_quantize_act_static(FAKE, 4, 256, 256, FAKE + 2, FAKE, FAKE, None) == 2  # scale alignment
+    assert raw.fg8_quantize_act_static(None, 0, 256, 256, None, None, None, None) == 0      # empty
+    assert raw.fg8_linear_static(FAKE, 16, 256, 256, 256, None, FAKE, FAKE, None, FAKE, 256, FAKE * 16, 1 << 40,
+                                 None) == 1
+    assert raw.fg8_linear_static(FAKE, 16, 256, 256, 256, FAKE, FAKE, FAKE, None, FAKE, 256, None, 1 << 40,
+                                 None) == 4
+
+
 def test_empty_m_is_a_noop(fg8):
     raw = _raw(fg8)
     assert raw.fg8_linear(None, 0, 256, 256, 256, None, None, None, None, 256, 0, None, 0, None) == 0
