@@ -38,6 +38,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_quantize_act_static,
     fg8_quantize_weight,
     fg8_scale_to_ue8m0,
+    fg8_set_test_stall,
     fg8_set_wait_limit_ns,
     fg8_status_string,
     fg8_version,

@@ -46,6 +46,7 @@ SIGNATURES = {
     "fg8_scale_to_ue8m0": (_INT, [_VP, _I64, _VP, _VP, _VP]),
     "fg8_check_device_status": (_INT, [_VP, _VP]),
     "fg8_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "fg8_set_test_stall": (None, [_INT]),
     "fg8_status_string": (ctypes.c_char_p, [_INT]),
     "fg8_version": (_INT, []),
 }
@@ -91,6 +92,10 @@ def fg8_version() -> int:
 
 def fg8_set_wait_limit_ns(ns: int) -> None:
     lib().fg8_set_wait_limit_ns(int(ns))
+
+
+def fg8_set_test_stall(on: bool) -> None:
+    lib().fg8_set_test_stall(1 if on else 0)
 
 
 def fg8_quantize_weight(w_bf16, N, K, ld_w, wq_e4m3, w_scale_inv, fmt, stream):

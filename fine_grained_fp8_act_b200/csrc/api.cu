@@ -23,6 +23,7 @@ constexpr size_t kHeaderBytes = kWorkspaceHeaderBytes;  // status word, split-K 
 constexpr size_t kAlign = 256;
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_test_stall{0};
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -187,6 +188,8 @@ const char* fg8_status_string(fg8_status st) {
 
 void fg8_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
+void fg8_set_test_stall(int on) { g_test_stall.store(on != 0 ? 1 : 0); }
+
 fg8_status fg8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w, void* wq_e4m3,
                                void* w_scale_inv, fg8_scale_fmt fmt, void* stream) {
   if (!fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K) return FG8_ERR_INVALID_ARG;
@@ -293,6 +296,7 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   g.bias = bias_bf16;
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
+  g.test_stall = g_test_stall.load();
   if (fmt == FG8_SCALE_FLOAT) {
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
@@ -340,6 +344,7 @@ fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, co
   g.bias = bias_bf16;
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
+  g.test_stall = g_test_stall.load();
   if (fmt == FG8_SCALE_FLOAT) {
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
@@ -393,6 +398,7 @@ fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64
     a.part = reinterpret_cast<float*>(ws + kHeaderBytes + extra);
     a.status = reinterpret_cast<uint32_t*>(ws);
     a.wait_limit_ns = g_wait_limit_ns.load();
+    a.test_stall = g_test_stall.load();
     return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
   }
   if (fg8_status st = fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes, stream);
@@ -434,6 +440,7 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
   g.bias = bias_bf16;
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
+  g.test_stall = g_test_stall.load();
   if (fmt == FG8_SCALE_FLOAT) {
     if (fg8_status st = cuda_status(launch_xs_transpose(static_cast<const float*>(x_scale), static_cast<int>(M), Kb,
                                                         L.ld_s, reinterpret_cast<float*>(ws + L.xs_off), s));

@@ -76,6 +76,7 @@ struct GemmArgs {
   const void* bias;   // bf16 [N] or nullptr
   uint32_t* status;   // device status word (0 = ok)
   uint64_t wait_limit_ns;
+  int test_stall;     // test hook: the MMA thread first waits on a barrier nothing completes
   // Optional: also quantize this layer's bf16 output as the activation of a
   // next layer (K_next = N, N_next outputs) straight into that layer's
   // workspace, exactly as its prepare step would.
@@ -122,6 +123,7 @@ struct SmallMArgs {
   float* part;            // [splits][M][N] fp32 when splits > 1
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int test_stall;         // test hook, as GemmArgs::test_stall
 };
 
 int small_m_splits(int N, int K);

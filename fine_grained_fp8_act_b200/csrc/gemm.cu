@@ -61,6 +61,7 @@ struct KParams {
   const uint16_t* bias;
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int test_stall;
   // output re-quantization for a next layer (REQUANT configs)
   uint8_t* nx_xq;
   void* nx_xs;
@@ -354,10 +355,15 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
 template <class C>
 __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint32_t tmem_base, uint64_t* full,
                                            uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* teardown,
-                                           volatile int* abort_flag) {
+                                           uint64_t* stall, volatile int* abort_flag) {
   const uint64_t limit = p.wait_limit_ns;
   Ring st, ab;
   bool ok = true;
+  // test hook: a barrier nothing arrives on, so the bounded wait runs out
+  if (p.test_stall && !mbar_wait(stall, 0, limit, abort_flag)) {
+    raise_abort(abort_flag, p.status);
+    ok = false;
+  }
   const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
@@ -652,7 +658,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bfull = tempty + C::kNumAcc;
   uint64_t* bempty = bfull + 2;
   uint64_t* teardown = bempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* stall = teardown + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -670,6 +677,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bempty + s, C::kEpiWarps);
     }
     mbar_init(teardown, 1);
+    mbar_init(stall, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -702,7 +710,7 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 0 && lane == 0)
       producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag);
     else if (warp == 1 && lane == 0 && cta_rank<C>() == 0)
-      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, abort_flag);
+      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, abort_flag);
     if constexpr (C::REQUANT) {
       if (warp == 2 || warp == 3)
         prepare_next_layer<C>(p, static_cast<int>(blockIdx.x) * 64 + (warp - 2) * 32 + lane,
@@ -790,6 +798,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.bias = static_cast<const uint16_t*>(g.bias);
   p.status = g.status;
   p.wait_limit_ns = g.wait_limit_ns;
+  p.test_stall = g.test_stall;
   p.nx_xq = g.nx_xq;
   p.nx_xs = g.nx_xs;
   p.nx_ld_s = g.nx_ld_s;

@@ -38,27 +38,29 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 // True once the phase with the given parity has completed.  A thread whose
 // phase is still open sleeps in the instruction until the phase completes or
-// about a millisecond has passed, instead of spinning.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// about `hint_ns` have passed, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns = 0) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 
 // Bounded wait: gives up (returns false) once `limit_ns` of global time has
-// passed or another role raised `*abort`.  Never spins forever.
+// passed or another role raised `*abort`.  Never spins forever.  Each poll
+// sleeps at most min(limit, 1 ms) in try_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                           const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = limit_ns < 1000000ull ? static_cast<uint32_t>(limit_ns) : 1000000u;
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     if ((i & 15u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (global_timer_ns() - t0 > limit_ns) return false;

@@ -67,6 +67,7 @@ struct SmParams {
   uint32_t* counters;   // [Nb], zero at launch; the last CTA of a tile resets its own
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int test_stall;
 };
 
 template <int FMT_, int MP_>
@@ -261,8 +262,14 @@ __device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, u
 template <class C>
 __device__ __forceinline__ void sm_mma(const SmParams& p, uint8_t* smem, uint32_t tmem, uint64_t* wfull,
                                        uint64_t* xfull, uint64_t* sempty, uint64_t* tfull, uint64_t* tempty,
-                                       uint64_t* teardown, int kb0, int kb1, volatile int* abort_flag) {
+                                       uint64_t* teardown, uint64_t* stall, int kb0, int kb1,
+                                       volatile int* abort_flag) {
   SmRing st, ab;
+  // test hook: a barrier nothing arrives on, so the bounded wait runs out
+  if (p.test_stall && !mbar_wait(stall, 0, p.wait_limit_ns, abort_flag)) {
+    sm_raise(abort_flag, p.status);
+    kb1 = kb0;
+  }
   for (int kb = kb0; kb < kb1; ++kb) {
     if (!mbar_wait(wfull + st.slot, st.phase, p.wait_limit_ns, abort_flag) ||
         !mbar_wait(xfull + st.slot, st.phase, p.wait_limit_ns, abort_flag)) {
@@ -421,7 +428,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint64_t* scfull = tempty + C::kNumAcc;
   uint64_t* scempty = scfull + C::kScSlots;
   uint64_t* teardown = scempty + C::kScSlots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* stall = teardown + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -444,6 +452,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       mbar_init(scempty + s, C::kEpiThreads / 32);
     }
     mbar_init(teardown, 1);
+    mbar_init(stall, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbarrier_init();
@@ -464,7 +473,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   if (warp == 0) {
     if (lane == 0) sm_producer<C>(&tmW, &tmX, p, smem, wfull, sempty, nt, kb0, kb1, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0) sm_mma<C>(p, smem, tmem, wfull, xfull, sempty, tfull, tempty, teardown, kb0, kb1, abort_flag);
+    if (lane == 0)
+      sm_mma<C>(p, smem, tmem, wfull, xfull, sempty, tfull, tempty, teardown, stall, kb0, kb1, abort_flag);
   } else if (warp < kEpiWarp0) {
     sm_quantizer<C>(p, smem, wfull, xfull, scfull, scempty, nt, kb0, kb1, abort_flag);
   } else {
@@ -534,6 +544,7 @@ cudaError_t launch_small_m_cfg(const SmallMArgs& a, cudaStream_t s) {
   p.counters = a.counters;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.test_stall = a.test_stall;
   const int nt = (a.N + 127) / 128;
   auto kern = fg8_small_m_kernel<C>;
   static int configured_device = -1;

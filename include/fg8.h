@@ -236,6 +236,14 @@ FG8_API fg8_status fg8_check_device_status(void* workspace, void* stream);
  * before it gives up with FG8_ERR_TIMEOUT (default 2e9).  Process-wide. */
 FG8_API void fg8_set_wait_limit_ns(uint64_t ns);
 
+/* Test hook for the timeout path (process-wide, off by default): when on,
+ * the MMA thread of every GEMM launched afterwards first waits on an
+ * mbarrier that nothing completes, so its bounded wait runs out after the
+ * wait limit; the kernel then records FG8_ERR_TIMEOUT in the status word,
+ * drains its own copies and tensor-core ops, frees TMEM and returns.  No
+ * fault and no unbounded wait are involved.  Not for production use. */
+FG8_API void fg8_set_test_stall(int on);
+
 /* Static description of a status code. */
 FG8_API const char* fg8_status_string(fg8_status status);
 
