@@ -39,7 +39,18 @@ import workloads as W  # noqa: E402
 
 METRIC = "block-scaled FP8 linear TFLOP/s and % of B200 dense FP8 peak; act-quant GB/s"
 L2_FLUSH_BYTES = 256 << 20
-SMALL_M_MAX = 32  # fg8_linear's fused few-token path
+SMALL_M_MAX, SMALL_M_ALWAYS, FUSED_M_MAX = 128, 32, 16  # fg8_linear's few-token dispatch
+
+
+def layer_path(g):
+    """Which kernels fg8_linear runs for this shape (the library's rule):
+    "fused" one few-token kernel that also quantizes x (UE8M0, M <= 16);
+    "small" the prepare step, then the few-token swap-AB kernel;
+    "tiled" the prepare step, then the tiled GEMM."""
+    small = g.M <= SMALL_M_ALWAYS or (g.M <= SMALL_M_MAX and (g.N + 255) // 256 * 4 <= 148)
+    if small and g.fmt == 1 and g.M <= FUSED_M_MAX:
+        return "fused"
+    return "small" if small else "tiled"
 FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 
 
@@ -287,17 +298,19 @@ def run_fg8(args, rank, world, local):
         L["x"] = x0 if i == 0 else plan[i - 1]["y"]
         assert L["x"].shape == (L["g"].M, L["g"].K), "consecutive layers must chain"
 
-    # Few tokens (M <= 128): fg8_linear runs one fused kernel per layer
-    # (quantize, swap-AB split-K GEMM, reduce).  Otherwise consecutive layers
-    # chain: the GEMM of layer i also quantizes its output for layer i+1
-    # (fg8_linear_run_chain), so layer i+1 has no act-quant launch.
-    small = plan[0]["g"].M <= SMALL_M_MAX
-    chain = not args.no_chain and not small
+    # Each layer runs what fg8_linear runs for its shape: few tokens take the
+    # swap-AB split-K kernel (after the prepare step, or with the
+    # quantization fused in), more take the tiled GEMM.  When every layer is
+    # tiled, consecutive layers chain: the GEMM of layer i also quantizes its
+    # output for layer i+1 (fg8_linear_run_chain), so layer i+1 has no
+    # act-quant launch.
+    paths = [layer_path(L["g"]) for L in plan]
+    chain = not args.no_chain and all(pth == "tiled" for pth in paths)
 
     def launch_layer(i, ev_mid=None):
         L = plan[i]
         g = L["g"]
-        if small:
+        if paths[i] == "fused":
             if ev_mid is not None:
                 ev_mid.record(stream)
             fg8.fg8_linear(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
@@ -402,7 +415,7 @@ def run_fg8(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(args.workload, dom)  # ncu DRAM bytes per launch, None if stale
-    roof["kernel"] = ("fg8_small_m_kernel" if small else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+    roof["kernel"] = ("fg8_small_m_kernel" if paths[dom] != "tiled" else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
     roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
@@ -412,10 +425,10 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        fused = small or (chain and i > 0)  # act-quant inside a GEMM kernel
-        per_kernel.append({"layer": gi.name, "act_quant_us": None if fused else qm[i] * 1e3,
+        fused = paths[i] == "fused" or (chain and i > 0)  # act-quant inside a GEMM kernel
+        per_kernel.append({"layer": gi.name, "path": paths[i], "act_quant_us": None if fused else qm[i] * 1e3,
                            "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
-                           "act_quant": ("fused into the few-token kernel" if small else
+                           "act_quant": ("fused into the few-token kernel" if paths[i] == "fused" else
                                          "fused into the previous GEMM" if fused else "own launch"),
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
                            "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
@@ -426,9 +439,9 @@ def run_fg8(args, rank, world, local):
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
 
     # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM;
-    # few tokens: one kernel per layer
-    prep = [1 + (1 if L["g"].fmt == 1 else 0) for L in plan]
-    launches_per_step = nl if small else (prep[0] if chain else sum(prep)) + nl
+    # fused few-token layers: one kernel
+    prep = [0 if pth == "fused" else 1 + (1 if L["g"].fmt == 1 else 0) for pth, L in zip(paths, plan)]
+    launches_per_step = (prep[0] if chain else sum(prep)) + nl
     out = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,

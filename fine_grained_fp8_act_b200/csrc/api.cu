@@ -145,14 +145,11 @@ size_t small_counter_bytes(int64_t N) {
   return nt > kHeaderCounters ? align_up(static_cast<size_t>(nt) * 4, kAlign) : 0;
 }
 
-// fg8_linear's workspace: the prepare/run layout, and for few tokens also
-// the small-M path's [header | (counters) | partials] (the same bytes reused).
+// fg8_linear's workspace: the prepare/run layout, then for few tokens the
+// small-M path's (counters beyond the header) and split-K partials.
 size_t linear_workspace_need(int64_t M, int64_t N, int64_t K, int fmt) {
   size_t need = linear_ws_layout(M, N, K, fmt).total;
-  if (M <= kSmallMMax) {
-    const size_t small = kHeaderBytes + small_counter_bytes(N) + small_m_partial_bytes(M, N, K);
-    if (small > need) need = small;
-  }
+  if (use_small_m(M, N)) need = align_up(need, kAlign) + small_counter_bytes(N) + small_m_partial_bytes(M, N, K);
   return need;
 }
 
@@ -168,6 +165,50 @@ fg8_status cuda_status(cudaError_t e) {
 }
 
 }  // namespace
+
+// The few-token kernel (small_m.cu) on fg8_linear's workspace: counters in
+// the header (or after the prepare layout for more than kHeaderCounters
+// weight tiles), split-K partials after the prepare layout.  fused: x is
+// quantized inside the kernel; otherwise the prepare step's codes and
+// scales are in the workspace already.
+fg8_status launch_small_path(bool fused, const void* x_bf16, int64_t ld_x, int64_t M, int64_t N, int64_t K,
+                             const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16, void* y_bf16,
+                             int64_t ld_y, int fmt, void* workspace, void* stream) {
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  const size_t small_off = align_up(L.total, kAlign);
+  SmallMArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.wq = wq_e4m3;
+  a.w_scale = w_scale_inv;
+  a.bias = bias_bf16;
+  a.y = y_bf16;
+  a.ld_y = ld_y;
+  a.splits = small_m_splits(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+  const size_t extra = small_counter_bytes(N);
+  a.zero_counters = extra > 0;
+  a.counters = reinterpret_cast<uint32_t*>(ws + (extra > 0 ? small_off : kHeaderCounterOffset));
+  a.part = reinterpret_cast<float*>(ws + small_off + extra);
+  a.preq = !fused;
+  if (a.preq) {
+    a.xq = ws + L.xq_off;
+    a.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    a.ld_s = L.ld_s;
+    a.sfa = ws + L.xs_off;
+    a.sfb = ws + L.wsc_off;
+    a.Kq = ceil_div(ceil_div(K, kGroup), 4);
+  }
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.test_stall = g_test_stall.load();
+  return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
+}
 
 extern "C" {
 
@@ -277,6 +318,12 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   if (ld_y % 8 != 0 || !aligned16(wq_e4m3) || !aligned16(y_bf16) || (bias_bf16 != nullptr && !aligned16(bias_bf16)) ||
       !aligned16(w_scale_inv))
     return FG8_ERR_ALIGNMENT;
+  if (use_small_m(M, N)) {  // few tokens: the swap-AB split-K kernel streaming the weights
+    if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
+      return st;
+    return launch_small_path(false, nullptr, 0, M, N, K, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt,
+                             workspace, stream);
+  }
   const LinearWs L = linear_ws_layout(M, N, K, fmt);
   if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
   DeviceInfo dev;
@@ -376,31 +423,9 @@ fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64
     return FG8_ERR_ALIGNMENT;
   if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
     return st;
-  if (M <= kSmallMMax) {  // few tokens: one fused kernel (quantize, swap-AB split-K GEMM, reduce)
-    DeviceInfo dev;
-    if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    SmallMArgs a{};
-    a.x = x_bf16;
-    a.ld_x = ld_x;
-    a.M = static_cast<int>(M);
-    a.N = static_cast<int>(N);
-    a.K = static_cast<int>(K);
-    a.wq = wq_e4m3;
-    a.w_scale = w_scale_inv;
-    a.bias = bias_bf16;
-    a.y = y_bf16;
-    a.ld_y = ld_y;
-    a.splits = small_m_splits(static_cast<int>(N), static_cast<int>(K));
-    const size_t extra = small_counter_bytes(N);
-    a.zero_counters = extra > 0;
-    a.counters = reinterpret_cast<uint32_t*>(ws + (extra > 0 ? kHeaderBytes : kHeaderCounterOffset));
-    a.part = reinterpret_cast<float*>(ws + kHeaderBytes + extra);
-    a.status = reinterpret_cast<uint32_t*>(ws);
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.test_stall = g_test_stall.load();
-    return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
-  }
+  if (use_small_m(M, N) && use_fused_small_m(M, fmt))  // one kernel: quantize, GEMM, reduce
+    return launch_small_path(true, x_bf16, ld_x, M, N, K, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt,
+                             workspace, stream);
   if (fg8_status st = fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes, stream);
       st != FG8_OK)
     return st;

@@ -104,29 +104,48 @@ constexpr size_t kWorkspaceHeaderBytes = 1024;
 constexpr size_t kHeaderCounterOffset = 64;
 constexpr int kHeaderCounters = static_cast<int>((kWorkspaceHeaderBytes - kHeaderCounterOffset) / 4);
 
-// Few tokens (M <= kSmallMMax): one kernel quantizes x, runs the swap-AB
-// split-K GEMM and reduces (small_m.cu).
-constexpr int kSmallMMax = 32;
+// Few tokens: a swap-AB split-K GEMM that streams the weights as the tensor
+// core's M side (small_m.cu), either on the prepare step's quantized
+// activations (preq) or, with UE8M0 scales and M <= kFusedMMax, with the
+// activation quantization fused into it.  fg8_linear takes it for
+// M <= kSmallMAlways, and up to kSmallMMax tokens while the tiled GEMM's grid
+// (ceil(N / 256) tiles of 128 tokens) would cover at most a quarter of the
+// 148 SMs; both rules depend on the shape only.
+constexpr int kSmallMMax = 128;
+constexpr int kSmallMAlways = 32;
+constexpr int kFusedMMax = 16;
+
+inline bool use_small_m(int64_t M, int64_t N) {
+  return M >= 1 && (M <= kSmallMAlways || (M <= kSmallMMax && (N + 255) / 256 * 4 <= 148));
+}
+inline bool use_fused_small_m(int64_t M, int fmt) { return fmt == 1 && M <= kFusedMMax; }
 
 struct SmallMArgs {
-  const void* x;          // bf16 [M, K], row stride ld_x
+  const void* x;          // bf16 [M, K], row stride ld_x (fused)
   int64_t ld_x;
+  bool preq;              // activations already quantized (the prepare step's layouts below)
+  const void* xq;         // e4m3 [M, K], row stride K
+  const float* xs_t;      // float: x scales K-major [Kb][ld_s]
+  int64_t ld_s;
+  const uint8_t* sfa;     // UE8M0: scale-factor tiles of x, and of W (sfb)
+  const uint8_t* sfb;
+  int Kq;
   int M, N, K;
   const void* wq;         // e4m3 [N, K]
   const void* w_scale;    // [ceil(N/128), ceil(K/128)] float32 or UE8M0 bytes
   const void* bias;       // bf16 [N] or nullptr
   void* y;                // bf16 [M, N], row stride ld_y
   int64_t ld_y;
-  int splits;             // small_m_splits(N, K)
+  int splits;             // small_m_splits(M, N, K)
   uint32_t* counters;     // [ceil(N/128)], zero at rest (or zeroed by the launch, below)
   bool zero_counters;     // counters outside the header: clear them before the kernel
-  float* part;            // [splits][M][N] fp32 when splits > 1
+  float* part;            // [ceil(N/128)][splits][M][128] fp32 when splits > 1
   uint32_t* status;
   uint64_t wait_limit_ns;
   int test_stall;         // test hook, as GemmArgs::test_stall
 };
 
-int small_m_splits(int N, int K);
+int small_m_splits(int M, int N, int K);
 // Bytes of fp32 split-K partials the small-M path needs (0 with one split).
 size_t small_m_partial_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s);

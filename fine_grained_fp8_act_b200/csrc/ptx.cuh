@@ -113,6 +113,14 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* src, 
                : "memory");
 }
 
+// 1-D bulk store shared -> global (16-byte aligned addresses, size % 16 == 0),
+// bulk-group completion.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 template <int N>
@@ -129,6 +137,12 @@ __device__ __forceinline__ void bulk_wait_group() {
 // async-proxy (TMA / tensor core) reads of them.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders global-memory accesses of the generic proxy (plain loads, stores,
+// atomics) with those of the async proxy (bulk copies), in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {

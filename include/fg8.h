@@ -109,10 +109,14 @@ FG8_API size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_s
  *               clears the status word, and after a failed call the whole
  *               header.  Calls sharing a workspace must not overlap on the
  *               device.
- * M <= 32 runs one kernel that quantizes x, streams the weights as the
- * tensor core's M side (128 weight rows per CTA, split over K) and reduces;
- * larger M quantizes x (fg8_linear_prepare) and runs the tiled GEMM
- * (fg8_linear_run).
+ * fg8_linear is fg8_linear_prepare (quantize x into the workspace) then
+ * fg8_linear_run (the GEMM), which picks its kernel by shape: for M <= 32,
+ * and for M <= 128 while ceil(N / 256) <= 37 (the tiled grid would cover at
+ * most a quarter of the SMs), the few-token kernel, which streams the
+ * weights as the tensor core's M side (128 weight rows per CTA, split over
+ * K) and reduces the splits; otherwise the tiled GEMM.  With UE8M0 scales
+ * and M <= 16 fg8_linear instead runs one few-token kernel that also
+ * quantizes x (no prepare launch).
  * Float scales are applied exactly per 128-K block in float32 (never rounded
  * to a power of two, [zh] §七 补充); UE8M0 scales go through the tensor
  * core's block-scaled MMA.  M == 0 is a no-op. */
@@ -126,9 +130,11 @@ FG8_API fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t 
  *   fg8_linear_prepare  quantizes x into the workspace in the GEMM's layouts
  *                       (and, for UE8M0, packs w_scale_inv's scale-factor tiles);
  *   fg8_linear_run      runs the GEMM from that workspace.
- * prepare followed by run on the same stream and workspace is fg8_linear for
- * M > 32 (for M <= 32 fg8_linear runs its fused few-token kernel, whose
- * split-K sums may round differently within the stated tolerance).
+ * prepare followed by run on the same stream and workspace is fg8_linear
+ * (bit for bit), except with UE8M0 scales and M <= 16, where fg8_linear
+ * quantizes inside its few-token kernel (same codes and scales; its sums
+ * may round differently within the stated tolerance).  The workspace is
+ * fg8_linear_workspace_bytes, as for fg8_linear.
  * Arguments and checks are those of fg8_linear. */
 FG8_API fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                                       const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,

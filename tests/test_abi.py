@@ -176,6 +176,11 @@ def test_workspace_sizes(fg8):
     b = f(8192, 18432, 7168, 1)
     assert b >= 8192 * 7168
     assert f(0, 256, 256, 0) > 0
+    # few tokens with a long K: the swap-AB kernel's split-K partials come on
+    # top (2 weight tiles, 64 K-blocks -> 32 splits, the 512 / M cap;
+    # fp32 [tiles][splits][M][128])
+    assert f(16, 256, 8192, 0) >= 32 * 16 * 256 * 4
+    assert f(16, 256, 8192, 0) > f(16, 256, 128, 0) + 32 * 16 * 256 * 4 - 64 * 1024
     # pre-quantized GEMM: header + scales in the GEMM's layouts (x: K-major
     # float32 over 128-row-padded M; W: 16-byte entries per 128x128 block)
     assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 0) >= 256 + 2 * 128 * 4 + 2 * 2 * 16

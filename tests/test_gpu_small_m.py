@@ -1,8 +1,10 @@
-"""The few-token path of fg8_linear (M <= 32): one kernel that quantizes x,
-runs the swap-AB split-K GEMM and reduces.  Checked against the oracle on
-every element, at token counts around each padding step (16, 32, and
-just past the path up to 128), shapes whose K-range is split over many
-CTAs, ragged weight tiles and K."""
+"""The few-token path of fg8_linear: the swap-AB split-K kernel that streams
+the weights as the tensor core's M side, on the prepare step's quantized
+activations (or, for UE8M0 scales and M <= 16, quantizing x itself), for
+M <= 32 and up to M = 128 while N is small enough.  Checked against the
+oracle on every element, at token counts around each padding step (16, 32,
+64, 128), shapes whose K-range is split over many CTAs, ragged weight tiles
+and K, and both sides of the shape rule that picks it."""
 import numpy as np
 import pytest
 import torch
@@ -60,10 +62,12 @@ def test_token_counts(fg8, orc, fmt, M):
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
 @pytest.mark.parametrize("M,N,K", [(16, 256, 8192), (5, 384, 2048), (128, 136, 4096), (64, 520, 6160), (1, 8, 16),
-                                   (33, 4096, 1024)])
+                                   (33, 4096, 1024), (3, 1032, 7168), (100, 264, 12288), (1, 256, 16384)])
 def test_split_k_shapes(fg8, orc, fmt, M, N, K):
     """Few weight tiles and a long K: the K-range is split over up to 64 CTAs
-    whose fp32 partials the last one adds up; ragged last weight tile and K."""
+    (at most 512 / M) whose fp32 partials the last one adds up, with each of
+    its three load batchings (M <= 8, M <= 32, larger) and split counts that
+    do not fill the last batch; ragged last weight tile, token batch and K."""
     _run(fg8, orc, M, N, K, fmt, seed=N + K)
 
 
@@ -99,6 +103,28 @@ def test_strided_x_and_y(fg8, orc, fmt):
     assert fg8.fg8_check_device_status(wsp.data_ptr(), s) == 0
     assert torch.isnan(ybuf[:, N:].float()).all()  # nothing written past N
     _check(orc, x.contiguous(), w, b, ybuf[:, :N].contiguous(), fmt)
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N", [(33, 9472), (33, 9480), (128, 9472), (40, 1040), (20, 1040)])
+def test_dispatch_and_prepare_run(fg8, orc, fmt, M, N):
+    """Past 32 tokens fg8_linear takes the few-token kernel while the tiled
+    GEMM's grid would cover at most a quarter of the SMs (N <= 9472) and the
+    tiled GEMM beyond.  Either way fg8_linear_prepare then fg8_linear_run
+    (which picks the kernel by the same rule) gives fg8_linear's bits."""
+    K = 256
+    x, w, b, wq, ws, y = _run(fg8, orc, M, N, K, fmt, seed=M + N)
+    nb = fg8.fg8_linear_workspace_bytes(M, N, K, fmt)
+    wsp = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    y2 = torch.full_like(y, float("nan"))
+    s = torch.cuda.current_stream().cuda_stream
+    if fmt == UE8M0 and M <= 16:
+        pytest.skip("fg8_linear quantizes inside the few-token kernel here")
+    fg8.fg8_linear_prepare(x.data_ptr(), M, N, K, K, ws.data_ptr(), fmt, wsp.data_ptr(), nb, s)  # raises on error
+    fg8.fg8_linear_run(wq.data_ptr(), ws.data_ptr(), b.data_ptr(), y2.data_ptr(), M, N, K, N, fmt, wsp.data_ptr(), nb, s)
+    torch.cuda.synchronize()
+    assert fg8.fg8_check_device_status(wsp.data_ptr(), s) == 0
+    assert torch.equal(y, y2)
 
 
 def test_repeated_calls_same_workspace(fg8, orc):
