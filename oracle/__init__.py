@@ -187,6 +187,53 @@ def linear(x_bf16, wq, ws, bias_bf16, fmt, rows=None):
     return linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows)
 
 
+# ------------------------------------------------------ MoE experts ------
+MOE_TILE = 128  # rows of one expert block in the contiguous grouped layout
+
+
+def grouped_linear(x_bf16, row_expert, wq, ws, bias_bf16, fmt):
+    """The expert GEMM of an MoE layer ([zh] §6.4 / [pt] "Caminho rápido do
+    DeepGEMM": FP8Experts sends each expert's tokens through the fine-grained
+    FP8 linear of [zh] §八 step 6, with that expert's e4m3 weights and block
+    scales; on Blackwell the expert kernels take UE8M0 scales).
+
+    Layout (a reading: the pages print no expert kernel interface): the
+    routed rows of x are sorted by expert, each expert's run padded to whole
+    blocks of MOE_TILE rows; block t = rows [128 t, 128 t + 128) is computed
+    with expert row_expert[128 t], and skipped when that is -1.  The
+    activation groups are per token, so x is quantized once for all experts.
+
+    x_bf16 [M, K] (bits), row_expert [M] int, wq [E, N, K], ws [E, Nb, Kb],
+    bias_bf16 [E, N] or None.  Returns (y64, bound, y_bf16, written): rows of
+    skipped blocks have written False, y64 NaN and y_bf16 0.
+    """
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    re = np.asarray(row_expert).astype(np.int64)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(ws, dtype=_scale_dtype(fmt))
+    M, K = x.shape
+    E, N, K2 = wq.shape
+    if K2 != K or re.shape != (M,) or ws.shape != (E, _kb(N), _kb(K)):
+        raise ValueError("shape mismatch")
+    if bias_bf16 is not None and np.shape(bias_bf16) != (E, N):
+        raise ValueError("bias shape mismatch")
+    xq, xs = quantize_act(x, fmt)
+    y64 = np.full((M, N), np.nan)
+    bound = np.zeros((M, N))
+    ybf = np.zeros((M, N), dtype=np.uint16)
+    written = np.zeros(M, dtype=bool)
+    for t in range(-(-M // MOE_TILE)):
+        e = int(re[t * MOE_TILE])
+        if e < 0:
+            continue
+        if e >= E:
+            raise ValueError(f"block {t}: expert {e} >= {E}")
+        rows = np.arange(t * MOE_TILE, min(M, (t + 1) * MOE_TILE))
+        a, b, c = linear_dequant(xq, xs, wq[e], ws[e], None if bias_bf16 is None else bias_bf16[e], fmt, rows=rows)
+        y64[rows], bound[rows], ybf[rows], written[rows] = a, b, c, True
+    return y64, bound, ybf, written
+
+
 # ------------------------------------------------ checkpoint conversions --
 def dequantize_weight(wq, ws, fmt: int) -> np.ndarray:
     """Fp8Dequantize: e4m3 [N, K] and its block scales -> bf16 bits [N, K]."""

@@ -553,3 +553,100 @@ def test_quantize_act_static_lossless_and_linear(orc):
             exact = sum(Fraction(float(x[m, k])) * Fraction(float(table[wq[n, k]])) * Fraction(float(ws[n // 128, k // 128]))
                         for k in range(K))
             assert abs(Fraction(y64[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+
+
+# ---------------------------------------------------------- MoE experts --
+def _lossless_rows(M, K, rng, exps):
+    """Rows whose 128-groups each have amax 448 * 2^i and every value on the
+    e4m3 grid times 2^i: both scale formats then give s = 2^i exactly and
+    quantization is lossless (all values are bf16 numbers)."""
+    table = torch_e4m3_table()
+    finite = table[np.isfinite(table)]
+    x = np.empty((M, K))
+    for m in range(M):
+        for g in range(K // 128):
+            i = exps[(m + g) % len(exps)]
+            v = rng.choice(finite, 128) * 2.0 ** i
+            v[rng.integers(128)] = 448.0 * 2.0 ** i * rng.choice([-1.0, 1.0])
+            x[m, g * 128:(g + 1) * 128] = v
+    return x
+
+
+def _bits(a):
+    return (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _moe_case(seed, fmt, E=3, K=256, M=4 * 128 + 50, tile_e=(2, 0, -1, 1, 0)):
+    rng = np.random.default_rng(seed)
+    N = K
+    x = _lossless_rows(M, K, rng, (-12, -9, -6))
+    perms = [rng.permutation(K) for _ in range(E)]
+    c = [448.0 * 2.0 ** j for j in (-14, -10, -7)][:E]
+    w = np.zeros((E, N, K))
+    for e in range(E):
+        w[e, np.arange(N), perms[e]] = c[e]   # W_e[n, pi_e(n)] = c_e
+    b = _bits(rng.normal(0, 0.1, (E, N)))
+    re = np.empty(M, dtype=np.int32)
+    for t, e in enumerate(tile_e):
+        re[t * 128:(t + 1) * 128] = e
+    re[128 - 10:128] = -1  # padding rows inside a computed block: computed with the block's expert
+    wq = np.empty((E, N, K), dtype=np.uint8)
+    ws = np.empty((E, N // 128, K // 128), dtype=np.float32 if fmt == FLOAT else np.uint8)
+    return x, perms, c, b, re, wq, ws, w
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+def test_grouped_linear_closed_form(orc, fmt):
+    """Experts W_e = c_e * P_e (a permutation, c_e = 448 * 2^j, block scales
+    exact) on losslessly quantized rows: y[r, n] = c_e * x[r, pi_e(n)] + b_e[n]
+    exactly, with e the expert of r's 128-row block; skipped blocks untouched."""
+    x, perms, c, b, re, wq, ws, w = _moe_case(7, fmt)
+    for e in range(w.shape[0]):
+        wq[e], ws[e] = orc.quantize_weight(_bits(w[e]), fmt)
+    y64, bound, ybf, written = orc.grouped_linear(_bits(x), re, wq, ws, b, fmt)
+    bf = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for t, e in enumerate((2, 0, -1, 1, 0)):
+        rows = np.arange(t * 128, min(x.shape[0], (t + 1) * 128))
+        if e < 0:
+            assert not written[rows].any() and np.isnan(y64[rows]).all()
+            continue
+        assert written[rows].all()
+        want = c[e] * x[rows][:, perms[e]] + bf[e]
+        assert np.array_equal(y64[rows], want), f"block {t} (expert {e})"
+
+
+def test_grouped_linear_block_order(orc):
+    """Moving whole 128-row blocks (rows and their expert) moves the outputs."""
+    rng = np.random.default_rng(3)
+    E, N, K, M = 3, 136, 384, 3 * 128 + 40
+    x = _bits(rng.normal(0, 1, (M, K)))
+    wq = np.empty((E, N, K), dtype=np.uint8)
+    ws = np.empty((E, 2, 3), dtype=np.uint8)
+    for e in range(E):
+        wq[e], ws[e] = orc.quantize_weight(_bits(rng.normal(0, 0.05, (N, K))), UE8M0)
+    re = np.repeat(np.array([1, 2, 0, 2], dtype=np.int32), 128)[:M]
+    y1 = orc.grouped_linear(x, re, wq, ws, None, UE8M0)[0]
+    order = [2, 0, 1]  # full blocks only; the ragged last block stays
+    idx = np.concatenate([np.arange(o * 128, o * 128 + 128) for o in order] + [np.arange(384, M)])
+    y2 = orc.grouped_linear(x[idx], re[idx], wq, ws, None, UE8M0)[0]
+    assert np.array_equal(y2, y1[idx])
+
+
+def test_grouped_linear_one_expert_is_the_dense_layer(orc):
+    """One expert owning every block is the dense layer of [zh] §八 step 6."""
+    rng = np.random.default_rng(4)
+    M, N, K = 200, 264, 256
+    x = _bits(rng.normal(0, 1, (M, K)))
+    wq, ws = orc.quantize_weight(_bits(rng.normal(0, 0.05, (N, K))), FLOAT)
+    b = _bits(rng.normal(0, 0.1, N))
+    y64, bound, ybf, written = orc.grouped_linear(x, np.zeros(M, np.int32), wq[None], ws[None], b[None], FLOAT)
+    d64, dbound, dbf = orc.linear(x, wq, ws, b, FLOAT)
+    assert written.all() and np.array_equal(y64, d64) and np.array_equal(ybf, dbf)
+
+
+def test_grouped_linear_rejects_unknown_expert(orc):
+    x = np.zeros((128, 128), np.uint16)
+    wq = np.zeros((2, 8, 128), np.uint8)
+    ws = np.ones((2, 1, 1), np.float32)
+    with pytest.raises(ValueError):
+        orc.grouped_linear(x, np.full(128, 2, np.int32), wq, ws, None, FLOAT)

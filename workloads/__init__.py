@@ -135,6 +135,57 @@ def make_inputs(cfg: str, gemm: Gemm, device="cpu", stage: int = 1) -> Tuple[tor
     return x, w, bias
 
 
+# ----------------------------------------------------- MoE experts ----
+# DeepSeek-V3-shaped routed experts (hidden 7168, expert intermediate 2048,
+# 256 experts, 8 per token); the expert kernels take UE8M0 scales on
+# Blackwell.  gate/up: K = 7168 -> N = 2 x 2048; down: K = 2048 -> N = 7168.
+MOE_BLOCK = 128
+DSV3_MOE = dict(experts=256, topk=8, hidden=7168, inter=2048, tokens=4096)
+
+
+def moe_routing(T: int, E: int, topk: int, seed: int, skew: float = 1.0):
+    """Seeded synthetic routing in the contiguous grouped layout.
+
+    Expert popularity is log-normal (sigma = skew); each token picks topk
+    distinct experts with probability proportional to popularity (Gumbel
+    top-k).  The T * topk routed rows are sorted by expert (then token) and
+    each expert's run is padded with rows of token -1 to a whole number of
+    MOE_BLOCK-row blocks.  Returns (row_token, row_expert) int64 / int32
+    tensors of the padded length: row_expert is -1 on padding rows.
+    """
+    g = _gen(seed, "cpu")
+    logp = torch.randn(E, generator=g, dtype=torch.float64) * skew
+    gumbel = -torch.log(-torch.log(torch.rand(T, E, generator=g, dtype=torch.float64).clamp_min(1e-300)))
+    picks = torch.topk(logp[None, :] + gumbel, topk, dim=1).indices  # [T, topk], distinct per token
+    tok = torch.arange(T).repeat_interleave(topk)
+    exp = picks.reshape(-1)
+    order = torch.argsort(exp * T + tok)
+    tok, exp = tok[order], exp[order]
+    counts = torch.bincount(exp, minlength=E)
+    padded = (counts + MOE_BLOCK - 1) // MOE_BLOCK * MOE_BLOCK
+    Mp = int(padded.sum())
+    row_token = torch.full((Mp,), -1, dtype=torch.int64)
+    row_expert = torch.full((Mp,), -1, dtype=torch.int32)
+    starts = torch.cumsum(padded, 0) - padded
+    src = 0
+    for e in range(E):
+        n = int(counts[e])
+        if n:
+            a = int(starts[e])
+            row_token[a:a + n] = tok[src:src + n]
+            row_expert[a:a + n] = e
+            src += n
+    return row_token, row_expert
+
+
+def gather_rows(x: torch.Tensor, row_token: torch.Tensor) -> torch.Tensor:
+    """x[row_token] with zero rows where row_token is -1."""
+    out = torch.zeros(row_token.numel(), x.shape[1], dtype=x.dtype, device=x.device)
+    keep = row_token >= 0
+    out[keep.to(x.device)] = x[row_token[keep].to(x.device)]
+    return out
+
+
 def bf16_bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (CPU copy)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view("uint16")
