@@ -33,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import workloads as W  # noqa: E402
@@ -521,6 +522,237 @@ def run_e2e(fg8, plan, args, stream, dev, world, chain):
             "steps": steps, "ms_per_step": ms / steps}
 
 
+# ---------------------------------------------------- MoE experts (fg8) ----
+def moe_shapes():
+    """[(name, K, N)] of the routed-expert layers: gate/up, then down."""
+    c = W.DSV3_MOE
+    return [("moe_dsv3_gate_up", c["hidden"], 2 * c["inter"]), ("moe_dsv3_down", c["inter"], c["hidden"])]
+
+
+def moe_config(rows_routed, rows_padded):
+    c = W.DSV3_MOE
+    return {"workload": "moe_dsv3", "model": "DeepSeek-V3-shaped routed experts (hidden 7168, expert "
+            "intermediate 2048, 256 experts, top-8), synthetic routing: log-normal expert popularity, sigma "
+            f"{c['skew']}",
+            "tokens": c["tokens"], "experts": c["experts"], "topk": c["topk"], "rows_routed": rows_routed,
+            "rows_padded": rows_padded, "layers": [[K, N] for _, K, N in moe_shapes()], "scale_fmt": "ue8m0",
+            "block": [128, 128], "act_group": 128, "layout": "contiguous grouped, expert runs padded to 128 rows",
+            "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the step events)"}
+
+
+def run_moe(args, rank, world, local):
+    """The MoE expert layers through fg8_grouped_linear (prepare + grouped GEMM per
+    layer).  TFLOP/s count the routed rows only (padding rows are work done but
+    not counted)."""
+    import fine_grained_fp8_act_b200 as fg8
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    c = W.DSV3_MOE
+    T, E, topk, fmt = c["tokens"], c["experts"], c["topk"], 1
+    rt, re = W.moe_routing(T, E, topk, seed=5, skew=c["skew"])
+    Mp, routed = int(re.numel()), T * topk
+    re_d = re.to(dev)
+    plan = []
+    for i, (name, K, N) in enumerate(moe_shapes()):
+        xt = W.x_student_t(T, K, seed=50 + i, device=dev)
+        if rank:
+            xt = xt.roll(rank, 0).contiguous()
+        x = W.gather_rows(xt, rt)
+        del xt
+        wq = ws = None
+        for e in range(E):  # one expert at a time: the bf16 stack would need twice the e4m3 bytes
+            q, sc = fg8.quantize_weight(W.w_row_groups(N, K, 0.015, seed=1000 * (i + 1) + e, device=dev), fmt)
+            if wq is None:  # the dtypes quantize_weight returns, so that the stores below copy bits
+                wq = torch.empty((E,) + tuple(q.shape), dtype=q.dtype, device=dev)
+                ws = torch.empty((E,) + tuple(sc.shape), dtype=sc.dtype, device=dev)
+            wq[e] = q
+            ws[e] = sc
+        nb = fg8.fg8_grouped_linear_workspace_bytes(Mp, E, N, K, fmt)
+        plan.append(dict(name=name, K=K, N=N, x=x, wq=wq, ws=ws, wsp=torch.zeros(nb, dtype=torch.uint8, device=dev),
+                         y=torch.empty(Mp, N, dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+
+    def prep(L):
+        fg8.fg8_grouped_linear_prepare(L["x"].data_ptr(), Mp, L["K"], L["K"], E, L["N"], L["ws"].data_ptr(), fmt,
+                                       L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+
+    def run(L):
+        fg8.fg8_grouped_linear_run(re_d.data_ptr(), E, L["wq"].data_ptr(), L["ws"].data_ptr(), None,
+                                   L["y"].data_ptr(), Mp, L["N"], L["K"], L["N"], fmt, L["wsp"].data_ptr(),
+                                   L["wsp"].numel(), sp)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()
+    for _ in range(args.warmup):
+        flush_l2()
+        for L in plan:
+            prep(L)
+            run(L)
+    torch.cuda.synchronize()
+    for L in plan:
+        if fg8.fg8_check_device_status(L["wsp"].data_ptr(), sp) != 0:
+            raise RuntimeError("device status after warm-up")
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush_l2()
+        step_ev[k][0].record(stream)
+        for L in plan:
+            prep(L)
+            run(L)
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    time.sleep(0.25)
+    clk = clocks.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    total_ms_max = max_over_ranks(total_ms, world, dev)
+    flops_step = sum(2.0 * routed * L["N"] * L["K"] for L in plan)
+    tflops = sum_over_ranks(flops_step * args.steps, world, dev) / (total_ms_max * 1e-3) / 1e12
+
+    # per-kernel pass: events around each layer's prepare and grouped GEMM
+    n_prof = max(3, min(args.steps, 20))
+    pm = [[] for _ in plan]
+    gm = [[] for _ in plan]
+    for _ in range(n_prof):
+        flush_l2()
+        for i, L in enumerate(plan):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            prep(L)
+            e[1].record(stream)
+            run(L)
+            e[2].record(stream)
+            pm[i].append(e)
+            gm[i].append(e)
+    torch.cuda.synchronize()
+    pm = [statistics.mean(e[0].elapsed_time(e[1]) for e in v) for v in pm]
+    gm = [statistics.mean(e[1].elapsed_time(e[2]) for e in v) for v in gm]
+    peaks = measured_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    dom = max(range(len(plan)), key=lambda i: gm[i])
+    L = plan[dom]
+    t_s = gm[dom] * 1e-3
+    Kb, Nb = -(-L["K"] // 128), -(-L["N"] // 128)
+    # every expert's weights once, the routed layout's codes, scales and output
+    moe_bytes = E * L["N"] * L["K"] + E * Nb * Kb + Mp * L["K"] + Mp * Kb + 2 * Mp * L["N"]
+    moe_flops = 2.0 * Mp * L["N"] * L["K"]  # the tensor cores run the padding rows too
+    if moe_flops / (fp8_peak * 1e12) >= moe_bytes / (peaks["hbm_gbs"] * 1e9):
+        roof = {"bound": "tensor", "achieved": moe_flops / t_s / 1e12, "peak": fp8_peak, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": moe_bytes / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": recorded_traffic("moe_dsv3", dom),
+                 "kernel": f"fg8_gemm_kernel, grouped ({L['name']}: {Mp} rows of which {routed} routed, "
+                           f"K={L['K']} N={L['N']}, {E} experts)",
+                 "kernel_us": gm[dom] * 1e3,
+                 "algorithmic": (f"{moe_bytes / 1e9:.3f} GB per launch (all experts' e4m3 weights + scales, the "
+                                 f"routed layout's e4m3 codes + scales, bf16 y); {moe_flops / 1e12:.3f} TFLOP "
+                                 f"(padded rows)"),
+                 "routed_tflops": 2.0 * routed * L["N"] * L["K"] / t_s / 1e12,
+                 "peak_source": (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 "
+                                 f"nominal), HBM {peaks['hbm_gbs']} GB/s"),
+                 "timing": f"kernel alone: CUDA events around each launch over {n_prof} flushed steps"})
+    per_kernel = [{"layer": L["name"], "path": "grouped", "prepare_us": pm[i] * 1e3,
+                   "act_quant_gbs": (3 * Mp * L["K"] + Mp * (-(-L["K"] // 128))) / (pm[i] * 1e-3) / 1e9,
+                   "gemm_us": gm[i] * 1e3,
+                   "gemm_tflops": 2.0 * routed * L["N"] * L["K"] / (gm[i] * 1e-3) / 1e12}
+                  for i, L in enumerate(plan)]
+
+    # end to end: routed rows and the expert index in from pinned host memory,
+    # both layers, the last layer's rows out
+    xh = [L["x"].to("cpu").pin_memory() for L in plan]
+    reh = re.pin_memory()
+    xd = [torch.empty_like(L["x"]) for L in plan]
+    red = torch.empty_like(re_d)
+    yh = torch.empty(plan[-1]["y"].shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def one():
+        red.copy_(reh, non_blocking=True)
+        for L, a, b in zip(plan, xh, xd):
+            b.copy_(a, non_blocking=True)
+            fg8.fg8_grouped_linear(b.data_ptr(), Mp, L["K"], L["K"], red.data_ptr(), E, L["N"], L["wq"].data_ptr(),
+                                   L["ws"].data_ptr(), None, L["y"].data_ptr(), L["N"], fmt, L["wsp"].data_ptr(),
+                                   L["wsp"].numel(), sp)
+        yh.copy_(plan[-1]["y"], non_blocking=True)
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": sum_over_ranks(flops_step * e2e_steps, world, dev) / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": sum(a.numel() * 2 for a in xh) + reh.numel() * 4,
+           "d2h_bytes_per_step": yh.numel() * 2, "steps": e2e_steps, "ms_per_step": ems / e2e_steps}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_moe(budget_s=args.cpu_seconds)
+    out = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": dict(moe_config(routed, Mp), parallelism=f"dp{world} (token rows, replicated experts, no collective)"),
+        "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
+        "per_kernel": per_kernel, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 3 * len(plan) * args.steps,  # act-quant, scale packing, grouped GEMM per layer
+        "clocks": clk, "wall_s": wall,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def cpu_baseline_moe(budget_s=15.0, rows=None):
+    """The CPU oracle's grouped layer, as it stands, on the first R rows of the
+    routed layout (all in the first expert block) of each expert layer; weights
+    of that block's expert quantized outside the timing.  TFLOP/s of those rows."""
+    import oracle
+    c = W.DSV3_MOE
+    rt, re = W.moe_routing(c["tokens"], c["experts"], c["topk"], seed=5, skew=c["skew"])
+    e0 = int(re[0])
+    ops = []
+    for i, (name, K, N) in enumerate(moe_shapes()):
+        xt = W.x_student_t(c["tokens"], K, seed=50 + i)
+        x = W.bf16_bits(W.gather_rows(xt, rt[:128]))
+        wq, ws = oracle.quantize_weight(W.bf16_bits(W.w_row_groups(N, K, 0.015, seed=1000 * (i + 1) + e0)), 1)
+        ops.append((K, N, x, wq[None], ws[None]))
+    rexp = np.zeros(128, dtype=np.int32)  # the block's expert, renumbered 0 in the one-expert table
+
+    def run(R):
+        t0 = time.perf_counter()
+        for K, N, x, wq, ws in ops:
+            oracle.grouped_linear(x[:R], rexp[:R], wq, ws, None, 1)
+        return time.perf_counter() - t0
+
+    if rows is None:
+        t = run(2)
+        rows = int(max(2, min(128, 2 * budget_s / max(t, 1e-6))))
+    t = run(rows)
+    flops = sum(2.0 * rows * N * K for K, N, _, _, _ in ops)
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"first {rows} routed rows (expert {e0}) through both expert layers ({t:.1f} s; weights "
+                      f"quantized outside the timing)", "seconds": t, "rows": rows}
+
+
 # ------------------------------------------------------ oracle (CPU) arm ----
 def cpu_baseline(workload, budget_s=15.0, rows=None):
     """The CPU oracle, as it stands, on a bounded sample of the workload: the
@@ -558,8 +790,33 @@ def cpu_baseline(workload, budget_s=15.0, rows=None):
             "seconds": t}
 
 
+def run_reference_moe(args):
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    probe = cpu_baseline_moe(rows=2)
+    rows = int(max(1, min(128, 2 * budget / max(probe["seconds"], 1e-6))))
+    for _ in range(args.warmup):
+        cpu_baseline_moe(rows=rows)
+    ts = [cpu_baseline_moe(rows=rows)["seconds"] for _ in range(args.steps)]
+    flops = sum(2.0 * rows * N * K for _, K, N in moe_shapes())
+    value = flops * len(ts) / sum(ts) / 1e12
+    c = W.DSV3_MOE
+    cpu = {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+           "sample": f"first {rows} routed rows through both expert layers per step"}
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: float32 quantization, double GEMM)",
+           "data": "synthetic", "impl": "reference",
+           "config": dict(moe_config(c["tokens"] * c["topk"], None), parallelism="cpu oracle, rank 0 only"),
+           "cpu_baseline": cpu,
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
+        return
+    if args.workload.startswith("moe_"):
+        run_reference_moe(args)
         return
     layers = workload_layers(args.workload)
     # size each step so warm-up + steps stay within ~2 minutes
@@ -608,6 +865,11 @@ def main(argv=None):
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload.startswith("moe_"):
+        if args.workload != "moe_dsv3":
+            raise SystemExit(f"unknown workload {args.workload}")
+        run_moe(args, rank, world, local)
         return
     run_fg8(args, rank, world, local)
 

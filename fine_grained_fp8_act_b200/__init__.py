@@ -27,6 +27,10 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_dequantize_weight,
     fg8_gemm_prequant,
     fg8_gemm_workspace_bytes,
+    fg8_grouped_linear,
+    fg8_grouped_linear_prepare,
+    fg8_grouped_linear_run,
+    fg8_grouped_linear_workspace_bytes,
     fg8_linear,
     fg8_linear_noalloc,
     fg8_linear_prepare,
@@ -49,6 +53,7 @@ from .layer import (  # noqa: F401
     FP8Linear,
     dequantize_weight,
     gemm_prequant,
+    grouped_linear,
     linear,
     linear_chain,
     linear_static,

@@ -34,6 +34,11 @@ SIGNATURES = {
     "fg8_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
     "fg8_linear": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_prepare": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _INT, _VP, _SZ, _VP]),
+    "fg8_grouped_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _INT]),
+    "fg8_grouped_linear": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP, _SZ,
+                                  _VP]),
+    "fg8_grouped_linear_prepare": (_INT, [_VP, _I64, _I64, _I64, _I64, _I64, _VP, _INT, _VP, _SZ, _VP]),
+    "fg8_grouped_linear_run": (_INT, [_VP, _I64, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run_chain": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _I64, _VP, _VP, _SZ,
                                      _VP]),
@@ -123,6 +128,29 @@ def fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, l
 def fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes, stream):
     _check("fg8_linear_prepare", lib().fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace,
                                                           workspace_bytes, stream))
+
+
+def fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt):
+    return lib().fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt)
+
+
+def fg8_grouped_linear(x_bf16, M, K, ld_x, row_expert, E, N, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt,
+                       workspace, workspace_bytes, stream):
+    _check("fg8_grouped_linear", lib().fg8_grouped_linear(x_bf16, M, K, ld_x, row_expert, E, N, wq_e4m3, w_scale_inv,
+                                                          bias_bf16, y_bf16, ld_y, fmt, workspace, workspace_bytes,
+                                                          stream))
+
+
+def fg8_grouped_linear_prepare(x_bf16, M, K, ld_x, E, N, w_scale_inv, fmt, workspace, workspace_bytes, stream):
+    _check("fg8_grouped_linear_prepare", lib().fg8_grouped_linear_prepare(x_bf16, M, K, ld_x, E, N, w_scale_inv, fmt,
+                                                                          workspace, workspace_bytes, stream))
+
+
+def fg8_grouped_linear_run(row_expert, E, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace,
+                           workspace_bytes, stream):
+    _check("fg8_grouped_linear_run", lib().fg8_grouped_linear_run(row_expert, E, wq_e4m3, w_scale_inv, bias_bf16,
+                                                                  y_bf16, M, N, K, ld_y, fmt, workspace,
+                                                                  workspace_bytes, stream))
 
 
 def fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes, stream):

@@ -166,6 +166,42 @@ fg8_status cuda_status(cudaError_t e) {
 
 }  // namespace
 
+// x's codes and scales into the workspace in the GEMM's layouts (the
+// activation half of fg8_linear_prepare).
+fg8_status prepare_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, int fmt, uint8_t* ws,
+                       const LinearWs& L, const DeviceInfo& dev, cudaStream_t s) {
+  ActQuantArgs a{};
+  a.x = x_bf16;
+  a.ld_x = ld_x;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.Kb = ceil_div(K, kGroup);
+  a.xq = ws + L.xq_off;
+  a.xs = ws + L.xs_off;
+  a.layout = fmt == FG8_SCALE_FLOAT ? kScaleKMajor : kScaleSfTiles;
+  a.ld_s = L.ld_s;
+  a.Kq = ceil_div(a.Kb, 4);
+  a.M_pad = ceil_div(M, 128) * 128;
+  return cuda_status(launch_act_quant(a, fmt, dev.sms, s));
+}
+
+// Grouped (MoE) workspace: fg8_linear's layout for the M routed rows, with
+// the UE8M0 weight scale-factor region holding every expert's tiles -- E x
+// ceil(N/128) tiles of 128 rows, plus one spare the 256-wide tile of the
+// last expert may read past its last block.
+int64_t grouped_sf_rows(int64_t E, int64_t N) { return (E * ceil_div(N, 128) + 1) * 128; }
+
+fg8_status check_grouped_shape(int64_t M, int64_t E, int64_t N, int64_t K, int fmt) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (E <= 0 || E > 65535 || E * N + 256 > kMaxDim || E * ceil_div(N, 128) * ceil_div(K, kGroup) > kMaxDim)
+    return FG8_ERR_INVALID_ARG;
+  return FG8_OK;
+}
+
+LinearWs grouped_ws_layout(int64_t M, int64_t E, int64_t N, int64_t K, int fmt) {
+  return linear_ws_layout(M, fmt == FG8_SCALE_UE8M0 ? grouped_sf_rows(E, N) : N, K, fmt);
+}
+
 // The few-token kernel (small_m.cu) on fg8_linear's workspace: counters in
 // the header (or after the prepare layout for more than kHeaderCounters
 // weight tiles), split-K partials after the prepare layout.  fused: x is
@@ -274,6 +310,99 @@ size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt f
   return gemm_ws_layout(M, N, K, fmt).total;
 }
 
+size_t fg8_grouped_linear_workspace_bytes(int64_t M, int64_t E, int64_t N, int64_t K, fg8_scale_fmt fmt) {
+  if (check_grouped_shape(M, E, N, K, fmt) != FG8_OK) return 0;
+  return grouped_ws_layout(M, E, N, K, fmt).total;
+}
+
+fg8_status fg8_grouped_linear_prepare(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, int64_t E, int64_t N,
+                                      const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_grouped_shape(M, E, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || w_scale_inv == nullptr) return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || !aligned16(x_bf16) || !aligned16(w_scale_inv)) return FG8_ERR_ALIGNMENT;
+  const LinearWs L = grouped_ws_layout(M, E, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (fg8_status st = prepare_act(x_bf16, M, K, ld_x, fmt, ws, L, dev, s); st != FG8_OK) return st;
+  if (fmt == FG8_SCALE_UE8M0)  // every expert's [Nb][Kb] bytes as one stack of 128-row tiles
+    return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv),
+                                      static_cast<int>(E * ceil_div(N, 128) * 128), sfb_rows(grouped_sf_rows(E, N)),
+                                      128, ceil_div(K, kGroup), ws + L.wsc_off, s));
+  return FG8_OK;
+}
+
+fg8_status fg8_grouped_linear_run(const int32_t* row_expert, int64_t E, const void* wq_e4m3, const void* w_scale_inv,
+                                  const void* bias_bf16, void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
+                                  fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_grouped_shape(M, E, N, K, fmt); st != FG8_OK) return st;
+  if (ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (row_expert == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_y % 8 != 0 || !aligned16(wq_e4m3) || !aligned16(y_bf16) || (bias_bf16 != nullptr && !aligned16(bias_bf16)) ||
+      !aligned16(w_scale_inv) || (reinterpret_cast<uintptr_t>(row_expert) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  const LinearWs L = grouped_ws_layout(M, E, N, K, fmt);
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Kb = ceil_div(K, kGroup);
+  GemmArgs g{};
+  g.xq = ws + L.xq_off;
+  g.wq = wq_e4m3;
+  g.y = y_bf16;
+  g.ld_y = ld_y;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.Kb = Kb;
+  g.Kq = ceil_div(Kb, 4);
+  g.bias = bias_bf16;
+  g.status = reinterpret_cast<uint32_t*>(ws);
+  g.wait_limit_ns = g_wait_limit_ns.load();
+  g.test_stall = g_test_stall.load();
+  if (fmt == FG8_SCALE_FLOAT) {
+    g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.ld_s = L.ld_s;
+    g.w_scale = static_cast<const float*>(w_scale_inv);
+  } else {
+    g.sfa = ws + L.xs_off;
+    g.sfb = ws + L.wsc_off;
+  }
+  g.row_expert = row_expert;
+  g.E = static_cast<int>(E);
+  g.sfb_tiles = ceil_div(N, 128);
+  return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
+fg8_status fg8_grouped_linear(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, const int32_t* row_expert,
+                              int64_t E, int64_t N, const void* wq_e4m3, const void* w_scale_inv,
+                              const void* bias_bf16, void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (fg8_status st = check_grouped_shape(M, E, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || row_expert == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
+      (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv) ||
+      (reinterpret_cast<uintptr_t>(row_expert) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  if (fg8_status st = fg8_grouped_linear_prepare(x_bf16, M, K, ld_x, E, N, w_scale_inv, fmt, workspace,
+                                                 workspace_bytes, stream);
+      st != FG8_OK)
+    return st;
+  return fg8_grouped_linear_run(row_expert, E, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace,
+                                workspace_bytes, stream);
+}
+
 fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                               const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes,
                               void* stream) {
@@ -288,23 +417,10 @@ fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t 
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
-  ActQuantArgs a{};
-  a.x = x_bf16;
-  a.ld_x = ld_x;
-  a.M = static_cast<int>(M);
-  a.K = static_cast<int>(K);
-  a.Kb = Kb;
-  a.xq = ws + L.xq_off;
-  a.xs = ws + L.xs_off;
-  a.layout = fmt == FG8_SCALE_FLOAT ? kScaleKMajor : kScaleSfTiles;
-  a.ld_s = L.ld_s;
-  a.Kq = Kq;
-  a.M_pad = ceil_div(M, 128) * 128;
-  if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
+  if (fg8_status st = prepare_act(x_bf16, M, K, ld_x, fmt, ws, L, dev, s); st != FG8_OK) return st;
   if (fmt == FG8_SCALE_UE8M0)
     return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), sfb_rows(N),
-                                      128, Kb, ws + L.wsc_off, s));
+                                      128, ceil_div(K, kGroup), ws + L.wsc_off, s));
   return FG8_OK;
 }
 

@@ -87,6 +87,13 @@ struct GemmArgs {
   const void* nx_w_scale; // next layer's weight scales [ceil(N_next/128), ceil(N/128)]
   void* nx_w_prep;        // UE8M0: ... packed into scale-factor tiles (unused for float)
   int nx_N;               // N_next
+  // Optional: grouped (MoE experts) -- the expert of each row [M] (a tile
+  // computes with its first row's expert; -1 skips it); wq [E][N][K],
+  // w_scale [E][Nb][Kb], bias [E][N]; sfb holds sfb_tiles 128-row
+  // scale-factor tiles per expert.  nullptr: one weight matrix.
+  const int32_t* row_expert;
+  int E;
+  int sfb_tiles;
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM

@@ -70,7 +70,28 @@ struct KParams {
   const void* nx_w_scale;
   void* nx_w_prep;
   int nx_N;
+  // grouped (MoE experts): the expert of each row, [M]; a tile computes
+  // with the expert of its first row (-1: the tile is skipped).  Weights
+  // [E][N][K] (one tensor map over E*N rows), float scales [E][Nb][Kb],
+  // bias [E][N], UE8M0 weight scale-factor tiles sfb_tiles per expert.
+  const int32_t* row_expert;  // nullptr: a plain GEMM (expert 0)
+  int E;
+  int sfb_tiles;
 };
+
+constexpr uint32_t kStatusBadExpert = 1u;  // FG8_ERR_INVALID_ARG
+
+// Expert of the tile whose first row is m0.  An index past the last expert
+// skips the tile like -1; the producer also records it in the status word.
+__device__ __forceinline__ int tile_expert(const KParams& p, int m0, bool report) {
+  if (p.row_expert == nullptr) return 0;
+  const int e = p.row_expert[m0];
+  if (e >= p.E) {
+    if (report) atomicExch(p.status, kStatusBadExpert);
+    return -1;
+  }
+  return e;
+}
 
 template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool PAIR_ = false, bool REQUANT_ = false>
 struct Cfg {
@@ -292,6 +313,9 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int n0 = nb * C::BN;
     const int m0 = mb * C::kTileM + rank * kBlockM;  // this CTA's rows
+    const int e = tile_expert(p, mb * C::kTileM, true);
+    if (e < 0) continue;  // every role skips the same tiles
+    const int wrow0 = e * p.N + n0;  // the expert's weight rows in the [E*N, K] tensor map
     // bias of the tile (clipped to N; nothing when there is no bias)
     if (!mbar_wait(bempty + bi.slot, bi.phase ^ 1u, limit, abort_flag)) {
       raise_abort(abort_flag, p.status);
@@ -301,7 +325,9 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       const int ncols = min(C::BN, p.N - n0);
       const uint32_t bytes = p.bias != nullptr ? static_cast<uint32_t>(ncols) * 2u : 0u;
       mbar_arrive_expect_tx(bfull + bi.slot, bytes);
-      if (bytes) bulk_load(smem + C::kOffBias + bi.slot * C::kBiasSlot, p.bias + n0, bytes, bfull + bi.slot);
+      if (bytes)
+        bulk_load(smem + C::kOffBias + bi.slot * C::kBiasSlot, p.bias + static_cast<int64_t>(e) * p.N + n0, bytes,
+                  bfull + bi.slot);
       bi_par[bi.slot] = bi.phase;
       bi_issued |= 1u << bi.slot;
       bi.template advance<2>();
@@ -320,11 +346,11 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
         if (rank == 0) mbar_arrive_expect_tx(full + st.slot, C::kStageTx);
         const uint32_t bar = mapa_shared(full + st.slot, 0);
         tma_load_2d_pair(sa, tmA, bar, kb * 128, m0);
-        tma_load_2d_pair(sa + C::kA, tmB, bar, kb * 128, n0 + rank * C::kBRows);
+        tma_load_2d_pair(sa + C::kA, tmB, bar, kb * 128, wrow0 + rank * C::kBRows);
       } else {
         mbar_arrive_expect_tx(full + st.slot, C::kStageTx + (sf ? C::kSfBytes : 0));
         tma_load_2d(sa, tmA, full + st.slot, kb * 128, m0);
-        tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, n0);
+        tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, wrow0);
       }
       if (sf) {
         uint8_t* sfs = sa + C::kA + C::kB;
@@ -333,7 +359,8 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
 #pragma unroll
         for (int h = 0; h < C::BN / 128; ++h)
           bulk_load(sfs + kSfChunkBytes * (1 + h),
-                    p.sfb + (static_cast<size_t>(n0 / 128 + h) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
+                    p.sfb + (static_cast<size_t>(e * p.sfb_tiles + n0 / 128 + h) * p.Kq + (kb >> 2)) * kSfChunkBytes,
+                    kSfChunkBytes,
                     full + st.slot);
       }
       st_par[st.slot] = st.phase;
@@ -367,6 +394,11 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
+    if (p.row_expert != nullptr) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      if (tile_expert(p, mb * C::kTileM, false) < 0) continue;
+    }
     for (int kb = 0; kb < p.Kb; ++kb) {
       if (!mbar_wait(full + st.slot, st.phase, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
@@ -443,16 +475,19 @@ struct ScaleStream {
   int xoff = 0;  // row of the thread in xs_t's K-major layout
   int woff = 0;  // offset of the weight block's row in w_scale
   __device__ __forceinline__ void start(const KParams& p, int t, int sub_row, int col) {
-    tile = t;
     kb = 0;
-    if (t < p.num_tiles) {
+    for (; t < p.num_tiles; t += tile_stride<C>()) {  // the next tile that is not skipped
       int mb, nb;
       tile_coords(t, p.num_m, p.num_n, mb, nb);
+      const int e = tile_expert(p, mb * C::kTileM, false);
+      if (e < 0) continue;
       xoff = mb * C::kTileM + sub_row;
       // a column block past N (ragged last tile) reads the last block: its
       // columns are never stored
-      woff = min((nb * C::BN + col) / 128, p.Nb - 1) * p.Kb;
+      woff = (e * p.Nb + min((nb * C::BN + col) / 128, p.Nb - 1)) * p.Kb;
+      break;
     }
+    tile = t;
   }
   // {sx, sw} of the next (tile, K-block), or zeros past the end of the walk.
   __device__ __forceinline__ float2 next(const KParams& p, int sub_row, int col) {
@@ -493,6 +528,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    if (tile_expert(p, mb * C::kTileM, false) < 0) continue;
     const int row0 = mb * C::kTileM + rank * kBlockM + q * 32;
     // the tile's bias (bias ring; zeros past N or without bias)
     if (!mbar_wait_warp(bfull + bi.slot, bi.phase, limit, abort_flag)) {
@@ -774,7 +810,8 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K, g.M, g.K, 128, kBlockM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K, g.N, g.K, 128, C::kBRows,
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K,
+                    static_cast<uint64_t>(g.N) * (g.row_expert != nullptr ? g.E : 1), g.K, 128, C::kBRows,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, static_cast<uint64_t>(g.ld_y) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
@@ -806,6 +843,9 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.nx_w_scale = g.nx_w_scale;
   p.nx_w_prep = g.nx_w_prep;
   p.nx_N = g.nx_N;
+  p.row_expert = g.row_expert;
+  p.E = g.row_expert != nullptr ? g.E : 1;
+  p.sfb_tiles = g.sfb_tiles;
   if (p.num_tiles == 0) return cudaSuccess;
 
   static int configured_device = -1;

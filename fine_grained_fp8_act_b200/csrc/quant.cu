@@ -198,18 +198,35 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const uint16_t* __res
 }
 
 // --------------------------------------------------------------- sf pack ----
+// One thread per 16-byte chunk of a scale-factor tile: chunk i of tile
+// (rows 128 t.., K-blocks 4 q..) holds the words of rows 128 t + 32 c + i,
+// c = 0..3, byte j of each being K-block 4 q + j (sf_tile_offset's layout).
+// Rows past R and K-blocks past Kb get 127 (2^0, never applied to data).
 __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict__ src, const int R, const int row_div,
-                                                      const int Kb, const int Kq, const int64_t total,
+                                                      const int Kb, const int Kq, const int64_t chunks,
                                                       uint8_t* __restrict__ dst) {
   grid_wait_prerequisites();
   grid_launch_dependents();
-  const int cols = Kq * 4;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / cols;
-    const int kb = static_cast<int>(i % cols);
-    const uint8_t b = (r < R && kb < Kb) ? src[(r / row_div) * Kb + kb] : static_cast<uint8_t>(127);
-    dst[sf_tile_offset(r, kb, Kq)] = b;
+    const int64_t tq = i >> 5;  // (tile, K-group) index: tile * Kq + q
+    const int lane = static_cast<int>(i & 31);
+    const int64_t tile = tq / Kq;
+    const int q = static_cast<int>(tq - tile * Kq);
+    uint32_t w[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t r = tile * 128 + c * 32 + lane;
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kb = 4 * q + j;
+        const uint32_t b = (r < R && kb < Kb) ? src[(r / row_div) * Kb + kb] : 127u;
+        v |= b << (8 * j);
+      }
+      w[c] = v;
+    }
+    *reinterpret_cast<uint4*>(dst + tq * kSfChunkBytes + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -286,9 +303,9 @@ cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div
                            cudaStream_t s) {
   const int Kq = (Kb + 3) / 4;
   if (R_pad % 128 != 0 || R_pad < R) return cudaErrorInvalidValue;
-  const int64_t total = R_pad * Kq * 4;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > 4096) blocks = 4096;
+  const int64_t chunks = R_pad / 128 * Kq * 32;  // 16-byte chunks, 32 per 512-byte tile
+  int64_t blocks = (chunks + 255) / 256;
+  if (blocks > 8192) blocks = 8192;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -298,7 +315,7 @@ cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_pack_kernel, src, R, row_div, Kb, Kq, total, dst);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_pack_kernel, src, R, row_div, Kb, Kq, chunks, dst);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

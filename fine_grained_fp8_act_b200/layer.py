@@ -112,6 +112,32 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: O
     return y
 
 
+def grouped_linear(x: torch.Tensor, row_expert: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor,
+                   bias: Optional[torch.Tensor] = None, scale_fmt="ue8m0", out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """MoE expert layer over the contiguous grouped layout: x [M, K] bf16 routed
+    rows sorted by expert (runs padded to 128-row blocks), row_expert [M]
+    int32 (block t uses row_expert[128 t]; -1 skips it), wq [E, N, K],
+    w_scale_inv [E, ceil(N/128), ceil(K/128)], bias [E, N] or None.  Rows of
+    skipped blocks of the returned y are left as allocated."""
+    fmt = scale_fmt_code(scale_fmt)
+    _check_bf16_matrix(x, "x")
+    M, K = x.shape
+    if wq.dim() != 3 or wq.shape[2] != K:
+        raise ValueError("wq must be [E, N, K]")
+    E, N = int(wq.shape[0]), int(wq.shape[1])
+    if row_expert.dtype != torch.int32 or row_expert.shape != (M,) or row_expert.device != x.device:
+        raise ValueError("row_expert must be int32 [M] on x's device")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(C.fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt), x.device, workspace)
+    with torch.cuda.device(x.device):
+        C.fg8_grouped_linear(x.data_ptr(), M, K, x.stride(0), row_expert.contiguous().data_ptr(), E, N,
+                             wq.data_ptr(), w_scale_inv.data_ptr(), 0 if bias is None else bias.data_ptr(),
+                             y.data_ptr(), y.stride(0), fmt, ws.data_ptr(), ws.numel() * ws.element_size(),
+                             _stream(x))
+    return y
+
+
 def linear_static(x: torch.Tensor, act_scale: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor,
                   bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -211,6 +211,49 @@ FG8_API fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, i
                                      const void* bias_bf16, void* y_bf16, int64_t ld_y, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* MoE experts ([zh] §6.4 and [pt] "Caminho rápido do DeepGEMM": FP8Experts
+ * sends each expert's tokens through this layer with that expert's e4m3
+ * weights and block scales; on Blackwell the expert kernels take UE8M0
+ * scales, float32 scales being the grouped_mm alternative -- both work here).
+ * The pages print no kernel interface; the layout taken is the contiguous
+ * grouped one: the routed rows of x are sorted by expert and each expert's
+ * run is padded to whole blocks of 128 rows.
+ *   x_bf16       [M, K] bf16, row stride ld_x: the routed rows
+ *   row_expert   [M] int32 (device, 4-byte aligned): block t = rows
+ *                [128 t, 128 t + 128) is computed with expert
+ *                row_expert[128 t]; -1 there skips the block (its y rows are
+ *                not written).  The other rows' entries are not read (padding
+ *                rows inside a computed block are computed with it).  An
+ *                entry >= E also skips its block and leaves
+ *                FG8_ERR_INVALID_ARG in the workspace's status word.
+ *   wq_e4m3      [E, N, K] e4m3fn (expert e's [N, K] matrix at e*N*K bytes)
+ *   w_scale_inv  [E, ceil(N/128), ceil(K/128)] float32 or UE8M0 bytes
+ *   bias_bf16    [E, N] bf16 or NULL
+ *   y_bf16       [M, N] bf16, row stride ld_y
+ *   workspace    >= fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt),
+ *                with the header rules of fg8_linear
+ * y[r] = fg8_linear of row r with expert e's weights, bit for bit the dense
+ * layer's arithmetic (per-token activation groups, exact float scale
+ * promotion or the block-scaled MMA for UE8M0).  Checks as fg8_linear, plus
+ * 1 <= E <= 65535 and E*N + 256 <= 2^31 - 1. */
+FG8_API size_t fg8_grouped_linear_workspace_bytes(int64_t M, int64_t E, int64_t N, int64_t K, fg8_scale_fmt fmt);
+FG8_API fg8_status fg8_grouped_linear(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                                      const int32_t* row_expert, int64_t E, int64_t N, const void* wq_e4m3,
+                                      const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y,
+                                      fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream);
+/* fg8_grouped_linear in two halves (as fg8_linear_prepare / fg8_linear_run):
+ * the prepare step quantizes x into the workspace (and, for UE8M0, packs
+ * every expert's weight scales into scale-factor tiles); the run step is
+ * the grouped GEMM.  prepare then run on one stream and workspace is
+ * fg8_grouped_linear, bit for bit.  Arguments and checks as there. */
+FG8_API fg8_status fg8_grouped_linear_prepare(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, int64_t E,
+                                              int64_t N, const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+FG8_API fg8_status fg8_grouped_linear_run(const int32_t* row_expert, int64_t E, const void* wq_e4m3,
+                                          const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t M,
+                                          int64_t N, int64_t K, int64_t ld_y, fg8_scale_fmt fmt, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
 /* Fp8Dequantize ([zh] §五 and §八 step 4: a pre-quantized checkpoint loaded
  * with dequantize=True folds each block's scale back into the weight):
  *   w[n, k] = bf16(value(wq[n, k]) * w_scale_inv[n / 128][k / 128]),
@@ -233,9 +276,10 @@ FG8_API fg8_status fg8_scale_to_ue8m0(const void* scale_f32, int64_t n, void* sc
                                       void* stream);
 
 /* Synchronizes `stream`, reads and clears the status word a previous
- * fg8_linear / fg8_gemm_prequant left in `workspace`: FG8_OK, or
- * FG8_ERR_TIMEOUT if one of its device-side waits gave up (the kernel then
- * returned early; y is unspecified). */
+ * fg8_linear / fg8_gemm_prequant / fg8_grouped_linear left in `workspace`:
+ * FG8_OK; FG8_ERR_TIMEOUT if one of its device-side waits gave up (the
+ * kernel then returned early; y is unspecified); FG8_ERR_INVALID_ARG if
+ * fg8_grouped_linear met an expert index >= E (those blocks were skipped). */
 FG8_API fg8_status fg8_check_device_status(void* workspace, void* stream);
 
 /* Upper bound, in nanoseconds, on any single device-side wait of the GEMM

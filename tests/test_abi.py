@@ -193,3 +193,28 @@ def test_scale_fmt_validation(fg8):
     for bad in ("Float", "e8m0", "fp32", 3, None):
         with pytest.raises(ValueError):
             scale_fmt_code(bad)
+
+
+def test_grouped_rejects_bad_args(fg8):
+    raw = _raw(fg8)
+    big = 1 << 40
+    args = lambda **kw: [kw.get(k, v) for k, v in (
+        ("x", FAKE), ("M", 256), ("K", 256), ("ld_x", 256), ("re", FAKE), ("E", 4), ("N", 256), ("wq", FAKE),
+        ("ws", FAKE), ("b", None), ("y", FAKE), ("ld_y", 256), ("fmt", 1), ("wsp", FAKE * 16), ("nb", big),
+        ("s", None))]
+    g = raw.fg8_grouped_linear
+    assert g(*args(E=0)) == 1
+    assert g(*args(E=70000)) == 1
+    assert g(*args(E=1 << 20, N=4096)) == 1      # E * N past 2^31
+    assert g(*args(fmt=2)) == 1
+    assert g(*args(re=None)) == 1
+    assert g(*args(K=200, ld_x=200)) == 2        # K % 16
+    assert g(*args(N=260, ld_y=264)) == 2        # N % 8
+    assert g(*args(re=FAKE + 2)) == 2            # int32 alignment
+    assert g(*args(nb=1024)) == 4                # workspace too small
+    assert g(*args(M=0, x=None, re=None, y=None)) == 0
+    f = raw.fg8_grouped_linear_workspace_bytes
+    # UE8M0: the weight scale-factor region holds every expert's 128-row tiles
+    assert f(256, 8, 256, 1024, 1) > f(256, 1, 256, 1024, 1) + 7 * 2 * 2 * 512 - 256
+    assert f(256, 8, 256, 1024, 0) == fg8.fg8_linear_workspace_bytes(256, 256, 1024, 0)
+    assert f(256, 0, 256, 1024, 0) == 0

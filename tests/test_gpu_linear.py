@@ -40,7 +40,7 @@ def check_y(y_gpu_bits, y64, bound, what=""):
     got = _as_f64(y_gpu_bits)
     err = np.abs(got - y64)
     tol = y_tolerance(bound)
-    bad = err > tol
+    bad = ~(err <= tol)  # NaN counts as out of tolerance
     if bad.any():
         i = tuple(np.argwhere(bad)[0])
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; first {i}: "

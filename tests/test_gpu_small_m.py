@@ -39,7 +39,7 @@ def _check(orc, x, w, b, y, fmt):
     y64, bound, _ = orc.linear(_bits(x), owq, ows, None if b is None else _bits(b), fmt)
     err = np.abs(_as_f64(_bits(y)) - y64)
     tol = y_tolerance(bound)
-    bad = err > tol
+    bad = ~(err <= tol)  # NaN counts as out of tolerance
     assert not bad.any(), f"{bad.sum()} of {bad.size} elements out of tolerance; worst {(err - tol).max()}"
 
 

@@ -140,7 +140,7 @@ def make_inputs(cfg: str, gemm: Gemm, device="cpu", stage: int = 1) -> Tuple[tor
 # 256 experts, 8 per token); the expert kernels take UE8M0 scales on
 # Blackwell.  gate/up: K = 7168 -> N = 2 x 2048; down: K = 2048 -> N = 7168.
 MOE_BLOCK = 128
-DSV3_MOE = dict(experts=256, topk=8, hidden=7168, inter=2048, tokens=4096)
+DSV3_MOE = dict(experts=256, topk=8, hidden=7168, inter=2048, tokens=4096, skew=0.5)
 
 
 def moe_routing(T: int, E: int, topk: int, seed: int, skew: float = 1.0):
