@@ -132,3 +132,36 @@ def test_layer_wrapper(fg8, orc):
     assert st == 0
     written = _check(orc, x, re, wq, ws, b, y2, UE8M0)
     assert torch.equal(y[torch.from_numpy(written).cuda()], y2[torch.from_numpy(written).cuda()])
+
+
+def test_moe_full_size_sampled(fg8, orc):
+    """The bench's MoE gate/up layer at full size (4096 tokens x top-8 on 256
+    experts, K = 7168 -> N = 4096, UE8M0) in the bench's launch
+    configuration; sampled rows of several blocks (first, middle, last routed
+    row) checked on every column against the oracle with the block's expert."""
+    c = W.DSV3_MOE
+    E, K, N = c["experts"], c["hidden"], 2 * c["inter"]
+    rt, re = W.moe_routing(c["tokens"], E, c["topk"], seed=5, skew=c["skew"])
+    x = W.gather_rows(W.x_student_t(c["tokens"], K, seed=50, device="cuda"), rt)
+    M = x.shape[0]
+    wq = torch.empty(E, N, K, dtype=torch.float8_e4m3fn, device="cuda")
+    ws = torch.empty(E, N // 128, K // 128, dtype=torch.float8_e8m0fnu, device="cuda")
+    for e in range(E):
+        q, s = fg8.quantize_weight(W.w_row_groups(N, K, 0.015, seed=1000 + e, device="cuda"), UE8M0)
+        wq[e] = q
+        ws[e] = s
+    re_d = re.cuda()
+    y, st = _run(fg8, x, re_d, wq, ws, None, UE8M0)
+    assert st == 0
+    blocks = M // 128
+    heads = re.view(-1, 128)[:, 0]
+    for t in sorted({0, 1, blocks // 2, blocks - 1}):
+        e = int(heads[t])
+        real = (re[t * 128:(t + 1) * 128] >= 0).nonzero().flatten()
+        rows = t * 128 + torch.unique(torch.stack([real[0], real[len(real) // 2], real[-1]]))
+        xb = W.bf16_bits(x[rows])
+        y64, bound, _, written = orc.grouped_linear(xb, np.zeros(len(rows), np.int32), _u8(wq[e:e + 1]),
+                                                    _u8(ws[e:e + 1]), None, UE8M0)
+        yg = (W.bf16_bits(y[rows]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        err = np.abs(yg - y64)
+        assert written.all() and (err <= y_tolerance(bound)).all(), f"block {t} (expert {e})"
