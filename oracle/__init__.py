@@ -54,6 +54,16 @@ def lib():
             f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                           ctypes.c_void_p, ctypes.c_void_p]
         L.orc_linear_dequant.restype = ctypes.c_int
+        for name in ("orc_quantize_act_g", "orc_quantize_weight_b"):
+            f = getattr(L, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                          ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        L.orc_linear_dequant_b.restype = ctypes.c_int
+        L.orc_linear_dequant_b.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.orc_dequantize_weight.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_int, ctypes.c_void_p, ctypes.c_int64]
         L.orc_dequantize_weight.restype = ctypes.c_int
@@ -72,6 +82,10 @@ def lib():
 
 def _ptr(a):
     return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _nb(k, block):
+    return -(-k // block)
 
 
 def _kb(k):
@@ -115,13 +129,17 @@ def bf16_from_double(v: float) -> int:
 
 
 # ------------------------------------------------------------- quantizers --
-def quantize_act(x_bf16: np.ndarray, fmt: int):
-    """x bf16 bits [M, K] -> (xq e4m3 [M, K], x_scale [M, ceil(K/128)] float32|uint8)."""
+def quantize_act(x_bf16: np.ndarray, fmt: int, block: int = GROUP):
+    """x bf16 bits [M, K] -> (xq e4m3 [M, K], x_scale [M, ceil(K/block)] float32|uint8).
+
+    block: the group width (the weight block's input-channel size; 128 by
+    default, [zh] §一; other block sizes such as (32, 32) are tested
+    configurations on the pages, [zh] §八)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     M, K = x.shape
     xq = np.empty((M, K), dtype=np.uint8)
-    xs = np.empty((M, _kb(K)), dtype=_scale_dtype(fmt))
-    rc = lib().orc_quantize_act(_ptr(x), M, K, K, fmt, _ptr(xq), _ptr(xs))
+    xs = np.empty((M, _nb(K, block)), dtype=_scale_dtype(fmt))
+    rc = lib().orc_quantize_act_g(_ptr(x), M, K, K, fmt, block, _ptr(xq), _ptr(xs))
     if rc != 0:
         raise ValueError("orc_quantize_act: bad argument")
     return xq, xs
@@ -138,19 +156,20 @@ def quantize_act_static(x_bf16: np.ndarray, scale: float):
     return xq, np.full((M, _kb(K)), np.float32(scale), dtype=np.float32)
 
 
-def quantize_weight(w_bf16: np.ndarray, fmt: int):
-    """W bf16 bits [N, K] -> (wq e4m3 [N, K], w_scale_inv [ceil(N/128), ceil(K/128)])."""
+def quantize_weight(w_bf16: np.ndarray, fmt: int, block: int = GROUP):
+    """W bf16 bits [N, K] -> (wq e4m3 [N, K], w_scale_inv [ceil(N/block), ceil(K/block)]);
+    block x block weight blocks (128 by default)."""
     w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
     N, K = w.shape
     wq = np.empty((N, K), dtype=np.uint8)
-    ws = np.empty((_kb(N), _kb(K)), dtype=_scale_dtype(fmt))
-    rc = lib().orc_quantize_weight(_ptr(w), N, K, K, fmt, _ptr(wq), _ptr(ws))
+    ws = np.empty((_nb(N, block), _nb(K, block)), dtype=_scale_dtype(fmt))
+    rc = lib().orc_quantize_weight_b(_ptr(w), N, K, K, fmt, block, _ptr(wq), _ptr(ws))
     if rc != 0:
         raise ValueError("orc_quantize_weight: bad argument")
     return wq, ws
 
 
-def linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows=None):
+def linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows=None, block: int = GROUP):
     """Reference y for quantized operands.
 
     Returns (y64 [R, N] float64, bound [R, N] float64, y_bf16 [R, N] uint16),
@@ -164,7 +183,7 @@ def linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows=None):
     N, K2 = wq.shape
     if K2 != K:
         raise ValueError("K mismatch")
-    if xs.shape != (M, _kb(K)) or ws.shape != (_kb(N), _kb(K)):
+    if xs.shape != (M, _nb(K, block)) or ws.shape != (_nb(N, block), _nb(K, block)):
         raise ValueError("scale shape mismatch")
     b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
     if b is not None and b.shape != (N,):
@@ -174,17 +193,18 @@ def linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows=None):
     y64 = np.empty((R, N), dtype=np.float64)
     bound = np.empty((R, N), dtype=np.float64)
     ybf = np.empty((R, N), dtype=np.uint16)
-    rc = lib().orc_linear_dequant(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(b), M, N, K, fmt,
-                                  _ptr(r), 0 if r is None else r.size, _ptr(y64), _ptr(bound), _ptr(ybf))
+    rc = lib().orc_linear_dequant_b(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(b), M, N, K, fmt, block,
+                                    _ptr(r), 0 if r is None else r.size, _ptr(y64), _ptr(bound), _ptr(ybf))
     if rc != 0:
         raise ValueError("orc_linear_dequant: bad argument")
     return y64, bound, ybf
 
 
-def linear(x_bf16, wq, ws, bias_bf16, fmt, rows=None):
-    """Whole layer: quantize x per token, then linear_dequant."""
-    xq, xs = quantize_act(x_bf16, fmt)
-    return linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows)
+def linear(x_bf16, wq, ws, bias_bf16, fmt, rows=None, block: int = GROUP):
+    """Whole layer: quantize x per token (1 x block groups), then linear_dequant
+    with block x block weight blocks."""
+    xq, xs = quantize_act(x_bf16, fmt, block)
+    return linear_dequant(xq, xs, wq, ws, bias_bf16, fmt, rows, block)
 
 
 # ------------------------------------------------------ MoE experts ------

@@ -180,22 +180,24 @@ void orc_e4m3_encode_many(const float* f, int64_t n, uint8_t* out) {
 }
 
 // Dynamic per-token activation quantization ([zh] §一, [pt]): token row m is
-// split into groups of 128 consecutive input channels (the last group holds
-// K mod 128 real channels); each group gets one scale from its own amax and
-// its elements are cast to e4m3fn.
+// split into groups of `group` consecutive input channels (128 by default; the
+// weight block's input-channel size, so (32, 32) blocks give 1x32 groups --
+// [zh] §八 lists such non-default block sizes among the tested ones); the last
+// group holds the remaining real channels; each group gets one scale from its
+// own amax and its elements are cast to e4m3fn.
 //   x      : bf16 bits, row m at x + m*ld_x
 //   xq     : e4m3fn bytes [M, K] row-major
-//   x_scale: [M, ceil(K/128)] row-major; float32 (fmt 0) or UE8M0 bytes (fmt 1)
+//   x_scale: [M, ceil(K/group)] row-major; float32 (fmt 0) or UE8M0 bytes (fmt 1)
 // Returns 0, or -1 on a bad argument.
-int orc_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, int fmt,
-                     uint8_t* xq, void* x_scale) {
-  if (M < 0 || K <= 0 || ld_x < K || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
-  const int Kb = ceil_div(K, kGroup);
+int orc_quantize_act_g(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, int fmt, int group,
+                       uint8_t* xq, void* x_scale) {
+  if (M < 0 || K <= 0 || ld_x < K || group <= 0 || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
+  const int Kb = ceil_div(K, group);
 #pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
     for (int g = 0; g < Kb; ++g) {
-      const int64_t k0 = static_cast<int64_t>(g) * kGroup;
-      const int64_t k1 = std::min<int64_t>(k0 + kGroup, K);
+      const int64_t k0 = static_cast<int64_t>(g) * group;
+      const int64_t k1 = std::min<int64_t>(k0 + group, K);
       float amax = 0.0f;
       for (int64_t k = k0; k < k1; ++k) amax = std::fmax(amax, std::fabs(bf16_to_float(x[m * ld_x + k])));
       const float s = group_scale(amax);
@@ -217,20 +219,25 @@ int orc_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, int 
   return 0;
 }
 
-// 2-D block weight quantization ([zh] §一: one scale per 128x128 sub-matrix,
-// weight_scale_inv shaped (ceil(out/128), ceil(in/128)); [zh] §三: bias is not
+int orc_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, int fmt, uint8_t* xq, void* x_scale) {
+  return orc_quantize_act_g(x, M, K, ld_x, fmt, kGroup, xq, x_scale);
+}
+
+// 2-D block weight quantization ([zh] §一: one scale per block x block
+// sub-matrix, 128 by default, weight_scale_inv shaped (ceil(out/block),
+// ceil(in/block)); [zh] §三: bias is not
 // quantized).  W is nn.Linear's [out=N, in=K].  Edge blocks use their real
 // elements only.  W ~= dequant(wq) = value(wq) * scale_inv.
-int orc_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ld_w, int fmt,
-                        uint8_t* wq, void* w_scale_inv) {
-  if (N <= 0 || K <= 0 || ld_w < K || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
-  const int Nb = ceil_div(N, kBlock);
-  const int Kb = ceil_div(K, kBlock);
+int orc_quantize_weight_b(const uint16_t* w, int64_t N, int64_t K, int64_t ld_w, int fmt, int block,
+                          uint8_t* wq, void* w_scale_inv) {
+  if (N <= 0 || K <= 0 || ld_w < K || block <= 0 || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
+  const int Nb = ceil_div(N, block);
+  const int Kb = ceil_div(K, block);
 #pragma omp parallel for collapse(2) schedule(static)
   for (int nb = 0; nb < Nb; ++nb) {
     for (int kb = 0; kb < Kb; ++kb) {
-      const int64_t n0 = static_cast<int64_t>(nb) * kBlock, n1 = std::min<int64_t>(n0 + kBlock, N);
-      const int64_t k0 = static_cast<int64_t>(kb) * kBlock, k1 = std::min<int64_t>(k0 + kBlock, K);
+      const int64_t n0 = static_cast<int64_t>(nb) * block, n1 = std::min<int64_t>(n0 + block, N);
+      const int64_t k0 = static_cast<int64_t>(kb) * block, k1 = std::min<int64_t>(k0 + block, K);
       float amax = 0.0f;
       for (int64_t n = n0; n < n1; ++n)
         for (int64_t k = k0; k < k1; ++k) amax = std::fmax(amax, std::fabs(bf16_to_float(w[n * ld_w + k])));
@@ -251,19 +258,24 @@ int orc_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ld_w, i
   return 0;
 }
 
+int orc_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ld_w, int fmt, uint8_t* wq,
+                        void* w_scale_inv) {
+  return orc_quantize_weight_b(w, N, K, ld_w, fmt, kBlock, wq, w_scale_inv);
+}
+
 // The linear layer on quantized operands ([zh] §八 step 6: FP8Linear.forward
 // hands quantized weights to fp8_linear):
 //   y[m,n] = sum_k xhat[m,k] * what[n,k] + bias[n],
-//   xhat = value(xq) * x_scale(m, k/128),  what = value(wq) * w_scale_inv(n/128, k/128),
+//   xhat = value(xq) * x_scale(m, k/block),  what = value(wq) * w_scale_inv(n/block, k/block),
 // summed in double in increasing k; bias (bf16, may be NULL) added in double.
 // Outputs, for each requested row (rows == NULL means all M rows, in order):
 //   y64   [R, N] the double result, bound [R, N] = sum_k |xhat*what|,
 //   y_bf16[R, N] the double result rounded once to bf16 (RNE).
-int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq, const void* w_scale_inv,
-                       const uint16_t* bias, int64_t M, int64_t N, int64_t K, int fmt,
-                       const int64_t* rows, int64_t n_rows, double* y64, double* bound, uint16_t* y_bf16) {
-  if (M < 0 || N <= 0 || K <= 0 || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
-  const int Kb = ceil_div(K, kBlock);
+int orc_linear_dequant_b(const uint8_t* xq, const void* x_scale, const uint8_t* wq, const void* w_scale_inv,
+                         const uint16_t* bias, int64_t M, int64_t N, int64_t K, int fmt, int block,
+                         const int64_t* rows, int64_t n_rows, double* y64, double* bound, uint16_t* y_bf16) {
+  if (M < 0 || N <= 0 || K <= 0 || block <= 0 || (fmt != ORC_FMT_FLOAT && fmt != ORC_FMT_UE8M0)) return -1;
+  const int Kb = ceil_div(K, block);
   const int64_t R = rows ? n_rows : M;
   auto xs_at = [&](int64_t m, int64_t g) -> double {
     return fmt == ORC_FMT_FLOAT ? static_cast<double>(static_cast<const float*>(x_scale)[m * Kb + g])
@@ -277,7 +289,7 @@ int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq
   std::vector<double> what(static_cast<size_t>(N * K));
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n)
-    for (int64_t k = 0; k < K; ++k) what[n * K + k] = e4m3_signed(wq[n * K + k]) * ws_at(n / kBlock, k / kBlock);
+    for (int64_t k = 0; k < K; ++k) what[n * K + k] = e4m3_signed(wq[n * K + k]) * ws_at(n / block, k / block);
 
   for (int64_t r = 0; r < R; ++r) {
     const int64_t m = rows ? rows[r] : r;
@@ -287,7 +299,7 @@ int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq
   for (int64_t r = 0; r < R; ++r) {
     const int64_t m = rows ? rows[r] : r;
     std::vector<double> xhat(static_cast<size_t>(K));
-    for (int64_t k = 0; k < K; ++k) xhat[k] = e4m3_signed(xq[m * K + k]) * xs_at(m, k / kGroup);
+    for (int64_t k = 0; k < K; ++k) xhat[k] = e4m3_signed(xq[m * K + k]) * xs_at(m, k / block);
     for (int64_t n = 0; n < N; ++n) {
       double acc = 0.0, mag = 0.0;
       const double* wr = &what[n * K];
@@ -303,6 +315,13 @@ int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq
     }
   }
   return 0;
+}
+
+int orc_linear_dequant(const uint8_t* xq, const void* x_scale, const uint8_t* wq, const void* w_scale_inv,
+                       const uint16_t* bias, int64_t M, int64_t N, int64_t K, int fmt, const int64_t* rows,
+                       int64_t n_rows, double* y64, double* bound, uint16_t* y_bf16) {
+  return orc_linear_dequant_b(xq, x_scale, wq, w_scale_inv, bias, M, N, K, fmt, kBlock, rows, n_rows, y64, bound,
+                              y_bf16);
 }
 
 // Fp8Dequantize ([zh] §五 and §八 step 4: a pre-quantized checkpoint loaded

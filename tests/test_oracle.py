@@ -298,7 +298,7 @@ def test_quantize_weight_blocks(orc, fmt, N, K):
 
 
 # ---------------------------------------------------------------- GEMM --
-def exact_linear(xq, xs, wq, ws, bias_bits, fmt):
+def exact_linear(xq, xs, wq, ws, bias_bits, fmt, block=128):
     """y[m,n] = sum_k xhat*what + bias as exact rationals (PyTorch decode of codes)."""
     t = torch_e4m3_table()
     M, K = xq.shape
@@ -307,8 +307,8 @@ def exact_linear(xq, xs, wq, ws, bias_bits, fmt):
     def sc(v):
         return Fraction(float(np.float32(v))) if fmt == FLOAT else e8m0_value_exact(v)
 
-    xh = [[Fraction(float(t[xq[m, k]])) * sc(xs[m, k // 128]) for k in range(K)] for m in range(M)]
-    wh = [[Fraction(float(t[wq[n, k]])) * sc(ws[n // 128, k // 128]) for k in range(K)] for n in range(N)]
+    xh = [[Fraction(float(t[xq[m, k]])) * sc(xs[m, k // block]) for k in range(K)] for m in range(M)]
+    wh = [[Fraction(float(t[wq[n, k]])) * sc(ws[n // block, k // block]) for k in range(K)] for n in range(N)]
     bias = None
     if bias_bits is not None:
         bias = (bias_bits.astype(np.uint32) << 16).view(np.float32)
@@ -650,3 +650,92 @@ def test_grouped_linear_rejects_unknown_expert(orc):
     ws = np.ones((2, 1, 1), np.float32)
     with pytest.raises(ValueError):
         orc.grouped_linear(x, np.full(128, 2, np.int32), wq, ws, None, FLOAT)
+
+
+# --------------------------------------------- non-default block size 32 --
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,K", [(3, 256), (2, 80), (1, 48)])
+def test_quantize_act_groups_block32(orc, fmt, M, K):
+    """1 x 32 groups (weight_block_size = (32, 32)): each group's scale from its
+    own 32 channels (a 16-wide last group from its 16), codes by brute force."""
+    g = torch.Generator().manual_seed(7 * M + K)
+    x = torch.randn(M, K, generator=g)
+    for j in range(-(-K // 32)):  # very different magnitudes per group: a wrong group index shows
+        x[:, 32 * j:32 * j + 32] *= 2.0 ** (3 * (j % 5) - 6)
+    x = x.to(torch.bfloat16)
+    xq, xs = orc.quantize_act(_bf16_bits(x), fmt, 32)
+    assert xs.shape == (M, -(-K // 32))
+    xf = x.float().numpy()
+    for m in range(M):
+        for j in range(-(-K // 32)):
+            k0, k1 = 32 * j, min(32 * j + 32, K)
+            _check_group(orc, xf[m, k0:k1], xq[m, k0:k1], xs[m, j], fmt)
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("N,K", [(64, 64), (40, 80), (96, 48)])
+def test_quantize_weight_blocks_block32(orc, fmt, N, K):
+    g = torch.Generator().manual_seed(N + 3 * K)
+    w = torch.randn(N, K, generator=g) * 0.02
+    Nb, Kb = -(-N // 32), -(-K // 32)
+    for nb in range(Nb):
+        for kb in range(Kb):
+            w[32 * nb:32 * nb + 32, 32 * kb:32 * kb + 32] *= 2.0 ** (3 * nb - 2 * kb)
+    w = w.to(torch.bfloat16)
+    wq, ws = orc.quantize_weight(_bf16_bits(w), fmt, 32)
+    assert ws.shape == (Nb, Kb)
+    wf = w.float().numpy()
+    for nb in range(Nb):
+        for kb in range(Kb):
+            blk = wf[32 * nb:min(32 * nb + 32, N), 32 * kb:min(32 * kb + 32, K)]
+            q = wq[32 * nb:min(32 * nb + 32, N), 32 * kb:min(32 * kb + 32, K)]
+            _check_group(orc, blk.ravel(), q.ravel(), ws[nb, kb], fmt)
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(2, 3, 80), (1, 40, 64), (3, 5, 48)])
+def test_linear_vs_exact_rationals_block32(orc, fmt, M, N, K):
+    g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
+    x = torch.randn(M, K, generator=g)
+    w = torch.randn(N, K, generator=g) * 0.02
+    for j in range(-(-K // 32)):  # scales that differ by group, so a k / 128 index would show
+        x[:, 32 * j:32 * j + 32] *= 2.0 ** (2 * j - 3)
+        w[:, 32 * j:32 * j + 32] *= 2.0 ** (1 - j)
+    xb, wb = _bf16_bits(x.to(torch.bfloat16)), _bf16_bits(w.to(torch.bfloat16))
+    bb = _bf16_bits((torch.randn(N, generator=g) * 0.1).to(torch.bfloat16))
+    xq, xs = orc.quantize_act(xb, fmt, 32)
+    wq, ws = orc.quantize_weight(wb, fmt, 32)
+    y64, bound, ybf = orc.linear_dequant(xq, xs, wq, ws, bb, fmt, block=32)
+    ye, be = exact_linear(xq, xs, wq, ws, bb, fmt, block=32)
+    gamma = K * 2.0 ** -52
+    for m in range(M):
+        for n in range(N):
+            assert abs(Fraction(y64[m, n]) - ye[m][n]) <= Fraction(gamma) * be[m][n] + Fraction(1, 2 ** 1074)
+            assert ybf[m, n] == frac_bf16_rne(Fraction(y64[m, n]))
+    y2 = orc.linear(xb, wq, ws, bb, fmt, block=32)[0]
+    assert np.array_equal(y2, y64)
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+def test_block32_equals_block128_when_scales_coincide(orc, fmt):
+    """When every 32-group of a 128-group (and every 32 x 32 block of a
+    128 x 128 block) has the same amax, the scales coincide and so do the
+    codes and y: block 32 reduces to the default layer."""
+    rng = np.random.default_rng(9)
+    M, N, K = 3, 136, 256
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    x = np.clip(x, -3.0, 3.0)
+    x[:, ::32] = 3.0                 # each 32-group holds the row's amax
+    w = np.clip(w, -0.05, 0.05)
+    for n0 in range(0, N, 32):       # each 32 x 32 block holds its 128 x 128 block's amax
+        w[n0, ::32] = 0.0625
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    wb = (w.view(np.uint32) >> 16).astype(np.uint16)
+    b = (rng.normal(0, 0.1, N).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    q32, s32 = orc.quantize_weight(wb, fmt, 32)
+    q128, s128 = orc.quantize_weight(wb, fmt)
+    assert np.array_equal(q32, q128)
+    y32 = orc.linear(xb, q32, s32, b, fmt, block=32)[0]
+    y128 = orc.linear(xb, q128, s128, b, fmt)[0]
+    assert np.array_equal(y32, y128)
