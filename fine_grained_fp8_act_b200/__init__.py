@@ -32,6 +32,8 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_grouped_linear_run,
     fg8_grouped_linear_workspace_bytes,
     fg8_linear,
+    fg8_linear_block,
+    fg8_linear_block_workspace_bytes,
     fg8_linear_noalloc,
     fg8_linear_prepare,
     fg8_linear_run,
@@ -39,8 +41,10 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear_static,
     fg8_linear_workspace_bytes,
     fg8_quantize_act,
+    fg8_quantize_act_block,
     fg8_quantize_act_static,
     fg8_quantize_weight,
+    fg8_quantize_weight_block,
     fg8_scale_to_ue8m0,
     fg8_set_test_stall,
     fg8_set_wait_limit_ns,

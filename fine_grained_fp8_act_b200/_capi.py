@@ -39,6 +39,10 @@ SIGNATURES = {
                                   _VP]),
     "fg8_grouped_linear_prepare": (_INT, [_VP, _I64, _I64, _I64, _I64, _I64, _VP, _INT, _VP, _SZ, _VP]),
     "fg8_grouped_linear_run": (_INT, [_VP, _I64, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
+    "fg8_quantize_act_block": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _INT, _INT, _VP]),
+    "fg8_quantize_weight_block": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _INT, _INT, _VP]),
+    "fg8_linear_block_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT, _INT]),
+    "fg8_linear_block": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run_chain": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _I64, _VP, _VP, _SZ,
                                      _VP]),
@@ -151,6 +155,26 @@ def fg8_grouped_linear_run(row_expert, E, wq_e4m3, w_scale_inv, bias_bf16, y_bf1
     _check("fg8_grouped_linear_run", lib().fg8_grouped_linear_run(row_expert, E, wq_e4m3, w_scale_inv, bias_bf16,
                                                                   y_bf16, M, N, K, ld_y, fmt, workspace,
                                                                   workspace_bytes, stream))
+
+
+def fg8_quantize_act_block(x_bf16, M, K, ld_x, xq_e4m3, x_scale, fmt, block, stream):
+    _check("fg8_quantize_act_block", lib().fg8_quantize_act_block(x_bf16, M, K, ld_x, xq_e4m3, x_scale, fmt, block,
+                                                                  stream))
+
+
+def fg8_quantize_weight_block(w_bf16, N, K, ld_w, wq_e4m3, w_scale_inv, fmt, block, stream):
+    _check("fg8_quantize_weight_block", lib().fg8_quantize_weight_block(w_bf16, N, K, ld_w, wq_e4m3, w_scale_inv, fmt,
+                                                                        block, stream))
+
+
+def fg8_linear_block_workspace_bytes(M, N, K, fmt, block):
+    return lib().fg8_linear_block_workspace_bytes(M, N, K, fmt, block)
+
+
+def fg8_linear_block(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, block, workspace,
+                     workspace_bytes, stream):
+    _check("fg8_linear_block", lib().fg8_linear_block(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                      ld_y, fmt, block, workspace, workspace_bytes, stream))
 
 
 def fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes, stream):

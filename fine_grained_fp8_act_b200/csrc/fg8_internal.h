@@ -32,12 +32,13 @@ __host__ __device__ inline size_t sf_tile_offset(int64_t r, int kb, int Kq) {
 struct ActQuantArgs {
   const void* x;      // bf16 [M, K], row stride ld_x
   int64_t ld_x;
-  int M, K, Kb;
+  int M, K, Kb;       // Kb: groups per row, ceil(K / group)
+  int group;          // group width: 128 (0 means 128) or 32
   uint8_t* xq;        // e4m3 [M, K], row stride K
   void* xs;           // scales, layout below
   int layout;         // ScaleLayout
   int64_t ld_s;       // kScaleKMajor: column stride (>= M)
-  int Kq;             // kScaleSfTiles: ceil(Kb / 4)
+  int Kq;             // kScaleSfTiles: ceil(Kb / 4) chunks of four groups per row tile
   int M_pad;          // kScaleSfTiles: rows rounded up to 128 (padding rows get scale 2^0)
   // static activation scheme (float scales only): one precomputed scale for
   // the whole tensor, read from device memory; nullptr = dynamic groups
@@ -48,6 +49,9 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
 
 cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
                                 cudaStream_t s);
+// 32 x 32 blocks (weight_block_size = (32, 32)): scales [ceil(N/32), ceil(K/32)].
+cudaError_t launch_weight_quant32(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
+                                  cudaStream_t s);
 
 // Pack a UE8M0 [R_src, Kb] row-major scale matrix into scale-factor tiles for
 // R rows, written for R_pad rows (a multiple of 128): row r takes
@@ -94,6 +98,10 @@ struct GemmArgs {
   const int32_t* row_expert;
   int E;
   int sfb_tiles;
+  // UE8M0 with 1 x 32 activation groups and 32 x 32 weight blocks: the
+  // scale-factor tiles hold ceil(K/32) scales per row, one chunk per K-block
+  // (Kq = ceil(K/128) chunks per row tile)
+  bool sf32;
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM

@@ -77,6 +77,11 @@ struct KParams {
   const int32_t* row_expert;  // nullptr: a plain GEMM (expert 0)
   int E;
   int sfb_tiles;
+  // UE8M0 scale granularity along K: one scale-factor chunk (4 scales per
+  // row) covers 4 K-blocks of 128 (sf_shift 2, 1 x 128 groups), or one
+  // K-block whose 4 MMA steps of K = 32 each take their own scale (sf_shift
+  // 0, 1 x 32 groups and 32 x 32 weight blocks)
+  int sf_shift;
 };
 
 constexpr uint32_t kStatusBadExpert = 1u;  // FG8_ERR_INVALID_ARG
@@ -113,8 +118,12 @@ struct Cfg {
   static constexpr int kCols = BN / 2;  // columns per epilogue thread
   static constexpr int kChunks = kCols / 32;
   static constexpr int kNumAcc = FMT == 0 ? 512 / BN : (BN == 256 ? 1 : 3);
+  // UE8M0 scale factors in TMEM: two sets (A: 4 columns, B: 4 per 128 rows),
+  // alternating per copy, so that a copy never lands under an MMA that may
+  // still read the previous set
   static constexpr int kSfaCol = kNumAcc * BN;
   static constexpr int kSfbCol = kSfaCol + 4;
+  static constexpr int kSfSetCols = 4 + BN / 32;
   static constexpr int kBiasSlot = BN * 2;
   // register split after launch (384 x 168): the wide float epilogue holds
   // 128 accumulators + 32 TMEM registers per thread, the others need less
@@ -134,7 +143,7 @@ struct Cfg {
   static_assert(kSmem <= kMaxSmem, "shared memory budget");
   static_assert(kStage % 1024 == 0, "stages keep 1024-byte alignment for the 128B swizzle");
   static_assert(kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
-  static_assert(kNumAcc * BN + (FMT == 1 ? 4 + BN / 32 : 0) <= 512, "TMEM columns");
+  static_assert(kNumAcc * BN + (FMT == 1 ? 2 * kSfSetCols : 0) <= 512, "TMEM columns");
   static_assert(!PAIR || (FMT == 0 && BN == 256), "CTA pairs: float scales, 256-wide tiles");
   static_assert(!REQUANT || (BN == 256 && !PAIR), "output re-quantization: one 128-column group per thread");
   // bytes the stage's full barrier (in the pair's first CTA) waits for
@@ -338,7 +347,7 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
         ok = false;
         break;
       }
-      const bool sf = C::FMT == 1 && (kb & 3) == 0;
+      const bool sf = C::FMT == 1 && (kb & ((1 << p.sf_shift) - 1)) == 0;
       uint8_t* sa = smem + st.slot * C::kStage;
       if constexpr (C::PAIR) {
         // both CTAs' tiles complete on the first CTA's full barrier, which
@@ -354,12 +363,13 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       }
       if (sf) {
         uint8_t* sfs = sa + C::kA + C::kB;
-        bulk_load(sfs, p.sfa + (static_cast<size_t>(m0 / kBlockM) * p.Kq + (kb >> 2)) * kSfChunkBytes, kSfChunkBytes,
-                  full + st.slot);
+        bulk_load(sfs, p.sfa + (static_cast<size_t>(m0 / kBlockM) * p.Kq + (kb >> p.sf_shift)) * kSfChunkBytes,
+                  kSfChunkBytes, full + st.slot);
 #pragma unroll
         for (int h = 0; h < C::BN / 128; ++h)
           bulk_load(sfs + kSfChunkBytes * (1 + h),
-                    p.sfb + (static_cast<size_t>(e * p.sfb_tiles + n0 / 128 + h) * p.Kq + (kb >> 2)) * kSfChunkBytes,
+                    p.sfb + (static_cast<size_t>(e * p.sfb_tiles + n0 / 128 + h) * p.Kq + (kb >> p.sf_shift)) *
+                                kSfChunkBytes,
                     kSfChunkBytes,
                     full + st.slot);
       }
@@ -391,8 +401,9 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
     raise_abort(abort_flag, p.status);
     ok = false;
   }
-  const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
-  const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
+  uint32_t sf_set = 1;  // the set the next copy goes to is sf_set ^ 1
+  uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
+  uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
   for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
     if (p.row_expert != nullptr) {
       int mb, nb;
@@ -417,11 +428,14 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
         tc_fence_after();
       }
       const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
-      if (C::FMT == 1 && (kb & 3) == 0) {
-        // UE8M0 scales of 128 rows x 4 K-blocks for A, and for B, into TMEM;
+      if (C::FMT == 1 && (kb & ((1 << p.sf_shift) - 1)) == 0) {
+        // UE8M0 scales of 128 rows x 4 K-blocks (or 4 K = 32 steps) for A, and for B, into TMEM;
         // issued before the MMAs that read them (tcgen05 ops of one thread
         // execute in issue order).
         const uint32_t sfs = b_addr + C::kB;
+        sf_set ^= 1u;
+        sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol + sf_set * C::kSfSetCols);
+        sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol + sf_set * C::kSfSetCols);
         tc_cp_32x128b_warpx4(sfa_t, smem_desc(sfs, 128, 128, 0));
 #pragma unroll
         for (int h = 0; h < C::BN / 128; ++h)
@@ -436,7 +450,8 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
         } else if (C::FMT == 0) {
           mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
         } else {
-          const uint32_t j = static_cast<uint32_t>(kb & 3);
+          // the byte of each row's scale word: the K-block's (1 x 128 groups) or the step's (1 x 32)
+          const uint32_t j = static_cast<uint32_t>(p.sf_shift == 0 ? k : (kb & 3));
           mma_mxf8f6f4(d, ad, bd, C::kIdescMx | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
                        (kb > 0 || k > 0) ? 1u : 0u);
         }
@@ -846,6 +861,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.row_expert = g.row_expert;
   p.E = g.row_expert != nullptr ? g.E : 1;
   p.sfb_tiles = g.sfb_tiles;
+  p.sf_shift = g.sf32 ? 0 : 2;
   if (p.num_tiles == 0) return cudaSuccess;
 
   static int configured_device = -1;

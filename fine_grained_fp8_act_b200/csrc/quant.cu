@@ -70,30 +70,33 @@ __device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32
 // saturate); the scale is still written per group, so the GEMM reads it
 // exactly as it reads dynamic scales.
 //
-// Eight lanes own one 128-channel group: lane l loads channels [16l, 16l+16)
-// with two 16-byte loads.  A warp covers 4 groups per pass and makes 2 passes
-// per iteration (all loads issued before any arithmetic), striding over the
-// grid.  amax: per-lane max, then 3 xor-shuffles inside the 8 lanes.
+// GL lanes own one group of 16*GL channels (8 lanes for the default 128, 2
+// for 1 x 32 groups): lane l loads channels [16l, 16l+16) with two 16-byte
+// loads.  A warp covers 32/GL groups per pass and makes 2 passes per
+// iteration (all loads issued before any arithmetic), striding over the
+// grid.  amax: per-lane max, then log2(GL) xor-shuffles inside the group.
 //   kScaleRowMajor: group g -> (m = g / Kb, kb = g % Kb)  (scales [M, Kb])
 //   kScaleKMajor / kScaleSfTiles: g -> (kb = g / rows, m = g % rows), so the
 //   scale writes of neighbouring lane-octets are neighbouring addresses.
-template <int FMT, int LAYOUT>
+template <int FMT, int LAYOUT, int GL>
 __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, const uint32_t total, const FastDiv div) {
   grid_wait_prerequisites();  // x may come from the preceding kernel (launched ahead of its end)
   grid_launch_dependents();   // the GEMM may set itself up meanwhile; it waits for our results
   constexpr int kPasses = 2;
-  const int lane = threadIdx.x & 31, oct = lane >> 3, l = lane & 7;
+  constexpr int kGpw = 32 / GL;  // groups per warp and pass
+  constexpr int G = 16 * GL;     // group width
+  const int lane = threadIdx.x & 31, oct = lane / GL, l = lane % GL;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const uint16_t* x = static_cast<const uint16_t*>(a.x);
 
-  for (uint32_t base = warp * (4 * kPasses); base < total; base += nwarps * (4 * kPasses)) {
+  for (uint32_t base = warp * (kGpw * kPasses); base < total; base += nwarps * (kGpw * kPasses)) {
     uint4 v[kPasses][2];
     int m[kPasses], kb[kPasses];
     bool has[kPasses], real[kPasses];
 #pragma unroll
     for (int u = 0; u < kPasses; ++u) {
-      const uint32_t g = base + u * 4 + oct;
+      const uint32_t g = base + u * kGpw + oct;
       has[u] = g < total;
       uint32_t qt, r;
       fast_divmod(div, g, qt, r);
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, co
         m[u] = static_cast<int>(r);
       }
       real[u] = has[u] && m[u] < a.M && kb[u] < a.Kb;
-      const int k = kb[u] * kGroup + l * 16;
+      const int k = kb[u] * G + l * 16;
       v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
       if (real[u] && k < a.K) {
         const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m[u]) * a.ld_x + k);
@@ -124,12 +127,12 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, co
 #pragma unroll
       for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-      for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+      for (int off = GL / 2; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
       // dynamic: the group's scale; static (float only): the tensor's one scale
       const float s = (FMT == 0 && a.static_scale != nullptr) ? *a.static_scale : group_scale(amax);
       const uint32_t sbyte = FMT == 1 ? e8m0_ceil_byte(s) : 0u;
       const uint4 packed = quantize16<FMT>(f, s, sbyte);
-      const int k = kb[u] * kGroup + l * 16;
+      const int k = kb[u] * G + l * 16;
       if (real[u] && k < a.K) *reinterpret_cast<uint4*>(a.xq + static_cast<int64_t>(m[u]) * a.K + k) = packed;
       if (l == 0 && has[u]) {
         if (LAYOUT == kScaleRowMajor) {
@@ -194,6 +197,55 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const uint16_t* __res
   if (t == 0) {
     if (FMT == 0) static_cast<float*>(ws)[static_cast<int64_t>(nb) * Kb + kb] = s;
     else static_cast<uint8_t*>(ws)[static_cast<int64_t>(nb) * Kb + kb] = static_cast<uint8_t>(sbyte);
+  }
+}
+
+// One warp per 32 x 32 block (weight_block_size = (32, 32)): lane i holds row
+// i of the block (32 channels, four 16-byte loads; a 16-wide last block when
+// K % 32 == 16), amax by 5 xor-shuffles, two 16-byte stores per row.
+template <int FMT>
+__global__ void __launch_bounds__(256) weight_quant32_kernel(const uint16_t* __restrict__ w, const int64_t ld_w,
+                                                             const int N, const int K, const int Nb, const int Kb,
+                                                             uint8_t* __restrict__ wq, void* __restrict__ ws) {
+  const int lane = threadIdx.x & 31;
+  const int64_t blk = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (blk >= static_cast<int64_t>(Nb) * Kb) return;
+  const int nb = static_cast<int>(blk / Kb), kb = static_cast<int>(blk % Kb);
+  const int n = nb * 32 + lane, k0 = kb * 32;
+  const bool row = n < N;
+  uint4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = k0 + 8 * i;
+    v[i] = (row && k < K) ? __ldg(reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * ld_w + k))
+                          : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float f[2][16];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float(&a0)[8] = *reinterpret_cast<float(*)[8]>(f[h]);
+    float(&a1)[8] = *reinterpret_cast<float(*)[8]>(f[h] + 8);
+    unpack_bf16x8(v[2 * h], a0);
+    unpack_bf16x8(v[2 * h + 1], a1);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[h][i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  const float s = group_scale(amax);
+  const uint32_t sbyte = FMT == 1 ? e8m0_ceil_byte(s) : 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = k0 + 16 * h;
+    if (row && k < K)
+      *reinterpret_cast<uint4*>(wq + static_cast<int64_t>(n) * K + k) = quantize16<FMT>(f[h], s, sbyte);
+  }
+  if (lane == 0) {
+    if (FMT == 0) static_cast<float*>(ws)[blk] = s;
+    else static_cast<uint8_t*>(ws)[blk] = static_cast<uint8_t>(sbyte);
   }
 }
 
@@ -263,7 +315,8 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   if (total == 0) return cudaSuccess;
   if (total > 0x7FFFFFF0LL) return cudaErrorInvalidValue;  // group index is 32-bit
   const FastDiv div = make_fastdiv(static_cast<uint32_t>(a.layout == kScaleRowMajor ? cols : rows));
-  const int64_t per_block = 8 * 8;  // 8 warps x 8 groups per iteration
+  const int gl = a.group == 32 ? 2 : 8;  // lanes per group
+  const int64_t per_block = 8 * (32 / gl) * 2;  // 8 warps x groups per warp x 2 passes
   int64_t blocks = (total + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
@@ -278,15 +331,35 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-#define FG8_AQ(F, L) cudaLaunchKernelEx(&cfg, act_quant_kernel<F, L>, a, t32, div)
-  if (fmt == 0) {
-    if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor);
-    else FG8_AQ(0, kScaleKMajor);
-  } else {
-    if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor);
-    else FG8_AQ(1, kScaleSfTiles);
+#define FG8_AQ(F, L, GL) cudaLaunchKernelEx(&cfg, act_quant_kernel<F, L, GL>, a, t32, div)
+  if (gl == 8) {
+    if (fmt == 0) {
+      if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor, 8);
+      else FG8_AQ(0, kScaleKMajor, 8);
+    } else {
+      if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 8);
+      else FG8_AQ(1, kScaleSfTiles, 8);
+    }
+  } else {  // 1 x 32 groups: row-major scales, or UE8M0 scale-factor tiles for the GEMM
+    if (a.layout == kScaleKMajor) return cudaErrorInvalidValue;
+    if (fmt == 0) FG8_AQ(0, kScaleRowMajor, 2);
+    else if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 2);
+    else FG8_AQ(1, kScaleSfTiles, 2);
   }
 #undef FG8_AQ
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_quant32(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
+                                  cudaStream_t s) {
+  const int Kb = (K + 31) / 32, Nb = (N + 31) / 32;
+  const int64_t blocks = (static_cast<int64_t>(Nb) * Kb + 7) / 8;
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  if (fmt == 0)
+    weight_quant32_kernel<0><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(w), ld_w, N, K, Nb, Kb, wq, ws);
+  else
+    weight_quant32_kernel<1><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(w), ld_w, N, K, Nb, Kb, wq, ws);
   return cudaGetLastError();
 }
 

@@ -211,6 +211,28 @@ FG8_API fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, i
                                      const void* bias_bf16, void* y_bf16, int64_t ld_y, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* Non-default block size ([zh] §八: the tests cover weight_block_size such
+ * as (32, 32)).  Reading: the activation groups follow the weight's
+ * input-channel block, so block = 32 means 1 x 32 activation groups and
+ * 32 x 32 weight blocks; scales are shaped [M, ceil(K/32)] and
+ * [ceil(N/32), ceil(K/32)].  block is 32 or 128 (128 forwards to the calls
+ * above).  The quantizers take either scale format; fg8_linear_block with
+ * block 32 takes UE8M0 only (FG8_ERR_INVALID_ARG for float): the tensor
+ * core's block-scaled MMA applies one scale per 32 K per row natively,
+ * float scales would need a register promotion per 32-K slice.  It always
+ * runs the tiled GEMM (no few-token kernel).  Other checks and errors as
+ * the 128 versions; the workspace is fg8_linear_block_workspace_bytes (0 for
+ * an unsupported combination), with the header rules of fg8_linear. */
+FG8_API fg8_status fg8_quantize_act_block(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* xq_e4m3,
+                                          void* x_scale, fg8_scale_fmt fmt, int block, void* stream);
+FG8_API fg8_status fg8_quantize_weight_block(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w, void* wq_e4m3,
+                                             void* w_scale_inv, fg8_scale_fmt fmt, int block, void* stream);
+FG8_API size_t fg8_linear_block_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt, int block);
+FG8_API fg8_status fg8_linear_block(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                    const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                    void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, int block, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* MoE experts ([zh] §6.4 and [pt] "Caminho rápido do DeepGEMM": FP8Experts
  * sends each expert's tokens through this layer with that expert's e4m3
  * weights and block scales; on Blackwell the expert kernels take UE8M0

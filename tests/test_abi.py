@@ -218,3 +218,21 @@ def test_grouped_rejects_bad_args(fg8):
     assert f(256, 8, 256, 1024, 1) > f(256, 1, 256, 1024, 1) + 7 * 2 * 2 * 512 - 256
     assert f(256, 8, 256, 1024, 0) == fg8.fg8_linear_workspace_bytes(256, 256, 1024, 0)
     assert f(256, 0, 256, 1024, 0) == 0
+
+
+def test_block_size_rejects_bad_args(fg8):
+    raw = _raw(fg8)
+    assert raw.fg8_quantize_act_block(FAKE, 4, 256, 256, FAKE, FAKE, 0, 64, None) == 1       # block 64
+    assert raw.fg8_quantize_act_block(FAKE, 4, 120, 128, FAKE, FAKE, 1, 32, None) == 2      # K % 16
+    assert raw.fg8_quantize_act_block(None, 0, 256, 256, None, None, 1, 32, None) == 0      # empty
+    assert raw.fg8_quantize_weight_block(FAKE, 0, 256, 256, FAKE, FAKE, 1, 32, None) == 1
+    assert raw.fg8_quantize_weight_block(FAKE, 256, 248, 248, FAKE, FAKE, 1, 32, None) == 2
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 0, 32) == 0                   # float at 32
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 64) == 0
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 128) == raw.fg8_linear_workspace_bytes(256, 256, 256, 1)
+    # x codes + 2 x-scale chunks (K = 256: 2 K-blocks) + 2 row tiles x 2 W chunks, beyond the header
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 32) >= 256 * 256 + 2 * 2 * 512 + 2 * 2 * 512
+    lb = raw.fg8_linear_block
+    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, 32, FAKE * 16, 1 << 40, None) == 1
+    assert lb(FAKE, 16, 256, 200, 200, FAKE, FAKE, None, FAKE, 256, 1, 32, FAKE * 16, 1 << 40, None) == 2
+    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 1, 32, None, 1 << 40, None) == 4
