@@ -71,10 +71,10 @@ def workload_layers(name):
     raise SystemExit(f"unknown workload {name}")
 
 
-def workload_config(name, layers):
+def workload_config(name, layers, block=128):
     g0 = layers[0][1]
     cfg = {"workload": name, "tokens": g0.M, "layers": [[g.K, g.N] for _, g, _ in layers],
-           "scale_fmt": "ue8m0" if g0.fmt else "float", "block": [128, 128], "act_group": 128,
+           "scale_fmt": "ue8m0" if g0.fmt else "float", "block": [block, block], "act_group": block,
            "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the step events)"}
     if name == "esm2_ffn":
         cfg.update({"model": "ESM-2 35M FFN shape (hidden 480, ffn 1920, 8 x 1022 tokens)"})
@@ -290,9 +290,10 @@ def run_fg8(args, rank, world, local):
         if i == 0:
             # weak scaling: every rank runs its own batch of the same shape
             x0 = x if rank == 0 else x.roll(rank, 0).contiguous()
-        wq, ws = fg8.quantize_weight(w, g.fmt)
+        wq, ws = fg8.quantize_weight(w, g.fmt, block=args.block)
         del w
-        wsp = torch.zeros(fg8.fg8_linear_workspace_bytes(g.M, g.N, g.K, g.fmt), dtype=torch.uint8, device=dev)
+        wsp = torch.zeros(fg8.fg8_linear_block_workspace_bytes(g.M, g.N, g.K, g.fmt, args.block), dtype=torch.uint8,
+                          device=dev)
         y = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
         plan.append(dict(g=g, wq=wq, ws=ws, b=b, wsp=wsp, y=y))
     for i, L in enumerate(plan):
@@ -305,12 +306,20 @@ def run_fg8(args, rank, world, local):
     # tiled, consecutive layers chain: the GEMM of layer i also quantizes its
     # output for layer i+1 (fg8_linear_run_chain), so layer i+1 has no
     # act-quant launch.
-    paths = [layer_path(L["g"]) for L in plan]
+    # block 32 (1 x 32 groups, 32 x 32 weight blocks): fg8_linear_block per layer
+    paths = [("block32" if args.block == 32 else layer_path(L["g"])) for L in plan]
     chain = not args.no_chain and all(pth == "tiled" for pth in paths)
 
     def launch_layer(i, ev_mid=None):
         L = plan[i]
         g = L["g"]
+        if paths[i] == "block32":  # act-quant, scale packing and GEMM in one call
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            fg8.fg8_linear_block(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["wq"].data_ptr(),
+                                 L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, 32,
+                                 L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+            return
         if paths[i] == "fused":
             if ev_mid is not None:
                 ev_mid.record(stream)
@@ -416,7 +425,9 @@ def run_fg8(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(args.workload, dom)  # ncu DRAM bytes per launch, None if stale
-    roof["kernel"] = ("fg8_small_m_kernel" if paths[dom] != "tiled" else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+    roof["kernel"] = ("fg8_gemm_kernel, 32 x 32 blocks, timed with its act-quant and scale packing"
+                      if paths[dom] == "block32" else
+                      "fg8_small_m_kernel" if paths[dom] != "tiled" else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
     roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
@@ -426,10 +437,12 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        fused = paths[i] == "fused" or (chain and i > 0)  # act-quant inside a GEMM kernel
+        fused = paths[i] in ("fused", "block32") or (chain and i > 0)  # act-quant not timed on its own
         per_kernel.append({"layer": gi.name, "path": paths[i], "act_quant_us": None if fused else qm[i] * 1e3,
                            "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
                            "act_quant": ("fused into the few-token kernel" if paths[i] == "fused" else
+                                         "timed with the GEMM (fg8_linear_block: act-quant, scale packing, GEMM)"
+                                         if paths[i] == "block32" else
                                          "fused into the previous GEMM" if fused else "own launch"),
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
                            "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
@@ -437,7 +450,7 @@ def run_fg8(args, rank, world, local):
     e2e = run_e2e(fg8, plan, args, stream, dev, world, chain)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds, block=args.block)
 
     # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM;
     # fused few-token layers: one kernel
@@ -447,7 +460,8 @@ def run_fg8(args, rank, world, local):
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": dict(workload_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)]),
+        "config": dict(workload_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)],
+                                       args.block),
                        parallelism=f"dp{world} (token rows, replicated weights, no collective)"),
         "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
         "act_quant_gbs": [k["act_quant_gbs"] for k in per_kernel if k["act_quant_gbs"] is not None],
@@ -499,9 +513,9 @@ def run_e2e(fg8, plan, args, stream, dev, world, chain):
             xin = x_dev
             for L in plan:
                 g = L["g"]
-                fg8.fg8_linear(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
-                               L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, L["wsp"].data_ptr(),
-                               L["wsp"].numel(), sp)
+                fg8.fg8_linear_block(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(),
+                                     L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt,
+                                     args.block, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
                 xin = L["y"]
         y_host.copy_(Ln["y"], non_blocking=True)
 
@@ -754,7 +768,7 @@ def cpu_baseline_moe(budget_s=15.0, rows=None):
 
 
 # ------------------------------------------------------ oracle (CPU) arm ----
-def cpu_baseline(workload, budget_s=15.0, rows=None):
+def cpu_baseline(workload, budget_s=15.0, rows=None, block=128):
     """The CPU oracle, as it stands, on a bounded sample of the workload: the
     first R token rows of the batch through every layer (quantize, dequantized
     double GEMM, bf16 out), weights quantized once outside the timing.
@@ -767,14 +781,14 @@ def cpu_baseline(workload, budget_s=15.0, rows=None):
         x, w, b = W.make_inputs(cfg, g, device="cpu", stage=stage)
         if i == 0:
             xb = W.bf16_bits(x)
-        wq, ws = oracle.quantize_weight(W.bf16_bits(w), g.fmt)
+        wq, ws = oracle.quantize_weight(W.bf16_bits(w), g.fmt, block)
         ops.append((g, wq, ws, W.bf16_bits(b)))
 
     def run(R):
         t0 = time.perf_counter()
         a = xb[:R]
         for g, wq, ws, bb in ops:
-            _, _, ybf = oracle.linear(a, wq, ws, bb, g.fmt)
+            _, _, ybf = oracle.linear(a, wq, ws, bb, g.fmt, block=block)
             a = ybf
         return time.perf_counter() - t0
 
@@ -821,13 +835,13 @@ def run_reference(args, rank, world):
     layers = workload_layers(args.workload)
     # size each step so warm-up + steps stay within ~2 minutes
     budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
-    probe = cpu_baseline(args.workload, rows=16)
+    probe = cpu_baseline(args.workload, rows=16, block=args.block)
     rows = int(max(1, min(layers[0][1].M, 16 * budget / max(probe["seconds"], 1e-6))))
     for _ in range(args.warmup):
-        cpu_baseline(args.workload, rows=rows)
+        cpu_baseline(args.workload, rows=rows, block=args.block)
     ts = []
     for _ in range(args.steps):
-        ts.append(cpu_baseline(args.workload, rows=rows)["seconds"])
+        ts.append(cpu_baseline(args.workload, rows=rows, block=args.block)["seconds"])
     flops = sum(2.0 * rows * g.N * g.K for _, g, _ in layers)
     tot = sum(ts)
     value = flops * len(ts) / tot / 1e12
@@ -837,7 +851,7 @@ def run_reference(args, rank, world):
            "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: float32 quantization, double GEMM)",
            "data": "synthetic", "impl": "reference",
-           "config": dict(workload_config(args.workload, layers), parallelism="cpu oracle, rank 0 only"),
+           "config": dict(workload_config(args.workload, layers, args.block), parallelism="cpu oracle, rank 0 only"),
            "cpu_baseline": cpu,
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -852,6 +866,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=128, choices=[128, 32],
+                    help="weight_block_size (block, block) and 1 x block activation groups; 32 takes UE8M0 workloads")
     ap.add_argument("--no-chain", action="store_true",
                     help="quantize every layer's input in its own launch instead of in the previous GEMM")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
@@ -863,6 +879,9 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_env()
+    if args.block == 32 and (args.workload.startswith("moe_") or
+                             any(g.fmt != 1 for _, g, _ in workload_layers(args.workload))):
+        raise SystemExit("--block 32 runs UE8M0 dense workloads (dsv3_mlp, square_m*_ue8m0)")
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -44,27 +44,30 @@ def _check_bf16_matrix(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must have unit stride in its last dimension")
 
 
-def quantize_weight(w: torch.Tensor, scale_fmt="float") -> Tuple[torch.Tensor, torch.Tensor]:
-    """W bf16 [N, K] -> (wq float8_e4m3fn [N, K], weight_scale_inv [ceil(N/128), ceil(K/128)])."""
+def quantize_weight(w: torch.Tensor, scale_fmt="float", block: int = 128) -> Tuple[torch.Tensor, torch.Tensor]:
+    """W bf16 [N, K] -> (wq float8_e4m3fn [N, K], weight_scale_inv [ceil(N/block), ceil(K/block)]);
+    block x block weight blocks, block 128 (default) or 32."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(w, "w")
     N, K = w.shape
     wq = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
-    ws = torch.empty((_cdiv(N, 128), _cdiv(K, 128)), dtype=_SCALE_DTYPES[fmt], device=w.device)
+    ws = torch.empty((_cdiv(N, block), _cdiv(K, block)), dtype=_SCALE_DTYPES[fmt], device=w.device)
     with torch.cuda.device(w.device):
-        C.fg8_quantize_weight(w.data_ptr(), N, K, w.stride(0), wq.data_ptr(), ws.data_ptr(), fmt, _stream(w))
+        C.fg8_quantize_weight_block(w.data_ptr(), N, K, w.stride(0), wq.data_ptr(), ws.data_ptr(), fmt, block,
+                                    _stream(w))
     return wq, ws
 
 
-def quantize_act(x: torch.Tensor, scale_fmt="float") -> Tuple[torch.Tensor, torch.Tensor]:
-    """x bf16 [M, K] -> (xq float8_e4m3fn [M, K], x_scale [M, ceil(K/128)])."""
+def quantize_act(x: torch.Tensor, scale_fmt="float", block: int = 128) -> Tuple[torch.Tensor, torch.Tensor]:
+    """x bf16 [M, K] -> (xq float8_e4m3fn [M, K], x_scale [M, ceil(K/block)]); 1 x block groups."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
-    xs = torch.empty((M, _cdiv(K, 128)), dtype=_SCALE_DTYPES[fmt], device=x.device)
+    xs = torch.empty((M, _cdiv(K, block)), dtype=_SCALE_DTYPES[fmt], device=x.device)
     with torch.cuda.device(x.device):
-        C.fg8_quantize_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), xs.data_ptr(), fmt, _stream(x))
+        C.fg8_quantize_act_block(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), xs.data_ptr(), fmt, block,
+                                 _stream(x))
     return xq, xs
 
 
@@ -94,8 +97,9 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
 
 def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: Optional[torch.Tensor] = None,
            scale_fmt="float", out: Optional[torch.Tensor] = None,
-           workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y [M, N] bf16 = dequant(quantize_act(x)) . dequant(wq)^T + bias."""
+           workspace: Optional[torch.Tensor] = None, block: int = 128) -> torch.Tensor:
+    """y [M, N] bf16 = dequant(quantize_act(x)) . dequant(wq)^T + bias.  block 32
+    (1 x 32 groups, 32 x 32 weight blocks) takes UE8M0 scales."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
     M, K = x.shape
@@ -103,12 +107,12 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: O
     if wq.shape != (N, K):
         raise ValueError("wq must be [N, K]")
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    nbytes = C.fg8_linear_workspace_bytes(M, N, K, fmt)
+    nbytes = C.fg8_linear_block_workspace_bytes(M, N, K, fmt, block)  # 0: the call below reports why
     ws = _workspace(nbytes, x.device, workspace)
     with torch.cuda.device(x.device):
-        C.fg8_linear(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(),
-                     0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0), fmt, ws.data_ptr(),
-                     ws.numel() * ws.element_size(), _stream(x))
+        C.fg8_linear_block(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(),
+                           0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0), fmt, block,
+                           ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
     return y
 
 
@@ -238,13 +242,16 @@ def scale_to_ue8m0(scale: torch.Tensor) -> Tuple[torch.Tensor, int]:
 
 class FP8Linear(torch.nn.Module):
     """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
-    weight float8_e4m3fn [out, in], weight_scale_inv per 128x128 block, bias
-    kept in bf16 (not quantized, [zh] §三)."""
+    weight float8_e4m3fn [out, in], weight_scale_inv per block x block block
+    (weight_block_size (128, 128) by default, or (32, 32) with UE8M0 scales),
+    bias kept in bf16 (not quantized, [zh] §三)."""
 
-    def __init__(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None, scale_fmt="float"):
+    def __init__(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None, scale_fmt="float",
+                 block: int = 128):
         super().__init__()
         self.scale_fmt = scale_fmt_code(scale_fmt)
-        wq, ws = quantize_weight(weight.to(torch.bfloat16).contiguous(), self.scale_fmt)
+        self.block = block
+        wq, ws = quantize_weight(weight.to(torch.bfloat16).contiguous(), self.scale_fmt, block)
         self.register_buffer("weight", wq)
         self.register_buffer("weight_scale_inv", ws)
         self.register_buffer("bias", None if bias is None else bias.to(torch.bfloat16).contiguous())
@@ -262,8 +269,9 @@ class FP8Linear(torch.nn.Module):
         lead = x.shape[:-1]
         x2 = x.reshape(-1, x.shape[-1]).to(torch.bfloat16).contiguous()
         M, N, K = x2.shape[0], self.out_features, self.in_features
-        need = C.fg8_linear_workspace_bytes(M, N, K, self.scale_fmt)
+        need = C.fg8_linear_block_workspace_bytes(M, N, K, self.scale_fmt, self.block)
         if self._ws is None or self._ws.numel() < need or self._ws.device != x2.device:
             self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x2.device)
-        y = linear(x2, self.weight, self.weight_scale_inv, self.bias, self.scale_fmt, workspace=self._ws)
+        y = linear(x2, self.weight, self.weight_scale_inv, self.bias, self.scale_fmt, workspace=self._ws,
+                   block=self.block)
         return y.reshape(*lead, N)

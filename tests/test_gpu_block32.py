@@ -109,3 +109,26 @@ def test_block128_through_block_calls_is_the_default(fg8, fmt):
     y2 = fg8.linear(x, wq.view(torch.float8_e4m3fn), ws if fmt == FLOAT else ws.view(torch.float8_e8m0fnu), b,
                     "ue8m0" if fmt else "float")
     assert torch.equal(y, y2)
+
+
+def test_layer_wrappers_block32(fg8, orc):
+    """quantize_weight / quantize_act / linear / FP8Linear with block = 32."""
+    M, N, K = 150, 264, 320
+    x = W.x_normal(M, K, seed=11).cuda()
+    w = W.normal((N, K), 0.02, seed=12).cuda()
+    b = W.normal((N,), 0.1, seed=13).cuda()
+    wq, ws = fg8.quantize_weight(w, "ue8m0", block=32)
+    assert ws.shape == (-(-N // 32), K // 32)
+    oq, os_ = orc.quantize_weight(W.bf16_bits(w), UE8M0, 32)
+    assert np.array_equal(_np(wq), oq) and np.array_equal(_np(ws), os_)
+    xq, xs = fg8.quantize_act(x, "ue8m0", block=32)
+    aq, as_ = orc.quantize_act(W.bf16_bits(x), UE8M0, 32)
+    assert np.array_equal(_np(xq), aq) and np.array_equal(_np(xs), as_)
+    y = fg8.linear(x, wq, ws, b, "ue8m0", block=32)
+    layer = fg8.FP8Linear(w, b, "ue8m0", block=32)
+    y2 = layer(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    y64, bound, _ = orc.linear(W.bf16_bits(x), oq, os_, W.bf16_bits(b), UE8M0, block=32)
+    yg = (W.bf16_bits(y).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert (np.abs(yg - y64) <= y_tolerance(bound)).all()
