@@ -181,9 +181,10 @@ def test_wide_tiles_ragged_n(fg8, orc, fmt, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(2176, 2304, 384), (4000, 2560, 1040), (8176, 1920, 480)])
-def test_cta_pair_tiles(fg8, orc, M, N, K):
-    """Float shapes large enough for the CTA-pair (256 x 256) tiles: a last
-    pair tile whose second CTA is entirely past M, ragged K, the ESM-2 shape."""
+def test_ragged_row_tiles(fg8, orc, M, N, K):
+    """Float shapes whose last 128-row tile is partly past M (and whose last
+    256 rows straddle M), ragged K, the ESM-2 shape; sampled rows around the
+    tile boundaries."""
     x = W.x_outliers(M, K, seed=M + 2 * K).cuda()
     w = W.w_row_groups(N, K, 0.02, seed=N + 5 * K).cuda()
     b = W.normal((N,), 0.1, seed=N + 7).cuda()
@@ -218,3 +219,37 @@ def test_fullsize_dsv3(fg8, orc, stage):
 @pytest.mark.parametrize("M", W.SQUARE_M)
 def test_fullsize_square(fg8, orc, M, fmt):
     full_size_case(fg8, orc, "square", W.square(M, fmt), 1)
+
+
+
+def _dequant(q, s, block=128):
+    """value(q) * scale, the scales expanded over their groups/blocks (fp32, on the GPU)."""
+    v = q.float()
+    sc = s.float()
+    rows = sc.repeat_interleave(block, dim=0)[:v.shape[0]] if sc.shape[0] != v.shape[0] else sc
+    return v * rows.repeat_interleave(block, dim=1)[:, :v.shape[1]]
+
+
+@pytest.mark.parametrize("cfg,gemm,stage", [("square", W.square(8192, FLOAT), 1), ("square", W.square(8192, UE8M0), 1),
+                                            ("dsv3", W.DSV3_UP, 1), ("llama", W.llama(4096, "gate_up"), 1),
+                                            ("esm2", W.ESM_W2, 2)])
+def test_fullsize_every_element_vs_fp32_matmul(fg8, cfg, gemm, stage):
+    """A library check beside the oracle's sampled rows: every element of y at
+    full size against an fp32 matmul (TF32 off) of the dequantized operands,
+    y_ref = x^ . w^T + bias, with the same tolerance 8e-3 * (|x^| . |w^|^T) + 1e-6."""
+    x, w, b = W.make_inputs(cfg, gemm, device="cuda", stage=stage)
+    fmt = gemm.fmt
+    wq, ws = fg8.quantize_weight(w, fmt)
+    xq, xs = fg8.quantize_act(x, fmt)
+    y = fg8.linear(x, wq, ws, b, fmt).float()
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        xh = _dequant(xq, xs)
+        wh = _dequant(wq, ws)
+        ref = xh @ wh.t() + b.float()
+        bound = xh.abs() @ wh.abs().t()
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    bad = ~((y - ref).abs() <= 8e-3 * bound + 1e-6)
+    assert int(bad.sum()) == 0, f"{int(bad.sum())} of {bad.numel()} elements out of tolerance"
