@@ -30,6 +30,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_grouped_linear,
     fg8_grouped_linear_prepare,
     fg8_grouped_linear_run,
+    fg8_grouped_row_expert,
     fg8_grouped_linear_workspace_bytes,
     fg8_linear,
     fg8_linear_block,

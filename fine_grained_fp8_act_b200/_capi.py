@@ -43,6 +43,7 @@ SIGNATURES = {
     "fg8_quantize_weight_block": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _INT, _INT, _VP]),
     "fg8_linear_block_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT, _INT]),
     "fg8_linear_block": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _INT, _VP, _SZ, _VP]),
+    "fg8_grouped_row_expert": (_INT, [_VP, _I64, _I64, _VP, _VP]),
     "fg8_linear_run": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_run_chain": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _I64, _VP, _VP, _SZ,
                                      _VP]),
@@ -175,6 +176,10 @@ def fg8_linear_block(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_b
                      workspace_bytes, stream):
     _check("fg8_linear_block", lib().fg8_linear_block(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
                                                       ld_y, fmt, block, workspace, workspace_bytes, stream))
+
+
+def fg8_grouped_row_expert(counts, E, cap, row_expert, stream):
+    _check("fg8_grouped_row_expert", lib().fg8_grouped_row_expert(counts, E, cap, row_expert, stream))
 
 
 def fg8_linear_run(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace, workspace_bytes, stream):

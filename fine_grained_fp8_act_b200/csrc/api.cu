@@ -315,6 +315,20 @@ size_t fg8_grouped_linear_workspace_bytes(int64_t M, int64_t E, int64_t N, int64
   return grouped_ws_layout(M, E, N, K, fmt).total;
 }
 
+fg8_status fg8_grouped_row_expert(const int32_t* counts, int64_t E, int64_t cap, int32_t* row_expert,
+                                  void* stream) {
+  if (E <= 0 || E > 65535 || cap < 0 || E * cap > kMaxDim) return FG8_ERR_INVALID_ARG;
+  if (cap == 0) return FG8_OK;
+  if (counts == nullptr || row_expert == nullptr) return FG8_ERR_INVALID_ARG;
+  if (cap % 128 != 0 || (reinterpret_cast<uintptr_t>(counts) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(row_expert) & 3u) != 0)
+    return FG8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  return cuda_status(launch_row_expert(counts, static_cast<int>(E), static_cast<int>(cap), row_expert, dev.sms,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 fg8_status fg8_grouped_linear_prepare(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, int64_t E, int64_t N,
                                       const void* w_scale_inv, fg8_scale_fmt fmt, void* workspace,
                                       size_t workspace_bytes, void* stream) {

@@ -74,6 +74,18 @@ __global__ void __launch_bounds__(256) scale_to_e8m0_kernel(const float* __restr
   }
 }
 
+// Batched expert layout -> the grouped layout's expert index: expert e owns
+// rows [e * cap, (e + 1) * cap), of which the first counts[e] are routed.
+__global__ void __launch_bounds__(256) row_expert_kernel(const int32_t* __restrict__ counts, const int E, const int cap,
+                                                         int32_t* __restrict__ row_expert) {
+  const int64_t total = static_cast<int64_t>(E) * cap;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(i / cap), r = static_cast<int>(i % cap);
+    row_expert[i] = r < counts[e] ? e : -1;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dequant_weight(const uint8_t* wq, int N, int K, const void* ws, int fmt, uint16_t* w, int64_t ld_w,
@@ -88,6 +100,16 @@ cudaError_t launch_dequant_weight(const uint8_t* wq, int N, int K, const void* w
     dequant_weight_kernel<0><<<static_cast<unsigned>(blocks), 256, 0, s>>>(wq, K, ws, Kb, w, ld_w, groups16);
   else
     dequant_weight_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(wq, K, ws, Kb, w, ld_w, groups16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_expert(const int32_t* counts, int E, int cap, int32_t* row_expert, int num_sms,
+                              cudaStream_t st) {
+  const int64_t total = static_cast<int64_t>(E) * cap;
+  if (total == 0) return cudaSuccess;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+  row_expert_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(counts, E, cap, row_expert);
   return cudaGetLastError();
 }
 

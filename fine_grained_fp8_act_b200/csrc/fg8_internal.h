@@ -168,6 +168,9 @@ cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s);
 // Checkpoint conversions (convert.cu).
 cudaError_t launch_dequant_weight(const uint8_t* wq, int N, int K, const void* ws, int fmt, uint16_t* w, int64_t ld_w,
                                   int num_sms, cudaStream_t s);
+// Batched expert layout (E slabs of cap rows, counts[e] routed) -> row_expert.
+cudaError_t launch_row_expert(const int32_t* counts, int E, int cap, int32_t* row_expert, int num_sms,
+                              cudaStream_t st);
 cudaError_t launch_scale_to_e8m0(const float* s, int64_t n, uint8_t* out, uint32_t* bad, int num_sms, cudaStream_t st);
 
 int choose_block_n(int M, int N, int num_sms);

@@ -263,6 +263,16 @@ FG8_API fg8_status fg8_grouped_linear(const void* x_bf16, int64_t M, int64_t K, 
                                       const int32_t* row_expert, int64_t E, int64_t N, const void* wq_e4m3,
                                       const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y,
                                       fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream);
+/* The batched expert layout ([zh] §6.4's batched_mm alternative: each
+ * expert's tokens in a slab of `cap` rows, x [E * cap, K]) as the grouped
+ * layout: writes row_expert [E * cap] (device int32), row e * cap + r =
+ * e for r < counts[e] (device int32 [E]) and -1 beyond, so blocks past an
+ * expert's count are skipped.  cap % 128 == 0 (FG8_ERR_ALIGNMENT otherwise:
+ * a 128-row block must not straddle two slabs); counts[e] > cap computes
+ * the whole slab.  Then fg8_grouped_linear on M = E * cap rows. */
+FG8_API fg8_status fg8_grouped_row_expert(const int32_t* counts, int64_t E, int64_t cap, int32_t* row_expert,
+                                          void* stream);
+
 /* fg8_grouped_linear in two halves (as fg8_linear_prepare / fg8_linear_run):
  * the prepare step quantizes x into the workspace (and, for UE8M0, packs
  * every expert's weight scales into scale-factor tiles); the run step is

@@ -236,3 +236,14 @@ def test_block_size_rejects_bad_args(fg8):
     assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, 32, FAKE * 16, 1 << 40, None) == 1
     assert lb(FAKE, 16, 256, 200, 200, FAKE, FAKE, None, FAKE, 256, 1, 32, FAKE * 16, 1 << 40, None) == 2
     assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 1, 32, None, 1 << 40, None) == 4
+
+
+def test_batched_row_expert_rejects_bad_args(fg8):
+    raw = _raw(fg8)
+    f = raw.fg8_grouped_row_expert
+    assert f(FAKE, 0, 256, FAKE, None) == 1
+    assert f(FAKE, 4, -1, FAKE, None) == 1
+    assert f(None, 4, 256, FAKE, None) == 1
+    assert f(FAKE, 4, 100, FAKE, None) == 2       # slabs must be whole 128-row blocks
+    assert f(FAKE + 2, 4, 256, FAKE, None) == 2
+    assert f(None, 4, 0, None, None) == 0         # nothing to write

@@ -165,3 +165,22 @@ def test_moe_full_size_sampled(fg8, orc):
         yg = (W.bf16_bits(y[rows]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         err = np.abs(yg - y64)
         assert written.all() and (err <= y_tolerance(bound)).all(), f"block {t} (expert {e})"
+
+
+def test_batched_layout(fg8, orc):
+    """The batched layout (E slabs of cap rows, counts[e] routed) through
+    fg8_grouped_row_expert and the grouped GEMM: the index matches its
+    definition, empty and partial slabs skip their trailing blocks."""
+    E, cap, K, N = 4, 256, 256, 136
+    counts = torch.tensor([0, 130, 300, 5], dtype=torch.int32, device="cuda")
+    re = torch.full((E * cap,), 7, dtype=torch.int32, device="cuda")
+    fg8.fg8_grouped_row_expert(counts.data_ptr(), E, cap, re.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    want = np.concatenate([np.where(np.arange(cap) < c, e, -1) for e, c in enumerate(counts.tolist())])
+    assert np.array_equal(re.cpu().numpy(), want.astype(np.int32))
+    x = W.x_normal(E * cap, K, seed=81).cuda()
+    wq, ws = _expert_stack(fg8, [W.normal((N, K), 0.02, seed=82 + e).cuda() for e in range(E)], UE8M0)
+    y, st = _run(fg8, x, re, wq, ws, None, UE8M0)
+    assert st == 0
+    written = _check(orc, x, re, wq, ws, None, y, UE8M0)
+    assert written.sum() == 0 + 256 + 256 + 128  # the blocks whose first row is routed
