@@ -39,6 +39,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "fg8_internal.h"
 #include "ptx.cuh"
 #include "quant_math.cuh"
@@ -715,6 +717,10 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    // the descriptors' fetch overlaps the barrier set-up before the first copy
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
@@ -731,11 +737,6 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(stall, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmY);
   }
   if (warp == 2) {
     if constexpr (C::PAIR) {
@@ -797,14 +798,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
+  // looked up once per process (thread-safe static initialisation)
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
@@ -864,10 +866,14 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.sf_shift = g.sf32 ? 0 : 2;
   if (p.num_tiles == 0) return cudaSuccess;
 
-  static int configured_device = -1;
-  static int max_clusters = 0;
+  // the shared-memory opt-in (and, for CTA pairs, the cluster occupancy) once
+  // per device: one bit per device; calls from several host threads may
+  // repeat it, which is harmless
+  static std::atomic<uint64_t> configured{0};
+  static std::atomic<int> max_clusters{0};
   int dev = 0;
   cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(C::kThreads);
@@ -886,7 +892,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  if (configured_device != dev) {
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     if constexpr (C::PAIR) {
@@ -897,12 +903,13 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
         cudaGetLastError();
         n = num_sms / 2;
       }
-      max_clusters = n;
+      max_clusters.store(n, std::memory_order_relaxed);
     }
-    configured_device = dev;
+    configured.fetch_or(bit, std::memory_order_release);
   }
   if constexpr (C::PAIR) {
-    const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+    const int mc = max_clusters.load(std::memory_order_relaxed);
+    const int clusters = p.num_tiles < mc ? p.num_tiles : mc;
     cfg.gridDim = dim3(2 * clusters);
   } else {
     cfg.gridDim = dim3(p.num_tiles < num_sms ? p.num_tiles : num_sms);

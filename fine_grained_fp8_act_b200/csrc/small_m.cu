@@ -48,6 +48,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "fg8_internal.h"
 #include "ptx.cuh"
 #include "quant_math.cuh"
@@ -621,6 +623,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   const int kb0 = static_cast<int>(static_cast<int64_t>(sp) * p.Kb / p.S);
   const int kb1 = static_cast<int>(static_cast<int64_t>(sp + 1) * p.Kb / p.S);
   if (threadIdx.x == 0) {
+    // the descriptors' fetch overlaps the barrier set-up before the first copy
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(wfull + s, 1);
       mbar_init(xfull + s, 1);
@@ -640,8 +645,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbarrier_init();
-    prefetch_tmap(&tmW);
-    prefetch_tmap(&tmX);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -683,14 +686,15 @@ typedef CUresult (*EncodeTiledFnSm)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFnSm encode_fn_sm() {
-  static EncodeTiledFnSm fn = nullptr;
-  if (fn == nullptr) {
+  // looked up once per process (thread-safe static initialisation)
+  static const EncodeTiledFnSm fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnSm>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFnSm>(ptr);
+    return static_cast<EncodeTiledFnSm>(nullptr);
+  }();
   return fn;
 }
 
@@ -751,13 +755,16 @@ cudaError_t launch_small_m_cfg(const SmallMArgs& a, cudaStream_t s) {
   p.test_stall = a.test_stall;
   const int nt = (a.N + 127) / 128;
   auto kern = fg8_small_m_kernel<C>;
-  static int configured_device = -1;
+  // the shared-memory opt-in, once per device (one bit per device; calls from
+  // several host threads may repeat it, which is harmless)
+  static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  const uint64_t bit = 1ull << (dev & 63);
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
+    configured.fetch_or(bit, std::memory_order_release);
   }
   if (a.splits > 1 && a.zero_counters) {  // arrival counters outside the header start at zero
     const cudaError_t e = cudaMemsetAsync(a.counters, 0, static_cast<size_t>(nt) * sizeof(uint32_t), s);
