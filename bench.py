@@ -481,59 +481,87 @@ def run_fg8(args, rank, world, local):
 
 
 def run_e2e(fg8, plan, args, stream, dev, world, chain):
-    """Same metric through the public calls with host buffers: pinned x -> device,
-    the layers (chained as in the device-timed step, else fg8_linear per layer),
-    y -> pinned host, every step inside the timed region."""
+    """Same metric through the public calls with host buffers, as a serving
+    loop runs it: every step copies its input from pinned host memory to the
+    device, runs the layers (chained as in the device-timed step, else
+    fg8_linear per layer) and copies its output back to pinned host memory,
+    all inside the timed region.  The copies go on their own streams, so a
+    step's input copy and the previous step's output copy overlap the
+    kernels; two device buffers each for the input and the output, ordered
+    by events, keep a copy from touching a buffer still in use."""
     L0, Ln = plan[0], plan[-1]
+    slots = 2
     x_host = L0["x"].to("cpu").pin_memory()
-    y_host = torch.empty(Ln["y"].shape, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(L0["x"])
+    y_host = [torch.empty(Ln["y"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(slots)]
+    x_dev = [torch.empty_like(L0["x"]) for _ in range(slots)]
+    y_dev = [torch.empty_like(Ln["y"]) for _ in range(slots)]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(slots)]     # x_dev[s] holds the step's input
+    ev_done = [torch.cuda.Event() for _ in range(slots)]   # the step's kernels are done with x_dev[s], y_dev[s] written
+    ev_out = [torch.cuda.Event() for _ in range(slots)]    # y_dev[s] has been copied out
     sp = stream.cuda_stream
     steps = max(3, min(args.steps, 50))
 
-    def one():
-        x_dev.copy_(x_host, non_blocking=True)
+    def layers(xin, yout):
         if chain:
             g = L0["g"]
-            fg8.fg8_linear_prepare(x_dev.data_ptr(), g.M, g.N, g.K, x_dev.stride(0), L0["ws"].data_ptr(), g.fmt,
+            fg8.fg8_linear_prepare(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L0["ws"].data_ptr(), g.fmt,
                                    L0["wsp"].data_ptr(), L0["wsp"].numel(), sp)
             for i, L in enumerate(plan):
                 g = L["g"]
+                y = yout if i + 1 == len(plan) else L["y"]
                 if i + 1 < len(plan):
                     Lx = plan[i + 1]
                     fg8.fg8_linear_run_chain(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(),
-                                             L["y"].data_ptr(), g.M, g.N, g.K, L["y"].stride(0), g.fmt,
+                                             y.data_ptr(), g.M, g.N, g.K, y.stride(0), g.fmt,
                                              L["wsp"].data_ptr(), L["wsp"].numel(), Lx["g"].N, Lx["ws"].data_ptr(),
                                              Lx["wsp"].data_ptr(), Lx["wsp"].numel(), sp)
                 else:
-                    fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(),
-                                       g.M, g.N, g.K, L["y"].stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(),
-                                       sp)
+                    fg8.fg8_linear_run(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(), y.data_ptr(),
+                                       g.M, g.N, g.K, y.stride(0), g.fmt, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
         else:
-            xin = x_dev
-            for L in plan:
+            for i, L in enumerate(plan):
                 g = L["g"]
+                y = yout if i + 1 == len(plan) else L["y"]
                 fg8.fg8_linear_block(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(),
-                                     L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt,
+                                     L["ws"].data_ptr(), L["b"].data_ptr(), y.data_ptr(), y.stride(0), g.fmt,
                                      args.block, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
-                xin = L["y"]
-        y_host.copy_(Ln["y"], non_blocking=True)
+                xin = y
 
-    for _ in range(3):
-        one()
+    def one(k, start=None):
+        s = k % slots
+        with torch.cuda.stream(h2d):
+            if start is not None:
+                h2d.wait_event(start)
+            h2d.wait_event(ev_done[s])           # the step two back has finished reading x_dev[s]
+            x_dev[s].copy_(x_host, non_blocking=True)
+            ev_in[s].record(h2d)
+        stream.wait_event(ev_in[s])
+        stream.wait_event(ev_out[s])             # y_dev[s] of the step two back has been copied out
+        layers(x_dev[s], y_dev[s])
+        ev_done[s].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_done[s])
+            y_host[s].copy_(y_dev[s], non_blocking=True)
+            ev_out[s].record(d2h)
+
+    for k in range(3):
+        one(k)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        one()
+    for k in range(steps):
+        one(k, e0 if k == 0 else None)
+    stream.wait_event(ev_out[(steps - 1) % slots])  # the last output is on the host (the d2h stream is in order)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     flops = sum_over_ranks(sum(gemm_flops(L["g"]) for L in plan) * steps, world, dev)
     return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 2,
-            "steps": steps, "ms_per_step": ms / steps}
+            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host[0].numel() * 2,
+            "steps": steps, "ms_per_step": ms / steps,
+            "overlap": "input and output copies on their own streams, overlapping the neighbouring steps' kernels"}
 
 
 # ---------------------------------------------------- MoE experts (fg8) ----
