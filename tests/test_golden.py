@@ -40,3 +40,23 @@ def test_group_and_block_width(orc):
     x = np.zeros((1, 129), dtype=np.uint16)
     _, xs = orc.quantize_act(x, 0)
     assert xs.shape == (1, 2)  # a group boundary every 128 channels
+
+
+def test_tested_block_size_in_oracle(orc):
+    """The non-default block size the pages' tests cover: 1 x 32 activation
+    groups and 32 x 32 weight blocks, scales shaped by the same ceil rule."""
+    g = _load()
+    bs = g["tested_block_size"]["value"]
+    assert bs == [32, 32]
+    x = np.zeros((2, 80), dtype=np.uint16)
+    w = np.zeros((40, 80), dtype=np.uint16)
+    for fmt in (0, 1):
+        _, xs = orc.quantize_act(x, fmt, bs[1])
+        _, ws = orc.quantize_weight(w, fmt, bs[0])
+        assert xs.shape == (2, 3) and ws.shape == (2, 3)
+
+
+def test_expert_workload_uses_the_blackwell_expert_format():
+    import bench
+    g = _load()
+    assert bench.moe_config(0, 0)["scale_fmt"] == g["blackwell_expert_scale_fmt"]["value"]
