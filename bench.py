@@ -460,9 +460,8 @@ def run_fg8(args, rank, world, local):
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": dict(workload_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)],
-                                       args.block),
-                       parallelism=f"dp{world} (token rows, replicated weights, no collective)"),
+        "config": dense_arm_config(args.workload, [(c, L["g"], s) for (c, _, s), L in zip(layers, plan)],
+                                   args.block, world),
         "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
         "act_quant_gbs": [k["act_quant_gbs"] for k in per_kernel if k["act_quant_gbs"] is not None],
         "chained": chain,
@@ -582,6 +581,25 @@ def moe_config(rows_routed, rows_padded):
             "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the step events)"}
 
 
+def dense_arm_config(workload, layers, block, world):
+    """The `config` of a dense workload's line, the same on both arms."""
+    return dict(workload_config(workload, layers, block),
+                parallelism=f"dp{world} (token rows, replicated weights, no collective)")
+
+
+def moe_layout():
+    """The seeded routing of the MoE workload: (row_token, row_expert, padded rows, routed rows)."""
+    c = W.DSV3_MOE
+    rt, re = W.moe_routing(c["tokens"], c["experts"], c["topk"], seed=5, skew=c["skew"])
+    return rt, re, int(re.numel()), c["tokens"] * c["topk"]
+
+
+def moe_arm_config(world):
+    """The `config` of the MoE workload's line, the same on both arms."""
+    _, _, Mp, routed = moe_layout()
+    return dict(moe_config(routed, Mp), parallelism=f"dp{world} (token rows, replicated experts, no collective)")
+
+
 def run_moe(args, rank, world, local):
     """The MoE expert layers through fg8_grouped_linear (prepare + grouped GEMM per
     layer).  TFLOP/s count the routed rows only (padding rows are work done but
@@ -594,8 +612,7 @@ def run_moe(args, rank, world, local):
     sp = stream.cuda_stream
     c = W.DSV3_MOE
     T, E, topk, fmt = c["tokens"], c["experts"], c["topk"], 1
-    rt, re = W.moe_routing(T, E, topk, seed=5, skew=c["skew"])
-    Mp, routed = int(re.numel()), T * topk
+    rt, re, Mp, routed = moe_layout()
     re_d = re.to(dev)
     plan = []
     for i, (name, K, N) in enumerate(moe_shapes()):
@@ -751,7 +768,7 @@ def run_moe(args, rank, world, local):
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": dict(moe_config(routed, Mp), parallelism=f"dp{world} (token rows, replicated experts, no collective)"),
+        "config": moe_arm_config(world),
         "pct_fp8_peak": 100.0 * tflops / world / fp8_peak,
         "per_kernel": per_kernel, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": 3 * len(plan) * args.steps,  # act-quant, scale packing, grouped GEMM per layer
@@ -763,13 +780,19 @@ def run_moe(args, rank, world, local):
         torch.distributed.destroy_process_group()
 
 
-def cpu_baseline_moe(budget_s=15.0, rows=None):
-    """The CPU oracle's grouped layer, as it stands, on the first R rows of the
-    routed layout (all in the first expert block) of each expert layer; weights
-    of that block's expert quantized outside the timing.  TFLOP/s of those rows."""
+def threads_note(rows, threads):
+    """The oracle's GEMM spreads sampled rows over its threads: say so when some stay idle there."""
+    return "" if rows >= threads else f"; the GEMM keeps {rows} of the {threads} threads busy"
+
+
+def oracle_moe_sample():
+    """Inputs of the CPU oracle's MoE sample, built once: the first expert block's
+    routed rows of each expert layer and that expert's quantized weights.
+    Returns (run, expert): run(R) times the oracle's grouped layer on the first
+    R rows (R <= 128) of both layers and returns (seconds, FLOPs)."""
     import oracle
     c = W.DSV3_MOE
-    rt, re = W.moe_routing(c["tokens"], c["experts"], c["topk"], seed=5, skew=c["skew"])
+    rt, re, _, _ = moe_layout()
     e0 = int(re[0])
     ops = []
     for i, (name, K, N) in enumerate(moe_shapes()):
@@ -783,24 +806,33 @@ def cpu_baseline_moe(budget_s=15.0, rows=None):
         t0 = time.perf_counter()
         for K, N, x, wq, ws in ops:
             oracle.grouped_linear(x[:R], rexp[:R], wq, ws, None, 1)
-        return time.perf_counter() - t0
+        return time.perf_counter() - t0, sum(2.0 * R * N * K for K, N, _, _, _ in ops)
 
+    return run, e0
+
+
+def cpu_baseline_moe(budget_s=15.0, rows=None):
+    """The CPU oracle's grouped layer, as it stands, on the first R rows of the
+    routed layout (all in the first expert block) of each expert layer; weights
+    of that block's expert quantized outside the timing.  TFLOP/s of those rows."""
+    import oracle
+    run, e0 = oracle_moe_sample()
     if rows is None:
-        t = run(2)
+        t, _ = run(2)
         rows = int(max(2, min(128, 2 * budget_s / max(t, 1e-6))))
-    t = run(rows)
-    flops = sum(2.0 * rows * N * K for K, N, _, _, _ in ops)
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+    t, flops = run(rows)
+    nt = oracle.num_threads()
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
             "sample": f"first {rows} routed rows (expert {e0}) through both expert layers ({t:.1f} s; weights "
-                      f"quantized outside the timing)", "seconds": t, "rows": rows}
+                      f"quantized outside the timing{threads_note(rows, nt)})", "seconds": t, "rows": rows}
 
 
 # ------------------------------------------------------ oracle (CPU) arm ----
-def cpu_baseline(workload, budget_s=15.0, rows=None, block=128):
-    """The CPU oracle, as it stands, on a bounded sample of the workload: the
-    first R token rows of the batch through every layer (quantize, dequantized
-    double GEMM, bf16 out), weights quantized once outside the timing.
-    Reported in TFLOP/s of the sampled rows."""
+def oracle_dense_sample(workload, block=128):
+    """Inputs of the CPU oracle's sample of a dense workload, built once (the
+    batch's bf16 rows, every layer's quantized weights and bias).  run(R) times
+    the first R token rows through every layer (quantize, dequantized double
+    GEMM, bf16 out) and returns (seconds, FLOPs)."""
     import oracle
     layers = workload_layers(workload)
     ops = []
@@ -818,37 +850,51 @@ def cpu_baseline(workload, budget_s=15.0, rows=None, block=128):
         for g, wq, ws, bb in ops:
             _, _, ybf = oracle.linear(a, wq, ws, bb, g.fmt, block=block)
             a = ybf
-        return time.perf_counter() - t0
+        return time.perf_counter() - t0, sum(2.0 * R * g.N * g.K for g, _, _, _ in ops)
 
+    return run
+
+
+def cpu_baseline(workload, budget_s=15.0, rows=None, block=128):
+    """The CPU oracle, as it stands, on a bounded sample of the workload: the
+    first R token rows of the batch through every layer, weights quantized once
+    outside the timing.  Reported in TFLOP/s of the sampled rows."""
+    import oracle
+    layers = workload_layers(workload)
+    run = oracle_dense_sample(workload, block)
     if rows is None:
         probe = 16
-        t = run(probe)
+        t, _ = run(probe)
         rows = int(max(16, min(layers[0][1].M, probe * budget_s / max(t, 1e-6))))
-    t = run(rows)
-    flops = sum(2.0 * rows * g.N * g.K for g, _, _, _ in ops)
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(ops)} layers "
-                      f"({t:.1f} s; weights quantized outside the timing)",
-            "seconds": t}
+    t, flops = run(rows)
+    nt = oracle.num_threads()
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
+            "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(layers)} layers "
+                      f"({t:.1f} s; weights quantized outside the timing{threads_note(rows, nt)})",
+            "seconds": t, "rows": rows}
 
 
-def run_reference_moe(args):
-    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
-    probe = cpu_baseline_moe(rows=2)
-    rows = int(max(1, min(128, 2 * budget / max(probe["seconds"], 1e-6))))
+def run_reference_moe(args, world):
+    import oracle
+    run, _ = oracle_moe_sample()
+    # size each step so warm-up + steps take about --ref-seconds (2 minutes by default)
+    budget = max(0.05, args.ref_seconds / max(1, args.steps + args.warmup))
+    t_probe, _ = run(2)
+    rows = int(max(1, min(128, 2 * budget / max(t_probe, 1e-6))))
     for _ in range(args.warmup):
-        cpu_baseline_moe(rows=rows)
-    ts = [cpu_baseline_moe(rows=rows)["seconds"] for _ in range(args.steps)]
+        run(rows)
+    ts = [run(rows)[0] for _ in range(args.steps)]
     flops = sum(2.0 * rows * N * K for _, K, N in moe_shapes())
     value = flops * len(ts) / sum(ts) / 1e12
-    c = W.DSV3_MOE
-    cpu = {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-           "sample": f"first {rows} routed rows through both expert layers per step"}
-    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+    nt = oracle.num_threads()
+    cpu = {"value": value, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
+           "sample": f"first {rows} routed rows through both expert layers per step on the host cores of "
+                     f"rank 0{threads_note(rows, nt)}"}
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: float32 quantization, double GEMM)",
            "data": "synthetic", "impl": "reference",
-           "config": dict(moe_config(c["tokens"] * c["topk"], None), parallelism="cpu oracle, rank 0 only"),
+           "config": moe_arm_config(world),
            "cpu_baseline": cpu,
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -858,28 +904,30 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     if args.workload.startswith("moe_"):
-        run_reference_moe(args)
+        run_reference_moe(args, world)
         return
+    import oracle
     layers = workload_layers(args.workload)
-    # size each step so warm-up + steps stay within ~2 minutes
-    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
-    probe = cpu_baseline(args.workload, rows=16, block=args.block)
-    rows = int(max(1, min(layers[0][1].M, 16 * budget / max(probe["seconds"], 1e-6))))
+    run = oracle_dense_sample(args.workload, args.block)
+    # size each step so warm-up + steps take about --ref-seconds (2 minutes by default)
+    budget = max(0.05, args.ref_seconds / max(1, args.steps + args.warmup))
+    t_probe, _ = run(16)
+    rows = int(max(1, min(layers[0][1].M, 16 * budget / max(t_probe, 1e-6))))
     for _ in range(args.warmup):
-        cpu_baseline(args.workload, rows=rows, block=args.block)
-    ts = []
-    for _ in range(args.steps):
-        ts.append(cpu_baseline(args.workload, rows=rows, block=args.block)["seconds"])
+        run(rows)
+    ts = [run(rows)[0] for _ in range(args.steps)]
     flops = sum(2.0 * rows * g.N * g.K for _, g, _ in layers)
     tot = sum(ts)
     value = flops * len(ts) / tot / 1e12
-    cpu = {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-           "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(layers)} layers per step"}
+    nt = oracle.num_threads()
+    cpu = {"value": value, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
+           "sample": f"first {rows} of {layers[0][1].M} token rows through all {len(layers)} layers per step "
+                     f"on the host cores of rank 0{threads_note(rows, nt)}"}
     out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: float32 quantization, double GEMM)",
            "data": "synthetic", "impl": "reference",
-           "config": dict(workload_config(args.workload, layers, args.block), parallelism="cpu oracle, rank 0 only"),
+           "config": dense_arm_config(args.workload, layers, args.block, world),
            "cpu_baseline": cpu,
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -894,6 +942,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: CPU seconds that the warm-up and timed steps together aim at")
     ap.add_argument("--block", type=int, default=128, choices=[128, 32],
                     help="weight_block_size (block, block) and 1 x block activation groups; 32 takes UE8M0 workloads")
     ap.add_argument("--no-chain", action="store_true",

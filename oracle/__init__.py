@@ -35,6 +35,8 @@ def lib():
         L = ctypes.CDLL(path)
         c_u8p = ctypes.POINTER(ctypes.c_uint8)
         L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_num_threads.restype = ctypes.c_int
+        L.orc_num_threads.argtypes = []
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_encode.restype = ctypes.c_uint8
         L.orc_e4m3_encode.argtypes = [ctypes.c_float]
@@ -97,6 +99,11 @@ def _scale_dtype(fmt):
 
 
 # ---------------------------------------------------------------- scalars --
+def num_threads() -> int:
+    """Host threads the oracle's OpenMP loops run on."""
+    return int(lib().orc_num_threads())
+
+
 def e4m3_value(code: int) -> float:
     return lib().orc_e4m3_value(int(code))
 

@@ -33,6 +33,8 @@
 #include <cstring>
 #include <vector>
 
+#include <omp.h>
+
 static_assert(FLT_EVAL_METHOD == 0, "float expressions must evaluate in float");
 
 namespace {
@@ -381,5 +383,9 @@ int orc_quantize_act_static(const uint16_t* x, int64_t M, int64_t K, int64_t ld_
     for (int64_t k = 0; k < K; ++k) xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) / s);
   return 0;
 }
+
+// Team size of the OpenMP loops above (OMP_NUM_THREADS, else the CPUs this
+// process may run on), for reporting how many host threads a timing used.
+int orc_num_threads(void) { return omp_get_max_threads(); }
 
 }  // extern "C"

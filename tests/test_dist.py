@@ -43,8 +43,8 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_reductions():
     port = _free_port()
-    out = mp.Manager().dict()
-    ctx = mp.get_context("spawn")
+    ctx = mp.get_context("spawn")  # never fork: this process may already run the oracle's OpenMP threads
+    out = ctx.Manager().dict()
     procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
     for p in procs:
         p.start()
