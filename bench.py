@@ -731,36 +731,61 @@ def run_moe(args, rank, world, local):
                   for i, L in enumerate(plan)]
 
     # end to end: routed rows and the expert index in from pinned host memory,
-    # both layers, the last layer's rows out
+    # both layers, the last layer's rows out.  As in the dense leg, the copies
+    # run on their own streams (a step's input copy and the previous step's
+    # output copy overlap the kernels) with two device slots ordered by events.
+    slots = 2
     xh = [L["x"].to("cpu").pin_memory() for L in plan]
     reh = re.pin_memory()
-    xd = [torch.empty_like(L["x"]) for L in plan]
-    red = torch.empty_like(re_d)
-    yh = torch.empty(plan[-1]["y"].shape, dtype=torch.bfloat16).pin_memory()
+    yh = [torch.empty(plan[-1]["y"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(slots)]
+    xd = [[torch.empty_like(L["x"]) for L in plan] for _ in range(slots)]
+    red = [torch.empty_like(re_d) for _ in range(slots)]
+    yd = [torch.empty_like(plan[-1]["y"]) for _ in range(slots)]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(slots)]    # slot s holds the step's inputs
+    ev_done = [torch.cuda.Event() for _ in range(slots)]  # the step's kernels are done with slot s
+    ev_out = [torch.cuda.Event() for _ in range(slots)]   # yd[s] has been copied out
     e2e_steps = max(3, min(args.steps, 20))
 
-    def one():
-        red.copy_(reh, non_blocking=True)
-        for L, a, b in zip(plan, xh, xd):
-            b.copy_(a, non_blocking=True)
-            fg8.fg8_grouped_linear(b.data_ptr(), Mp, L["K"], L["K"], red.data_ptr(), E, L["N"], L["wq"].data_ptr(),
-                                   L["ws"].data_ptr(), None, L["y"].data_ptr(), L["N"], fmt, L["wsp"].data_ptr(),
+    def one(k, start=None):
+        s = k % slots
+        with torch.cuda.stream(h2d):
+            if start is not None:
+                h2d.wait_event(start)
+            h2d.wait_event(ev_done[s])  # the step two back has finished reading slot s
+            red[s].copy_(reh, non_blocking=True)
+            for a, b in zip(xh, xd[s]):
+                b.copy_(a, non_blocking=True)
+            ev_in[s].record(h2d)
+        stream.wait_event(ev_in[s])
+        stream.wait_event(ev_out[s])    # yd[s] of the step two back has been copied out
+        for i, (L, b) in enumerate(zip(plan, xd[s])):
+            y = yd[s] if i + 1 == len(plan) else L["y"]
+            fg8.fg8_grouped_linear(b.data_ptr(), Mp, L["K"], L["K"], red[s].data_ptr(), E, L["N"], L["wq"].data_ptr(),
+                                   L["ws"].data_ptr(), None, y.data_ptr(), L["N"], fmt, L["wsp"].data_ptr(),
                                    L["wsp"].numel(), sp)
-        yh.copy_(plan[-1]["y"], non_blocking=True)
-    for _ in range(3):
-        one()
+        ev_done[s].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_done[s])
+            yh[s].copy_(yd[s], non_blocking=True)
+            ev_out[s].record(d2h)
+
+    for k in range(3):
+        one(k)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        one()
+    for k in range(e2e_steps):
+        one(k, e0 if k == 0 else None)
+    stream.wait_event(ev_out[(e2e_steps - 1) % slots])  # the last output is on the host (d2h runs in order)
     e1.record(stream)
     torch.cuda.synchronize()
     ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e = {"value": sum_over_ranks(flops_step * e2e_steps, world, dev) / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": sum(a.numel() * 2 for a in xh) + reh.numel() * 4,
-           "d2h_bytes_per_step": yh.numel() * 2, "steps": e2e_steps, "ms_per_step": ems / e2e_steps}
+           "d2h_bytes_per_step": yh[0].numel() * 2, "steps": e2e_steps, "ms_per_step": ems / e2e_steps,
+           "overlap": "input and output copies on their own streams, overlapping the neighbouring steps' kernels"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_moe(budget_s=args.cpu_seconds)
