@@ -37,11 +37,63 @@ def _cdiv(a: int, b: int) -> int:
     return (a + b - 1) // b
 
 
+# The C ABI takes raw pointers and cannot see how large a buffer is, so every
+# operand a kernel reads or writes is checked here against the shape, dtype and
+# device the call implies before its pointer is passed on.  e4m3 codes and UE8M0
+# scales may also come as raw uint8 bytes (the same bits).
+_E4M3 = (torch.float8_e4m3fn, torch.uint8)
+
+
+def _scale_dtypes(fmt: int):
+    return (torch.float32,) if fmt == C.FG8_SCALE_FLOAT else (torch.float8_e8m0fnu, torch.uint8)
+
+
 def _check_bf16_matrix(t: torch.Tensor, name: str):
-    if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_cuda:
-        raise ValueError(f"{name} must be a 2-D bf16 CUDA tensor")
-    if t.stride(1) != 1:
-        raise ValueError(f"{name} must have unit stride in its last dimension")
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D bf16 tensor")
+    if t.stride(1) != 1 or (t.shape[0] > 1 and t.stride(0) < t.shape[1]):
+        raise ValueError(f"{name} must have unit stride in its last dimension and rows that do not overlap")
+
+
+def _check_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _check_tensor(t, name: str, shape, dtypes, device):
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_weight(wq, w_scale_inv, lead, N: int, K: int, fmt: int, block: int, device):
+    """wq e4m3 [*lead, N, K] and its block scales [*lead, ceil(N/block), ceil(K/block)]."""
+    _check_tensor(wq, "wq", (*lead, N, K), _E4M3, device)
+    _check_tensor(w_scale_inv, "w_scale_inv", (*lead, _cdiv(N, block), _cdiv(K, block)), _scale_dtypes(fmt), device)
+
+
+def _check_bias(bias, shape, device) -> int:
+    if bias is None:
+        return 0
+    _check_tensor(bias, "bias", shape, (torch.bfloat16,), device)
+    return bias.data_ptr()
+
+
+def _output(out, M: int, N: int, device) -> torch.Tensor:
+    """out as given (bf16 [M, N], unit column stride, row stride >= N) or a new tensor."""
+    if out is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    _check_bf16_matrix(out, "out")
+    if tuple(out.shape) != (M, N) or out.device != device:
+        raise ValueError(f"out must be [{M}, {N}] on {device}")
+    return out
 
 
 def quantize_weight(w: torch.Tensor, scale_fmt="float", block: int = 128) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -49,6 +101,7 @@ def quantize_weight(w: torch.Tensor, scale_fmt="float", block: int = 128) -> Tup
     block x block weight blocks, block 128 (default) or 32."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(w, "w")
+    _check_cuda(w, "w")
     N, K = w.shape
     wq = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
     ws = torch.empty((_cdiv(N, block), _cdiv(K, block)), dtype=_SCALE_DTYPES[fmt], device=w.device)
@@ -62,6 +115,7 @@ def quantize_act(x: torch.Tensor, scale_fmt="float", block: int = 128) -> Tuple[
     """x bf16 [M, K] -> (xq float8_e4m3fn [M, K], x_scale [M, ceil(K/block)]); 1 x block groups."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
+    _check_cuda(x, "x")
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     xs = torch.empty((M, _cdiv(K, block)), dtype=_SCALE_DTYPES[fmt], device=x.device)
@@ -77,6 +131,7 @@ def quantize_act_static(x: torch.Tensor, act_scale: torch.Tensor) -> Tuple[torch
     _check_bf16_matrix(x, "x")
     if act_scale.dtype != torch.float32 or act_scale.numel() != 1 or act_scale.device != x.device:
         raise ValueError("act_scale must be one float32 on x's device")
+    _check_cuda(x, "x")
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     xs = torch.empty((M, _cdiv(K, 128)), dtype=torch.float32, device=x.device)
@@ -88,6 +143,8 @@ def quantize_act_static(x: torch.Tensor, act_scale: torch.Tensor) -> Tuple[torch
 
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
     if workspace is not None:
+        if workspace.device != device or not workspace.is_contiguous():
+            raise ValueError(f"workspace must be a contiguous tensor on {device}")
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError(f"workspace too small: need {nbytes} bytes")
         return workspace
@@ -103,16 +160,19 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: O
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
     M, K = x.shape
-    N = wq.shape[0]
-    if wq.shape != (N, K):
+    if wq.dim() != 2:
         raise ValueError("wq must be [N, K]")
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    N = int(wq.shape[0])
+    _check_weight(wq, w_scale_inv, (), N, K, fmt, block, x.device)
+    bp = _check_bias(bias, (N,), x.device)
+    y = _output(out, M, N, x.device)
+    _check_cuda(x, "x")
     nbytes = C.fg8_linear_block_workspace_bytes(M, N, K, fmt, block)  # 0: the call below reports why
     ws = _workspace(nbytes, x.device, workspace)
     with torch.cuda.device(x.device):
-        C.fg8_linear_block(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(),
-                           0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0), fmt, block,
-                           ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
+        C.fg8_linear_block(x.data_ptr(), M, N, K, x.stride(0), wq.data_ptr(), w_scale_inv.data_ptr(), bp,
+                           y.data_ptr(), y.stride(0), fmt, block, ws.data_ptr(), ws.numel() * ws.element_size(),
+                           _stream(x))
     return y
 
 
@@ -127,18 +187,19 @@ def grouped_linear(x: torch.Tensor, row_expert: torch.Tensor, wq: torch.Tensor, 
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
     M, K = x.shape
-    if wq.dim() != 3 or wq.shape[2] != K:
+    if wq.dim() != 3:
         raise ValueError("wq must be [E, N, K]")
     E, N = int(wq.shape[0]), int(wq.shape[1])
-    if row_expert.dtype != torch.int32 or row_expert.shape != (M,) or row_expert.device != x.device:
-        raise ValueError("row_expert must be int32 [M] on x's device")
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check_weight(wq, w_scale_inv, (E,), N, K, fmt, 128, x.device)
+    _check_tensor(row_expert, "row_expert", (M,), (torch.int32,), x.device)
+    bp = _check_bias(bias, (E, N), x.device)
+    y = _output(out, M, N, x.device)
+    _check_cuda(x, "x")
     ws = _workspace(C.fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt), x.device, workspace)
     with torch.cuda.device(x.device):
-        C.fg8_grouped_linear(x.data_ptr(), M, K, x.stride(0), row_expert.contiguous().data_ptr(), E, N,
-                             wq.data_ptr(), w_scale_inv.data_ptr(), 0 if bias is None else bias.data_ptr(),
-                             y.data_ptr(), y.stride(0), fmt, ws.data_ptr(), ws.numel() * ws.element_size(),
-                             _stream(x))
+        C.fg8_grouped_linear(x.data_ptr(), M, K, x.stride(0), row_expert.data_ptr(), E, N, wq.data_ptr(),
+                             w_scale_inv.data_ptr(), bp, y.data_ptr(), y.stride(0), fmt, ws.data_ptr(),
+                             ws.numel() * ws.element_size(), _stream(x))
     return y
 
 
@@ -150,13 +211,18 @@ def linear_static(x: torch.Tensor, act_scale: torch.Tensor, wq: torch.Tensor, w_
     if act_scale.dtype != torch.float32 or act_scale.numel() != 1 or act_scale.device != x.device:
         raise ValueError("act_scale must be one float32 on x's device")
     M, K = x.shape
-    N = wq.shape[0]
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if wq.dim() != 2:
+        raise ValueError("wq must be [N, K]")
+    N = int(wq.shape[0])
+    _check_weight(wq, w_scale_inv, (), N, K, C.FG8_SCALE_FLOAT, 128, x.device)
+    bp = _check_bias(bias, (N,), x.device)
+    y = _output(out, M, N, x.device)
+    _check_cuda(x, "x")
     ws = _workspace(C.fg8_linear_workspace_bytes(M, N, K, C.FG8_SCALE_FLOAT), x.device, workspace)
     with torch.cuda.device(x.device):
         C.fg8_linear_static(x.data_ptr(), M, N, K, x.stride(0), act_scale.data_ptr(), wq.data_ptr(),
-                            w_scale_inv.data_ptr(), 0 if bias is None else bias.data_ptr(), y.data_ptr(), y.stride(0),
-                            ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
+                            w_scale_inv.data_ptr(), bp, y.data_ptr(), y.stride(0), ws.data_ptr(),
+                            ws.numel() * ws.element_size(), _stream(x))
     return y
 
 
@@ -165,15 +231,22 @@ def gemm_prequant(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_s
                   workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The GEMM on already-quantized activations (layouts of quantize_act)."""
     fmt = scale_fmt_code(scale_fmt)
-    M, K = xq.shape
-    N = wq.shape[0]
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    if not isinstance(xq, torch.Tensor) or xq.dim() != 2 or wq.dim() != 2:
+        raise ValueError("xq must be [M, K] and wq [N, K]")
+    M, K = int(xq.shape[0]), int(xq.shape[1])
+    N = int(wq.shape[0])
+    _check_tensor(xq, "xq", (M, K), _E4M3, xq.device)
+    _check_tensor(x_scale, "x_scale", (M, _cdiv(K, 128)), _scale_dtypes(fmt), xq.device)
+    _check_weight(wq, w_scale_inv, (), N, K, fmt, 128, xq.device)
+    bp = _check_bias(bias, (N,), xq.device)
+    y = _output(out, M, N, xq.device)
+    _check_cuda(xq, "xq")
     nbytes = C.fg8_gemm_workspace_bytes(M, N, K, fmt)
     ws = _workspace(nbytes, xq.device, workspace)
     with torch.cuda.device(xq.device):
-        C.fg8_gemm_prequant(xq.data_ptr(), x_scale.data_ptr(), wq.data_ptr(), w_scale_inv.data_ptr(),
-                            0 if bias is None else bias.data_ptr(), y.data_ptr(), M, N, K, y.stride(0), fmt,
-                            ws.data_ptr(), ws.numel() * ws.element_size(), _stream(xq))
+        C.fg8_gemm_prequant(xq.data_ptr(), x_scale.data_ptr(), wq.data_ptr(), w_scale_inv.data_ptr(), bp,
+                            y.data_ptr(), M, N, K, y.stride(0), fmt, ws.data_ptr(), ws.numel() * ws.element_size(),
+                            _stream(xq))
     return y
 
 
@@ -187,11 +260,18 @@ def linear_chain(x: torch.Tensor, layers, scale_fmt="float", workspaces=None):
     M = x.shape[0]
     dims = []
     k = x.shape[1]
-    for i, (wq, _, _) in enumerate(layers):
+    for i, (wq, wsc, b) in enumerate(layers):
         if wq.dim() != 2 or wq.shape[1] != k:
             raise ValueError(f"layer {i}: wq must be [N, {k}]")
-        dims.append((wq.shape[0], k))
-        k = wq.shape[0]
+        n = int(wq.shape[0])
+        try:
+            _check_weight(wq, wsc, (), n, k, fmt, 128, x.device)
+            _check_bias(b, (n,), x.device)
+        except ValueError as e:
+            raise ValueError(f"layer {i}: {e}") from None
+        dims.append((n, k))
+        k = n
+    _check_cuda(x, "x")
     if workspaces is None:
         workspaces = [None] * len(layers)
     wss = [_workspace(C.fg8_linear_workspace_bytes(M, n, kk, fmt), x.device, w)
@@ -218,9 +298,11 @@ def linear_chain(x: torch.Tensor, layers, scale_fmt="float", workspaces=None):
 def dequantize_weight(wq: torch.Tensor, w_scale_inv: torch.Tensor, scale_fmt="float") -> torch.Tensor:
     """Fp8Dequantize: (e4m3 [N, K], block scales) -> bf16 [N, K] with each block's scale folded in."""
     fmt = scale_fmt_code(scale_fmt)
-    N, K = wq.shape
-    if w_scale_inv.shape != (_cdiv(N, 128), _cdiv(K, 128)) or w_scale_inv.dtype != _SCALE_DTYPES[fmt]:
-        raise ValueError("w_scale_inv must be [ceil(N/128), ceil(K/128)] of the format's dtype")
+    if not isinstance(wq, torch.Tensor) or wq.dim() != 2:
+        raise ValueError("wq must be [N, K]")
+    N, K = int(wq.shape[0]), int(wq.shape[1])
+    _check_weight(wq, w_scale_inv, (), N, K, fmt, 128, wq.device)
+    _check_cuda(wq, "wq")
     w = torch.empty((N, K), dtype=torch.bfloat16, device=wq.device)
     with torch.cuda.device(wq.device):
         C.fg8_dequantize_weight(wq.data_ptr(), N, K, w_scale_inv.data_ptr(), fmt, w.data_ptr(), K, _stream(wq))

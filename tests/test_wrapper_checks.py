@@ -1,0 +1,107 @@
+"""The Python binding's operand checks, on CPU.
+
+The C ABI takes raw pointers, so a scale tensor of the wrong shape or dtype
+would be read out of bounds by a kernel.  The wrappers check every operand
+against the shape, dtype and device the call implies before passing a
+pointer on; these tests feed each wrapper one wrong operand at a time and
+expect a ValueError naming it.  With every operand right but on the CPU the
+last check (CUDA device) fires, so no CPU pointer ever reaches the library.
+"""
+import pytest
+import torch
+
+import fine_grained_fp8_act_b200 as fg8
+
+BF16, F32, U8 = torch.bfloat16, torch.float32, torch.uint8
+E4M3, E8M0 = torch.float8_e4m3fn, torch.float8_e8m0fnu
+M, N, K = 40, 264, 400          # ragged against 128 and 32
+Nb, Kb = 3, 4                   # ceil(264 / 128), ceil(400 / 128)
+
+
+def _dense(fmt="float", block=128):
+    nb, kb = -(-N // block), -(-K // block)
+    x = torch.zeros(M, K, dtype=BF16)
+    wq = torch.zeros(N, K, dtype=E4M3)
+    ws = torch.zeros(nb, kb, dtype=F32 if fmt == "float" else E8M0)
+    b = torch.zeros(N, dtype=BF16)
+    return x, wq, ws, b
+
+
+def _raises(match, fn, *a, **k):
+    with pytest.raises(ValueError, match=match):
+        fn(*a, **k)
+
+
+@pytest.mark.parametrize("fmt", ["float", "ue8m0"])
+def test_linear_operands(fmt):
+    x, wq, ws, b = _dense(fmt)
+    _raises("must be a CUDA tensor", fg8.linear, x, wq, ws, b, fmt)
+    _raises("wq must be", fg8.linear, x, wq.to(BF16), ws, b, fmt)
+    _raises("wq must have shape", fg8.linear, x, wq[:, :K - 16].contiguous(), ws, b, fmt)
+    _raises("wq must be contiguous", fg8.linear, x, torch.zeros(K, N, dtype=E4M3).t(), ws, b, fmt)
+    _raises("w_scale_inv must have shape", fg8.linear, x, wq, ws[:, :Kb - 1].contiguous(), b, fmt)
+    _raises("w_scale_inv must have shape", fg8.linear, x, wq, ws.t().contiguous(), b, fmt)
+    other = torch.zeros(Nb, Kb, dtype=E8M0 if fmt == "float" else F32)
+    _raises("w_scale_inv must be", fg8.linear, x, wq, other, b, fmt)
+    _raises("bias must have shape", fg8.linear, x, wq, ws, b[:N - 1].contiguous(), fmt)
+    _raises("bias must be", fg8.linear, x, wq, ws, b.float(), fmt)
+    _raises("out must be", fg8.linear, x, wq, ws, b, fmt, out=torch.empty(M, N + 1, dtype=BF16)[:, :N - 1])
+    _raises("out must have unit stride", fg8.linear, x, wq, ws, b, fmt, out=torch.empty(N, M, dtype=BF16).t())
+    _raises("x must be a 2-D bf16", fg8.linear, x.float(), wq, ws, b, fmt)
+    _raises("x must have unit stride", fg8.linear, x.as_strided((M, K), (K // 2, 1)), wq, ws, b, fmt)
+    # raw bytes are the same bits: accepted (up to the device check)
+    wsb = ws.view(U8) if fmt == "ue8m0" else ws
+    _raises("must be a CUDA tensor", fg8.linear, x, wq.view(U8), wsb, None, fmt)
+    # row-strided x and out are fine
+    xs = torch.zeros(M, K + 64, dtype=BF16)[:, :K]
+    _raises("must be a CUDA tensor", fg8.linear, xs, wq, ws, b, fmt, out=torch.empty(M, N + 8, dtype=BF16)[:, :N])
+
+
+def test_linear_block32_operands():
+    x, wq, ws, b = _dense("ue8m0", block=32)
+    assert ws.shape == (9, 13)
+    _raises("must be a CUDA tensor", fg8.linear, x, wq, ws, b, "ue8m0", block=32)
+    _raises("w_scale_inv must have shape", fg8.linear, x, wq, ws, b, "ue8m0", block=128)
+    _, _, ws128, _ = _dense("ue8m0")
+    _raises("w_scale_inv must have shape", fg8.linear, x, wq, ws128, b, "ue8m0", block=32)
+
+
+def test_grouped_linear_operands():
+    E = 3
+    x = torch.zeros(256, K, dtype=BF16)
+    re = torch.zeros(256, dtype=torch.int32)
+    wq = torch.zeros(E, N, K, dtype=E4M3)
+    ws = torch.zeros(E, Nb, Kb, dtype=E8M0)
+    b = torch.zeros(E, N, dtype=BF16)
+    _raises("must be a CUDA tensor", fg8.grouped_linear, x, re, wq, ws, b)
+    _raises("wq must be", fg8.grouped_linear, x, re, wq[0], ws, b)
+    _raises("w_scale_inv must have shape", fg8.grouped_linear, x, re, wq, ws[:E - 1].contiguous(), b)
+    _raises("w_scale_inv must be", fg8.grouped_linear, x, re, wq, ws.float(), b)
+    _raises("row_expert must be", fg8.grouped_linear, x, re.long(), wq, ws, b)
+    _raises("row_expert must have shape", fg8.grouped_linear, x, re[:255].contiguous(), wq, ws, b)
+    _raises("bias must have shape", fg8.grouped_linear, x, re, wq, ws, b[0].contiguous())
+    _raises("must be a CUDA tensor", fg8.grouped_linear, x, re, wq, ws.view(U8), None)
+
+
+def test_static_prequant_chain_dequant_operands():
+    x, wq, ws, b = _dense("float")
+    s = torch.ones(1, dtype=F32)
+    _raises("must be a CUDA tensor", fg8.linear_static, x, s, wq, ws, b)
+    _raises("w_scale_inv must be", fg8.linear_static, x, s, wq, ws.to(E8M0), b)
+    _raises("wq must have shape", fg8.linear_static, x, s, torch.zeros(N, K + 16, dtype=E4M3), ws, b)
+
+    xq = torch.zeros(M, K, dtype=E4M3)
+    xs = torch.zeros(M, Kb, dtype=F32)
+    _raises("must be a CUDA tensor", fg8.gemm_prequant, xq, xs, wq, ws, b, "float")
+    _raises("x_scale must have shape", fg8.gemm_prequant, xq, xs.t().contiguous(), wq, ws, b, "float")
+    _raises("x_scale must be", fg8.gemm_prequant, xq, xs.to(E8M0), wq, ws, b, "float")
+    _raises("xq must be", fg8.gemm_prequant, xq.to(BF16), xs, wq, ws, b, "float")
+
+    wq2 = torch.zeros(K, N, dtype=E4M3)
+    ws2 = torch.zeros(Kb, Nb, dtype=F32)
+    _raises("must be a CUDA tensor", fg8.linear_chain, x, [(wq, ws, b), (wq2, ws2, None)])
+    _raises("layer 1: w_scale_inv must have shape", fg8.linear_chain, x, [(wq, ws, b), (wq2, ws, None)])
+    _raises("layer 1: wq must be", fg8.linear_chain, x, [(wq, ws, b), (wq, ws, None)])
+
+    _raises("must be a CUDA tensor", fg8.dequantize_weight, wq, ws, "float")
+    _raises("w_scale_inv must have shape", fg8.dequantize_weight, wq, ws[:1].contiguous(), "float")
