@@ -76,9 +76,9 @@ typedef enum fg8_status {
  *               FG8_SCALE_FLOAT, UE8M0 bytes for FG8_SCALE_UE8M0.
  * W ~= value(wq) * scale_inv per 128x128 block; edge blocks use their real
  * elements only.  One CTA per block on a 2-D grid, so N <= 65535 * 128
- * rows (8,388,480): a larger N fails to launch (FG8_ERR_CUDA, nothing
- * written); quantize such a matrix in row slices that start at multiples
- * of 128 rows and are at most that high. */
+ * rows (8,388,480): a larger N returns FG8_ERR_INVALID_ARG before any
+ * launch; quantize such a matrix in row slices that start at multiples of
+ * 128 rows and are at most that high. */
 FG8_API fg8_status fg8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w,
                                void* wq_e4m3, void* w_scale_inv, fg8_scale_fmt fmt, void* stream);
 

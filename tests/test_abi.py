@@ -155,6 +155,8 @@ def test_quantizers_reject_bad_args(fg8):
     assert raw.fg8_quantize_weight(FAKE, 0, 256, 256, FAKE, FAKE, 0, None) == 1
     assert raw.fg8_quantize_weight(FAKE, 256, 248, 248, FAKE, FAKE, 1, None) == 2
     assert raw.fg8_quantize_weight(None, 256, 256, 256, FAKE, FAKE, 1, None) == 1
+    # one CTA per 128 x 128 block on a 2-D grid: at most 65535 row blocks
+    assert raw.fg8_quantize_weight(FAKE, 65535 * 128 + 1, 256, 256, FAKE, FAKE, 0, None) == 1
 
 
 def test_valid_call_without_gpu_reports_unsupported_device(fg8):
