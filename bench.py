@@ -272,6 +272,34 @@ def gemm_flops(g):
     return 2.0 * g.M * g.N * g.K
 
 
+def weight_quant_bytes(g, block):
+    """HBM bytes of quantizing one weight: bf16 read, e4m3 written, block scales written."""
+    nb, kb = -(-g.N // block), -(-g.K // block)
+    return 3 * g.N * g.K + nb * kb * (4 if g.fmt == 0 else 1)
+
+
+def time_weight_quant(fg8, w, wq, ws, fmt, block, flush_l2, reps=10):
+    """The one-time weight quantization (outside the step), timed after the
+    step's measurement so the clocks are those of a loaded GPU: mean
+    CUDA-event time in ms of `reps` launches of the C entry point into scratch
+    copies of wq / ws on the current stream, L2 flushed before each (the
+    flush's device time also covers the host's enqueue of the launch)."""
+    stream = torch.cuda.current_stream(w.device)
+    wq_t, ws_t = torch.empty_like(wq), torch.empty_like(ws)
+    N, K = w.shape
+    evs = []
+    for _ in range(reps):
+        flush_l2()
+        e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        e[0].record(stream)
+        fg8.fg8_quantize_weight_block(w.data_ptr(), N, K, w.stride(0), wq_t.data_ptr(), ws_t.data_ptr(), fmt, block,
+                                      stream.cuda_stream)
+        e[1].record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
 # ------------------------------------------------------------ fg8 arm ----
 def run_fg8(args, rank, world, local):
     import fine_grained_fp8_act_b200 as fg8
@@ -291,11 +319,10 @@ def run_fg8(args, rank, world, local):
             # weak scaling: every rank runs its own batch of the same shape
             x0 = x if rank == 0 else x.roll(rank, 0).contiguous()
         wq, ws = fg8.quantize_weight(w, g.fmt, block=args.block)
-        del w
         wsp = torch.zeros(fg8.fg8_linear_block_workspace_bytes(g.M, g.N, g.K, g.fmt, args.block), dtype=torch.uint8,
                           device=dev)
         y = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
-        plan.append(dict(g=g, wq=wq, ws=ws, b=b, wsp=wsp, y=y))
+        plan.append(dict(g=g, wq=wq, ws=ws, b=b, wsp=wsp, y=y, w=w))  # w: the weight-quant timing below
     for i, L in enumerate(plan):
         L["x"] = x0 if i == 0 else plan[i - 1]["y"]
         assert L["x"].shape == (L["g"].M, L["g"].K), "consecutive layers must chain"
@@ -402,6 +429,9 @@ def run_fg8(args, rank, world, local):
         step(evs[k])
     torch.cuda.synchronize()
     quant_ms = [[e[2 * i].elapsed_time(e[1 + 2 * i]) for e in evs] for i in range(nl)]
+    for L in plan:
+        L["wq_ms"] = time_weight_quant(fg8, L["w"], L["wq"], L["ws"], L["g"].fmt, args.block, flush_l2)
+        del L["w"]
     gemm_ms = [[e[1 + 2 * i].elapsed_time(e[2 + 2 * i]) for e in evs] for i in range(nl)]
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, world, dev)
@@ -445,7 +475,10 @@ def run_fg8(args, rank, world, local):
                                          if paths[i] == "block32" else
                                          "fused into the previous GEMM" if fused else "own launch"),
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
-                           "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak})
+                           "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak,
+                           # one-time, on load (not in the step): the weight's own quantization launch
+                           "weight_quant_us": L["wq_ms"] * 1e3,
+                           "weight_quant_gbs": weight_quant_bytes(gi, args.block) / (L["wq_ms"] * 1e-3) / 1e9})
 
     e2e = run_e2e(fg8, plan, args, stream, dev, world, chain)
     cpu = None
