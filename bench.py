@@ -159,11 +159,15 @@ class ClockSampler:
             if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax = float(parts[1])
-                power.append(float(parts[2]))
+                s, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
+            sm.append(s)
+            smax = mx
+            try:
+                power.append(float(parts[2]))
+            except ValueError:  # power may read [N/A]; the clocks still count
+                pass
             for nm, v in zip(names, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
