@@ -257,6 +257,11 @@ def linear_chain(x: torch.Tensor, layers, scale_fmt="float", workspaces=None):
     bit, what `linear` gives for that layer on y_{i-1}.  Returns [y_0, ..., y_last]."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
+    layers = list(layers)
+    if not layers:
+        raise ValueError("layers must hold at least one (wq, w_scale_inv, bias) triple")
+    if workspaces is not None and len(workspaces) != len(layers):
+        raise ValueError(f"workspaces must hold one entry (a tensor or None) per layer: {len(layers)}")
     M = x.shape[0]
     dims = []
     k = x.shape[1]

@@ -102,6 +102,8 @@ def test_static_prequant_chain_dequant_operands():
     _raises("must be a CUDA tensor", fg8.linear_chain, x, [(wq, ws, b), (wq2, ws2, None)])
     _raises("layer 1: w_scale_inv must have shape", fg8.linear_chain, x, [(wq, ws, b), (wq2, ws, None)])
     _raises("layer 1: wq must be", fg8.linear_chain, x, [(wq, ws, b), (wq, ws, None)])
+    _raises("at least one", fg8.linear_chain, x, [])
+    _raises("one entry", fg8.linear_chain, x, [(wq, ws, b), (wq2, ws2, None)], workspaces=[None])
 
     _raises("must be a CUDA tensor", fg8.dequantize_weight, wq, ws, "float")
     _raises("w_scale_inv must have shape", fg8.dequantize_weight, wq, ws[:1].contiguous(), "float")
