@@ -335,10 +335,37 @@ class FP8Linear(torch.nn.Module):
 
     def __init__(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None, scale_fmt="float",
                  block: int = 128):
+        """Quantizes `weight` (bf16 [out, in], or any float dtype, cast to bf16) on its device."""
         super().__init__()
-        self.scale_fmt = scale_fmt_code(scale_fmt)
+        fmt = scale_fmt_code(scale_fmt)
+        wq, ws = quantize_weight(weight.to(torch.bfloat16).contiguous(), fmt, block)
+        self._hold(wq, ws, bias, fmt, block)
+
+    @classmethod
+    def from_quantized(cls, weight: torch.Tensor, weight_scale_inv: torch.Tensor,
+                       bias: Optional[torch.Tensor] = None, scale_fmt="float", block: int = 128) -> "FP8Linear":
+        """The layer over a weight that is already quantized, as a pre-quantized
+        checkpoint stores it ([zh] §五): `weight` e4m3 [out, in] and
+        `weight_scale_inv` [ceil(out/block), ceil(in/block)], float32, or UE8M0
+        for scale_fmt "ue8m0" (a checkpoint's float32 power-of-two scales
+        convert exactly with scale_to_ue8m0).  Raw uint8 bytes are taken as
+        those dtypes.  No kernel runs; the tensors are kept, not copied."""
+        fmt = scale_fmt_code(scale_fmt)
+        if not isinstance(weight, torch.Tensor) or weight.dim() != 2:
+            raise ValueError("weight must be [out, in]")
+        N, K = int(weight.shape[0]), int(weight.shape[1])
+        _check_weight(weight, weight_scale_inv, (), N, K, fmt, block, weight.device)
+        if bias is not None:
+            bias = bias.to(torch.bfloat16).contiguous()
+            _check_bias(bias, (N,), weight.device)
+        layer = cls.__new__(cls)
+        torch.nn.Module.__init__(layer)
+        layer._hold(weight.view(torch.float8_e4m3fn), weight_scale_inv.view(_SCALE_DTYPES[fmt]), bias, fmt, block)
+        return layer
+
+    def _hold(self, wq, ws, bias, fmt, block):
+        self.scale_fmt = fmt
         self.block = block
-        wq, ws = quantize_weight(weight.to(torch.bfloat16).contiguous(), self.scale_fmt, block)
         self.register_buffer("weight", wq)
         self.register_buffer("weight_scale_inv", ws)
         self.register_buffer("bias", None if bias is None else bias.to(torch.bfloat16).contiguous())

@@ -107,3 +107,28 @@ def test_static_prequant_chain_dequant_operands():
 
     _raises("must be a CUDA tensor", fg8.dequantize_weight, wq, ws, "float")
     _raises("w_scale_inv must have shape", fg8.dequantize_weight, wq, ws[:1].contiguous(), "float")
+
+
+@pytest.mark.parametrize("fmt,block", [("float", 128), ("ue8m0", 128), ("ue8m0", 32)])
+def test_fp8linear_from_quantized(fmt, block):
+    """A layer over a pre-quantized checkpoint's tensors: kept as given (raw
+    bytes viewed as float8), checked against the block shape rule, and its
+    forward refuses CPU tensors instead of computing on the host."""
+    _, wq, ws, b = _dense(fmt, block)
+    layer = fg8.FP8Linear.from_quantized(wq, ws, b, fmt, block=block)
+    assert (layer.in_features, layer.out_features, layer.block) == (K, N, block)
+    assert layer.weight.data_ptr() == wq.data_ptr() and layer.weight_scale_inv.data_ptr() == ws.data_ptr()
+    assert set(layer.state_dict()) == {"weight", "weight_scale_inv", "bias"}
+    raw = fg8.FP8Linear.from_quantized(wq.view(U8), ws.view(U8) if fmt == "ue8m0" else ws, None, fmt, block=block)
+    assert raw.weight.dtype == E4M3 and raw.weight_scale_inv.dtype == (F32 if fmt == "float" else E8M0)
+    assert raw.bias is None
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        layer(torch.zeros(2, 3, K, dtype=BF16))
+    other = 128 if block == 32 else 32
+    _raises("w_scale_inv must have shape", fg8.FP8Linear.from_quantized, wq, ws, b, fmt, block=other)
+    _raises("bias must have shape", fg8.FP8Linear.from_quantized, wq, ws, b[:N - 8], fmt, block=block)
+    _raises("weight must be", fg8.FP8Linear.from_quantized, wq[0], ws, b, fmt, block=block)
+    # a state dict moves between layers built this way
+    twin = fg8.FP8Linear.from_quantized(torch.ones_like(wq), torch.ones_like(ws), torch.ones_like(b), fmt, block)
+    twin.load_state_dict(layer.state_dict())
+    assert torch.equal(twin.weight.view(U8), wq.view(U8)) and torch.equal(twin.bias, b)
