@@ -31,7 +31,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # FG8_ORACLE_LIB: a library compiled from another copy of the source
+        # (the mutation tests load deliberately broken copies this way)
+        path = os.environ.get("FG8_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         c_u8p = ctypes.POINTER(ctypes.c_uint8)
         L.orc_e4m3_value.restype = ctypes.c_double

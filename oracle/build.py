@@ -12,12 +12,18 @@ SRC = os.path.join(HERE, "fg8_oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+def compile_library(src: str, out: str) -> str:
+    """Compile one oracle source file into a shared library at `out`."""
+    cmd = ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+           "-fPIC", "-shared", "-Wall", "-Wextra", src, "-o", out]
+    subprocess.run(cmd, check=True)
+    return out
+
+
 def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
-    cmd = ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
-           "-fPIC", "-shared", "-Wall", "-Wextra", SRC, "-o", LIB + ".tmp"]
-    subprocess.run(cmd, check=True)
+    compile_library(SRC, LIB + ".tmp")
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -278,6 +278,39 @@ def test_quantize_act_ragged_tail_uses_real_elements(orc):
     assert orc.e4m3_value(int(xq[0, 128])) == -448.0
 
 
+
+def test_quantize_act_quotient_is_a_correctly_rounded_division(orc):
+    """The element quotient is RN_f32(x / s), not x times a rounded reciprocal
+    of s.  The two differ by at most one float32 ulp, which changes the e4m3
+    code only when x / s sits on a rounding midpoint, so the group is built
+    for that: its amax fixes a non-power-of-two scale s, and every other
+    element is a bf16 value x with x / s exactly an e4m3 midpoint.  Expected
+    codes: numpy's IEEE float32 division, then PyTorch's RNE cast."""
+    codes = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    mids = (codes[:-1] + codes[1:]) / 2
+    rows, separating = [], 0
+    for amax in (0.765625, 1.53125, 0.8203125, 1.421875):
+        s = np.float32(amax) / np.float32(448)
+        xs = (mids * np.float64(s)).astype(np.float32)
+        exact = (xs.astype(np.float64) == mids * np.float64(s)) & ((xs.view(np.uint32) & 0xFFFF) == 0) & (xs < amax)
+        xs = xs[exact]
+        assert 0 < xs.size < 128
+        row = np.zeros(128, dtype=np.float32)
+        row[0] = amax
+        row[1:1 + xs.size] = xs
+        row[64:64 + xs.size // 2] = -xs[: xs.size // 2]  # negative ones too
+        rows.append(row)
+        recip = (xs * (np.float32(1) / s)).astype(np.float32)
+        e4 = lambda q: torch.from_numpy(np.ascontiguousarray(q)).to(torch.float8_e4m3fn).view(torch.uint8)
+        separating += int((e4(recip) != e4(xs / s)).sum())
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    xq, xsc = orc.quantize_act(_bf16_bits(x), FLOAT)
+    xf = x.float().numpy()
+    want_q = (xf / xsc.astype(np.float32)).astype(np.float32)  # IEEE float32 division, row scale broadcast
+    want = torch.from_numpy(want_q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(xq, want)
+    assert separating >= 8  # cases on which a reciprocal-multiply quotient would round differently
+
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
 @pytest.mark.parametrize("N,K", [(256, 256), (200, 144), (130, 480), (16, 32)])
 def test_quantize_weight_blocks(orc, fmt, N, K):

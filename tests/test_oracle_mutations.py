@@ -1,0 +1,86 @@
+"""The oracle's pins catch planted mistakes (CPU only; test infrastructure).
+
+Each case copies the oracle's C++ source with one plausible mistake planted
+in it: a rounding or tie rule, a constant, a dropped term or element, a wrong
+or transposed index, a lost sign.  The copy is compiled into a temporary
+directory, and the oracle's pin tests (tests/test_oracle.py) are run against
+it in a child process; at least one pin must fail.  An unmodified copy,
+built the same way, must pass them all (the control).  Every planted mistake
+keeps each memory access inside its buffer.
+"""
+import concurrent.futures
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "fg8_oracle.cpp")
+
+# name: (text in the source, planted replacement)
+MUTATIONS = {
+    "e4m3 ties away from even": ("pick = (lo & 1) == 0 ? lo : hi;", "pick = hi;"),
+    "e4m3 saturates to NaN": ("if (a >= kE4m3Max) return sign | 0x7E;", "if (a >= kE4m3Max) return sign | 0x7F;"),
+    "e4m3 drops the sign of zero": ("const uint8_t sign = std::signbit(f) ? 0x80 : 0x00;",
+                                    "const uint8_t sign = f < 0.0f ? 0x80 : 0x00;"),
+    "UE8M0 rounds down": ("return static_cast<uint8_t>(mant == 0 ? biased : biased + 1);",
+                          "return static_cast<uint8_t>(biased);"),
+    "UE8M0 moves exact powers up": ("return static_cast<uint8_t>(mant == 0 ? biased : biased + 1);",
+                                    "return static_cast<uint8_t>(biased + 1);"),
+    "scale constant 440": ("float s = amax / 448.0f;", "float s = amax / 440.0f;"),
+    "scale floor dropped": ("if (s < floor_s) s = floor_s;", "(void)floor_s;"),
+    "quotient by reciprocal": ("const float quotient = bf16_to_float(x[m * ld_x + k]) / s_used;",
+                               "const float quotient = bf16_to_float(x[m * ld_x + k]) * (1.0f / s_used);"),
+    "act amax skips a group's last element": (
+        "for (int64_t k = k0; k < k1; ++k) amax = std::fmax(amax, std::fabs(bf16_to_float(x[m * ld_x + k])));",
+        "for (int64_t k = k0; k < k1 - 1; ++k) amax = std::fmax(amax, std::fabs(bf16_to_float(x[m * ld_x + k])));"),
+    "weight amax skips a block's last row": (
+        "for (int64_t n = n0; n < n1; ++n)\n        for (int64_t k = k0; k < k1; ++k) amax",
+        "for (int64_t n = n0; n < n1 - 1; ++n)\n        for (int64_t k = k0; k < k1; ++k) amax"),
+    "weight scales stored transposed": ("static_cast<float*>(w_scale_inv)[nb * Kb + kb] = s;",
+                                        "static_cast<float*>(w_scale_inv)[kb * Nb + nb] = s;"),
+    "GEMM uses the first group's x scale": ("xhat[k] = e4m3_signed(xq[m * K + k]) * xs_at(m, k / block);",
+                                            "xhat[k] = e4m3_signed(xq[m * K + k]) * xs_at(m, 0);"),
+    "GEMM drops the bias": ("if (bias) acc += static_cast<double>(bf16_to_float(bias[n]));", "if (bias) acc += 0.0;"),
+    "GEMM bound without magnitudes": ("mag += std::fabs(p);", "mag += p;"),
+    "GEMM drops the last k": ("for (int64_t k = 0; k < K; ++k) {\n        const double p",
+                              "for (int64_t k = 0; k < K - 1; ++k) {\n        const double p"),
+    "bf16 output truncated": ("const double r = std::nearbyint(scaled);", "const double r = std::floor(scaled);"),
+    "dequant ignores the column block": ("const int64_t blk = (n / kBlock) * Kb + k / kBlock;",
+                                         "const int64_t blk = (n / kBlock) * Kb;"),
+    "static scale multiplies": ("xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) / s);",
+                                "xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) * s);"),
+}
+
+
+def _build(tmp, i, name):
+    from oracle import build
+    src = open(SRC).read()
+    if name is not None:
+        old, new = MUTATIONS[name]
+        assert src.count(old) == 1, f"{name}: the text to mutate is not unique in the oracle source"
+        src = src.replace(old, new)
+    path = os.path.join(tmp, f"m{i}.cpp")
+    with open(path, "w") as f:
+        f.write(src)
+    return build.compile_library(path, os.path.join(tmp, f"libm{i}.so"))
+
+
+def _run_pins(lib):
+    env = dict(os.environ, FG8_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle.py"), "-x", "-q",
+                        "-p", "no:cacheprovider", "-m", "not gpu"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-600:]
+
+
+def test_every_planted_mistake_fails_a_pin(tmp_path):
+    names = [None] + list(MUTATIONS)
+    with concurrent.futures.ThreadPoolExecutor(4) as pool:
+        libs = list(pool.map(lambda a: _build(str(tmp_path), *a), enumerate(names)))
+        results = dict(zip(names, pool.map(_run_pins, libs)))
+    rc, out = results[None]
+    assert rc == 0, f"the unmodified copy must pass every pin:\n{out}"
+    # pytest exit status 1: some test failed (not a crash, a usage error or an empty run)
+    survivors = {n: results[n] for n in MUTATIONS if results[n][0] != 1}
+    assert not survivors, "planted mistakes no pin caught: " + "; ".join(
+        f"{n} (exit {rc})" for n, (rc, _) in survivors.items())
