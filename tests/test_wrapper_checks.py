@@ -132,3 +132,27 @@ def test_fp8linear_from_quantized(fmt, block):
     twin = fg8.FP8Linear.from_quantized(torch.ones_like(wq), torch.ones_like(ws), torch.ones_like(b), fmt, block)
     twin.load_state_dict(layer.state_dict())
     assert torch.equal(twin.weight.view(U8), wq.view(U8)) and torch.equal(twin.bias, b)
+
+
+@pytest.mark.parametrize("fmt,block", [("float", 128), ("ue8m0", 32)])
+def test_fp8linear_init_holds_what_quantize_weight_returns(monkeypatch, orc, fmt, block):
+    """FP8Linear(weight) keeps quantize_weight's outputs as its buffers (the
+    device quantizer replaced by the oracle here, so this runs on CPU)."""
+    from fine_grained_fp8_act_b200 import layer as L
+    code = 0 if fmt == "float" else 1
+
+    def on_host(w, f, b):
+        assert (f, b) == (code, block) and w.dtype == BF16 and w.is_contiguous()
+        q, s = orc.quantize_weight(w.view(torch.int16).numpy().view("uint16"), f, b)
+        s = torch.from_numpy(s)
+        return torch.from_numpy(q).view(E4M3), (s if f == 0 else s.view(E8M0))
+    monkeypatch.setattr(L, "quantize_weight", on_host)
+    w = torch.randn(N, K).mul(0.02)                       # float32: cast to bf16 by the layer
+    b = torch.randn(N)
+    layer = fg8.FP8Linear(w, b, fmt, block=block)
+    q, s = on_host(w.to(BF16).contiguous(), code, block)
+    assert torch.equal(layer.weight.view(U8), q.view(U8)) and torch.equal(layer.weight_scale_inv.view(U8), s.view(U8))
+    assert layer.bias.dtype == BF16 and torch.equal(layer.bias, b.to(BF16))
+    assert (layer.scale_fmt, layer.block, layer.in_features, layer.out_features) == (code, block, K, N)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        layer(torch.zeros(5, K, dtype=BF16))
