@@ -685,6 +685,30 @@ def test_grouped_linear_rejects_unknown_expert(orc):
         orc.grouped_linear(x, np.full(128, 2, np.int32), wq, ws, None, FLOAT)
 
 
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+def test_grouped_linear_block_expert_is_its_first_row(orc, fmt):
+    """Only row_expert[128 t] selects block t's expert (or skips it): the
+    other rows of a block may hold anything, -1 and other experts included,
+    and the whole block is still the dense layer of that one expert."""
+    rng = np.random.default_rng(11)
+    E, N, K, M = 3, 136, 256, 2 * 128 + 40
+    x = _bits(rng.normal(0, 1, (M, K)))
+    wq = np.empty((E, N, K), dtype=np.uint8)
+    ws = np.empty((E, 2, 2), dtype=np.float32 if fmt == FLOAT else np.uint8)
+    for e in range(E):
+        wq[e], ws[e] = orc.quantize_weight(_bits(rng.normal(0, 0.05, (N, K))), fmt)
+    b = _bits(rng.normal(0, 0.1, (E, N)))
+    re = np.ones(M, dtype=np.int32)
+    re[0], re[64], re[65], re[127] = 2, -1, 0, -1     # block 0: expert 2, whatever its other rows say
+    re[128], re[129:256] = -1, 2                      # block 1: skipped
+    re[256], re[257:] = 0, -1                         # block 2 (40 rows): expert 0
+    y64, _, ybf, written = orc.grouped_linear(x, re, wq, ws, b, fmt)
+    assert written[:128].all() and not written[128:256].any() and written[256:].all()
+    for rows, e in ((np.arange(0, 128), 2), (np.arange(256, M), 0)):
+        d64, _, dbf = orc.linear(x, wq[e], ws[e], b[e], fmt, rows=rows)
+        assert np.array_equal(y64[rows], d64) and np.array_equal(ybf[rows], dbf)
+
 # --------------------------------------------- non-default block size 32 --
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
 @pytest.mark.parametrize("M,K", [(3, 256), (2, 80), (1, 48)])

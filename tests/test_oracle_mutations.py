@@ -1,15 +1,18 @@
 """The oracle's pins catch planted mistakes (CPU only; test infrastructure).
 
-Each case copies the oracle's C++ source with one plausible mistake planted
-in it: a rounding or tie rule, a constant, a dropped term or element, a wrong
-or transposed index, a lost sign.  The copy is compiled into a temporary
-directory, and the oracle's pin tests (tests/test_oracle.py) are run against
-it in a child process; at least one pin must fail.  An unmodified copy,
-built the same way, must pass them all (the control).  Every planted mistake
-keeps each memory access inside its buffer.
+Each case copies the oracle with one plausible mistake planted in it: a
+rounding or tie rule, a constant, a dropped term or element, a wrong or
+transposed index, a lost sign (in the C++ source), or a wrong tile, expert,
+bias or skip rule (in the Python grouped layer).  A C++ copy is compiled into
+a temporary directory; a Python copy runs from a temporary copy of the tree.
+The oracle's pin tests (tests/test_oracle.py) then run against it in a child
+process, and at least one pin must fail.  An unmodified copy, built the same
+way, must pass them all (the control).  Every planted mistake keeps each
+memory access inside its buffer.
 """
 import concurrent.futures
 import os
+import shutil
 import subprocess
 import sys
 
@@ -52,6 +55,36 @@ MUTATIONS = {
 }
 
 
+# Python grouped layer (oracle/__init__.py): name: (text, planted replacement)
+PY_MUTATIONS = {
+    "grouped tile of 64 rows": ("MOE_TILE = 128", "MOE_TILE = 64"),
+    "grouped expert from the block's last row": ("        e = int(re[t * MOE_TILE])\n",
+                                                 "        e = int(re[min(M, (t + 1) * MOE_TILE) - 1])\n"),
+    "grouped -1 blocks computed with expert 0": ("        if e < 0:\n            continue\n",
+                                                 "        if e < 0:\n            e = 0\n"),
+    "grouped bias of expert 0": ("None if bias_bf16 is None else bias_bf16[e], fmt, rows=rows)",
+                                 "None if bias_bf16 is None else bias_bf16[0], fmt, rows=rows)"),
+    "grouped scales of expert 0": ("wq[e], ws[e],", "wq[e], ws[0],"),
+}
+
+
+def _py_tree(tmp, i, name):
+    """A copy of the oracle, tests and input generators with one Python mistake planted."""
+    root = os.path.join(tmp, f"tree{i}")
+    skip = shutil.ignore_patterns("__pycache__", "*.so", "*.so.tmp")
+    for d in ("oracle", "tests", "workloads"):
+        shutil.copytree(os.path.join(ROOT, d), os.path.join(root, d), ignore=skip)
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), root)
+    if name is not None:
+        path = os.path.join(root, "oracle", "__init__.py")
+        src = open(path).read()
+        old, new = PY_MUTATIONS[name]
+        assert src.count(old) == 1, f"{name}: the text to mutate is not unique in the oracle's Python"
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+    return root
+
+
 def _build(tmp, i, name):
     from oracle import build
     src = open(SRC).read()
@@ -65,22 +98,28 @@ def _build(tmp, i, name):
     return build.compile_library(path, os.path.join(tmp, f"libm{i}.so"))
 
 
-def _run_pins(lib):
+def _run_pins(lib, root=ROOT):
     env = dict(os.environ, FG8_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle.py"), "-x", "-q",
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(root, "tests", "test_oracle.py"), "-x", "-q",
                         "-p", "no:cacheprovider", "-m", "not gpu"],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+                       cwd=root, env=env, capture_output=True, text=True, timeout=900)
     return r.returncode, r.stdout[-600:]
 
 
 def test_every_planted_mistake_fails_a_pin(tmp_path):
+    from oracle import build
     names = [None] + list(MUTATIONS)
     with concurrent.futures.ThreadPoolExecutor(4) as pool:
         libs = list(pool.map(lambda a: _build(str(tmp_path), *a), enumerate(names)))
+        py_names = ["tree control"] + list(PY_MUTATIONS)
+        trees = [_py_tree(str(tmp_path), i, None if i == 0 else n) for i, n in enumerate(py_names)]
         results = dict(zip(names, pool.map(_run_pins, libs)))
-    rc, out = results[None]
-    assert rc == 0, f"the unmodified copy must pass every pin:\n{out}"
+        real = build.build()
+        results.update(zip(py_names, pool.map(lambda t: _run_pins(real, t), trees)))
+    for control in (None, "tree control"):
+        rc, out = results[control]
+        assert rc == 0, f"an unmodified copy ({control or 'compiled'}) must pass every pin:\n{out}"
     # pytest exit status 1: some test failed (not a crash, a usage error or an empty run)
-    survivors = {n: results[n] for n in MUTATIONS if results[n][0] != 1}
+    survivors = {n: results[n] for n in list(MUTATIONS) + list(PY_MUTATIONS) if results[n][0] != 1}
     assert not survivors, "planted mistakes no pin caught: " + "; ".join(
         f"{n} (exit {rc})" for n, (rc, _) in survivors.items())
