@@ -52,6 +52,12 @@ MUTATIONS = {
                                          "const int64_t blk = (n / kBlock) * Kb;"),
     "static scale multiplies": ("xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) / s);",
                                 "xq[m * K + k] = e4m3_encode(bf16_to_float(x[m * ld_x + k]) * s);"),
+    "1 x 32 groups span 128 channels": ("const int64_t k1 = std::min<int64_t>(k0 + group, K);",
+                                        "const int64_t k1 = std::min<int64_t>(k0 + kGroup, K);"),
+    "GEMM weight row block fixed at 128": ("ws_at(n / block, k / block)", "ws_at(n / kBlock, k / block)"),
+    "e4m3 subnormals off by a factor 2": ("mag = std::ldexp(static_cast<double>(mant), -9);",
+                                          "mag = std::ldexp(static_cast<double>(mant), -10);"),
+    "scale conversion accepts non-powers": ("if (f == 0.5 && e >= -127 && e <= 127)", "if (e >= -127 && e <= 127)"),
 }
 
 
