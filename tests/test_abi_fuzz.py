@@ -160,3 +160,98 @@ def test_block32_linear_host_checks(lib):
                 broken.add(WORKSPACE)
         got = lib.fg8_linear_block(x, M, N, K, ld_x, wq, ws, bias, y, ld_y, fmt, block, wsp, nbytes, None)
         _check(got, broken, M, f"fg8_linear_block case {i}: M={M} N={N} K={K} fmt={fmt} block={block}")
+
+
+def _check_allowed(got, allowed, what):
+    assert got in allowed, f"{what}: status {got}, expected one of {sorted(allowed)}"
+
+
+@pytest.mark.parametrize("block", [None, 128, 32, 64])
+def test_quantize_act_host_checks(lib, block):
+    """fg8_quantize_act (block None) and fg8_quantize_act_block."""
+    rng = np.random.default_rng(4 + (block or 0))
+    for i in range(800):
+        M = _dim(rng, [0, 1, 129, 8192])
+        K = _dim(rng, [16, 48, 400, 7168])
+        fmt = int(rng.choice([0, 1, 1, 2]))
+        ld_x = K + int(rng.choice([0, 0, 8, -8, 4]))
+        x, xq, xs = (_ptr(rng, 16) for _ in range(3))
+        invalid = fmt not in (0, 1) or not (0 <= M <= MAXD and 0 < K <= MAXD) or ld_x < K or \
+            block not in (None, 128, 32)
+        if invalid:
+            allowed = {INVALID}
+        elif M == 0:
+            allowed = {OK}
+        else:
+            broken = set()
+            if None in (x, xq, xs):
+                broken.add(INVALID)
+            if K % 16 or ld_x % 8 or not all(_aligned(p, 16) for p in (x, xq) if p is not None):
+                broken.add(ALIGN)
+            allowed = broken or {UNSUPPORTED}
+        if block is None:
+            got = lib.fg8_quantize_act(x, M, K, ld_x, xq, xs, fmt, None)
+        else:
+            got = lib.fg8_quantize_act_block(x, M, K, ld_x, xq, xs, fmt, block, None)
+        _check_allowed(got, allowed, f"quantize_act block={block} case {i}: M={M} K={K} fmt={fmt} ld={ld_x}")
+
+
+@pytest.mark.parametrize("block", [None, 128, 32, 16])
+def test_quantize_weight_host_checks(lib, block):
+    """fg8_quantize_weight (block None) and fg8_quantize_weight_block."""
+    rng = np.random.default_rng(40 + (block or 0))
+    for i in range(800):
+        N = int(rng.choice([65535 * 128, 65535 * 128 + 1])) if rng.random() < 0.05 else _dim(rng, [1, 264, 4096])
+        K = _dim(rng, [16, 48, 400, 7168])
+        fmt = int(rng.choice([0, 1, 1, 2]))
+        ld_w = K + int(rng.choice([0, 0, 8, -8, 4]))
+        w, wq, ws = (_ptr(rng, 16) for _ in range(3))
+        b = 128 if block is None else block
+        invalid = fmt not in (0, 1) or not (0 < N <= MAXD and 0 < K <= MAXD) or ld_w < K or b not in (128, 32) or \
+            None in (w, wq, ws)
+        if not invalid and b == 128 and -(-N // 128) > 65535:
+            invalid = True
+        if not invalid and b == 32 and -(-N // 32) * -(-K // 32) > MAXD // 8:
+            invalid = True
+        align = not invalid and (K % 16 or ld_w % 8 or not (_aligned(w, 16) and _aligned(wq, 16)))
+        allowed = ({INVALID} | ({ALIGN} if (K % 16 or ld_w % 8) else set())) if invalid else \
+            ({ALIGN} if align else {UNSUPPORTED})
+        if block is None:
+            got = lib.fg8_quantize_weight(w, N, K, ld_w, wq, ws, fmt, None)
+        else:
+            got = lib.fg8_quantize_weight_block(w, N, K, ld_w, wq, ws, fmt, block, None)
+        _check_allowed(got, allowed, f"quantize_weight block={block} case {i}: N={N} K={K} fmt={fmt} ld={ld_w}")
+
+
+def test_dequantize_and_scale_conversion_host_checks(lib):
+    rng = np.random.default_rng(9)
+    for i in range(800):
+        N = _dim(rng, [1, 300, 4096])
+        K = _dim(rng, [16, 400, 7168])
+        fmt = int(rng.choice([0, 1, 1, 7]))
+        ld_w = K + int(rng.choice([0, 0, 8, -8, 4]))
+        wq, ws, w = (_ptr(rng, 16) for _ in range(3))
+        invalid = fmt not in (0, 1) or not (0 < N <= MAXD and 0 < K <= MAXD) or ld_w < K or N * K > 2**40 or \
+            None in (wq, ws, w)
+        align = K % 16 or ld_w % 8 or not (_aligned(wq, 16) and _aligned(w, 16))
+        allowed = ({INVALID} | ({ALIGN} if (K % 16 or ld_w % 8) else set())) if invalid else \
+            ({ALIGN} if align else {UNSUPPORTED})
+        got = lib.fg8_dequantize_weight(wq, N, K, ws, fmt, w, ld_w, None)
+        _check_allowed(got, allowed, f"dequantize_weight case {i}: N={N} K={K} fmt={fmt} ld={ld_w}")
+
+        n = int(rng.choice([-1, 0, 1, 1000, 2**20]))
+        s, out = _ptr(rng, 4), _ptr(rng, 1)
+        cnt = None if rng.random() < 0.3 else BASE + int(rng.choice([0, 0, 4, 2]))
+        if n < 0:
+            allowed = {INVALID}
+        elif n == 0:
+            allowed = {OK}
+        else:
+            broken = set()
+            if s is None or out is None:
+                broken.add(INVALID)
+            if (s is not None and s % 4) or (cnt is not None and cnt % 4):
+                broken.add(ALIGN)
+            allowed = broken or {UNSUPPORTED}
+        got = lib.fg8_scale_to_ue8m0(s, n, out, cnt, None)
+        _check_allowed(got, allowed, f"scale_to_ue8m0 case {i}: n={n}")
