@@ -206,6 +206,12 @@ FG8_API fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, c
  *               fg8_gemm_prequant reads)
  *   fg8_linear_static: as fg8_linear with scale_fmt FLOAT (the same
  *               workspace, fg8_linear_workspace_bytes(M, N, K, FLOAT)).
+ *               Exception to the check-before-launch rule: before its first
+ *               launch it checks only that the workspace holds the quantized
+ *               activations.  For few tokens, a workspace large enough for
+ *               that but short of fg8_linear_workspace_bytes is refused
+ *               (FG8_ERR_WORKSPACE) only after the quantization has been
+ *               enqueued, and y is not written.
  * Checks and errors as fg8_quantize_act / fg8_linear. */
 FG8_API fg8_status fg8_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
                                            const float* act_scale, void* xq_e4m3, void* x_scale, void* stream);
