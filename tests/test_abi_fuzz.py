@@ -255,3 +255,23 @@ def test_dequantize_and_scale_conversion_host_checks(lib):
             allowed = broken or {UNSUPPORTED}
         got = lib.fg8_scale_to_ue8m0(s, n, out, cnt, None)
         _check_allowed(got, allowed, f"scale_to_ue8m0 case {i}: n={n}")
+
+
+def test_batched_row_expert_host_checks(lib):
+    rng = np.random.default_rng(12)
+    for i in range(800):
+        E = int(rng.choice([1, 8, 256, 65535, 65536, 0, -3]))
+        cap = int(rng.choice([0, 128, 256, 640, 100, -128, 2**31]))
+        counts = None if rng.random() < 0.06 else BASE + int(rng.choice([0, 0, 2]))
+        re = None if rng.random() < 0.06 else BASE + int(rng.choice([0, 0, 2]))
+        if not (0 < E <= 65535) or cap < 0 or E * cap > MAXD:
+            allowed = {INVALID}
+        elif cap == 0:
+            allowed = {OK}
+        elif counts is None or re is None:
+            allowed = {INVALID} | ({ALIGN} if cap % 128 else set())
+        else:
+            align = cap % 128 or counts % 4 or re % 4
+            allowed = {ALIGN} if align else {UNSUPPORTED}
+        got = lib.fg8_grouped_row_expert(counts, E, cap, re, None)
+        _check_allowed(got, allowed, f"grouped_row_expert case {i}: E={E} cap={cap}")
