@@ -331,7 +331,9 @@ class FP8Linear(torch.nn.Module):
     """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
     weight float8_e4m3fn [out, in], weight_scale_inv per block x block block
     (weight_block_size (128, 128) by default, or (32, 32) with UE8M0 scales),
-    bias kept in bf16 (not quantized, [zh] §三)."""
+    bias kept in bf16 (not quantized, [zh] §三).  The layer keeps one device
+    workspace, so forwards of the same layer on different CUDA streams must
+    not overlap in time (use one layer object per concurrent stream)."""
 
     def __init__(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None, scale_fmt="float",
                  block: int = 128):
