@@ -997,13 +997,17 @@ def run_reference(args, rank, world):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="esm2_ffn")
-    ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1, help="ranks (one per GPU, launched by torchrun when > 1)")
+    ap.add_argument("--steps", type=int, default=200, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=10, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--workload", default="esm2_ffn",
+                    help="esm2_ffn (default), dsv3_mlp, llama_m<M> (e.g. llama_m16), "
+                         "square_m<M>_float or square_m<M>_ue8m0 (K = N = 12288), moe_dsv3")
+    ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"],
+                    help="fg8: this library; reference: the CPU oracle on a bounded sample")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time the oracle baseline of the fg8 arm aims at (rank 0, one GPU)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle baseline of the fg8 arm")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: CPU seconds that the warm-up and timed steps together aim at")
     ap.add_argument("--block", type=int, default=128, choices=[128, 32],
