@@ -227,5 +227,7 @@ def fg8_scale_to_ue8m0(scale_f32, n, scale_e8m0, invalid_count, stream):
 
 
 def fg8_check_device_status(workspace, stream) -> int:
-    """Returns the status code (FG8_OK or FG8_ERR_TIMEOUT); does not raise."""
+    """Returns the status code the previous calls on this workspace left: FG8_OK,
+    FG8_ERR_TIMEOUT, or FG8_ERR_INVALID_ARG for an expert index >= E in a
+    grouped call; synchronizes the stream and clears the word; does not raise."""
     return int(lib().fg8_check_device_status(workspace, stream))
