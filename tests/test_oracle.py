@@ -154,6 +154,32 @@ def test_e4m3_encode_vs_torch_all_bf16_patterns(orc):
         assert np.array_equal(got, ref), scale
 
 
+def test_bf16_rounding_brute_force(orc):
+    """The output rounding, double -> bf16 round-to-nearest-even, against a
+    brute-force search: the two bf16 neighbours of |v| among all finite bf16
+    values (exact in double), the nearer one, the even mantissa on a tie.
+    Random magnitudes over the whole range, bf16 subnormals, exact
+    midpoints and their one-ulp neighbours, signed zeros."""
+    bits = np.arange(0x0000, 0x7F80, dtype=np.uint32)                 # +0 ... largest finite
+    vals = (bits << 16).view(np.float32).astype(np.float64)
+    rng = np.random.default_rng(17)
+    mids = (vals[:-1] + vals[1:]) / 2                                  # exact: 8-bit significands
+    pick = rng.choice(mids.size, 400, replace=False)
+    cases = list(mids[pick]) + list(np.nextafter(mids[pick], 0)) + list(np.nextafter(mids[pick], np.inf))
+    cases += list(rng.uniform(-1, 1, 300) * np.exp2(rng.integers(-135, 127, 300)))
+    cases += [0.0, -0.0, 1.0, -3.0, vals[-1], -vals[-1], 2.0 ** -133, 2.0 ** -134, 1.5 * 2.0 ** -134]
+    for v in cases:
+        a = abs(v)
+        i = int(np.searchsorted(vals, a, side="right")) - 1            # vals[i] <= a < vals[i + 1]
+        if vals[i] == a:
+            b = i
+        else:
+            mid = (vals[i] + vals[i + 1]) / 2
+            b = i if a < mid else i + 1 if a > mid else (i if i % 2 == 0 else i + 1)
+        want = int(bits[b]) | (0x8000 if np.signbit(v) else 0)
+        assert orc.bf16_from_double(float(v)) == want, (v, hex(want))
+
+
 # ----------------------------------------------------------------- UE8M0 --
 def test_e8m0_decode_matches_torch(orc):
     t = torch.arange(255, dtype=torch.uint8).view(torch.float8_e8m0fnu).to(torch.float64).numpy()

@@ -58,6 +58,7 @@ MUTATIONS = {
     "e4m3 subnormals off by a factor 2": ("mag = std::ldexp(static_cast<double>(mant), -9);",
                                           "mag = std::ldexp(static_cast<double>(mant), -10);"),
     "scale conversion accepts non-powers": ("if (f == 0.5 && e >= -127 && e <= 127)", "if (e >= -127 && e <= 127)"),
+    "bf16 subnormal quantum off by one": ("if (q < -133) q = -133;", "if (q < -132) q = -132;"),
 }
 
 
