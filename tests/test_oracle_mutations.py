@@ -59,6 +59,9 @@ MUTATIONS = {
                                           "mag = std::ldexp(static_cast<double>(mant), -10);"),
     "scale conversion accepts non-powers": ("if (f == 0.5 && e >= -127 && e <= 127)", "if (e >= -127 && e <= 127)"),
     "bf16 subnormal quantum off by one": ("if (q < -133) q = -133;", "if (q < -132) q = -132;"),
+    "GEMM decode drops the sign": ("return (code & 0x80) ? -mag : mag;", "return mag;"),
+    "sampled rows read from the top": ("const int64_t m = rows ? rows[r] : r;\n    std::vector<double> xhat",
+                                       "const int64_t m = r;\n    std::vector<double> xhat"),
 }
 
 
