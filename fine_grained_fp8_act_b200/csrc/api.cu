@@ -246,6 +246,26 @@ fg8_status launch_small_path(bool fused, const void* x_bf16, int64_t ld_x, int64
   return cuda_status(launch_small_m(a, fmt, static_cast<cudaStream_t>(stream)));
 }
 
+namespace fg8 {
+
+// fg8_linear's argument checks (everything but the workspace), in the order
+// fg8_linear applies them; FG8_OK for M == 0 with a valid shape.
+int check_linear_args_status(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
+                             const void* w_scale_inv, const void* bias_bf16, const void* y_bf16, int64_t ld_y,
+                             int fmt) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (M == 0) return FG8_OK;
+  if (x_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
+    return FG8_ERR_INVALID_ARG;
+  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
+      (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv))
+    return FG8_ERR_ALIGNMENT;
+  return FG8_OK;
+}
+
+}  // namespace fg8
+
 extern "C" {
 
 int fg8_version(void) { return 100; }
@@ -667,14 +687,11 @@ fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, co
 fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
                       const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt,
                       void* workspace, size_t workspace_bytes, void* stream) {
-  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
-  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (const int st = fg8::check_linear_args_status(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                  ld_y, fmt);
+      st != FG8_OK)
+    return static_cast<fg8_status>(st);
   if (M == 0) return FG8_OK;
-  if (x_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
-    return FG8_ERR_INVALID_ARG;
-  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
-      (bias_bf16 != nullptr && !aligned16(bias_bf16)) || !aligned16(w_scale_inv))
-    return FG8_ERR_ALIGNMENT;
   if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
     return st;
   if (use_small_m(M, N) && use_fused_small_m(M, fmt))  // one kernel: quantize, GEMM, reduce
@@ -780,7 +797,10 @@ fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, int64_t K
       (reinterpret_cast<uintptr_t>(act_scale) & 3u) != 0)
     return FG8_ERR_ALIGNMENT;
   const LinearWs L = linear_ws_layout(M, N, K, fmt);
-  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  // the whole workspace the GEMM step needs (few tokens: split-K partials
+  // too), checked before the quantization is enqueued
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
+    return st;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

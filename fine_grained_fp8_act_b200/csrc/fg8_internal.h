@@ -175,6 +175,13 @@ cudaError_t launch_scale_to_e8m0(const float* s, int64_t n, uint8_t* out, uint32
 
 int choose_block_n(int M, int N, int num_sms);
 
+// fg8_linear's host-side argument checks, workspace excepted (api.cu); an
+// fg8_status value.  Entry points built on fg8_linear run them before their
+// own set-up so that a bad call touches no device state.
+int check_linear_args_status(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
+                             const void* w_scale_inv, const void* bias_bf16, const void* y_bf16, int64_t ld_y,
+                             int fmt);
+
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s);
 
 }  // namespace fg8

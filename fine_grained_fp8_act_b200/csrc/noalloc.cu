@@ -58,16 +58,15 @@ void* scratch_for_current_device() {
 extern "C" fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                                          const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
                                          void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* stream) {
-  if (M == 0) {  // nothing to compute; argument checks as fg8_linear
-    return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, nullptr, 0,
-                      stream);
-  }
+  // fg8_linear's own argument checks come first, so a bad call returns its
+  // status without touching the scratch or the device
+  if (const int st = fg8::check_linear_args_status(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                  ld_y, fmt);
+      st != FG8_OK)
+    return static_cast<fg8_status>(st);
+  if (M == 0) return FG8_OK;
   const size_t need = fg8_linear_workspace_bytes(M, N, K, fmt);
-  if (need == 0) {  // bad shape or format: let fg8_linear report which
-    return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, nullptr, 0,
-                      stream);
-  }
-  if (need > kNoAllocScratchBytes) return FG8_ERR_WORKSPACE;  // shape too large for the fixed scratch
+  if (need == 0 || need > kNoAllocScratchBytes) return FG8_ERR_WORKSPACE;  // too large for the fixed scratch
   void* scratch = scratch_for_current_device();
   if (scratch == nullptr) return FG8_ERR_CUDA;
   // The scratch keeps the previous call's bytes; the only part that must

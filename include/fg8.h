@@ -180,6 +180,8 @@ FG8_API fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale
  *     call's contents; each call clears the part that must start at zero.
  *     Calls that overlap on the GPU (different streams, or concurrent host
  *     threads) race on it: serialize them.
+ *   - Arguments are checked exactly as fg8_linear checks them, before the
+ *     scratch is looked up or touched: a refused call changes nothing.
  *   - Device-side wait timeouts are not reported through this entry point. */
 FG8_API fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                                       const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
@@ -205,13 +207,8 @@ FG8_API fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, c
  *               float32, every entry set to the scale (the layout
  *               fg8_gemm_prequant reads)
  *   fg8_linear_static: as fg8_linear with scale_fmt FLOAT (the same
- *               workspace, fg8_linear_workspace_bytes(M, N, K, FLOAT)).
- *               Exception to the check-before-launch rule: before its first
- *               launch it checks only that the workspace holds the quantized
- *               activations.  For few tokens, a workspace large enough for
- *               that but short of fg8_linear_workspace_bytes is refused
- *               (FG8_ERR_WORKSPACE) only after the quantization has been
- *               enqueued, and y is not written.
+ *               workspace, fg8_linear_workspace_bytes(M, N, K, FLOAT), checked
+ *               in full before anything is launched).
  * Checks and errors as fg8_quantize_act / fg8_linear. */
 FG8_API fg8_status fg8_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
                                            const float* act_scale, void* xq_e4m3, void* x_scale, void* stream);

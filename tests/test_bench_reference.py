@@ -51,10 +51,22 @@ def _check_line(out, workload, world, threads, steps):
 
 
 def test_reference_arm_dense_line():
-    lines = _run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3",
-                  "--ref-seconds", "5"], 4)
+    lines = _run([sys.executable, "bench.py", "--impl", "reference", "--workload", "esm2_ffn", "--steps", "2",
+                  "--warmup", "3", "--ref-seconds", "5"], 4)
     assert len(lines) == 1
     _check_line(json.loads(lines[0]), "esm2_ffn", 1, 4, 2)
+
+
+def test_reference_arm_default_workload_is_the_largest_config():
+    """With no --workload both arms run the largest single-GPU configuration:
+    16384 tokens through the square 12288 layer, float scales."""
+    import bench
+    layers = bench.workload_layers(bench.DEFAULT_WORKLOAD)
+    assert [(g.M, g.K, g.N, g.fmt) for _, g, _ in layers] == [(16384, 12288, 12288, 0)]
+    lines = _run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                  "--ref-seconds", "4"], 4)
+    assert len(lines) == 1
+    _check_line(json.loads(lines[0]), bench.DEFAULT_WORKLOAD, 1, 4, 1)
 
 
 def test_reference_arm_moe_line():
@@ -71,7 +83,8 @@ def test_reference_arm_two_ranks():
     prints, reporting the world size; rank 1 exits 0 without output."""
     lines = _run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
                   "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl",
-                  "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--ref-seconds", "4"], 2)
+                  "reference", "--workload", "esm2_ffn", "--gpus", "2", "--steps", "1", "--warmup", "3",
+                  "--ref-seconds", "4"], 2)
     assert len(lines) == 1
     _check_line(json.loads(lines[0]), "esm2_ffn", 2, 2, 1)
 

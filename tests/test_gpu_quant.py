@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import workloads as W
+from _ws_layout import decode
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +56,55 @@ def test_act_quant_bitexact(fg8, orc, fmt, M, K):
     oq, os_ = orc.quantize_act(W.bf16_bits(x), fmt)
     _assert_same(_u8(xq), oq, "xq")
     _assert_same(_scale_bits(xs, fmt), _oracle_scale_bits(os_, fmt), "x_scale")
+
+
+# The launcher caps the grid at 8 CTAs per SM (64 groups of 128 per CTA, so
+# 75,776 groups per pass over 148 SMs; 256 groups of 32 per CTA, 303,104 per
+# pass): these shapes need 6 and more passes of the grid-stride loop.
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,K", [(8192, 7168), (4096, 14336), (16384, 1040)])
+def test_act_quant_bitexact_multi_pass(fg8, orc, fmt, M, K):
+    x = W.x_student_t(M, K, seed=M + K)
+    assert M * ((K + 127) // 128) > 2 * 75776
+    xq, xs = fg8.quantize_act(x.cuda(), fmt)
+    torch.cuda.synchronize()
+    oq, os_ = orc.quantize_act(W.bf16_bits(x), fmt)
+    _assert_same(_u8(xq), oq, "xq")
+    _assert_same(_scale_bits(xs, fmt), _oracle_scale_bits(os_, fmt), "x_scale")
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+def test_act_quant_block32_multi_pass(fg8, orc, fmt):
+    M, K = 4096, 4112  # 4096 x 129 groups of 32 = 528,384 groups; ragged last group
+    x = W.x_outliers(M, K, seed=77)
+    xq, xs = fg8.quantize_act(x.cuda(), fmt, block=32)
+    torch.cuda.synchronize()
+    oq, os_ = orc.quantize_act(W.bf16_bits(x), fmt, block=32)
+    _assert_same(_u8(xq), oq, "xq")
+    _assert_same(_scale_bits(xs, fmt), _oracle_scale_bits(os_, fmt), "x_scale")
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,K", [(8192, 7168), (300, 1040)])
+def test_prepare_layouts_vs_oracle(fg8, orc, fmt, M, K):
+    """The prepare step of fg8_linear writes the codes and, in the GEMM's own
+    layouts (K-major float32, or UE8M0 scale-factor tiles), the scales: decoded
+    back to row-major they must be the oracle's bit for bit, across every pass
+    of the grid."""
+    N = 256
+    x = W.x_outliers(M, K, seed=M + 2 * K)
+    ws_scale = torch.ones(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device="cuda")
+    if fmt == UE8M0:
+        ws_scale = torch.full(ws_scale.shape, 127, dtype=torch.uint8, device="cuda")
+    wsp = torch.zeros(fg8.fg8_linear_workspace_bytes(M, N, K, fmt), dtype=torch.uint8, device="cuda")
+    xd = x.cuda()
+    fg8.fg8_linear_prepare(xd.data_ptr(), M, N, K, xd.stride(0), ws_scale.data_ptr(), fmt, wsp.data_ptr(),
+                           wsp.numel(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    gq, gs = decode(wsp.cpu().numpy(), M, K, fmt)
+    oq, os_ = orc.quantize_act(W.bf16_bits(x), fmt)
+    _assert_same(np.ascontiguousarray(gq), oq, "xq in the workspace")
+    _assert_same(np.ascontiguousarray(gs), _oracle_scale_bits(os_, fmt), "x scales in the workspace")
 
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
