@@ -8,13 +8,15 @@
 //
 // One persistent CTA per SM walks 128 x BN output tiles (BN = 128 or 256).
 // 384 threads in three warpgroups; the first gives up registers
-// (setmaxnreg 40-56) to the two epilogue warpgroups (setmaxnreg 224-232):
+// (setmaxnreg 40-80) to the two epilogue warpgroups (setmaxnreg 208-232):
 //   warp 0      producer: per 128-wide K-block, TMA loads of the A tile
 //               (128 x 128 e4m3) and B tile (BN x 128 e4m3) into a STAGES-deep
 //               ring (128-byte swizzle); bulk copies of UE8M0 scale-factor
 //               tiles (every 4th K-block) and of the tile's bias (bias ring).
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32) per K-block.
 //   warp 2      TMEM allocator.
+//   warp 3      float scales: per K-block, the 128 rows' x scales and the
+//               tile's weight-block scales into a shared-memory scale ring.
 //   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4)..+31; warpgroup g
 //               owns columns [g*BN/2, (g+1)*BN/2).
 //
@@ -22,10 +24,10 @@
 // TMEM buffer (512/BN of them); the epilogue promotes it in registers,
 // acc += P_kb * (sx * sw) starting from acc = bias, applying the float32
 // scales exactly as given --
-// never rounded to a power of two (§七 补充 names that hazard).  Each thread
-// loads its own sx (its row) and sw (its columns' weight block) from global
-// memory two K-blocks ahead, and reads P_kb from TMEM 32 columns at a time
-// with the next 32 in flight while it promotes the current ones.
+// never rounded to a power of two (§七 补充 names that hazard).  The scales
+// come from the scale ring (warp 3 runs ahead of the epilogue); P_kb is read
+// from TMEM 32 columns at a time with the next 32 in flight while the current
+// ones are promoted by packed two-lane FMAs (each lane rounds as a scalar FMA).
 // UE8M0 scales (FMT 1): tcgen05.mma.kind::mxf8f6f4.block_scale applies the
 // power-of-two scales inside the tensor core (one per 32 K-elements; four
 // equal ones per 128-block), accumulating the whole K range in TMEM.
@@ -100,19 +102,14 @@ __device__ __forceinline__ int tile_expert(const KParams& p, int m0, bool report
   return e;
 }
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool PAIR_ = false, bool REQUANT_ = false>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
   // REQUANT: the epilogue also quantizes its bf16 output rows, one 128-column
   // group per thread, for a next layer (needs the 256-wide tile).
   static constexpr bool REQUANT = REQUANT_;
-  // PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
-  // MMAs; each CTA holds 128 rows of A and of the result, and BN/2 rows of B.
-  static constexpr bool PAIR = PAIR_;
-  static constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
-  static constexpr int kBRows = PAIR ? BN / 2 : BN;
   static constexpr int kA = kBlockM * 128;
-  static constexpr int kB = kBRows * 128;
+  static constexpr int kB = BN * 128;
   static constexpr int kSfBytes = FMT == 1 ? kSfChunkBytes * (1 + BN / 128) : 0;
   static constexpr int kStage = (kA + kB + kSfBytes + 1023) / 1024 * 1024;
   static constexpr int kEpiWarps = 8;
@@ -127,8 +124,12 @@ struct Cfg {
   static constexpr int kSfbCol = kSfaCol + 4;
   static constexpr int kSfSetCols = 4 + BN / 32;
   static constexpr int kBiasSlot = BN * 2;
+  // float scale ring: per K-block the 128 rows' x scales, then the weight
+  // scales of the tile's BN/128 column blocks (padded to 16 bytes)
+  static constexpr int kSRing = FMT == 0 ? 4 : 0;
+  static constexpr int kScaleSlot = 128 * 4 + 16;
   // register split after launch (384 x 168): the wide float epilogue holds
-  // 128 accumulators + 32 TMEM registers per thread, the others need less
+  // 128 accumulators + 64 TMEM registers per thread, the others need less
   static constexpr uint32_t kRegsLow = (FMT == 0 && BN == 256) ? 40 : (BN == 128 ? 80 : 56);
   static constexpr uint32_t kRegsHigh = (FMT == 0 && BN == 256) ? 232 : (BN == 128 ? 208 : 224);
   static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch allocation");
@@ -140,21 +141,19 @@ struct Cfg {
   // shared memory map (offsets from the 1024-aligned base)
   static constexpr int kOffStaging = STAGES * kStage;
   static constexpr int kOffBias = kOffStaging + kEpiWarps * kOutBufs * kOutBuf;
-  static constexpr int kOffBar = kOffBias + 2 * kBiasSlot;
+  static constexpr int kOffScale = kOffBias + 2 * kBiasSlot;
+  static constexpr int kOffBar = kOffScale + kSRing * kScaleSlot;
   static constexpr int kSmem = 1024 + kOffBar + 512;
   static_assert(kSmem <= kMaxSmem, "shared memory budget");
   static_assert(kStage % 1024 == 0, "stages keep 1024-byte alignment for the 128B swizzle");
-  static_assert(kOffBias % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
+  static_assert(kOffBias % 16 == 0 && kOffScale % 16 == 0 && kOffBar % 8 == 0, "alignment of rings");
   static_assert(kNumAcc * BN + (FMT == 1 ? 2 * kSfSetCols : 0) <= 512, "TMEM columns");
-  static_assert(!PAIR || (FMT == 0 && BN == 256), "CTA pairs: float scales, 256-wide tiles");
-  static_assert(!REQUANT || (BN == 256 && !PAIR), "output re-quantization: one 128-column group per thread");
-  // bytes the stage's full barrier (in the pair's first CTA) waits for
-  static constexpr uint32_t kStageTx = (PAIR ? 2 : 1) * (kA + kB);
-  // arrivals that free a TMEM buffer: every epilogue warp of the pair
-  static constexpr uint32_t kTmemEmptyCount = (PAIR ? 2 : 1) * kEpiWarps;
-  // instruction descriptors (M = 128 or 256, K-major A and B, e4m3 x e4m3 -> f32)
-  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
-  static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kTileM >> 4) << 24);
+  static_assert(!REQUANT || BN == 256, "output re-quantization: one 128-column group per thread");
+  // bytes the stage's full barrier waits for
+  static constexpr uint32_t kStageTx = kA + kB;
+  // instruction descriptors (M = 128, K-major A and B, e4m3 x e4m3 -> f32)
+  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24);
+  static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBlockM >> 4) << 24);
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
@@ -166,24 +165,6 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb
   const int r = t - g * span;
   mb = first_m + r % gm;
   nb = r / gm;
-}
-
-// Persistent tile walk: single CTAs stride over tiles by the grid, CTA pairs
-// by the number of clusters.
-template <class C>
-__device__ __forceinline__ int tile_start() {
-  if constexpr (C::PAIR) return static_cast<int>(cluster_id_x());
-  else return static_cast<int>(blockIdx.x);
-}
-template <class C>
-__device__ __forceinline__ int tile_stride() {
-  if constexpr (C::PAIR) return static_cast<int>(nclusters_x());
-  else return static_cast<int>(gridDim.x);
-}
-template <class C>
-__device__ __forceinline__ int cta_rank() {
-  if constexpr (C::PAIR) return static_cast<int>(cluster_ctarank());
-  else return 0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
@@ -222,17 +203,6 @@ struct Ring {
     }
   }
 };
-
-// An epilogue warp's release of a TMEM buffer: the MMA issuer waits on the
-// barrier of the pair's first CTA, so the second CTA arrives there remotely.
-template <class C>
-__device__ __forceinline__ void release_tmem(uint64_t* bar) {
-  if constexpr (C::PAIR) {
-    mbar_arrive_cluster(mapa_shared(bar, 0));
-  } else {
-    mbar_arrive(bar);
-  }
-}
 
 // Quantize one output row's 128-column group (bf16-rounded values in `v`) as
 // the next layer's activation group: the same arithmetic, hence the same bits,
@@ -318,13 +288,12 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
   uint32_t st_issued = 0, bi_issued = 0;
   uint32_t st_par[C::STAGES], bi_par[2];
   bool ok = true;
-  const int rank = cta_rank<C>();
-  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
+  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int n0 = nb * C::BN;
-    const int m0 = mb * C::kTileM + rank * kBlockM;  // this CTA's rows
-    const int e = tile_expert(p, mb * C::kTileM, true);
+    const int m0 = mb * kBlockM;
+    const int e = tile_expert(p, m0, true);
     if (e < 0) continue;  // every role skips the same tiles
     const int wrow0 = e * p.N + n0;  // the expert's weight rows in the [E*N, K] tensor map
     // bias of the tile (clipped to N; nothing when there is no bias)
@@ -351,18 +320,9 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       }
       const bool sf = C::FMT == 1 && (kb & ((1 << p.sf_shift) - 1)) == 0;
       uint8_t* sa = smem + st.slot * C::kStage;
-      if constexpr (C::PAIR) {
-        // both CTAs' tiles complete on the first CTA's full barrier, which
-        // the first CTA arms with the pair's total byte count
-        if (rank == 0) mbar_arrive_expect_tx(full + st.slot, C::kStageTx);
-        const uint32_t bar = mapa_shared(full + st.slot, 0);
-        tma_load_2d_pair(sa, tmA, bar, kb * 128, m0);
-        tma_load_2d_pair(sa + C::kA, tmB, bar, kb * 128, wrow0 + rank * C::kBRows);
-      } else {
-        mbar_arrive_expect_tx(full + st.slot, C::kStageTx + (sf ? C::kSfBytes : 0));
-        tma_load_2d(sa, tmA, full + st.slot, kb * 128, m0);
-        tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, wrow0);
-      }
+      mbar_arrive_expect_tx(full + st.slot, C::kStageTx + (sf ? C::kSfBytes : 0));
+      tma_load_2d(sa, tmA, full + st.slot, kb * 128, m0);
+      tma_load_2d(sa + C::kA, tmB, full + st.slot, kb * 128, wrow0);
       if (sf) {
         uint8_t* sfs = sa + C::kA + C::kB;
         bulk_load(sfs, p.sfa + (static_cast<size_t>(m0 / kBlockM) * p.Kq + (kb >> p.sf_shift)) * kSfChunkBytes,
@@ -381,12 +341,8 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
     }
   }
   // Every issued copy must have landed before the CTA's shared memory goes away.
-  // (A pair's tile loads complete on the first CTA's barriers: it waits for
-  // both CTAs' copies there; the kernel's final cluster barrier keeps the
-  // second CTA alive until then.)
-  if (rank == 0)
-    for (int s = 0; s < C::STAGES; ++s)
-      if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
+  for (int s = 0; s < C::STAGES; ++s)
+    if ((st_issued >> s) & 1u) (void)mbar_wait(full + s, st_par[s], kTeardownNs, nullptr);
   for (int s = 0; s < 2; ++s)
     if ((bi_issued >> s) & 1u) (void)mbar_wait(bfull + s, bi_par[s], kTeardownNs, nullptr);
 }
@@ -406,11 +362,11 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   uint32_t sf_set = 1;  // the set the next copy goes to is sf_set ^ 1
   uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
-  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
+  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
     if (p.row_expert != nullptr) {
       int mb, nb;
       tile_coords(tile, p.num_m, p.num_n, mb, nb);
-      if (tile_expert(p, mb * C::kTileM, false) < 0) continue;
+      if (tile_expert(p, mb * kBlockM, false) < 0) continue;
     }
     for (int kb = 0; kb < p.Kb; ++kb) {
       if (!mbar_wait(full + st.slot, st.phase, limit, abort_flag)) {
@@ -447,9 +403,7 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
       for (int k = 0; k < 4; ++k) {
         const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
         const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
-        if (C::PAIR) {
-          mma_f8f6f4_pair(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
-        } else if (C::FMT == 0) {
+        if (C::FMT == 0) {
           mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
         } else {
           // the byte of each row's scale word: the K-block's (1 x 128 groups) or the step's (1 x 32)
@@ -458,70 +412,65 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
                        (kb > 0 || k > 0) ? 1u : 0u);
         }
       }
-      if constexpr (C::PAIR) {
-        tc_commit_pair(empty + st.slot, 0x3);  // frees the stage in both CTAs
-      } else {
-        tc_commit(empty + st.slot);
-      }
+      tc_commit(empty + st.slot);
       if (C::FMT == 0 || kb == p.Kb - 1) {
-        if constexpr (C::PAIR) {
-          tc_commit_pair(tfull + ab.slot, 0x3);
-        } else {
-          tc_commit(tfull + ab.slot);
-        }
+        tc_commit(tfull + ab.slot);
         ab.template advance<C::kNumAcc>();
       }
       st.template advance<C::STAGES>();
     }
   }
   // All issued tensor-core ops must finish before TMEM is released.
-  if constexpr (C::PAIR) {
-    tc_commit_pair(teardown, 0x1);
-  } else {
-    tc_commit(teardown);
-  }
+  tc_commit(teardown);
   (void)mbar_wait(teardown, 0, kTeardownNs, nullptr);
 }
 
-// The float scales one epilogue thread applies, in the order it applies them:
-// for each tile of the CTA's walk and each of its K-blocks, sx(the thread's
-// row, kb) and sw(the 128-column weight block of the thread's columns, kb).
+// Float scales, one warp: for each tile of the CTA's walk and each of its
+// K-blocks, the x scales of the tile's 128 rows (K-major layout: 128
+// consecutive floats, lane l takes rows l, l+32, l+64, l+96) and the weight
+// scale of each of the tile's 128-column blocks go into the next slot of the
+// scale ring, which the epilogue warps release.  The ring lets these global
+// loads run several K-blocks ahead of their use.
 template <class C>
-struct ScaleStream {
-  int tile = 0, kb = 0;
-  int xoff = 0;  // row of the thread in xs_t's K-major layout
-  int woff = 0;  // offset of the weight block's row in w_scale
-  __device__ __forceinline__ void start(const KParams& p, int t, int sub_row, int col) {
-    kb = 0;
-    for (; t < p.num_tiles; t += tile_stride<C>()) {  // the next tile that is not skipped
-      int mb, nb;
-      tile_coords(t, p.num_m, p.num_n, mb, nb);
-      const int e = tile_expert(p, mb * C::kTileM, false);
-      if (e < 0) continue;
-      xoff = mb * C::kTileM + sub_row;
-      // a column block past N (ragged last tile) reads the last block: its
-      // columns are never stored
-      woff = (e * p.Nb + min((nb * C::BN + col) / 128, p.Nb - 1)) * p.Kb;
-      break;
+__device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
+                                             volatile int* abort_flag, int lane) {
+  const uint64_t limit = p.wait_limit_ns;
+  Ring sr;
+  for (int tile = static_cast<int>(blockIdx.x); tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
+    int mb, nb;
+    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    const int e = tile_expert(p, mb * kBlockM, false);
+    if (e < 0) continue;
+    const float* xs = p.xs_t + mb * kBlockM + lane;
+    // a column block past N (ragged last tile) reads the last block: its
+    // columns are never stored
+    const int wb = e * p.Nb + min(nb * C::BN / 128 + (lane & 1), p.Nb - 1);
+    const float* ws = p.w_scale + static_cast<int64_t>(wb) * p.Kb;
+    for (int kb = 0; kb < p.Kb; ++kb) {
+      if (!mbar_wait_warp(sempty + sr.slot, sr.phase ^ 1u, limit, abort_flag)) {
+        raise_abort(abort_flag, p.status);
+        return;
+      }
+      float* slot = reinterpret_cast<float*>(smem + C::kOffScale + sr.slot * C::kScaleSlot);
+      const float* src = xs + static_cast<int64_t>(kb) * p.ld_s;
+      const float a0 = src[0], a1 = src[32], a2 = src[64], a3 = src[96];
+      const float w = lane < C::BN / 128 ? ws[kb] : 0.0f;
+      slot[lane] = a0;
+      slot[lane + 32] = a1;
+      slot[lane + 64] = a2;
+      slot[lane + 96] = a3;
+      if (lane < C::BN / 128) slot[128 + lane] = w;
+      mbar_arrive(sfull + sr.slot);  // one arrival per lane, each releasing its own stores
+      sr.template advance<C::kSRing>();
     }
-    tile = t;
   }
-  // {sx, sw} of the next (tile, K-block), or zeros past the end of the walk.
-  __device__ __forceinline__ float2 next(const KParams& p, int sub_row, int col) {
-    float2 v = make_float2(0.0f, 0.0f);
-    if (tile < p.num_tiles) {
-      v.x = p.xs_t[static_cast<int64_t>(kb) * p.ld_s + xoff];
-      v.y = p.w_scale[woff + kb];
-      if (++kb == p.Kb) start(p, tile + tile_stride<C>(), sub_row, col);
-    }
-    return v;
-  }
-};
+}
 
 template <class C>
 __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& p, uint8_t* smem, uint32_t tmem_base,
                                          uint64_t* tfull, uint64_t* tempty, uint64_t* bfull, uint64_t* bempty,
-                                         volatile int* abort_flag, int warp, int lane) {
+                                         uint64_t* sfull, uint64_t* sempty, volatile int* abort_flag, int warp,
+                                         int lane) {
   const uint64_t limit = p.wait_limit_ns;
   const int ew = warp - 4;
   const int q = warp & 3;      // TMEM lane quadrant
@@ -529,24 +478,14 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   const int col0 = wg * C::kCols;
   uint8_t* stg = smem + C::kOffStaging + ew * C::kOutBufs * C::kOutBuf;
   const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-  Ring ab, bi;
+  Ring ab, bi, sr;
   bool ok = true;
-  const int rank = cta_rank<C>();
-  const int sub_row = rank * kBlockM + q * 32 + lane;  // this thread's row inside a tile
-  // float path: scales of the current and the next K-block in registers, the
-  // one after that in flight
-  ScaleStream<C> ss;
-  float2 s_now = make_float2(0.0f, 0.0f), s_nxt = make_float2(0.0f, 0.0f);
-  if constexpr (C::FMT == 0) {
-    ss.start(p, tile_start<C>(), sub_row, col0);
-    s_now = ss.next(p, sub_row, col0);
-    s_nxt = ss.next(p, sub_row, col0);
-  }
-  for (int tile = tile_start<C>(); ok && tile < p.num_tiles; tile += tile_stride<C>()) {
+  const int sub_row = q * 32 + lane;  // this thread's row inside a tile
+  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
-    if (tile_expert(p, mb * C::kTileM, false) < 0) continue;
-    const int row0 = mb * C::kTileM + rank * kBlockM + q * 32;
+    if (tile_expert(p, mb * kBlockM, false) < 0) continue;
+    const int row0 = mb * kBlockM + q * 32;
     // the tile's bias (bias ring; zeros past N or without bias)
     if (!mbar_wait_warp(bfull + bi.slot, bi.phase, limit, abort_flag)) {
       raise_abort(abort_flag, p.status);
@@ -572,9 +511,18 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       if (lane == 0) mbar_arrive(bempty + bi.slot);
       bi.template advance<2>();
       for (int kb = 0; kb < p.Kb; ++kb) {
-        const float s = s_now.x * s_now.y;  // sx(m, kb) * sw(block, kb)
-        s_now = s_nxt;
-        s_nxt = ss.next(p, sub_row, col0);
+        // sx(m, kb) * sw(block, kb) from the scale ring
+        if (!mbar_wait_warp(sfull + sr.slot, sr.phase, limit, abort_flag)) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        const float* slot = reinterpret_cast<const float*>(smem + C::kOffScale + sr.slot * C::kScaleSlot);
+        const float sc = slot[sub_row] * slot[128 + wg * (C::BN / 256)];
+        const float2 s2 = make_float2(sc, sc);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sempty + sr.slot);
+        sr.template advance<C::kSRing>();
         if (!mbar_wait_warp(tfull + ab.slot, ab.phase, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
           ok = false;
@@ -598,14 +546,18 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
           if (!more) {  // every column of this K-block is in registers: hand the buffer back
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) release_tmem<C>(tempty + ab.slot);
+            if (lane == 0) mbar_arrive(tempty + ab.slot);
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[(c + h) * 32 + j] =
-                  __float_as_uint(__fmaf_rn(__uint_as_float(r[h][j]), s, __uint_as_float(acc[(c + h) * 32 + j])));
+            for (int j = 0; j < 32; j += 2) {  // acc += P * s, two lanes per packed FMA
+              uint32_t* a = acc + (c + h) * 32 + j;
+              const float2 o = __ffma2_rn(make_float2(__uint_as_float(r[h][j]), __uint_as_float(r[h][j + 1])), s2,
+                                          make_float2(__uint_as_float(a[0]), __uint_as_float(a[1])));
+              a[0] = __float_as_uint(o.x);
+              a[1] = __float_as_uint(o.y);
+            }
             if (more) tmem_ld32(taddr + (c + 2 + h) * 32, r[h]);
           }
           if (more) {
@@ -631,7 +583,7 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       for (int c = 0; c < C::kChunks; ++c) tmem_reg_fence(acc + c * 32);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) release_tmem<C>(tempty + ab.slot);
+      if (lane == 0) mbar_arrive(tempty + ab.slot);
       ab.template advance<C::kNumAcc>();
     }
 
@@ -710,10 +662,14 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* tempty = tfull + C::kNumAcc;
   uint64_t* bfull = tempty + C::kNumAcc;
   uint64_t* bempty = bfull + 2;
-  uint64_t* teardown = bempty + 2;
+  uint64_t* sfull = bempty + 2;
+  uint64_t* sempty = sfull + C::kSRing;
+  uint64_t* teardown = sempty + C::kSRing;
   uint64_t* stall = teardown + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert(C::kOffBar + 8 * (2 * C::STAGES + 2 * C::kNumAcc + 4 + 2 * C::kSRing + 2) + 8 <= C::kOffBar + 512,
+                "barrier block");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -727,11 +683,15 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int a = 0; a < C::kNumAcc; ++a) {
       mbar_init(tfull + a, 1);
-      mbar_init(tempty + a, C::kTmemEmptyCount);
+      mbar_init(tempty + a, C::kEpiWarps);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bfull + s, 1);
       mbar_init(bempty + s, C::kEpiWarps);
+    }
+    for (int s = 0; s < C::kSRing; ++s) {
+      mbar_init(sfull + s, 32);             // every lane of the scale warp
+      mbar_init(sempty + s, C::kEpiWarps);
     }
     mbar_init(teardown, 1);
     mbar_init(stall, 1);
@@ -739,17 +699,11 @@ __global__ void __launch_bounds__(384, 1)
     fence_mbarrier_init();
   }
   if (warp == 2) {
-    if constexpr (C::PAIR) {
-      tmem_alloc_pair(tmem_slot, 512);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, 512);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  if constexpr (C::PAIR) cluster_sync();  // the peer's barriers are initialised before any use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Everything above overlapped the preceding kernel (programmatic dependent
@@ -761,34 +715,25 @@ __global__ void __launch_bounds__(384, 1)
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
       producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag);
-    else if (warp == 1 && lane == 0 && cta_rank<C>() == 0)
+    else if (warp == 1 && lane == 0)
       mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, abort_flag);
-    if constexpr (C::REQUANT) {
+    if constexpr (C::FMT == 0) {
+      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, abort_flag, lane);
+    }
+    if constexpr (C::REQUANT && C::FMT == 1) {
       if (warp == 2 || warp == 3)
         prepare_next_layer<C>(p, static_cast<int>(blockIdx.x) * 64 + (warp - 2) * 32 + lane,
                               static_cast<int>(gridDim.x) * 64);
     }
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
-    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, abort_flag, warp, lane);
+    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, sfull, sempty, abort_flag, warp, lane);
   }
 
-  if (C::PAIR && *abort_flag) {
-    // after an abort the peer may still have copies in flight into this CTA:
-    // give them a bounded moment to land before the pair tears down
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 50000ull) {
-    }
-  }
   __syncthreads();
-  if constexpr (C::PAIR) cluster_sync();  // the first CTA's MMAs use this CTA's shared memory and TMEM
   if (warp == 2) {
     tc_fence_after();
-    if constexpr (C::PAIR) {
-      tmem_dealloc_pair(tmem_base, 512);
-    } else {
-      tmem_dealloc(tmem_base, 512);
-    }
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -828,7 +773,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K, g.M, g.K, 128, kBlockM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K,
-                    static_cast<uint64_t>(g.N) * (g.row_expert != nullptr ? g.E : 1), g.K, 128, C::kBRows,
+                    static_cast<uint64_t>(g.N) * (g.row_expert != nullptr ? g.E : 1), g.K, 128, C::BN,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, static_cast<uint64_t>(g.ld_y) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
@@ -841,7 +786,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.Kb = g.Kb;
   p.Kq = g.Kq;
   p.Nb = (g.N + 127) / 128;
-  p.num_m = (g.M + C::kTileM - 1) / C::kTileM;
+  p.num_m = (g.M + kBlockM - 1) / kBlockM;
   p.num_n = (g.N + C::BN - 1) / C::BN;
   p.num_tiles = p.num_m * p.num_n;
   p.xs_t = g.xs_t;
@@ -866,16 +811,19 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.sf_shift = g.sf32 ? 0 : 2;
   if (p.num_tiles == 0) return cudaSuccess;
 
-  // the shared-memory opt-in (and, for CTA pairs, the cluster occupancy) once
-  // per device: one bit per device; calls from several host threads may
-  // repeat it, which is harmless
+  // the shared-memory opt-in once per device: one bit per device; calls from
+  // several host threads may repeat it, which is harmless
   static std::atomic<uint64_t> configured{0};
-  static std::atomic<int> max_clusters{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit, std::memory_order_release);
+  }
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
@@ -885,35 +833,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if constexpr (C::PAIR) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 2;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
-  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    if constexpr (C::PAIR) {
-      // how many CTA pairs fit on the device at once (SMs pair up within a GPC)
-      cfg.gridDim = dim3(2 * (num_sms / 2));
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        n = num_sms / 2;
-      }
-      max_clusters.store(n, std::memory_order_relaxed);
-    }
-    configured.fetch_or(bit, std::memory_order_release);
-  }
-  if constexpr (C::PAIR) {
-    const int mc = max_clusters.load(std::memory_order_relaxed);
-    const int clusters = p.num_tiles < mc ? p.num_tiles : mc;
-    cfg.gridDim = dim3(2 * clusters);
-  } else {
-    cfg.gridDim = dim3(p.num_tiles < num_sms ? p.num_tiles : num_sms);
-  }
+  cfg.gridDim = dim3(p.num_tiles < num_sms ? p.num_tiles : num_sms);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -936,23 +856,24 @@ int choose_block_n(int M, int N, int num_sms) {
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s) {
-  if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
-    const bool short_k = g.Kb <= 32;
-    if (fmt == 0) {
-      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, false, true>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 2, false, true>>(g, num_sms, s);
-    }
-    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, false, true>>(g, num_sms, s);
-    return launch_cfg<Cfg<256, 1, 4, 1, false, true>>(g, num_sms, s);
-  }
-  const int bn = choose_block_n(g.M, g.N, num_sms);
   // Short K: few K-blocks per tile, so the tile's output path dominates --
   // give every output chunk its own staging box and keep one stage fewer.
+  // Long K: four stages (the float path's scale ring takes the shared memory
+  // of the second staging box per warp).
   const bool short_k = g.Kb <= 32;
+  if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
+    if (fmt == 0) {
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 1, true>>(g, num_sms, s);
+    }
+    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, true>>(g, num_sms, s);
+    return launch_cfg<Cfg<256, 1, 4, 1, true>>(g, num_sms, s);
+  }
+  const int bn = choose_block_n(g.M, g.N, num_sms);
   if (fmt == 0) {
     if (bn == 256) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 2>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 1>>(g, num_sms, s);
     }
     return launch_cfg<Cfg<128, 0, 5, 2>>(g, num_sms, s);
   }

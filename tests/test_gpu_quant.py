@@ -62,7 +62,7 @@ def test_act_quant_bitexact(fg8, orc, fmt, M, K):
 # 75,776 groups per pass over 148 SMs; 256 groups of 32 per CTA, 303,104 per
 # pass): these shapes need 6 and more passes of the grid-stride loop.
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("M,K", [(8192, 7168), (4096, 14336), (16384, 1040)])
+@pytest.mark.parametrize("M,K", [(8192, 7168), (4096, 14336), (24000, 1040)])
 def test_act_quant_bitexact_multi_pass(fg8, orc, fmt, M, K):
     x = W.x_student_t(M, K, seed=M + K)
     assert M * ((K + 127) // 128) > 2 * 75776
