@@ -126,7 +126,7 @@ struct Cfg {
   static constexpr int kBiasSlot = BN * 2;
   // float scale ring: per K-block the 128 rows' x scales, then the weight
   // scales of the tile's BN/128 column blocks (padded to 16 bytes)
-  static constexpr int kSRing = FMT == 0 ? 4 : 0;
+  static constexpr int kSRing = FMT == 0 ? 8 : 0;
   static constexpr int kScaleSlot = 128 * 4 + 16;
   // register split after launch (384 x 168): the wide float epilogue holds
   // 128 accumulators + 64 TMEM registers per thread, the others need less
@@ -426,11 +426,12 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
 }
 
 // Float scales, one warp: for each tile of the CTA's walk and each of its
-// K-blocks, the x scales of the tile's 128 rows (K-major layout: 128
-// consecutive floats, lane l takes rows l, l+32, l+64, l+96) and the weight
-// scale of each of the tile's 128-column blocks go into the next slot of the
-// scale ring, which the epilogue warps release.  The ring lets these global
-// loads run several K-blocks ahead of their use.
+// K-blocks, the x scales of the tile's 128 rows (K-major layout: 512
+// contiguous bytes, 16 per lane) and the weight scale of each of the tile's
+// 128-column blocks are copied asynchronously (cp.async) into the next slot
+// of the scale ring; each lane's copies complete the slot's barrier as they
+// land, so up to kSRing K-blocks of scale loads are in flight and their
+// latency stays off the epilogue's path.  The epilogue warps release slots.
 template <class C>
 __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
                                              volatile int* abort_flag, int lane) {
@@ -441,7 +442,7 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
     const int e = tile_expert(p, mb * kBlockM, false);
     if (e < 0) continue;
-    const float* xs = p.xs_t + mb * kBlockM + lane;
+    const float* xs = p.xs_t + mb * kBlockM + 4 * lane;
     // a column block past N (ragged last tile) reads the last block: its
     // columns are never stored
     const int wb = e * p.Nb + min(nb * C::BN / 128 + (lane & 1), p.Nb - 1);
@@ -449,21 +450,17 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
     for (int kb = 0; kb < p.Kb; ++kb) {
       if (!mbar_wait_warp(sempty + sr.slot, sr.phase ^ 1u, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
+        cp_async_wait_all();
         return;
       }
       float* slot = reinterpret_cast<float*>(smem + C::kOffScale + sr.slot * C::kScaleSlot);
-      const float* src = xs + static_cast<int64_t>(kb) * p.ld_s;
-      const float a0 = src[0], a1 = src[32], a2 = src[64], a3 = src[96];
-      const float w = lane < C::BN / 128 ? ws[kb] : 0.0f;
-      slot[lane] = a0;
-      slot[lane + 32] = a1;
-      slot[lane + 64] = a2;
-      slot[lane + 96] = a3;
-      if (lane < C::BN / 128) slot[128 + lane] = w;
-      mbar_arrive(sfull + sr.slot);  // one arrival per lane, each releasing its own stores
+      cp_async16(slot + 4 * lane, xs + static_cast<int64_t>(kb) * p.ld_s);
+      if (lane < C::BN / 128) cp_async4(slot + 128 + lane, ws + kb);
+      cp_async_mbar_arrive(sfull + sr.slot);  // one arrival per lane, when its copies have landed
       sr.template advance<C::kSRing>();
     }
   }
+  cp_async_wait_all();  // the CTA's shared memory must outlive every copy in flight
 }
 
 template <class C>
