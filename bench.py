@@ -344,18 +344,19 @@ def run_fg8(args, rank, world, local):
     # tiled, consecutive layers chain: the GEMM of layer i also quantizes its
     # output for layer i+1 (fg8_linear_run_chain), so layer i+1 has no
     # act-quant launch.
-    # block 32 (1 x 32 groups, 32 x 32 weight blocks): fg8_linear_block per layer
-    paths = [("block32" if args.block == 32 else layer_path(L["g"])) for L in plan]
+    # block 32 / 64 (1 x b groups, b x b weight blocks): fg8_linear_block per layer
+    paths = [("small_block" if args.block != 128 else layer_path(L["g"])) for L in plan]
     chain = not args.no_chain and all(pth == "tiled" for pth in paths)
 
     def launch_layer(i, ev_mid=None):
         L = plan[i]
         g = L["g"]
-        if paths[i] == "block32":  # act-quant, scale packing and GEMM in one call
+        if paths[i] == "small_block":  # act-quant, scale packing and GEMM in one call
             if ev_mid is not None:
                 ev_mid.record(stream)
             fg8.fg8_linear_block(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["wq"].data_ptr(),
-                                 L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt, 32,
+                                 L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt,
+                                 args.block,
                                  L["wsp"].data_ptr(), L["wsp"].numel(), sp)
             return
         if paths[i] == "fused":
@@ -469,8 +470,8 @@ def run_fg8(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": gemm_bytes(g) / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(args.workload, dom)  # ncu DRAM bytes per launch, None if stale
-    roof["kernel"] = ("fg8_gemm_kernel, 32 x 32 blocks, timed with its act-quant and scale packing"
-                      if paths[dom] == "block32" else
+    roof["kernel"] = (f"fg8_gemm_kernel, {args.block} x {args.block} blocks, timed with its act-quant "
+                      f"and scale packing" if paths[dom] == "small_block" else
                       "fg8_small_m_kernel" if paths[dom] != "tiled" else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
@@ -481,12 +482,12 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        fused = paths[i] in ("fused", "block32") or (chain and i > 0)  # act-quant not timed on its own
+        fused = paths[i] in ("fused", "small_block") or (chain and i > 0)  # act-quant not timed on its own
         per_kernel.append({"layer": gi.name, "path": paths[i], "act_quant_us": None if fused else qm[i] * 1e3,
                            "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
                            "act_quant": ("fused into the few-token kernel" if paths[i] == "fused" else
                                          "timed with the GEMM (fg8_linear_block: act-quant, scale packing, GEMM)"
-                                         if paths[i] == "block32" else
+                                         if paths[i] == "small_block" else
                                          "fused into the previous GEMM" if fused else "own launch"),
                            "gemm_us": gm[i] * 1e3, "gemm_tflops": gemm_flops(gi) / (gm[i] * 1e-3) / 1e12,
                            "gemm_pct_fp8_peak": 100.0 * gemm_flops(gi) / (gm[i] * 1e-3) / 1e12 / fp8_peak,
@@ -1024,8 +1025,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle baseline of the fg8 arm")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: CPU seconds that the warm-up and timed steps together aim at")
-    ap.add_argument("--block", type=int, default=128, choices=[128, 32],
-                    help="weight_block_size (block, block) and 1 x block activation groups; 32 takes UE8M0 workloads")
+    ap.add_argument("--block", type=int, default=128, choices=[128, 64, 32],
+                    help="weight_block_size (block, block) and 1 x block activation groups (either scale format)")
     ap.add_argument("--no-chain", action="store_true",
                     help="quantize every layer's input in its own launch instead of in the previous GEMM")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
@@ -1037,9 +1038,8 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_env()
-    if args.block == 32 and (args.workload.startswith("moe_") or
-                             any(g.fmt != 1 for _, g, _ in workload_layers(args.workload))):
-        raise SystemExit("--block 32 runs UE8M0 dense workloads (dsv3_mlp, square_m*_ue8m0)")
+    if args.block != 128 and args.workload.startswith("moe_"):
+        raise SystemExit("--block 32 / 64 runs the dense workloads (the expert GEMM takes 128 x 128 blocks)")
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

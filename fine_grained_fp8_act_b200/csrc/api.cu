@@ -367,7 +367,7 @@ fg8_status fg8_grouped_linear_prepare(const void* x_bf16, int64_t M, int64_t K, 
   if (fmt == FG8_SCALE_UE8M0)  // every expert's [Nb][Kb] bytes as one stack of 128-row tiles
     return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv),
                                       static_cast<int>(E * ceil_div(N, 128) * 128), sfb_rows(grouped_sf_rows(E, N)),
-                                      128, ceil_div(K, kGroup), ws + L.wsc_off, s));
+                                      128, ceil_div(K, kGroup), 1, ws + L.wsc_off, s));
   return FG8_OK;
 }
 
@@ -437,14 +437,16 @@ fg8_status fg8_grouped_linear(const void* x_bf16, int64_t M, int64_t K, int64_t 
                                 workspace_bytes, stream);
 }
 
-// ---- non-default block size: weight_block_size = (32, 32) ([zh] §八) ----
-// 1 x 32 activation groups and 32 x 32 weight blocks.  The layer takes UE8M0
-// scales: the block-scaled MMA applies one scale per 32 K per row natively,
-// whereas float scales would need a register promotion per 32-K slice.
+// ---- non-default block sizes: weight_block_size = (32, 32) or (64, 64) ([zh] §八) ----
+// 1 x b activation groups and b x b weight blocks.  UE8M0: the block-scaled
+// MMA applies one scale per 32 K per row (a 64-block's scale on both of its
+// steps); float: the GEMM promotes every b-wide slice of K in registers.
+bool small_block(int block) { return block == 32 || block == 64; }
+
 fg8_status fg8_quantize_act_block(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* xq_e4m3,
                                   void* x_scale, fg8_scale_fmt fmt, int block, void* stream) {
   if (block == 128) return fg8_quantize_act(x_bf16, M, K, ld_x, xq_e4m3, x_scale, fmt, stream);
-  if (block != 32 || !fmt_ok(fmt) || M < 0 || K <= 0 || M > kMaxDim || K > kMaxDim || ld_x < K)
+  if (!small_block(block) || !fmt_ok(fmt) || M < 0 || K <= 0 || M > kMaxDim || K > kMaxDim || ld_x < K)
     return FG8_ERR_INVALID_ARG;
   if (M == 0) return FG8_OK;
   if (x_bf16 == nullptr || xq_e4m3 == nullptr || x_scale == nullptr) return FG8_ERR_INVALID_ARG;
@@ -456,8 +458,8 @@ fg8_status fg8_quantize_act_block(const void* x_bf16, int64_t M, int64_t K, int6
   a.ld_x = ld_x;
   a.M = static_cast<int>(M);
   a.K = static_cast<int>(K);
-  a.Kb = ceil_div(K, 32);
-  a.group = 32;
+  a.Kb = ceil_div(K, block);
+  a.group = block;
   a.xq = static_cast<uint8_t*>(xq_e4m3);
   a.xs = x_scale;
   a.layout = kScaleRowMajor;
@@ -467,39 +469,47 @@ fg8_status fg8_quantize_act_block(const void* x_bf16, int64_t M, int64_t K, int6
 fg8_status fg8_quantize_weight_block(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w, void* wq_e4m3,
                                      void* w_scale_inv, fg8_scale_fmt fmt, int block, void* stream) {
   if (block == 128) return fg8_quantize_weight(w_bf16, N, K, ld_w, wq_e4m3, w_scale_inv, fmt, stream);
-  if (block != 32 || !fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K)
+  if (!small_block(block) || !fmt_ok(fmt) || N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim || ld_w < K)
     return FG8_ERR_INVALID_ARG;
   if (w_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr) return FG8_ERR_INVALID_ARG;
-  if (ceil_div(N, 32) * static_cast<int64_t>(ceil_div(K, 32)) > kMaxDim / 8) return FG8_ERR_INVALID_ARG;
+  if (ceil_div(N, block) * static_cast<int64_t>(ceil_div(K, block)) > kMaxDim / 8) return FG8_ERR_INVALID_ARG;
   if (K % 16 != 0 || ld_w % 8 != 0 || !aligned16(w_bf16) || !aligned16(wq_e4m3)) return FG8_ERR_ALIGNMENT;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
-  return cuda_status(launch_weight_quant32(w_bf16, ld_w, static_cast<int>(N), static_cast<int>(K),
-                                           static_cast<uint8_t*>(wq_e4m3), w_scale_inv, fmt,
-                                           static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_weight_quant_small(w_bf16, ld_w, static_cast<int>(N), static_cast<int>(K), block,
+                                               static_cast<uint8_t*>(wq_e4m3), w_scale_inv, fmt,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
-// Workspace of the 32-block layer: [header | xq | x scale-factor tiles | W
-// scale-factor tiles], one 512-byte chunk per 128 rows and K-block of 128
-// (its four bytes per row are the four 1 x 32 scales).
-struct Block32Ws {
+// Workspace of the small-block layer: [header | xq | x scales | W scales]
+//   UE8M0: x and W scale-factor tiles, one 512-byte chunk per 128 rows and
+//          K-block of 128 (its four bytes per row are the four 32-K steps' scales)
+//   float: x scales K-major [ceil(K/b)][ld_s] float32 (W scales read as given)
+struct SmallBlockWs {
   size_t xq_off, sfa_off, sfb_off, total;
+  int64_t ld_s;
 };
 
-Block32Ws block32_ws_layout(int64_t M, int64_t N, int64_t K) {
-  Block32Ws w;
+SmallBlockWs small_block_ws_layout(int64_t M, int64_t N, int64_t K, int fmt, int block) {
+  SmallBlockWs w;
   const int Kb = ceil_div(K, kGroup);
   w.xq_off = kHeaderBytes;
   w.sfa_off = align_up(w.xq_off + static_cast<size_t>(M) * K, kAlign);
-  w.sfb_off = align_up(w.sfa_off + static_cast<size_t>(ceil_div(M, 128)) * Kb * kSfChunkBytes, kAlign);
-  w.total = align_up(w.sfb_off + static_cast<size_t>(sfb_rows(N) / 128) * Kb * kSfChunkBytes, kAlign);
+  w.ld_s = kmajor_ld(M);
+  if (fmt == FG8_SCALE_FLOAT) {
+    w.sfb_off = align_up(w.sfa_off + static_cast<size_t>(ceil_div(K, block)) * w.ld_s * sizeof(float), kAlign);
+    w.total = w.sfb_off;
+  } else {
+    w.sfb_off = align_up(w.sfa_off + static_cast<size_t>(ceil_div(M, 128)) * Kb * kSfChunkBytes, kAlign);
+    w.total = align_up(w.sfb_off + static_cast<size_t>(sfb_rows(N) / 128) * Kb * kSfChunkBytes, kAlign);
+  }
   return w;
 }
 
 size_t fg8_linear_block_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt, int block) {
   if (block == 128) return fg8_linear_workspace_bytes(M, N, K, fmt);
-  if (block != 32 || fmt != FG8_SCALE_UE8M0 || check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
-  return block32_ws_layout(M, N, K).total;
+  if (!small_block(block) || check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
+  return small_block_ws_layout(M, N, K, fmt, block).total;
 }
 
 fg8_status fg8_linear_block(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
@@ -508,16 +518,14 @@ fg8_status fg8_linear_block(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   if (block == 128)
     return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, workspace,
                       workspace_bytes, stream);
-  if (block != 32 || fmt != FG8_SCALE_UE8M0) return FG8_ERR_INVALID_ARG;
-  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
-  if (ld_x < K || ld_y < N) return FG8_ERR_INVALID_ARG;
+  if (!small_block(block)) return FG8_ERR_INVALID_ARG;
+  if (const int st = fg8::check_linear_args_status(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                  ld_y, fmt);
+      st != FG8_OK)
+    return static_cast<fg8_status>(st);
   if (M == 0) return FG8_OK;
-  if (x_bf16 == nullptr || wq_e4m3 == nullptr || w_scale_inv == nullptr || y_bf16 == nullptr)
-    return FG8_ERR_INVALID_ARG;
-  if (ld_x % 8 != 0 || ld_y % 8 != 0 || !aligned16(x_bf16) || !aligned16(wq_e4m3) || !aligned16(y_bf16) ||
-      (bias_bf16 != nullptr && !aligned16(bias_bf16)))
-    return FG8_ERR_ALIGNMENT;
-  const Block32Ws L = block32_ws_layout(M, N, K);
+  if (ceil_div(N, block) * static_cast<int64_t>(ceil_div(K, block)) > kMaxDim / 8) return FG8_ERR_INVALID_ARG;
+  const SmallBlockWs L = small_block_ws_layout(M, N, K, fmt, block);
   if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
@@ -529,19 +537,33 @@ fg8_status fg8_linear_block(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   a.ld_x = ld_x;
   a.M = static_cast<int>(M);
   a.K = static_cast<int>(K);
-  a.Kb = ceil_div(K, 32);
-  a.group = 32;
+  a.Kb = ceil_div(K, block);
+  a.group = block;
   a.xq = ws + L.xq_off;
   a.xs = ws + L.sfa_off;
-  a.layout = kScaleSfTiles;
-  a.Kq = Kb;  // = ceil(ceil(K/32) / 4): a chunk's four bytes are the K-block's four 1 x 32 scales
-  a.M_pad = ceil_div(M, 128) * 128;
-  if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
-  if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N),
-                                                 sfb_rows(N), 32, ceil_div(K, 32), ws + L.sfb_off, s));
-      st != FG8_OK)
-    return st;
   GemmArgs g{};
+  if (fmt == FG8_SCALE_FLOAT) {
+    a.layout = kScaleKMajor;
+    a.ld_s = L.ld_s;
+    if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
+    g.xs_t = reinterpret_cast<const float*>(ws + L.sfa_off);
+    g.ld_s = L.ld_s;
+    g.w_scale = static_cast<const float*>(w_scale_inv);
+    g.wblk = block;
+  } else {
+    a.layout = kScaleSfTiles;
+    a.Kq = Kb;  // one chunk per K-block of 128: its four bytes are the four 32-K steps' scales
+    a.M_pad = ceil_div(M, 128) * 128;
+    if (fg8_status st = cuda_status(launch_act_quant(a, fmt, dev.sms, s)); st != FG8_OK) return st;
+    if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N),
+                                                   sfb_rows(N), block, ceil_div(K, block), block / 32,
+                                                   ws + L.sfb_off, s));
+        st != FG8_OK)
+      return st;
+    g.sfa = ws + L.sfa_off;
+    g.sfb = ws + L.sfb_off;
+    g.sf32 = true;
+  }
   g.xq = ws + L.xq_off;
   g.wq = wq_e4m3;
   g.y = y_bf16;
@@ -555,9 +577,6 @@ fg8_status fg8_linear_block(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
   g.test_stall = g_test_stall.load();
-  g.sfa = ws + L.sfa_off;
-  g.sfb = ws + L.sfb_off;
-  g.sf32 = true;
   return cuda_status(launch_gemm(g, fmt, dev.sms, s));
 }
 
@@ -578,7 +597,7 @@ fg8_status fg8_linear_prepare(const void* x_bf16, int64_t M, int64_t N, int64_t 
   if (fg8_status st = prepare_act(x_bf16, M, K, ld_x, fmt, ws, L, dev, s); st != FG8_OK) return st;
   if (fmt == FG8_SCALE_UE8M0)
     return cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N), sfb_rows(N),
-                                      128, ceil_div(K, kGroup), ws + L.wsc_off, s));
+                                      128, ceil_div(K, kGroup), 1, ws + L.wsc_off, s));
   return FG8_OK;
 }
 
@@ -747,11 +766,11 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
     g.w_scale = static_cast<const float*>(w_scale_inv);
   } else {
     if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(x_scale), static_cast<int>(M),
-                                                   (M + 127) / 128 * 128, 1, Kb, ws + L.xs_off, s));
+                                                   (M + 127) / 128 * 128, 1, Kb, 1, ws + L.xs_off, s));
         st != FG8_OK)
       return st;
     if (fg8_status st = cuda_status(launch_sf_pack(static_cast<const uint8_t*>(w_scale_inv), static_cast<int>(N),
-                                                   sfb_rows(N), 128, Kb, ws + L.wsc_off, s));
+                                                   sfb_rows(N), 128, Kb, 1, ws + L.wsc_off, s));
         st != FG8_OK)
       return st;
     g.sfa = ws + L.xs_off;

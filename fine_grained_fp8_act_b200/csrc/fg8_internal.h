@@ -33,7 +33,7 @@ struct ActQuantArgs {
   const void* x;      // bf16 [M, K], row stride ld_x
   int64_t ld_x;
   int M, K, Kb;       // Kb: groups per row, ceil(K / group)
-  int group;          // group width: 128 (0 means 128) or 32
+  int group;          // group width: 128 (0 means 128), 64 or 32
   uint8_t* xq;        // e4m3 [M, K], row stride K
   void* xs;           // scales, layout below
   int layout;         // ScaleLayout
@@ -49,14 +49,15 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
 
 cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
                                 cudaStream_t s);
-// 32 x 32 blocks (weight_block_size = (32, 32)): scales [ceil(N/32), ceil(K/32)].
-cudaError_t launch_weight_quant32(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
-                                  cudaStream_t s);
+// block x block weight blocks, block 32 or 64 (weight_block_size = (block,
+// block)): scales [ceil(N/block), ceil(K/block)].
+cudaError_t launch_weight_quant_small(const void* w, int64_t ld_w, int N, int K, int block, uint8_t* wq, void* ws,
+                                      int fmt, cudaStream_t s);
 
 // Pack a UE8M0 [R_src, Kb] row-major scale matrix into scale-factor tiles for
-// R rows, written for R_pad rows (a multiple of 128): row r takes
-// src[(r / row_div) * Kb + kb]; padding rows and K-blocks get byte 127 (2^0).
-cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, uint8_t* dst,
+// R rows, written for R_pad rows (a multiple of 128): row r, slot j takes
+// src[(r / row_div) * Kb + j / kdiv]; padding rows and slots get byte 127 (2^0).
+cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, int kdiv, uint8_t* dst,
                            cudaStream_t s);
 
 // Rows of weight scale-factor tiles: N rounded up to the widest GEMM tile.
@@ -98,10 +99,14 @@ struct GemmArgs {
   const int32_t* row_expert;
   int E;
   int sfb_tiles;
-  // UE8M0 with 1 x 32 activation groups and 32 x 32 weight blocks: the
-  // scale-factor tiles hold ceil(K/32) scales per row, one chunk per K-block
-  // (Kq = ceil(K/128) chunks per row tile)
+  // UE8M0 with 1 x 32 / 1 x 64 activation groups and 32 x 32 / 64 x 64
+  // weight blocks: the scale-factor tiles hold one scale per 32 K per row,
+  // one chunk per K-block (Kq = ceil(K/128) chunks per row tile)
   bool sf32;
+  // float scales: the block size b (0 means 128; 32 or 64): 1 x b x-scale
+  // groups, K-major [ceil(K/b)][ld_s], and b x b weight blocks
+  // [ceil(N/b)][ceil(K/b)]; the GEMM promotes every b-wide slice of K
+  int wblk;
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM

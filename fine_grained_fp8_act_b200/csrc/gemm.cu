@@ -84,8 +84,13 @@ struct KParams {
   // UE8M0 scale granularity along K: one scale-factor chunk (4 scales per
   // row) covers 4 K-blocks of 128 (sf_shift 2, 1 x 128 groups), or one
   // K-block whose 4 MMA steps of K = 32 each take their own scale (sf_shift
-  // 0, 1 x 32 groups and 32 x 32 weight blocks)
+  // 0, 1 x 32 or 1 x 64 groups and 32 x 32 or 64 x 64 weight blocks)
   int sf_shift;
+  // float scales at block size wblk (128, 64 or 32): every K-block of 128 is
+  // promoted in gsteps = 128 / wblk slices of MMA steps (kps_shift = log2 of
+  // the steps per slice), Kg = ceil(K / wblk) slices in all; x scales
+  // [Kg][ld_s], weight scales [Nbs = ceil(N / wblk)][Kg]
+  int wblk, gsteps, kps_shift, Kg, Nbs;
 };
 
 constexpr uint32_t kStatusBadExpert = 1u;  // FG8_ERR_INVALID_ARG
@@ -102,12 +107,16 @@ __device__ __forceinline__ int tile_expert(const KParams& p, int m0, bool report
   return e;
 }
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false, bool SUBK_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
   // REQUANT: the epilogue also quantizes its bf16 output rows, one 128-column
   // group per thread, for a next layer (needs the 256-wide tile).
   static constexpr bool REQUANT = REQUANT_;
+  // SUBK (float scales at block 64 or 32): every K-block is promoted in
+  // 64- or 32-wide slices, and the weight scale changes every 64 or 32
+  // columns of a thread's row; without it, one scale per K-block and thread.
+  static constexpr bool SUBK = SUBK_;
   static constexpr int kA = kBlockM * 128;
   static constexpr int kB = BN * 128;
   static constexpr int kSfBytes = FMT == 1 ? kSfChunkBytes * (1 + BN / 128) : 0;
@@ -124,10 +133,10 @@ struct Cfg {
   static constexpr int kSfbCol = kSfaCol + 4;
   static constexpr int kSfSetCols = 4 + BN / 32;
   static constexpr int kBiasSlot = BN * 2;
-  // float scale ring: per K-block the 128 rows' x scales, then the weight
-  // scales of the tile's BN/128 column blocks (padded to 16 bytes)
+  // float scale ring: per promotion slice the 128 rows' x scales, then the
+  // weight scales of the tile's column blocks (up to 8: BN / 32)
   static constexpr int kSRing = FMT == 0 ? 8 : 0;
-  static constexpr int kScaleSlot = 128 * 4 + 16;
+  static constexpr int kScaleSlot = 128 * 4 + 32;
   // register split after launch (384 x 168): the wide float epilogue holds
   // 128 accumulators + 64 TMEM registers per thread, the others need less
   static constexpr uint32_t kRegsLow = (FMT == 0 && BN == 256) ? 40 : (BN == 128 ? 80 : 56);
@@ -152,8 +161,10 @@ struct Cfg {
   // bytes the stage's full barrier waits for
   static constexpr uint32_t kStageTx = kA + kB;
   // instruction descriptors (M = 128, K-major A and B, e4m3 x e4m3 -> f32)
-  static constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24);
-  static constexpr uint32_t kIdescMx = (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBlockM >> 4) << 24);
+  // (kind::f8f6f4 for float scales, kind::mxf8f6f4 block-scaled for UE8M0)
+  static constexpr uint32_t kIdesc = FMT == 0
+                                         ? (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24)
+                                         : (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBlockM >> 4) << 24);
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
@@ -377,46 +388,86 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
       tc_fence_after();
       const uint32_t a_addr = smem_u32(smem + st.slot * C::kStage);
       const uint32_t b_addr = a_addr + C::kA;
-      if (C::FMT == 0 || kb == 0) {
+      if constexpr (C::FMT == 0 && !C::SUBK) {
+        // float: the K-block's 4 MMA steps of K = 32 into its own TMEM buffer
         if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-      const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
-      if (C::FMT == 1 && (kb & ((1 << p.sf_shift) - 1)) == 0) {
-        // UE8M0 scales of 128 rows x 4 K-blocks (or 4 K = 32 steps) for A, and for B, into TMEM;
-        // issued before the MMAs that read them (tcgen05 ops of one thread
-        // execute in issue order).
-        const uint32_t sfs = b_addr + C::kB;
-        sf_set ^= 1u;
-        sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol + sf_set * C::kSfSetCols);
-        sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol + sf_set * C::kSfSetCols);
-        tc_cp_32x128b_warpx4(sfa_t, smem_desc(sfs, 128, 128, 0));
+        const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
 #pragma unroll
-        for (int h = 0; h < C::BN / 128; ++h)
-          tc_cp_32x128b_warpx4(sfb_t + 4 * h, smem_desc(sfs + kSfChunkBytes * (1 + h), 128, 128, 0));
-      }
+        for (int k = 0; k < 4; ++k)
+          mma_f8f6f4(d, smem_desc(a_addr + k * 32, 16, 1024, 2), smem_desc(b_addr + k * 32, 16, 1024, 2), C::kIdesc,
+                     k > 0 ? 1u : 0u);
+        tc_commit(empty + st.slot);
+        tc_commit(tfull + ab.slot);
+        ab.template advance<C::kNumAcc>();
+        st.template advance<C::STAGES>();
+        continue;
+      } else if constexpr (C::FMT == 0) {
+        // float at block 64 / 32: every promotion slice (2 or 1 MMA steps of
+        // K = 32) into its own TMEM buffer; slices past the last real one are skipped
+        const int kps = 1 << p.kps_shift;
+        const int nsl = min(p.gsteps, p.Kg - kb * p.gsteps);
+        for (int k = 0; k < 4 && (k >> p.kps_shift) < nsl; ++k) {
+          const int j = k & (kps - 1);
+          if (j == 0) {
+            if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
+              raise_abort(abort_flag, p.status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
+          mma_f8f6f4(d, smem_desc(a_addr + k * 32, 16, 1024, 2), smem_desc(b_addr + k * 32, 16, 1024, 2),
+                     C::kIdesc, j > 0 ? 1u : 0u);
+          if (j == kps - 1) {
+            tc_commit(tfull + ab.slot);
+            ab.template advance<C::kNumAcc>();
+          }
+        }
+        if (!ok) break;
+      } else {
+        if (kb == 0) {
+          if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
+            raise_abort(abort_flag, p.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const uint32_t d = tmem_base + static_cast<uint32_t>(ab.slot * C::BN);
+        if ((kb & ((1 << p.sf_shift) - 1)) == 0) {
+          // UE8M0 scales of 128 rows x 4 K-blocks (or 4 K = 32 steps) for A, and for B, into TMEM;
+          // issued before the MMAs that read them (tcgen05 ops of one thread
+          // execute in issue order).
+          const uint32_t sfs = b_addr + C::kB;
+          sf_set ^= 1u;
+          sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol + sf_set * C::kSfSetCols);
+          sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol + sf_set * C::kSfSetCols);
+          tc_cp_32x128b_warpx4(sfa_t, smem_desc(sfs, 128, 128, 0));
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
-        const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
-        if (C::FMT == 0) {
-          mma_f8f6f4(d, ad, bd, C::kIdescF8, k > 0 ? 1u : 0u);
-        } else {
-          // the byte of each row's scale word: the K-block's (1 x 128 groups) or the step's (1 x 32)
+          for (int h = 0; h < C::BN / 128; ++h)
+            tc_cp_32x128b_warpx4(sfb_t + 4 * h, smem_desc(sfs + kSfChunkBytes * (1 + h), 128, 128, 0));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
+          const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
+          // the byte of each row's scale word: the K-block's (1 x 128 groups) or the step's (1 x 32, 1 x 64)
           const uint32_t j = static_cast<uint32_t>(p.sf_shift == 0 ? k : (kb & 3));
-          mma_mxf8f6f4(d, ad, bd, C::kIdescMx | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
+          mma_mxf8f6f4(d, ad, bd, C::kIdesc | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
                        (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        if (kb == p.Kb - 1) {
+          tc_commit(tfull + ab.slot);
+          ab.template advance<C::kNumAcc>();
         }
       }
       tc_commit(empty + st.slot);
-      if (C::FMT == 0 || kb == p.Kb - 1) {
-        tc_commit(tfull + ab.slot);
-        ab.template advance<C::kNumAcc>();
-      }
       st.template advance<C::STAGES>();
     }
   }
@@ -426,11 +477,12 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
 }
 
 // Float scales, one warp: for each tile of the CTA's walk and each of its
-// K-blocks, the x scales of the tile's 128 rows (K-major layout: 512
+// promotion slices (the K-blocks, or their 64- / 32-wide parts for smaller
+// blocks), the x scales of the tile's 128 rows (K-major layout: 512
 // contiguous bytes, 16 per lane) and the weight scale of each of the tile's
-// 128-column blocks are copied asynchronously (cp.async) into the next slot
-// of the scale ring; each lane's copies complete the slot's barrier as they
-// land, so up to kSRing K-blocks of scale loads are in flight and their
+// column blocks are copied asynchronously (cp.async) into the next slot of
+// the scale ring; each lane's copies complete the slot's barrier as they
+// land, so up to kSRing slices of scale loads are in flight and their
 // latency stays off the epilogue's path.  The epilogue warps release slots.
 template <class C>
 __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
@@ -443,19 +495,20 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
     const int e = tile_expert(p, mb * kBlockM, false);
     if (e < 0) continue;
     const float* xs = p.xs_t + mb * kBlockM + 4 * lane;
-    // a column block past N (ragged last tile) reads the last block: its
-    // columns are never stored
-    const int wb = e * p.Nb + min(nb * C::BN / 128 + (lane & 1), p.Nb - 1);
-    const float* ws = p.w_scale + static_cast<int64_t>(wb) * p.Kb;
-    for (int kb = 0; kb < p.Kb; ++kb) {
+    // the weight-scale block of lane j's slot (j < BN / wblk); a block past N
+    // (ragged last tile) reads the last block: its columns are never stored
+    const int nwb = C::BN / p.wblk;
+    const int wb = e * p.Nbs + min(nb * C::BN / p.wblk + (lane & 7), p.Nbs - 1);
+    const float* ws = p.w_scale + static_cast<int64_t>(wb) * p.Kg;
+    for (int g = 0; g < p.Kg; ++g) {
       if (!mbar_wait_warp(sempty + sr.slot, sr.phase ^ 1u, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
         cp_async_wait_all();
         return;
       }
       float* slot = reinterpret_cast<float*>(smem + C::kOffScale + sr.slot * C::kScaleSlot);
-      cp_async16(slot + 4 * lane, xs + static_cast<int64_t>(kb) * p.ld_s);
-      if (lane < C::BN / 128) cp_async4(slot + 128 + lane, ws + kb);
+      cp_async16(slot + 4 * lane, xs + static_cast<int64_t>(g) * p.ld_s);
+      if (lane < nwb) cp_async4(slot + 128 + lane, ws + g);
       cp_async_mbar_arrive(sfull + sr.slot);  // one arrival per lane, when its copies have landed
       sr.template advance<C::kSRing>();
     }
@@ -507,16 +560,22 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       __syncwarp();
       if (lane == 0) mbar_arrive(bempty + bi.slot);
       bi.template advance<2>();
-      for (int kb = 0; kb < p.Kb; ++kb) {
-        // sx(m, kb) * sw(block, kb) from the scale ring
+      for (int g = 0; g < p.Kg; ++g) {
+        // sx(m, g) * sw(block of the chunk's columns, g) from the scale ring
         if (!mbar_wait_warp(sfull + sr.slot, sr.phase, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
           ok = false;
           break;
         }
         const float* slot = reinterpret_cast<const float*>(smem + C::kOffScale + sr.slot * C::kScaleSlot);
-        const float sc = slot[sub_row] * slot[128 + wg * (C::BN / 256)];
-        const float2 s2 = make_float2(sc, sc);
+        const float sx = slot[sub_row];
+        constexpr int kScales = C::SUBK ? C::kChunks : 1;  // one per 32-column chunk, or one for the thread
+        float2 s2[kScales];
+#pragma unroll
+        for (int c = 0; c < kScales; ++c) {
+          const float sc = sx * slot[128 + ((col0 + 32 * c) >> (p.kps_shift + 5))];  // wblk = 32 << kps_shift
+          s2[c] = make_float2(sc, sc);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(sempty + sr.slot);
         sr.template advance<C::kSRing>();
@@ -550,7 +609,8 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {  // acc += P * s, two lanes per packed FMA
               uint32_t* a = acc + (c + h) * 32 + j;
-              const float2 o = __ffma2_rn(make_float2(__uint_as_float(r[h][j]), __uint_as_float(r[h][j + 1])), s2,
+              const float2 o = __ffma2_rn(make_float2(__uint_as_float(r[h][j]), __uint_as_float(r[h][j + 1])),
+                                          s2[C::SUBK ? c + h : 0],
                                           make_float2(__uint_as_float(a[0]), __uint_as_float(a[1])));
               a[0] = __float_as_uint(o.x);
               a[1] = __float_as_uint(o.y);
@@ -806,6 +866,11 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.E = g.row_expert != nullptr ? g.E : 1;
   p.sfb_tiles = g.sfb_tiles;
   p.sf_shift = g.sf32 ? 0 : 2;
+  p.wblk = g.wblk == 0 ? 128 : g.wblk;
+  p.gsteps = 128 / p.wblk;
+  p.kps_shift = p.wblk == 128 ? 2 : (p.wblk == 64 ? 1 : 0);
+  p.Kg = (g.K + p.wblk - 1) / p.wblk;
+  p.Nbs = (g.N + p.wblk - 1) / p.wblk;
   if (p.num_tiles == 0) return cudaSuccess;
 
   // the shared-memory opt-in once per device: one bit per device; calls from
@@ -867,6 +932,13 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
     return launch_cfg<Cfg<256, 1, 4, 1, true>>(g, num_sms, s);
   }
   const int bn = choose_block_n(g.M, g.N, num_sms);
+  if (fmt == 0 && g.wblk != 0 && g.wblk != 128) {  // float at block 64 / 32
+    if (bn == 256) {
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, false, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<256, 0, 4, 1, false, true>>(g, num_sms, s);
+    }
+    return launch_cfg<Cfg<128, 0, 5, 2, false, true>>(g, num_sms, s);
+  }
   if (fmt == 0) {
     if (bn == 256) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);

@@ -70,8 +70,8 @@ __device__ __forceinline__ void fast_divmod(const FastDiv& f, uint32_t n, uint32
 // saturate); the scale is still written per group, so the GEMM reads it
 // exactly as it reads dynamic scales.
 //
-// GL lanes own one group of 16*GL channels (8 lanes for the default 128, 2
-// for 1 x 32 groups): lane l loads channels [16l, 16l+16) with two 16-byte
+// GL lanes own one group of 16*GL channels (8 lanes for the default 128, 4
+// for 1 x 64 groups, 2 for 1 x 32): lane l loads channels [16l, 16l+16) with two 16-byte
 // loads.  A warp covers 32/GL groups per pass and makes 2 passes per
 // iteration (all loads issued before any arithmetic), striding over the
 // grid.  amax: per-lane max, then log2(GL) xor-shuffles inside the group.
@@ -140,6 +140,12 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActQuantArgs a, co
           else static_cast<uint8_t*>(a.xs)[static_cast<int64_t>(m[u]) * a.Kb + kb[u]] = static_cast<uint8_t>(sbyte);
         } else if (LAYOUT == kScaleKMajor) {
           if (real[u]) static_cast<float*>(a.xs)[static_cast<int64_t>(kb[u]) * a.ld_s + m[u]] = s;
+        } else if (G == 64) {
+          // the tensor core takes one scale per 32 K: a 1 x 64 group's byte
+          // goes to both of its steps (the same word, bytes 2j and 2j+1)
+          const uint32_t b = real[u] ? sbyte : 127u;
+          *reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(a.xs) + sf_tile_offset(m[u], 2 * kb[u], a.Kq)) =
+              static_cast<uint16_t>(b | (b << 8));
         } else {
           static_cast<uint8_t*>(a.xs)[sf_tile_offset(m[u], kb[u], a.Kq)] =
               real[u] ? static_cast<uint8_t>(sbyte) : static_cast<uint8_t>(127);
@@ -200,48 +206,56 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const uint16_t* __res
   }
 }
 
-// One warp per 32 x 32 block (weight_block_size = (32, 32)): lane i holds row
-// i of the block (32 channels, four 16-byte loads; a 16-wide last block when
-// K % 32 == 16), amax by 5 xor-shuffles, two 16-byte stores per row.
-template <int FMT>
-__global__ void __launch_bounds__(256) weight_quant32_kernel(const uint16_t* __restrict__ w, const int64_t ld_w,
-                                                             const int N, const int K, const int Nb, const int Kb,
-                                                             uint8_t* __restrict__ wq, void* __restrict__ ws) {
+// One warp per B x B block, B = 32 or 64 (weight_block_size = (B, B)): lane i
+// holds rows i, i + 32, ... of the block (B channels each, B/8 16-byte loads;
+// the last block of a row may be 16-wide multiples when K % B != 0), amax by
+// 5 xor-shuffles, 16-byte stores of 16 codes.
+template <int FMT, int B>
+__global__ void __launch_bounds__(256) weight_quant_small_kernel(const uint16_t* __restrict__ w, const int64_t ld_w,
+                                                                 const int N, const int K, const int Nb, const int Kb,
+                                                                 uint8_t* __restrict__ wq, void* __restrict__ ws) {
+  constexpr int R = B / 32;  // rows per lane
+  constexpr int L = B / 8;   // 16-byte loads per row
   const int lane = threadIdx.x & 31;
   const int64_t blk = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (blk >= static_cast<int64_t>(Nb) * Kb) return;
   const int nb = static_cast<int>(blk / Kb), kb = static_cast<int>(blk % Kb);
-  const int n = nb * 32 + lane, k0 = kb * 32;
-  const bool row = n < N;
-  uint4 v[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int k = k0 + 8 * i;
-    v[i] = (row && k < K) ? __ldg(reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * ld_w + k))
-                          : make_uint4(0u, 0u, 0u, 0u);
-  }
-  float f[2][16];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float(&a0)[8] = *reinterpret_cast<float(*)[8]>(f[h]);
-    float(&a1)[8] = *reinterpret_cast<float(*)[8]>(f[h] + 8);
-    unpack_bf16x8(v[2 * h], a0);
-    unpack_bf16x8(v[2 * h + 1], a1);
-  }
+  const int k0 = kb * B;
+  uint4 v[R][L];
   float amax = 0.0f;
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+  for (int r = 0; r < R; ++r) {
+    const int n = nb * B + lane + 32 * r;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[h][i]));
+    for (int i = 0; i < L; ++i) {
+      const int k = k0 + 8 * i;
+      v[r][i] = (n < N && k < K) ? __ldg(reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * ld_w + k))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+      float f[8];
+      unpack_bf16x8(v[r][i], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    }
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
   const float s = group_scale(amax);
   const uint32_t sbyte = FMT == 1 ? e8m0_ceil_byte(s) : 0u;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int k = k0 + 16 * h;
-    if (row && k < K)
-      *reinterpret_cast<uint4*>(wq + static_cast<int64_t>(n) * K + k) = quantize16<FMT>(f[h], s, sbyte);
+  for (int r = 0; r < R; ++r) {
+    const int n = nb * B + lane + 32 * r;
+#pragma unroll
+    for (int h = 0; h < L / 2; ++h) {
+      const int k = k0 + 16 * h;
+      if (n < N && k < K) {
+        float f[16];
+        float(&a0)[8] = *reinterpret_cast<float(*)[8]>(f);
+        float(&a1)[8] = *reinterpret_cast<float(*)[8]>(f + 8);
+        unpack_bf16x8(v[r][2 * h], a0);
+        unpack_bf16x8(v[r][2 * h + 1], a1);
+        *reinterpret_cast<uint4*>(wq + static_cast<int64_t>(n) * K + k) = quantize16<FMT>(f, s, sbyte);
+      }
+    }
   }
   if (lane == 0) {
     if (FMT == 0) static_cast<float*>(ws)[blk] = s;
@@ -254,8 +268,10 @@ __global__ void __launch_bounds__(256) weight_quant32_kernel(const uint16_t* __r
 // (rows 128 t.., K-blocks 4 q..) holds the words of rows 128 t + 32 c + i,
 // c = 0..3, byte j of each being K-block 4 q + j (sf_tile_offset's layout).
 // Rows past R and K-blocks past Kb get 127 (2^0, never applied to data).
+// Slot kb takes source column kb / kdiv (kdiv 2: a 64-wide block's scale for
+// both of its 32-wide MMA steps).
 __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict__ src, const int R, const int row_div,
-                                                      const int Kb, const int Kq, const int64_t chunks,
+                                                      const int Kb, const int kdiv, const int Kq, const int64_t chunks,
                                                       uint8_t* __restrict__ dst) {
   grid_wait_prerequisites();
   grid_launch_dependents();
@@ -272,7 +288,7 @@ __global__ void __launch_bounds__(256) sf_pack_kernel(const uint8_t* __restrict_
       uint32_t v = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int kb = 4 * q + j;
+        const int kb = (4 * q + j) / kdiv;
         const uint32_t b = (r < R && kb < Kb) ? src[(r / row_div) * Kb + kb] : 127u;
         v |= b << (8 * j);
       }
@@ -303,10 +319,15 @@ cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, fl
 }
 
 cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaStream_t s) {
+  const int G = a.group == 0 ? 128 : a.group;
+  if (G != 32 && G != 64 && G != 128) return cudaErrorInvalidValue;
   int rows, cols;
   if (a.layout == kScaleSfTiles) {
     rows = a.M_pad;
-    cols = a.Kq * 4;
+    // group slots of the scale-factor tiles: a chunk holds 4 K-blocks of 128
+    // (groups of 128; Kq chunks per row tile), or one K-block of 128 (smaller
+    // groups; Kq = K-blocks per row, 128 / G groups each)
+    cols = G == 128 ? a.Kq * 4 : a.Kq * (128 / G);
   } else {
     rows = a.M;
     cols = a.Kb;
@@ -315,7 +336,7 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
   if (total == 0) return cudaSuccess;
   if (total > 0x7FFFFFF0LL) return cudaErrorInvalidValue;  // group index is 32-bit
   const FastDiv div = make_fastdiv(static_cast<uint32_t>(a.layout == kScaleRowMajor ? cols : rows));
-  const int gl = a.group == 32 ? 2 : 8;  // lanes per group
+  const int gl = G / 16;  // lanes per group
   const int64_t per_block = 8 * (32 / gl) * 2;  // 8 warps x groups per warp x 2 passes
   int64_t blocks = (total + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
@@ -340,26 +361,46 @@ cudaError_t launch_act_quant(const ActQuantArgs& a, int fmt, int num_sms, cudaSt
       if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 8);
       else FG8_AQ(1, kScaleSfTiles, 8);
     }
-  } else {  // 1 x 32 groups: row-major scales, or UE8M0 scale-factor tiles for the GEMM
-    if (a.layout == kScaleKMajor) return cudaErrorInvalidValue;
-    if (fmt == 0) FG8_AQ(0, kScaleRowMajor, 2);
-    else if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 2);
-    else FG8_AQ(1, kScaleSfTiles, 2);
+  } else if (gl == 4) {  // 1 x 64 groups
+    if (fmt == 0) {
+      if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor, 4);
+      else if (a.layout == kScaleKMajor) FG8_AQ(0, kScaleKMajor, 4);
+      else return cudaErrorInvalidValue;
+    } else {
+      if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 4);
+      else if (a.layout == kScaleSfTiles) FG8_AQ(1, kScaleSfTiles, 4);
+      else return cudaErrorInvalidValue;
+    }
+  } else {  // 1 x 32 groups
+    if (fmt == 0) {
+      if (a.layout == kScaleRowMajor) FG8_AQ(0, kScaleRowMajor, 2);
+      else if (a.layout == kScaleKMajor) FG8_AQ(0, kScaleKMajor, 2);
+      else return cudaErrorInvalidValue;
+    } else {
+      if (a.layout == kScaleRowMajor) FG8_AQ(1, kScaleRowMajor, 2);
+      else if (a.layout == kScaleSfTiles) FG8_AQ(1, kScaleSfTiles, 2);
+      else return cudaErrorInvalidValue;
+    }
   }
 #undef FG8_AQ
   return cudaGetLastError();
 }
 
-cudaError_t launch_weight_quant32(const void* w, int64_t ld_w, int N, int K, uint8_t* wq, void* ws, int fmt,
-                                  cudaStream_t s) {
-  const int Kb = (K + 31) / 32, Nb = (N + 31) / 32;
+cudaError_t launch_weight_quant_small(const void* w, int64_t ld_w, int N, int K, int block, uint8_t* wq, void* ws,
+                                      int fmt, cudaStream_t s) {
+  if (block != 32 && block != 64) return cudaErrorInvalidValue;
+  const int Kb = (K + block - 1) / block, Nb = (N + block - 1) / block;
   const int64_t blocks = (static_cast<int64_t>(Nb) * Kb + 7) / 8;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
-  if (fmt == 0)
-    weight_quant32_kernel<0><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(w), ld_w, N, K, Nb, Kb, wq, ws);
-  else
-    weight_quant32_kernel<1><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(w), ld_w, N, K, Nb, Kb, wq, ws);
+  const dim3 grid(static_cast<unsigned>(blocks)), thr(256);
+  const uint16_t* wp = static_cast<const uint16_t*>(w);
+  if (block == 32) {
+    if (fmt == 0) weight_quant_small_kernel<0, 32><<<grid, thr, 0, s>>>(wp, ld_w, N, K, Nb, Kb, wq, ws);
+    else weight_quant_small_kernel<1, 32><<<grid, thr, 0, s>>>(wp, ld_w, N, K, Nb, Kb, wq, ws);
+  } else {
+    if (fmt == 0) weight_quant_small_kernel<0, 64><<<grid, thr, 0, s>>>(wp, ld_w, N, K, Nb, Kb, wq, ws);
+    else weight_quant_small_kernel<1, 64><<<grid, thr, 0, s>>>(wp, ld_w, N, K, Nb, Kb, wq, ws);
+  }
   return cudaGetLastError();
 }
 
@@ -372,9 +413,9 @@ cudaError_t launch_weight_quant(const void* w, int64_t ld_w, int N, int K, uint8
   return cudaGetLastError();
 }
 
-cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, uint8_t* dst,
+cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div, int Kb, int kdiv, uint8_t* dst,
                            cudaStream_t s) {
-  const int Kq = (Kb + 3) / 4;
+  const int Kq = (Kb * kdiv + 3) / 4;
   if (R_pad % 128 != 0 || R_pad < R) return cudaErrorInvalidValue;
   const int64_t chunks = R_pad / 128 * Kq * 32;  // 16-byte chunks, 32 per 512-byte tile
   int64_t blocks = (chunks + 255) / 256;
@@ -388,7 +429,7 @@ cudaError_t launch_sf_pack(const uint8_t* src, int R, int64_t R_pad, int row_div
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_pack_kernel, src, R, row_div, Kb, Kq, chunks, dst);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_pack_kernel, src, R, row_div, Kb, kdiv, Kq, chunks, dst);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

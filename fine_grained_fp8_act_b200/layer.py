@@ -98,7 +98,7 @@ def _output(out, M: int, N: int, device) -> torch.Tensor:
 
 def quantize_weight(w: torch.Tensor, scale_fmt="float", block: int = 128) -> Tuple[torch.Tensor, torch.Tensor]:
     """W bf16 [N, K] -> (wq float8_e4m3fn [N, K], weight_scale_inv [ceil(N/block), ceil(K/block)]);
-    block x block weight blocks, block 128 (default) or 32."""
+    block x block weight blocks, block 128 (default), 64 or 32."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(w, "w")
     _check_cuda(w, "w")
@@ -155,8 +155,9 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
 def linear(x: torch.Tensor, wq: torch.Tensor, w_scale_inv: torch.Tensor, bias: Optional[torch.Tensor] = None,
            scale_fmt="float", out: Optional[torch.Tensor] = None,
            workspace: Optional[torch.Tensor] = None, block: int = 128) -> torch.Tensor:
-    """y [M, N] bf16 = dequant(quantize_act(x)) . dequant(wq)^T + bias.  block 32
-    (1 x 32 groups, 32 x 32 weight blocks) takes UE8M0 scales."""
+    """y [M, N] bf16 = dequant(quantize_act(x)) . dequant(wq)^T + bias.  block 64
+    or 32: 1 x block activation groups and block x block weight blocks, either
+    scale format."""
     fmt = scale_fmt_code(scale_fmt)
     _check_bf16_matrix(x, "x")
     M, K = x.shape
@@ -330,7 +331,7 @@ def scale_to_ue8m0(scale: torch.Tensor) -> Tuple[torch.Tensor, int]:
 class FP8Linear(torch.nn.Module):
     """Inference linear layer holding a quantized weight ([zh] §一 FP8Linear):
     weight float8_e4m3fn [out, in], weight_scale_inv per block x block block
-    (weight_block_size (128, 128) by default, or (32, 32) with UE8M0 scales),
+    (weight_block_size (128, 128) by default, or (64, 64) or (32, 32)),
     bias kept in bf16 (not quantized, [zh] §三).  The layer keeps one device
     workspace, so forwards of the same layer on different CUDA streams must
     not overlap in time (use one layer object per concurrent stream)."""

@@ -217,18 +217,20 @@ FG8_API fg8_status fg8_linear_static(const void* x_bf16, int64_t M, int64_t N, i
                                      const void* bias_bf16, void* y_bf16, int64_t ld_y, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
-/* Non-default block size ([zh] §八: the tests cover weight_block_size such
+/* Non-default block sizes ([zh] §八: the tests cover weight_block_size such
  * as (32, 32)).  Reading: the activation groups follow the weight's
- * input-channel block, so block = 32 means 1 x 32 activation groups and
- * 32 x 32 weight blocks; scales are shaped [M, ceil(K/32)] and
- * [ceil(N/32), ceil(K/32)].  block is 32 or 128 (128 forwards to the calls
- * above).  The quantizers take either scale format; fg8_linear_block with
- * block 32 takes UE8M0 only (FG8_ERR_INVALID_ARG for float): the tensor
- * core's block-scaled MMA applies one scale per 32 K per row natively,
- * float scales would need a register promotion per 32-K slice.  It always
- * runs the tiled GEMM (no few-token kernel).  Other checks and errors as
- * the 128 versions; the workspace is fg8_linear_block_workspace_bytes (0 for
- * an unsupported combination), with the header rules of fg8_linear. */
+ * input-channel block, so block = b means 1 x b activation groups and b x b
+ * weight blocks; scales are shaped [M, ceil(K/b)] and [ceil(N/b), ceil(K/b)].
+ * block is 32, 64 or 128 (128 forwards to the calls above); every call takes
+ * either scale format.  In fg8_linear_block, UE8M0 scales go through the
+ * tensor core's block-scaled MMA (one scale per 32 K per row; a 64-block's
+ * scale on both of its steps), and float32 scales are promoted in float32
+ * registers per b-wide slice of K, exactly as the 128 layer promotes per
+ * K-block: y = bias + sum over slices of P_slice * (sx * sw).  It always runs
+ * the tiled GEMM (no few-token kernel).  Other checks and errors as the 128
+ * versions (block sizes other than 32, 64 and 128 are FG8_ERR_INVALID_ARG);
+ * the workspace is fg8_linear_block_workspace_bytes (0 for an unsupported
+ * combination), with the header rules of fg8_linear. */
 FG8_API fg8_status fg8_quantize_act_block(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* xq_e4m3,
                                           void* x_scale, fg8_scale_fmt fmt, int block, void* stream);
 FG8_API fg8_status fg8_quantize_weight_block(const void* w_bf16, int64_t N, int64_t K, int64_t ld_w, void* wq_e4m3,

@@ -224,19 +224,29 @@ def test_grouped_rejects_bad_args(fg8):
 
 def test_block_size_rejects_bad_args(fg8):
     raw = _raw(fg8)
-    assert raw.fg8_quantize_act_block(FAKE, 4, 256, 256, FAKE, FAKE, 0, 64, None) == 1       # block 64
+    assert raw.fg8_quantize_act_block(FAKE, 4, 256, 256, FAKE, FAKE, 0, 16, None) == 1       # block 16
+    assert raw.fg8_quantize_act_block(FAKE, 4, 256, 256, FAKE, FAKE, 0, 96, None) == 1       # block 96
     assert raw.fg8_quantize_act_block(FAKE, 4, 120, 128, FAKE, FAKE, 1, 32, None) == 2      # K % 16
+    assert raw.fg8_quantize_act_block(FAKE, 4, 120, 128, FAKE, FAKE, 0, 64, None) == 2
     assert raw.fg8_quantize_act_block(None, 0, 256, 256, None, None, 1, 32, None) == 0      # empty
     assert raw.fg8_quantize_weight_block(FAKE, 0, 256, 256, FAKE, FAKE, 1, 32, None) == 1
     assert raw.fg8_quantize_weight_block(FAKE, 256, 248, 248, FAKE, FAKE, 1, 32, None) == 2
-    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 0, 32) == 0                   # float at 32
-    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 64) == 0
-    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 128) == raw.fg8_linear_workspace_bytes(256, 256, 256, 1)
-    # x codes + 2 x-scale chunks (K = 256: 2 K-blocks) + 2 row tiles x 2 W chunks, beyond the header
-    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, 32) >= 256 * 256 + 2 * 2 * 512 + 2 * 2 * 512
+    assert raw.fg8_quantize_weight_block(FAKE, 256, 256, 256, FAKE, FAKE, 0, 48, None) == 1
+    for fmt in (0, 1):
+        assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, fmt, 16) == 0
+        assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, fmt, 128) == \
+            raw.fg8_linear_workspace_bytes(256, 256, 256, fmt)
+    # UE8M0: x codes + 2 x-scale chunks (K = 256: 2 K-blocks) + 2 row tiles x 2 W chunks, beyond the header
+    for blk in (32, 64):
+        assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 1, blk) >= 256 * 256 + 2 * 2 * 512 + 2 * 2 * 512
+    # float: x codes + K-major float32 x scales [K / blk][256]
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 0, 32) >= 256 * 256 + 8 * 256 * 4
+    assert raw.fg8_linear_block_workspace_bytes(256, 256, 256, 0, 64) >= 256 * 256 + 4 * 256 * 4
     lb = raw.fg8_linear_block
-    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, 32, FAKE * 16, 1 << 40, None) == 1
+    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, 16, FAKE * 16, 1 << 40, None) == 1
+    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 2, 32, FAKE * 16, 1 << 40, None) == 1
     assert lb(FAKE, 16, 256, 200, 200, FAKE, FAKE, None, FAKE, 256, 1, 32, FAKE * 16, 1 << 40, None) == 2
+    assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 0, 64, None, 1 << 40, None) == 4
     assert lb(FAKE, 16, 256, 256, 256, FAKE, FAKE, None, FAKE, 256, 1, 32, None, 1 << 40, None) == 4
 
 

@@ -128,19 +128,21 @@ def test_grouped_linear_host_checks(lib):
         _check(got, broken, M, f"fg8_grouped_linear case {i}: M={M} E={E} N={N} K={K} fmt={fmt}")
 
 
-def test_block32_linear_host_checks(lib):
+def test_small_block_linear_host_checks(lib):
+    """fg8_linear_block at blocks 32 and 64 (both scale formats; other block
+    sizes and formats refused)."""
     rng = np.random.default_rng(3)
-    for i in range(1200):
+    for i in range(1600):
         M = _dim(rng, [0, 1, 200, 2048])
         N = _dim(rng, [8, 264, 4096])
         K = _dim(rng, [16, 32, 400])
         fmt = int(rng.choice([0, 1, 1, 3]))
-        block = int(rng.choice([32, 32, 32, 64, 16]))
+        block = int(rng.choice([32, 32, 64, 64, 16]))
         ld_x = K + int(rng.choice([0, 0, 8, -8, 4]))
         ld_y = N + int(rng.choice([0, 0, 8, -8, 4]))
         x, wq, ws, y = (_ptr(rng, 16) for _ in range(4))
         bias = None if rng.random() < 0.3 else _ptr(rng, 16)
-        shape_ok = block == 32 and fmt == 1 and 0 <= M <= MAXD and 0 < N <= MAXD and 0 < K <= MAXD
+        shape_ok = block in (32, 64) and fmt in (0, 1) and 0 <= M <= MAXD and 0 < N <= MAXD and 0 < K <= MAXD
         need = (lib.fg8_linear_block_workspace_bytes(M, N, K, fmt, block)
                 if shape_ok and K % 16 == 0 and N % 8 == 0 else 0)
         wsp = _ptr(rng, 256)
@@ -153,7 +155,7 @@ def test_block32_linear_host_checks(lib):
         if shape_ok and M > 0:
             if None in (x, wq, ws, y):
                 broken.add(INVALID)
-            if ld_x % 8 or ld_y % 8 or not all(_aligned(p, 16) for p in (x, wq, y) if p is not None) or \
+            if ld_x % 8 or ld_y % 8 or not all(_aligned(p, 16) for p in (x, wq, ws, y) if p is not None) or \
                     (bias is not None and not _aligned(bias, 16)):
                 broken.add(ALIGN)
             if not _aligned(wsp, 256) or nbytes < need:
@@ -177,7 +179,7 @@ def test_quantize_act_host_checks(lib, block):
         ld_x = K + int(rng.choice([0, 0, 8, -8, 4]))
         x, xq, xs = (_ptr(rng, 16) for _ in range(3))
         invalid = fmt not in (0, 1) or not (0 <= M <= MAXD and 0 < K <= MAXD) or ld_x < K or \
-            block not in (None, 128, 32)
+            block not in (None, 128, 64, 32)
         if invalid:
             allowed = {INVALID}
         elif M == 0:
@@ -196,7 +198,7 @@ def test_quantize_act_host_checks(lib, block):
         _check_allowed(got, allowed, f"quantize_act block={block} case {i}: M={M} K={K} fmt={fmt} ld={ld_x}")
 
 
-@pytest.mark.parametrize("block", [None, 128, 32, 16])
+@pytest.mark.parametrize("block", [None, 128, 64, 32, 16])
 def test_quantize_weight_host_checks(lib, block):
     """fg8_quantize_weight (block None) and fg8_quantize_weight_block."""
     rng = np.random.default_rng(40 + (block or 0))
@@ -207,11 +209,11 @@ def test_quantize_weight_host_checks(lib, block):
         ld_w = K + int(rng.choice([0, 0, 8, -8, 4]))
         w, wq, ws = (_ptr(rng, 16) for _ in range(3))
         b = 128 if block is None else block
-        invalid = fmt not in (0, 1) or not (0 < N <= MAXD and 0 < K <= MAXD) or ld_w < K or b not in (128, 32) or \
-            None in (w, wq, ws)
+        invalid = fmt not in (0, 1) or not (0 < N <= MAXD and 0 < K <= MAXD) or ld_w < K or \
+            b not in (128, 64, 32) or None in (w, wq, ws)
         if not invalid and b == 128 and -(-N // 128) > 65535:
             invalid = True
-        if not invalid and b == 32 and -(-N // 32) * -(-K // 32) > MAXD // 8:
+        if not invalid and b in (32, 64) and -(-N // b) * -(-K // b) > MAXD // 8:
             invalid = True
         align = not invalid and (K % 16 or ld_w % 8 or not (_aligned(w, 16) and _aligned(wq, 16)))
         allowed = ({INVALID} | ({ALIGN} if (K % 16 or ld_w % 8) else set())) if invalid else \

@@ -123,20 +123,22 @@ def test_dequantize_stays_in_bounds(fg8, fmt):
     assert cw.intact()
 
 
-def test_block32_layer_stays_in_bounds(fg8):
+@pytest.mark.parametrize("blk,sfmt", [(32, "ue8m0"), (64, "ue8m0"), (32, "float"), (64, "float")])
+def test_small_block_layer_stays_in_bounds(fg8, blk, sfmt):
+    fmt = UE8M0 if sfmt == "ue8m0" else 0
     M, N, K = 200, 264, 400
     ld_y = N + 8
     x = W.x_student_t(M, K, seed=8).cuda()
     b = W.normal((N,), 0.1, seed=9).cuda()
-    wq, ws = fg8.quantize_weight(W.w_row_groups(N, K, 0.02, seed=10).cuda(), "ue8m0", block=32)
+    wq, ws = fg8.quantize_weight(W.w_row_groups(N, K, 0.02, seed=10).cuda(), sfmt, block=blk)
     cy = Canary(M * ld_y * 2, "cuda")
     y = cy.matrix(BF16, M, N, ld_y)
-    need = fg8.fg8_linear_block_workspace_bytes(M, N, K, UE8M0, 32)
+    need = fg8.fg8_linear_block_workspace_bytes(M, N, K, fmt, blk)
     cw = Canary(need, "cuda")
     cw.zeroed()
     fg8.fg8_linear_block(x.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), b.data_ptr(), cy.ptr(), ld_y,
-                         UE8M0, 32, cw.ptr(), need, _s())
+                         fmt, blk, cw.ptr(), need, _s())
     assert fg8.fg8_check_device_status(cw.ptr(), _s()) == 0
     torch.cuda.synchronize()
-    assert torch.equal(y, fg8.linear(x, wq, ws, b, "ue8m0", block=32))
+    assert torch.equal(y, fg8.linear(x, wq, ws, b, sfmt, block=blk))
     assert cy.intact() and cw.intact()

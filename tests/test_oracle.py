@@ -735,90 +735,97 @@ def test_grouped_linear_block_expert_is_its_first_row(orc, fmt):
         d64, _, dbf = orc.linear(x, wq[e], ws[e], b[e], fmt, rows=rows)
         assert np.array_equal(y64[rows], d64) and np.array_equal(ybf[rows], dbf)
 
-# --------------------------------------------- non-default block size 32 --
+# ------------------------------------- non-default block sizes 32 and 64 --
+@pytest.mark.parametrize("blk", [32, 64])
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("M,K", [(3, 256), (2, 80), (1, 48)])
-def test_quantize_act_groups_block32(orc, fmt, M, K):
-    """1 x 32 groups (weight_block_size = (32, 32)): each group's scale from its
-    own 32 channels (a 16-wide last group from its 16), codes by brute force."""
-    g = torch.Generator().manual_seed(7 * M + K)
+@pytest.mark.parametrize("M,K", [(3, 256), (2, 80), (1, 48), (2, 208)])
+def test_quantize_act_groups_small_blocks(orc, fmt, M, K, blk):
+    """1 x blk groups (weight_block_size = (blk, blk)): each group's scale from
+    its own blk channels (a shorter last group from its real ones), codes by
+    brute force."""
+    g = torch.Generator().manual_seed(7 * M + K + blk)
     x = torch.randn(M, K, generator=g)
-    for j in range(-(-K // 32)):  # very different magnitudes per group: a wrong group index shows
-        x[:, 32 * j:32 * j + 32] *= 2.0 ** (3 * (j % 5) - 6)
+    for j in range(-(-K // blk)):  # very different magnitudes per group: a wrong group index shows
+        x[:, blk * j:blk * j + blk] *= 2.0 ** (3 * (j % 5) - 6)
     x = x.to(torch.bfloat16)
-    xq, xs = orc.quantize_act(_bf16_bits(x), fmt, 32)
-    assert xs.shape == (M, -(-K // 32))
+    xq, xs = orc.quantize_act(_bf16_bits(x), fmt, blk)
+    assert xs.shape == (M, -(-K // blk))
     xf = x.float().numpy()
     for m in range(M):
-        for j in range(-(-K // 32)):
-            k0, k1 = 32 * j, min(32 * j + 32, K)
+        for j in range(-(-K // blk)):
+            k0, k1 = blk * j, min(blk * j + blk, K)
             _check_group(orc, xf[m, k0:k1], xq[m, k0:k1], xs[m, j], fmt)
 
 
+@pytest.mark.parametrize("blk", [32, 64])
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("N,K", [(64, 64), (40, 80), (96, 48)])
-def test_quantize_weight_blocks_block32(orc, fmt, N, K):
-    g = torch.Generator().manual_seed(N + 3 * K)
+@pytest.mark.parametrize("N,K", [(64, 64), (40, 80), (96, 48), (136, 208)])
+def test_quantize_weight_blocks_small_blocks(orc, fmt, N, K, blk):
+    g = torch.Generator().manual_seed(N + 3 * K + blk)
     w = torch.randn(N, K, generator=g) * 0.02
-    Nb, Kb = -(-N // 32), -(-K // 32)
+    Nb, Kb = -(-N // blk), -(-K // blk)
     for nb in range(Nb):
         for kb in range(Kb):
-            w[32 * nb:32 * nb + 32, 32 * kb:32 * kb + 32] *= 2.0 ** (3 * nb - 2 * kb)
+            w[blk * nb:blk * nb + blk, blk * kb:blk * kb + blk] *= 2.0 ** (3 * nb - 2 * kb)
     w = w.to(torch.bfloat16)
-    wq, ws = orc.quantize_weight(_bf16_bits(w), fmt, 32)
+    wq, ws = orc.quantize_weight(_bf16_bits(w), fmt, blk)
     assert ws.shape == (Nb, Kb)
     wf = w.float().numpy()
     for nb in range(Nb):
         for kb in range(Kb):
-            blk = wf[32 * nb:min(32 * nb + 32, N), 32 * kb:min(32 * kb + 32, K)]
-            q = wq[32 * nb:min(32 * nb + 32, N), 32 * kb:min(32 * kb + 32, K)]
-            _check_group(orc, blk.ravel(), q.ravel(), ws[nb, kb], fmt)
+            blkv = wf[blk * nb:min(blk * nb + blk, N), blk * kb:min(blk * kb + blk, K)]
+            q = wq[blk * nb:min(blk * nb + blk, N), blk * kb:min(blk * kb + blk, K)]
+            _check_group(orc, blkv.ravel(), q.ravel(), ws[nb, kb], fmt)
 
 
+@pytest.mark.parametrize("blk", [32, 64])
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("M,N,K", [(2, 3, 80), (1, 40, 64), (3, 5, 48)])
-def test_linear_vs_exact_rationals_block32(orc, fmt, M, N, K):
-    g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
+@pytest.mark.parametrize("M,N,K", [(2, 3, 80), (1, 40, 64), (3, 5, 48), (2, 70, 144)])
+def test_linear_vs_exact_rationals_small_blocks(orc, fmt, M, N, K, blk):
+    g = torch.Generator().manual_seed(M * 31 + N * 7 + K + blk)
     x = torch.randn(M, K, generator=g)
     w = torch.randn(N, K, generator=g) * 0.02
-    for j in range(-(-K // 32)):  # scales that differ by group, so a k / 128 index would show
-        x[:, 32 * j:32 * j + 32] *= 2.0 ** (2 * j - 3)
-        w[:, 32 * j:32 * j + 32] *= 2.0 ** (1 - j)
+    for j in range(-(-K // blk)):  # scales that differ by group, so a k / 128 index would show
+        x[:, blk * j:blk * j + blk] *= 2.0 ** (2 * j - 3)
+        w[:, blk * j:blk * j + blk] *= 2.0 ** (1 - j)
+    for i in range(-(-N // blk)):  # and by row block, so a n / 128 index would show
+        w[blk * i:blk * i + blk, :] *= 2.0 ** (3 - 2 * i)
     xb, wb = _bf16_bits(x.to(torch.bfloat16)), _bf16_bits(w.to(torch.bfloat16))
     bb = _bf16_bits((torch.randn(N, generator=g) * 0.1).to(torch.bfloat16))
-    xq, xs = orc.quantize_act(xb, fmt, 32)
-    wq, ws = orc.quantize_weight(wb, fmt, 32)
-    y64, bound, ybf = orc.linear_dequant(xq, xs, wq, ws, bb, fmt, block=32)
-    ye, be = exact_linear(xq, xs, wq, ws, bb, fmt, block=32)
+    xq, xs = orc.quantize_act(xb, fmt, blk)
+    wq, ws = orc.quantize_weight(wb, fmt, blk)
+    y64, bound, ybf = orc.linear_dequant(xq, xs, wq, ws, bb, fmt, block=blk)
+    ye, be = exact_linear(xq, xs, wq, ws, bb, fmt, block=blk)
     gamma = K * 2.0 ** -52
     for m in range(M):
         for n in range(N):
             assert abs(Fraction(y64[m, n]) - ye[m][n]) <= Fraction(gamma) * be[m][n] + Fraction(1, 2 ** 1074)
             assert ybf[m, n] == frac_bf16_rne(Fraction(y64[m, n]))
-    y2 = orc.linear(xb, wq, ws, bb, fmt, block=32)[0]
+    y2 = orc.linear(xb, wq, ws, bb, fmt, block=blk)[0]
     assert np.array_equal(y2, y64)
 
 
+@pytest.mark.parametrize("blk", [32, 64])
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-def test_block32_equals_block128_when_scales_coincide(orc, fmt):
-    """When every 32-group of a 128-group (and every 32 x 32 block of a
+def test_small_blocks_equal_block128_when_scales_coincide(orc, fmt, blk):
+    """When every blk-group of a 128-group (and every blk x blk block of a
     128 x 128 block) has the same amax, the scales coincide and so do the
-    codes and y: block 32 reduces to the default layer."""
-    rng = np.random.default_rng(9)
+    codes and y: the smaller block reduces to the default layer."""
+    rng = np.random.default_rng(9 + blk)
     M, N, K = 3, 136, 256
     x = rng.normal(0, 1, (M, K)).astype(np.float32)
     w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
     x = np.clip(x, -3.0, 3.0)
-    x[:, ::32] = 3.0                 # each 32-group holds the row's amax
+    x[:, ::blk] = 3.0                 # each blk-group holds the row's amax
     w = np.clip(w, -0.05, 0.05)
-    for n0 in range(0, N, 32):       # each 32 x 32 block holds its 128 x 128 block's amax
-        w[n0, ::32] = 0.0625
+    for n0 in range(0, N, blk):       # each blk x blk block holds its 128 x 128 block's amax
+        w[n0, ::blk] = 0.0625
     xb = (x.view(np.uint32) >> 16).astype(np.uint16)
     wb = (w.view(np.uint32) >> 16).astype(np.uint16)
     b = (rng.normal(0, 0.1, N).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
-    q32, s32 = orc.quantize_weight(wb, fmt, 32)
+    qs, ss = orc.quantize_weight(wb, fmt, blk)
     q128, s128 = orc.quantize_weight(wb, fmt)
-    assert np.array_equal(q32, q128)
-    y32 = orc.linear(xb, q32, s32, b, fmt, block=32)[0]
+    assert np.array_equal(qs, q128)
+    ys = orc.linear(xb, qs, ss, b, fmt, block=blk)[0]
     y128 = orc.linear(xb, q128, s128, b, fmt)[0]
-    assert np.array_equal(y32, y128)
+    assert np.array_equal(ys, y128)
