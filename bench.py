@@ -347,6 +347,15 @@ def run_fg8(args, rank, world, local):
     # block 32 / 64 (1 x b groups, b x b weight blocks): fg8_linear_block per layer
     paths = [("small_block" if args.block != 128 else layer_path(L["g"])) for L in plan]
     chain = not args.no_chain and all(pth == "tiled" for pth in paths)
+    # --fused-quant: a tiled layer with K <= 4096 whose input is not already
+    # quantized by the previous GEMM takes fg8_linear_fused, its act-quant
+    # inside the GEMM's launch (in-kernel units published with flags).
+    for i, L in enumerate(plan):
+        if paths[i] == "tiled" and args.fused_quant and -(-L["g"].K // 128) <= 32 and (i == 0 or not chain):
+            paths[i] = "tiled_fused_quant"
+            g = L["g"]
+            L["wsp"] = torch.zeros(fg8.fg8_linear_fused_workspace_bytes(g.M, g.N, g.K, g.fmt), dtype=torch.uint8,
+                                   device=dev)
 
     def launch_layer(i, ev_mid=None):
         L = plan[i]
@@ -358,6 +367,17 @@ def run_fg8(args, rank, world, local):
                                  L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt,
                                  args.block,
                                  L["wsp"].data_ptr(), L["wsp"].numel(), sp)
+            return
+        if paths[i] == "tiled_fused_quant":  # act-quant inside the GEMM's launch (+ the next layer's requant)
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            nxt = plan[i + 1] if chain and i + 1 < len(plan) else None
+            fg8.fg8_linear_fused(L["x"].data_ptr(), g.M, g.N, g.K, L["x"].stride(0), L["wq"].data_ptr(),
+                                 L["ws"].data_ptr(), L["b"].data_ptr(), L["y"].data_ptr(), L["y"].stride(0), g.fmt,
+                                 L["wsp"].data_ptr(), L["wsp"].numel(), 0 if nxt is None else nxt["g"].N,
+                                 None if nxt is None else nxt["ws"].data_ptr(),
+                                 None if nxt is None else nxt["wsp"].data_ptr(),
+                                 0 if nxt is None else nxt["wsp"].numel(), sp)
             return
         if paths[i] == "fused":
             if ev_mid is not None:
@@ -472,7 +492,9 @@ def run_fg8(args, rank, world, local):
     roof["traffic"] = recorded_traffic(args.workload, dom)  # ncu DRAM bytes per launch, None if stale
     roof["kernel"] = (f"fg8_gemm_kernel, {args.block} x {args.block} blocks, timed with its act-quant "
                       f"and scale packing" if paths[dom] == "small_block" else
-                      "fg8_small_m_kernel" if paths[dom] != "tiled" else "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+                      "fg8_small_m_kernel" if paths[dom] not in ("tiled", "tiled_fused_quant") else
+                      "fg8_gemm_kernel") + f" ({g.name}: M={g.M} K={g.K} N={g.N})" + (
+        ", act-quant of x inside the launch" if paths[dom] == "tiled_fused_quant" else "") + (
         ", epilogue also quantizes y for the next layer" if chain and dom + 1 < nl else "")
     roof["kernel_us"] = gm[dom] * 1e3
     roof["peak_source"] = (f"{peaks['source']}: bf16 {peaks['bf16_tflops']} TF/s x {FP8_PER_BF16} (fp8:bf16 nominal), "
@@ -482,10 +504,12 @@ def run_fg8(args, rank, world, local):
     per_kernel = []
     for i, L in enumerate(plan):
         gi = L["g"]
-        fused = paths[i] in ("fused", "small_block") or (chain and i > 0)  # act-quant not timed on its own
+        fused = paths[i] in ("fused", "small_block", "tiled_fused_quant") or (chain and i > 0)  # not timed alone
         per_kernel.append({"layer": gi.name, "path": paths[i], "act_quant_us": None if fused else qm[i] * 1e3,
                            "act_quant_gbs": None if fused else quant_bytes(gi) / (qm[i] * 1e-3) / 1e9,
                            "act_quant": ("fused into the few-token kernel" if paths[i] == "fused" else
+                                         "inside the GEMM's launch (fg8_linear_fused)"
+                                         if paths[i] == "tiled_fused_quant" else
                                          "timed with the GEMM (fg8_linear_block: act-quant, scale packing, GEMM)"
                                          if paths[i] == "small_block" else
                                          "fused into the previous GEMM" if fused else "own launch"),
@@ -495,14 +519,15 @@ def run_fg8(args, rank, world, local):
                            "weight_quant_us": L["wq_ms"] * 1e3,
                            "weight_quant_gbs": weight_quant_bytes(gi, args.block) / (L["wq_ms"] * 1e-3) / 1e9})
 
-    e2e = run_e2e(fg8, plan, args, stream, dev, world, chain)
+    e2e = run_e2e(fg8, plan, args, stream, dev, world, chain, paths)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds, block=args.block)
 
     # prepare: act-quant (+ the weight-scale packing launch for UE8M0), then the GEMM;
-    # fused few-token layers: one kernel
-    prep = [0 if pth == "fused" else 1 + (1 if L["g"].fmt == 1 else 0) for pth, L in zip(paths, plan)]
+    # fused few-token layers and act-quant inside the GEMM: one kernel
+    prep = [0 if pth in ("fused", "tiled_fused_quant") else 1 + (1 if L["g"].fmt == 1 else 0)
+            for pth, L in zip(paths, plan)]
     launches_per_step = (prep[0] if chain else sum(prep)) + nl
     out = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -528,7 +553,7 @@ def run_fg8(args, rank, world, local):
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(fg8, plan, args, stream, dev, world, chain):
+def run_e2e(fg8, plan, args, stream, dev, world, chain, paths):
     """Same metric through the public calls with host buffers, as a serving
     loop runs it: every step copies its input from pinned host memory to the
     device, runs the layers (chained as in the device-timed step, else
@@ -550,15 +575,27 @@ def run_e2e(fg8, plan, args, stream, dev, world, chain):
     sp = stream.cuda_stream
     steps = max(3, min(args.steps, 50))
 
+    def fused_layer(L, xin, y, nxt):
+        g = L["g"]
+        fg8.fg8_linear_fused(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(), L["ws"].data_ptr(),
+                             L["b"].data_ptr(), y.data_ptr(), y.stride(0), g.fmt, L["wsp"].data_ptr(),
+                             L["wsp"].numel(), 0 if nxt is None else nxt["g"].N,
+                             None if nxt is None else nxt["ws"].data_ptr(),
+                             None if nxt is None else nxt["wsp"].data_ptr(), 0 if nxt is None else nxt["wsp"].numel(),
+                             sp)
+
     def layers(xin, yout):
         if chain:
             g = L0["g"]
-            fg8.fg8_linear_prepare(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L0["ws"].data_ptr(), g.fmt,
-                                   L0["wsp"].data_ptr(), L0["wsp"].numel(), sp)
+            if paths[0] != "tiled_fused_quant":
+                fg8.fg8_linear_prepare(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L0["ws"].data_ptr(), g.fmt,
+                                       L0["wsp"].data_ptr(), L0["wsp"].numel(), sp)
             for i, L in enumerate(plan):
                 g = L["g"]
                 y = yout if i + 1 == len(plan) else L["y"]
-                if i + 1 < len(plan):
+                if i == 0 and paths[0] == "tiled_fused_quant":
+                    fused_layer(L, xin, y, plan[1] if len(plan) > 1 else None)
+                elif i + 1 < len(plan):
                     Lx = plan[i + 1]
                     fg8.fg8_linear_run_chain(L["wq"].data_ptr(), L["ws"].data_ptr(), L["b"].data_ptr(),
                                              y.data_ptr(), g.M, g.N, g.K, y.stride(0), g.fmt,
@@ -571,6 +608,10 @@ def run_e2e(fg8, plan, args, stream, dev, world, chain):
             for i, L in enumerate(plan):
                 g = L["g"]
                 y = yout if i + 1 == len(plan) else L["y"]
+                if paths[i] == "tiled_fused_quant":
+                    fused_layer(L, xin, y, None)
+                    xin = y
+                    continue
                 fg8.fg8_linear_block(xin.data_ptr(), g.M, g.N, g.K, xin.stride(0), L["wq"].data_ptr(),
                                      L["ws"].data_ptr(), L["b"].data_ptr(), y.data_ptr(), y.stride(0), g.fmt,
                                      args.block, L["wsp"].data_ptr(), L["wsp"].numel(), sp)
@@ -1029,6 +1070,9 @@ def main(argv=None):
                     help="weight_block_size (block, block) and 1 x block activation groups (either scale format)")
     ap.add_argument("--no-chain", action="store_true",
                     help="quantize every layer's input in its own launch instead of in the previous GEMM")
+    ap.add_argument("--fused-quant", action="store_true",
+                    help="quantize a tiled layer's input inside its GEMM's launch (fg8_linear_fused) instead of in "
+                         "the separate act-quant launch the GEMM overlaps (the default: measured faster)")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="store the DRAM bytes of the GEMM launches in an ncu raw CSV export for --workload, then exit")
     args = ap.parse_args(argv)

@@ -35,6 +35,8 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear,
     fg8_linear_block,
     fg8_linear_block_workspace_bytes,
+    fg8_linear_fused,
+    fg8_linear_fused_workspace_bytes,
     fg8_linear_noalloc,
     fg8_linear_prepare,
     fg8_linear_run,

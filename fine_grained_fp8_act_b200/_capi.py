@@ -48,6 +48,9 @@ SIGNATURES = {
     "fg8_linear_run_chain": (_INT, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _I64, _VP, _VP, _SZ,
                                      _VP]),
     "fg8_linear_noalloc": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP]),
+    "fg8_linear_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
+    "fg8_linear_fused": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP, _SZ, _I64, _VP,
+                                _VP, _SZ, _VP]),
     "fg8_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
     "fg8_gemm_prequant": (_INT, [_VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_quantize_act_static": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),
@@ -193,6 +196,20 @@ def fg8_linear_run_chain(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y,
                                                               fmt, workspace, workspace_bytes, next_N,
                                                               next_w_scale_inv, next_workspace, next_workspace_bytes,
                                                               stream))
+
+
+def fg8_linear_fused_workspace_bytes(M, N, K, fmt) -> int:
+    return int(lib().fg8_linear_fused_workspace_bytes(M, N, K, fmt))
+
+
+def fg8_linear_fused(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, workspace,
+                     workspace_bytes, next_N=0, next_w_scale_inv=None, next_workspace=None, next_workspace_bytes=0,
+                     stream=None):
+    """fg8_linear with the activation quantization inside the GEMM kernel (optionally
+    also quantizing y for a next layer, as fg8_linear_run_chain)."""
+    _check("fg8_linear_fused", lib().fg8_linear_fused(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                      ld_y, fmt, workspace, workspace_bytes, next_N,
+                                                      next_w_scale_inv, next_workspace, next_workspace_bytes, stream))
 
 
 def fg8_linear_noalloc(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, stream):

@@ -723,6 +723,105 @@ fg8_status fg8_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64
                         stream);
 }
 
+// ---- the activation quantization inside the tiled GEMM (fg8_linear_fused) ----
+// Layout: fg8_linear's workspace, then one 32-bit flag per 128-row x 128-channel
+// unit of x (ceil(M/128) * ceil(K/128)); the header's words at byte 8 hold
+// the call epoch and the kernel's counters.
+size_t fused_flags_off(int64_t M, int64_t N, int64_t K, int fmt) {
+  return align_up(linear_workspace_need(M, N, K, fmt), kAlign);
+}
+size_t fused_need(int64_t M, int64_t N, int64_t K, int fmt) {
+  return fused_flags_off(M, N, K, fmt) +
+         align_up(static_cast<size_t>(ceil_div(M, 128)) * ceil_div(K, kGroup) * sizeof(uint32_t), kAlign);
+}
+// The in-kernel quantization pays off where a separate act-quant launch is
+// latency-bound: short K (up to 32 K-blocks, the short-K tile configuration)
+// and enough tokens for the tiled GEMM.
+bool can_quantize_in_gemm(int64_t M, int64_t N, int64_t K) {
+  return !use_small_m(M, N) && ceil_div(K, kGroup) <= 32;
+}
+
+size_t fg8_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
+  if (check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
+  return fused_need(M, N, K, fmt);
+}
+
+fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x, const void* wq_e4m3,
+                            const void* w_scale_inv, const void* bias_bf16, void* y_bf16, int64_t ld_y,
+                            fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, int64_t next_N,
+                            const void* next_w_scale_inv, void* next_workspace, size_t next_workspace_bytes,
+                            void* stream) {
+  if (const int st = fg8::check_linear_args_status(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16,
+                                                  ld_y, fmt);
+      st != FG8_OK)
+    return static_cast<fg8_status>(st);
+  const bool chain = next_w_scale_inv != nullptr;
+  if (chain) {  // the next layer: K = N, next_N outputs
+    if (fg8_status st = check_gemm_shape(M, next_N, N, fmt); st != FG8_OK) return st;
+    if (!aligned16(next_w_scale_inv)) return FG8_ERR_ALIGNMENT;
+  }
+  if (M == 0) return FG8_OK;
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, fused_need(M, N, K, fmt)); st != FG8_OK) return st;
+  const LinearWs Ln = linear_ws_layout(M, chain ? next_N : 8, N, fmt);
+  if (chain)
+    if (fg8_status st = check_workspace(next_workspace, next_workspace_bytes, Ln.total); st != FG8_OK) return st;
+  if (!can_quantize_in_gemm(M, N, K)) {  // long K or few tokens: the separate prepare step
+    if (!chain)
+      return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, workspace,
+                        workspace_bytes, stream);
+    if (fg8_status st = fg8_linear_prepare(x_bf16, M, N, K, ld_x, w_scale_inv, fmt, workspace, workspace_bytes,
+                                           stream);
+        st != FG8_OK)
+      return st;
+    return fg8_linear_run_chain(wq_e4m3, w_scale_inv, bias_bf16, y_bf16, M, N, K, ld_y, fmt, workspace,
+                                workspace_bytes, next_N, next_w_scale_inv, next_workspace, next_workspace_bytes,
+                                stream);
+  }
+  DeviceInfo dev;
+  if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const LinearWs L = linear_ws_layout(M, N, K, fmt);
+  const int Kb = ceil_div(K, kGroup), Kq = ceil_div(Kb, 4);
+  GemmArgs g{};
+  g.xq = ws + L.xq_off;
+  g.wq = wq_e4m3;
+  g.y = y_bf16;
+  g.ld_y = ld_y;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.Kb = Kb;
+  g.Kq = Kq;
+  g.bias = bias_bf16;
+  g.status = reinterpret_cast<uint32_t*>(ws);
+  g.wait_limit_ns = g_wait_limit_ns.load();
+  g.test_stall = g_test_stall.load();
+  if (fmt == FG8_SCALE_FLOAT) {
+    g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
+    g.ld_s = L.ld_s;
+    g.w_scale = static_cast<const float*>(w_scale_inv);
+  } else {
+    g.sfa = ws + L.xs_off;
+    g.sfb = ws + L.wsc_off;
+    g.qwsc = w_scale_inv;
+  }
+  g.qx = x_bf16;
+  g.ld_qx = ld_x;
+  g.qflags = reinterpret_cast<uint32_t*>(ws + fused_flags_off(M, N, K, fmt));
+  g.qepoch = reinterpret_cast<uint32_t*>(ws + kHeaderEpochOffset);
+  if (chain) {
+    uint8_t* wn = static_cast<uint8_t*>(next_workspace);
+    g.nx_xq = wn + Ln.xq_off;
+    g.nx_xs = wn + Ln.xs_off;
+    g.nx_ld_s = Ln.ld_s;
+    g.nx_Kq = ceil_div(ceil_div(N, kGroup), 4);
+    g.nx_w_scale = next_w_scale_inv;
+    g.nx_w_prep = wn + Ln.wsc_off;
+    g.nx_N = static_cast<int>(next_N);
+  }
+  return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
+}
+
 fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const void* wq_e4m3, const void* w_scale_inv,
                              const void* bias_bf16, void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_y,
                              fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, void* stream) {
@@ -877,8 +976,11 @@ fg8_status fg8_check_device_status(void* workspace, void* stream) {
   }
   if (word != 0) {
     // a kernel gave up mid-way: its split-K counters may be left counting,
-    // so the whole header starts from zero again
-    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+    // so the header starts from zero again -- all but the epoch word of the
+    // in-GEMM quantization, which only ever advances
+    uint8_t* h = static_cast<uint8_t*>(workspace);
+    if (cudaMemsetAsync(h + kHeaderEpochOffset + 4, 0, kHeaderBytes - kHeaderEpochOffset - 4, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
       cudaGetLastError();
       return FG8_ERR_CUDA;
     }

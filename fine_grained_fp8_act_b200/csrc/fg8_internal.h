@@ -107,6 +107,18 @@ struct GemmArgs {
   // groups, K-major [ceil(K/b)][ld_s], and b x b weight blocks
   // [ceil(N/b)][ceil(K/b)]; the GEMM promotes every b-wide slice of K
   int wblk;
+  // Optional: quantize x inside the GEMM kernel (1 x 128 groups) instead of
+  // reading a prepare step's output.  Before their tiles, all CTAs
+  // quantize 128-row x 128-channel units of bf16 x (unit rb * Kb + kb on CTA
+  // unit % grid) into xq and the x scales (sfa / xs_t, the prepare step's
+  // layouts), and mark each unit done in qflags[unit] with the call's epoch
+  // + 1; the roles that read a unit wait for its flag.  The last CTA to
+  // finish advances the epoch in the workspace header.
+  const void* qx;         // bf16 [M, K], row stride ld_qx; nullptr = off
+  int64_t ld_qx;
+  uint32_t* qflags;       // [ceil(M/128) * Kb]
+  uint32_t* qepoch;       // the header's words: epoch, finished-CTA count, weight-packing CTA count
+  const void* qwsc;       // UE8M0: this layer's weight scales [Nb][Kb], packed into sfb by phase one
 };
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM
@@ -121,6 +133,7 @@ cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, fl
 // per 128-row weight tile, zero at rest: the last CTA of a tile resets its
 // counter).  Zeroed by the caller before first use.
 constexpr size_t kWorkspaceHeaderBytes = 1024;
+constexpr size_t kHeaderEpochOffset = 8;  // fused act-quant: epoch word, then the finished-CTA count
 constexpr size_t kHeaderCounterOffset = 64;
 constexpr int kHeaderCounters = static_cast<int>((kWorkspaceHeaderBytes - kHeaderCounterOffset) / 4);
 

@@ -91,6 +91,19 @@ struct KParams {
   // the steps per slice), Kg = ceil(K / wblk) slices in all; x scales
   // [Kg][ld_s], weight scales [Nbs = ceil(N / wblk)][Kg]
   int wblk, gsteps, kps_shift, Kg, Nbs;
+  // x quantized inside the kernel (QIN configs): bf16 x, the unit flags and
+  // the epoch / finished-CTA words; xq_w, xs_w: where the codes and scales go
+  const uint16_t* qx;
+  int64_t ld_qx;
+  uint32_t* qflags;
+  uint32_t* qepoch;
+  uint8_t* xq_w;
+  void* xs_w;
+  int M_pad;
+  // UE8M0 QIN: this layer's weight scales [Nb][Kb] as given, packed by phase
+  // one into the scale-factor tiles the producer reads (sfb_w = sfb)
+  const uint8_t* wsc_src;
+  uint8_t* sfb_w;
 };
 
 constexpr uint32_t kStatusBadExpert = 1u;  // FG8_ERR_INVALID_ARG
@@ -107,9 +120,11 @@ __device__ __forceinline__ int tile_expert(const KParams& p, int m0, bool report
   return e;
 }
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false, bool SUBK_ = false>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false, bool SUBK_ = false, bool QIN_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
+  // QIN: the kernel quantizes its own x (1 x 128 groups) before the tiles
+  static constexpr bool QIN = QIN_;
   // REQUANT: the epilogue also quantizes its bf16 output rows, one 128-column
   // group per thread, for a next layer (needs the 256-wide tile).
   static constexpr bool REQUANT = REQUANT_;
@@ -288,17 +303,163 @@ __device__ __forceinline__ void prepare_next_layer(const KParams& p, int idx, in
   }
 }
 
+// ------------------------------------------------- in-kernel act-quant ----
+// A unit: rows [128 rb, 128 rb + 128) of x, K-block kb -- 128 groups of
+// 1 x 128, eight lanes per group (two 16-byte loads each), the same
+// arithmetic as the stand-alone quantizer (quant_math.cuh), written in the
+// layouts the GEMM reads: codes [M, K] row stride K; float scales K-major
+// [Kb][ld_s]; UE8M0 bytes in the scale-factor tiles (rows past M, and the
+// K-block slots past Kb in the last chunk, get 2^0).  With 384 threads (48
+// groups at a time) a unit takes kUnitPasses passes; the loads of a batch of
+// kUnitBatch units are all issued before any of them is quantized.
+constexpr int kUnitPasses = 3;
+constexpr int kUnitBatch = 2;
+
+struct UnitLoad {
+  uint4 v[kUnitPasses][2];
+};
+
+template <class C>
+__device__ __forceinline__ void load_unit(const KParams& p, int u, UnitLoad& d) {
+  const int rb = u / p.Kb, kb = u - (u / p.Kb) * p.Kb;
+  const int oct = static_cast<int>(threadIdx.x) >> 3, l = static_cast<int>(threadIdx.x) & 7;
+#pragma unroll
+  for (int i = 0; i < kUnitPasses; ++i) {
+    const int r = oct + i * (C::kThreads >> 3);
+    const int m = rb * kBlockM + r;
+    const int k = kb * 128 + l * 16;
+    d.v[i][0] = d.v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+    if (r < kBlockM && m < p.M && k < p.K) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.qx + static_cast<int64_t>(m) * p.ld_qx + k);
+      d.v[i][0] = __ldg(src);
+      d.v[i][1] = __ldg(src + 1);
+    }
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void quantize_unit(const KParams& p, int u, const UnitLoad& d) {
+  const int rb = u / p.Kb, kb = u - (u / p.Kb) * p.Kb;
+  const int oct = static_cast<int>(threadIdx.x) >> 3, l = static_cast<int>(threadIdx.x) & 7;
+#pragma unroll
+  for (int i = 0; i < kUnitPasses; ++i) {
+    const int r = oct + i * (C::kThreads >> 3);
+    if (i * (C::kThreads >> 3) + (static_cast<int>(threadIdx.x) & ~31) / 8 >= kBlockM) break;  // whole warps stop
+    const int m = rb * kBlockM + r;
+    const bool real = r < kBlockM && m < p.M;
+    const int k = kb * 128 + l * 16;
+    float f[16];
+    float(&f0)[8] = *reinterpret_cast<float(*)[8]>(f);
+    float(&f1)[8] = *reinterpret_cast<float(*)[8]>(f + 8);
+    qm::unpack_bf16x8(d.v[i][0], f0);
+    qm::unpack_bf16x8(d.v[i][1], f1);
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(f[j]));
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const float s = qm::group_scale(amax);
+    const uint32_t sbyte = C::FMT == 1 ? qm::e8m0_ceil_byte(s) : 0u;
+    const uint4 packed = qm::quantize16<C::FMT>(f, s, sbyte);
+    if (real && k < p.K) *reinterpret_cast<uint4*>(p.xq_w + static_cast<int64_t>(m) * p.K + k) = packed;
+    if (l == 0 && r < kBlockM) {
+      if constexpr (C::FMT == 0) {
+        if (real) static_cast<float*>(p.xs_w)[static_cast<int64_t>(kb) * p.ld_s + m] = s;
+      } else {
+        uint8_t* sf = static_cast<uint8_t*>(p.xs_w);
+        sf[sf_tile_offset(m, kb, p.Kq)] = real ? static_cast<uint8_t>(sbyte) : static_cast<uint8_t>(127);
+        if (kb == p.Kb - 1)
+          for (int kx = p.Kb; kx < 4 * p.Kq; ++kx) sf[sf_tile_offset(m, kx, p.Kq)] = static_cast<uint8_t>(127);
+      }
+    }
+  }
+}
+
+// Phase one of a QIN launch, by every thread of the CTA.  UE8M0: first its
+// share of the weight scale-factor tiles (16-byte pieces, the prepare step's
+// packing), counted in the header's third word.  Then its share of the
+// units (unit u = rb * Kb + kb on CTA u % grid, in increasing u, so the row
+// blocks the first tiles need come first), each published with the epoch.
+template <class C>
+__device__ __forceinline__ void quantize_own_units(const KParams& p, uint32_t epoch) {
+  static_assert(kUnitPasses * (C::kThreads / 8) >= kBlockM, "a unit's 128 groups in kUnitPasses passes");
+  if constexpr (C::FMT == 1) {
+    const int64_t pieces = sfb_rows(p.N) / 128 * p.Kq * 32;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * C::kThreads + threadIdx.x; i < pieces;
+         i += static_cast<int64_t>(gridDim.x) * C::kThreads) {
+      const int64_t tq = i >> 5;
+      const int lane = static_cast<int>(i & 31);
+      const int64_t tile = tq / p.Kq;
+      const int q = static_cast<int>(tq - tile * p.Kq);
+      uint32_t w[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int64_t r = tile * 128 + c * 32 + lane;
+        uint32_t v = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int kb = 4 * q + j;
+          const uint32_t b = (r < p.N && kb < p.Kb) ? p.wsc_src[(r / 128) * p.Kb + kb] : 127u;
+          v |= b << (8 * j);
+        }
+        w[c] = v;
+      }
+      *reinterpret_cast<uint4*>(p.sfb_w + tq * kSfChunkBytes + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_global();  // read by bulk copies (async proxy) in every CTA
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(p.qepoch + 2, 1u);
+    }
+  }
+  const int units = p.num_m * p.Kb;
+  const int step = static_cast<int>(gridDim.x);
+  for (int u0 = static_cast<int>(blockIdx.x); u0 < units; u0 += kUnitBatch * step) {
+    UnitLoad d[kUnitBatch];
+#pragma unroll
+    for (int j = 0; j < kUnitBatch; ++j)
+      if (u0 + j * step < units) load_unit<C>(p, u0 + j * step, d[j]);
+#pragma unroll
+    for (int j = 0; j < kUnitBatch; ++j) {
+      const int u = u0 + j * step;
+      if (u >= units) break;
+      quantize_unit<C>(p, u, d[j]);
+      fence_proxy_async_global();  // the codes are read by TMA (async proxy) in other CTAs
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        st_release_gpu(p.qflags + u, epoch + 1u);
+      }
+    }
+  }
+}
+
+// Wait until unit (rb, kb) of this call is quantized (QIN configs).
+template <class C>
+__device__ __forceinline__ bool unit_ready(const KParams& p, uint32_t epoch, int rb, int kb,
+                                           volatile int* abort_flag) {
+  if constexpr (!C::QIN) {
+    return true;
+  } else {
+    if (!flag_wait(p.qflags + rb * p.Kb + kb, epoch + 1u, p.wait_limit_ns, abort_flag)) return false;
+    fence_proxy_async_global();
+    return true;
+  }
+}
+
 // ---------------------------------------------------------------- roles ----
 template <class C>
 __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
                                          uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* bfull,
-                                         uint64_t* bempty, volatile int* abort_flag) {
+                                         uint64_t* bempty, volatile int* abort_flag, uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
   Ring st, bi;
   // most recent issue phase per slot, for the drain at the end
   uint32_t st_issued = 0, bi_issued = 0;
   uint32_t st_par[C::STAGES], bi_par[2];
   bool ok = true;
+  bool w_packed = false;
   for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
     int mb, nb;
     tile_coords(tile, p.num_m, p.num_n, mb, nb);
@@ -330,6 +491,21 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
         break;
       }
       const bool sf = C::FMT == 1 && (kb & ((1 << p.sf_shift) - 1)) == 0;
+      if constexpr (C::QIN) {  // the A tile (and, UE8M0, the chunk's four K-blocks of scales) quantized
+        bool ready = true;
+        if (C::FMT == 1 && !w_packed) {  // every CTA's share of the weight scale-factor tiles is in place
+          ready = flag_wait(p.qepoch + 2, gridDim.x, limit, abort_flag);
+          fence_proxy_async_global();
+          w_packed = true;
+        }
+        const int last = C::FMT == 1 && sf ? min(kb + 3, p.Kb - 1) : kb;
+        for (int kx = kb; ready && kx <= last; ++kx) ready = unit_ready<C>(p, epoch, mb, kx, abort_flag);
+        if (!ready) {
+          raise_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+      }
       uint8_t* sa = smem + st.slot * C::kStage;
       mbar_arrive_expect_tx(full + st.slot, C::kStageTx + (sf ? C::kSfBytes : 0));
       tma_load_2d(sa, tmA, full + st.slot, kb * 128, m0);
@@ -486,7 +662,7 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
 // latency stays off the epilogue's path.  The epilogue warps release slots.
 template <class C>
 __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
-                                             volatile int* abort_flag, int lane) {
+                                             volatile int* abort_flag, int lane, uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
   Ring sr;
   for (int tile = static_cast<int>(blockIdx.x); tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
@@ -502,6 +678,11 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
     const float* ws = p.w_scale + static_cast<int64_t>(wb) * p.Kg;
     for (int g = 0; g < p.Kg; ++g) {
       if (!mbar_wait_warp(sempty + sr.slot, sr.phase ^ 1u, limit, abort_flag)) {
+        raise_abort(abort_flag, p.status);
+        cp_async_wait_all();
+        return;
+      }
+      if (!__all_sync(0xFFFFFFFFu, unit_ready<C>(p, epoch, mb, g, abort_flag))) {  // QIN: this unit's scales
         raise_abort(abort_flag, p.status);
         cp_async_wait_all();
         return;
@@ -767,15 +948,20 @@ __global__ void __launch_bounds__(384, 1)
   // launch); from here on its outputs (quantized activations, scales) are read.
   grid_wait_prerequisites();
   grid_launch_dependents();  // the next kernel may take SMs as this grid's CTAs finish
+  uint32_t epoch = 0;
+  if constexpr (C::QIN) {
+    epoch = ld_acquire_gpu(p.qepoch);
+    quantize_own_units<C>(p, epoch);
+  }
 
   if (warp < 4) {
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
-      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag);
+      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag, epoch);
     else if (warp == 1 && lane == 0)
       mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, abort_flag);
     if constexpr (C::FMT == 0) {
-      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, abort_flag, lane);
+      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, abort_flag, lane, epoch);
     }
     if constexpr (C::REQUANT && C::FMT == 1) {
       if (warp == 2 || warp == 3)
@@ -791,6 +977,19 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
+  }
+  if constexpr (C::QIN) {
+    // the last CTA out advances the epoch: every CTA has read it and every
+    // unit flag of this call holds epoch + 1, which no later call waits for
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.qepoch + 1, 1u) == gridDim.x - 1) {
+        p.qepoch[1] = 0u;
+        p.qepoch[2] = 0u;
+        __threadfence();
+        atomicAdd(p.qepoch, 1u);
+      }
+    }
   }
 }
 
@@ -871,6 +1070,15 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.kps_shift = p.wblk == 128 ? 2 : (p.wblk == 64 ? 1 : 0);
   p.Kg = (g.K + p.wblk - 1) / p.wblk;
   p.Nbs = (g.N + p.wblk - 1) / p.wblk;
+  p.qx = static_cast<const uint16_t*>(g.qx);
+  p.ld_qx = g.ld_qx;
+  p.qflags = g.qflags;
+  p.qepoch = g.qepoch;
+  p.xq_w = static_cast<uint8_t*>(const_cast<void*>(g.xq));
+  p.xs_w = C::FMT == 0 ? static_cast<void*>(const_cast<float*>(g.xs_t)) : static_cast<void*>(const_cast<uint8_t*>(g.sfa));
+  p.M_pad = (g.M + kBlockM - 1) / kBlockM * kBlockM;
+  p.wsc_src = static_cast<const uint8_t*>(g.qwsc);
+  p.sfb_w = const_cast<uint8_t*>(g.sfb);
   if (p.num_tiles == 0) return cudaSuccess;
 
   // the shared-memory opt-in once per device: one bit per device; calls from
@@ -923,6 +1131,19 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   // Long K: four stages (the float path's scale ring takes the shared memory
   // of the second staging box per warp).
   const bool short_k = g.Kb <= 32;
+  if (g.qx != nullptr) {  // x quantized inside the kernel: short K only (see can_quantize_in_gemm)
+    if (!short_k || g.wblk > 0 && g.wblk != 128 || g.row_expert != nullptr) return cudaErrorInvalidValue;
+    const bool requant = g.nx_xq != nullptr;
+    const int bnq = requant ? 256 : choose_block_n(g.M, g.N, num_sms);
+    if (fmt == 0) {
+      if (requant) return launch_cfg<Cfg<256, 0, 3, 4, true, false, true>>(g, num_sms, s);
+      if (bnq == 256) return launch_cfg<Cfg<256, 0, 3, 4, false, false, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<128, 0, 5, 2, false, false, true>>(g, num_sms, s);
+    }
+    if (requant) return launch_cfg<Cfg<256, 1, 3, 4, true, false, true>>(g, num_sms, s);
+    if (bnq == 256) return launch_cfg<Cfg<256, 1, 3, 4, false, false, true>>(g, num_sms, s);
+    return launch_cfg<Cfg<128, 1, 5, 2, false, false, true>>(g, num_sms, s);
+  }
   if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
     if (fmt == 0) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, true>>(g, num_sms, s);

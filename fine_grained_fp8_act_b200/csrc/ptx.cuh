@@ -76,6 +76,33 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, u
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, limit_ns, abort));
 }
 
+// ------------------------------------------------ flags in global memory ----
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait for *flag == want (acquire): false once `limit_ns` passed or
+// another role raised `*abort`.
+__device__ __forceinline__ bool flag_wait(const uint32_t* flag, uint32_t want, uint64_t limit_ns,
+                                          const volatile int* abort) {
+  if (ld_acquire_gpu(flag) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == want) return true;
+    if ((i & 15u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // ------------------------------------------ programmatic dependent launch ----
 // Lets the next kernel in the stream (launched with programmatic stream
 // serialization) start its prologue once every CTA of this grid got here.

@@ -109,8 +109,8 @@ FG8_API size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_s
  *               split-K arrival counters, which the kernels leave at zero.
  *               Zero the header once before first use (e.g. allocate the
  *               workspace zero-filled); fg8_check_device_status reads and
- *               clears the status word, and after a failed call the whole
- *               header.  Calls sharing a workspace must not overlap on the
+ *               clears the status word, and after a failed call the rest of
+ *               the header but the epoch word of fg8_linear_fused.  Calls sharing a workspace must not overlap on the
  *               device.
  * fg8_linear is fg8_linear_prepare (quantize x into the workspace) then
  * fg8_linear_run (the GEMM), which picks its kernel by shape: for M <= 32,
@@ -161,6 +161,38 @@ FG8_API fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale
                                         fg8_scale_fmt fmt, void* workspace, size_t workspace_bytes, int64_t next_N,
                                         const void* next_w_scale_inv, void* next_workspace,
                                         size_t next_workspace_bytes, void* stream);
+
+/* fg8_linear with the activation quantization inside the GEMM kernel ([zh]
+ * §八 step 6 / §6.1 make the per-token quantization part of fp8_linear; here
+ * it is fused into the tiled GEMM's launch instead of running as a separate
+ * prepare kernel).  Before its tiles, every CTA of the GEMM quantizes a share
+ * of x in 128-row x 128-channel units (the same codes and scales as
+ * fg8_quantize_act, in the GEMM's layouts) and publishes each unit with a
+ * flag; the roles that read a unit wait for its flag (bounded waits).  Used
+ * where it pays off -- the tiled path (M above the few-token range) with
+ * K <= 4096 (up to 32 K-blocks); other shapes run exactly fg8_linear (or,
+ * with a next layer, fg8_linear_prepare + fg8_linear_run_chain).
+ *   Arguments as fg8_linear, plus an optional next layer as in
+ *   fg8_linear_run_chain: with next_w_scale_inv non-NULL the epilogue also
+ *   quantizes y for a layer with next_N outputs into next_workspace
+ *   (>= fg8_linear_workspace_bytes(M, next_N, N, fmt)), after which
+ *   fg8_linear_run(next layer, next_workspace) computes that layer.  With
+ *   next_w_scale_inv NULL, next_N, next_workspace and next_workspace_bytes
+ *   are ignored.
+ *   workspace   >= fg8_linear_fused_workspace_bytes(M, N, K, fmt), 256-byte
+ *               aligned, ZERO-FILLED IN FULL before its first use: beyond
+ *               fg8_linear's layout it holds one flag per unit of x, and the
+ *               header holds the call epoch the flags are compared with (an
+ *               epoch that only advances; fg8_check_device_status keeps it).
+ *               Do not zero the header alone between fused calls on one
+ *               workspace.  Calls sharing a workspace must not overlap.
+ * Same results, bit for bit, as fg8_linear (and fg8_linear_run_chain). */
+FG8_API size_t fg8_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
+FG8_API fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
+                                    const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
+                                    void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* workspace,
+                                    size_t workspace_bytes, int64_t next_N, const void* next_w_scale_inv,
+                                    void* next_workspace, size_t next_workspace_bytes, void* stream);
 
 /* fg8_linear without a caller workspace, for callers that cannot allocate
  * device memory (for example a host framework that owns all device memory
