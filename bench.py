@@ -346,7 +346,7 @@ def run_fg8(args, rank, world, local):
     # act-quant launch.
     # block 32 / 64 (1 x b groups, b x b weight blocks): fg8_linear_block per layer
     paths = [("small_block" if args.block != 128 else layer_path(L["g"])) for L in plan]
-    chain = not args.no_chain and all(pth == "tiled" for pth in paths)
+    chain = not args.no_chain and len(plan) > 1 and all(pth == "tiled" for pth in paths)
     # --fused-quant: a tiled layer with K <= 4096 whose input is not already
     # quantized by the previous GEMM takes fg8_linear_fused, its act-quant
     # inside the GEMM's launch (in-kernel units published with flags).

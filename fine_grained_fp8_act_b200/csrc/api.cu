@@ -765,7 +765,10 @@ fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   const LinearWs Ln = linear_ws_layout(M, chain ? next_N : 8, N, fmt);
   if (chain)
     if (fg8_status st = check_workspace(next_workspace, next_workspace_bytes, Ln.total); st != FG8_OK) return st;
-  if (!can_quantize_in_gemm(M, N, K)) {  // long K or few tokens: the separate prepare step
+  if (!chain && use_small_m(M, N) && M <= kFusedMMax)  // few tokens: the few-token kernel quantizes x itself
+    return launch_small_path(true, x_bf16, ld_x, M, N, K, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt,
+                             workspace, stream);
+  if (!can_quantize_in_gemm(M, N, K)) {  // long K, or 17 to 128 tokens: the separate prepare step
     if (!chain)
       return fg8_linear(x_bf16, M, N, K, ld_x, wq_e4m3, w_scale_inv, bias_bf16, y_bf16, ld_y, fmt, workspace,
                         workspace_bytes, stream);

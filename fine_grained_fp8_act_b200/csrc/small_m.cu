@@ -120,7 +120,6 @@ struct SmCfg {
   static constexpr int kSmem = kSmemUsed < 120 * 1024 ? 120 * 1024 : kSmemUsed;
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(STAGES >= 4 && (PREQ || (STAGES % kQ == 0 && 8 % kQ == 0)), "ring depth");
-  static_assert(PREQ || FMT == 1, "fused quantization: UE8M0 scales (float scales take the prepare step)");
   static_assert(MP % 16 == 0 && MP >= 16 && MP <= (PREQ ? 128 : 32), "token padding");
   static_assert(kOffXq % 1024 == 0 && kOffXb == kW, "the swizzled B operand starts on a 1024-byte boundary");
   static_assert(kNumAcc * MP <= (FMT == 0 ? 512 : 256), "TMEM columns");
@@ -258,7 +257,8 @@ __device__ __forceinline__ void sm_producer_pq(const CUtensorMap* tmW, const CUt
 // ... (kQ K-blocks in flight at once), 8 lanes per token, 4 tokens per pass.
 template <class C>
 __device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, uint64_t* wfull, uint64_t* xfull,
-                                             int nt, int kb0, int kb1, volatile int* abort_flag) {
+                                             uint64_t* scfull, uint64_t* scempty, int nt, int kb0, int kb1,
+                                             volatile int* abort_flag) {
   const int qw = (static_cast<int>(threadIdx.x) >> 5) - kQuantWarp0;
   const int lane = static_cast<int>(threadIdx.x) & 31, l = lane & 7, r_in = lane >> 3;
   if (qw >= C::kQ) return;
@@ -275,6 +275,16 @@ __device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, u
     uint8_t* stage = smem + slot * C::kStage;
     uint8_t* xs = stage + C::kOffXq;
     const uint8_t* xb = stage + C::kOffXb;
+    // float: the K-block's token scales go to the epilogue's scale ring (slot
+    // i % 8: with kQ dividing 8, always this warp's), once the epilogue has
+    // released the slot's previous K-block
+    const int sc_slot = i % C::kScSlots;
+    float* scs = reinterpret_cast<float*>(smem + C::kOffSc + sc_slot * C::MP * 4);
+    if (C::FMT == 0 && !mbar_wait_warp(scempty + sc_slot, static_cast<uint32_t>((i / C::kScSlots) & 1) ^ 1u,
+                                       p.wait_limit_ns, abort_flag)) {
+      sm_raise(abort_flag, p.status);
+      break;
+    }
     constexpr int kPasses = C::MP / 4;
     constexpr int kBatch = kPasses < 4 ? kPasses : 4;
 #pragma unroll
@@ -308,15 +318,19 @@ __device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, u
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
         const float s = qm::group_scale(amax);
-        const uint32_t sb = qm::e8m0_ceil_byte(s);
-        const uint4 q = qm::quantize16<1>(f, s, sb);
+        const uint32_t sb = C::FMT == 1 ? qm::e8m0_ceil_byte(s) : 0u;
+        const uint4 q = qm::quantize16<C::FMT>(f, s, sb);
         // row `row`, 16-byte chunk l of the 128-byte row, 128-byte swizzle (8-row atoms)
         *reinterpret_cast<uint4*>(xs + (row >> 3) * 1024 + (row & 7) * 128 + ((l ^ (row & 7)) << 4)) = q;
-        if (l == 0)  // tcgen05.cp source: token row r -> word (r % 32) * 16 + (r / 32) * 4, byte 0
-          *reinterpret_cast<uint32_t*>(xs + C::kX + (row & 31) * 16 + (row >> 5) * 4) = row < p.M ? sb : 127u;
+        if (l == 0) {
+          if constexpr (C::FMT == 1)  // tcgen05.cp source: token row r -> word (r % 32) * 16 + (r / 32) * 4, byte 0
+            *reinterpret_cast<uint32_t*>(xs + C::kX + (row & 31) * 16 + (row >> 5) * 4) = row < p.M ? sb : 127u;
+          else
+            scs[row] = s;  // rows past M: a finite scale whose products are never stored
+        }
       }
     }
-    {
+    if constexpr (C::FMT == 1) {
       // every weight row of the tile has the block's scale; token rows past
       // MP get a finite scale the MMA never uses
       const uint32_t wb = p.ws_b[static_cast<int64_t>(nt) * p.Kb + kb];
@@ -329,7 +343,10 @@ __device__ __forceinline__ void sm_quantizer(const SmParams& p, uint8_t* smem, u
     }
     fence_proxy_async_smem();  // the tensor core reads what these threads wrote
     __syncwarp();
-    if (lane == 0) mbar_arrive(xfull + slot);
+    if (lane == 0) {
+      mbar_arrive(xfull + slot);
+      if (C::FMT == 0) mbar_arrive(scfull + sc_slot);  // the epilogue reads the scales
+    }
   }
 }
 
@@ -669,7 +686,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (lane == 0)
       sm_mma<C>(p, smem, tmem, wfull, xfull, sempty, tfull, tempty, teardown, stall, kb0, kb1, abort_flag);
   } else if (warp < C::kEpiWarp0) {
-    if constexpr (!C::PREQ) sm_quantizer<C>(p, smem, wfull, xfull, nt, kb0, kb1, abort_flag);
+    if constexpr (!C::PREQ) sm_quantizer<C>(p, smem, wfull, xfull, scfull, scempty, nt, kb0, kb1, abort_flag);
   } else {
     sm_epilogue<C>(p, smem, tmem, tfull, tempty, scfull, scempty, rbar, nt, sp, kb0, kb1, abort_flag, last_flag,
                    go_flag);
@@ -823,8 +840,9 @@ cudaError_t launch_small_m(const SmallMArgs& a, int fmt, cudaStream_t s) {
     if (mp == 64) return launch_small_m_cfg<SmCfg<1, 64, true>>(a, s);
     return launch_small_m_cfg<SmCfg<1, 128, true>>(a, s);
   }
-  // fused quantization: UE8M0 scales, M <= 16 (one token padding)
-  if (fmt != 1 || a.M < 1 || a.M > kFusedMMax) return cudaErrorInvalidValue;
+  // fused quantization: M <= 16 (one token padding)
+  if (a.M < 1 || a.M > kFusedMMax) return cudaErrorInvalidValue;
+  if (fmt == 0) return launch_small_m_cfg<SmCfg<0, 16>>(a, s);
   return launch_small_m_cfg<SmCfg<1, 16>>(a, s);
 }
 

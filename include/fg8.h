@@ -168,10 +168,15 @@ FG8_API fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale
  * prepare kernel).  Before its tiles, every CTA of the GEMM quantizes a share
  * of x in 128-row x 128-channel units (the same codes and scales as
  * fg8_quantize_act, in the GEMM's layouts) and publishes each unit with a
- * flag; the roles that read a unit wait for its flag (bounded waits).  Used
- * where it pays off -- the tiled path (M above the few-token range) with
- * K <= 4096 (up to 32 K-blocks); other shapes run exactly fg8_linear (or,
- * with a next layer, fg8_linear_prepare + fg8_linear_run_chain).
+ * flag; the roles that read a unit wait for its flag (bounded waits).  This
+ * covers the tiled path (M above the few-token range) with K <= 4096 (up to
+ * 32 K-blocks).  With M <= 16 (and no next layer) the few-token kernel
+ * quantizes x itself, in quantizer warps, for either scale format.  Other
+ * shapes run exactly fg8_linear (or, with a next layer, fg8_linear_prepare +
+ * fg8_linear_run_chain).  Measured on B200, the separate quantization launch
+ * that fg8_linear overlaps with the GEMM is faster for float scales, which is
+ * why fg8_linear keeps it; this entry point is for callers that want a single
+ * launch per layer.
  *   Arguments as fg8_linear, plus an optional next layer as in
  *   fg8_linear_run_chain: with next_w_scale_inv non-NULL the epilogue also
  *   quantizes y for a layer with next_N outputs into next_workspace
@@ -186,7 +191,9 @@ FG8_API fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale
  *               epoch that only advances; fg8_check_device_status keeps it).
  *               Do not zero the header alone between fused calls on one
  *               workspace.  Calls sharing a workspace must not overlap.
- * Same results, bit for bit, as fg8_linear (and fg8_linear_run_chain). */
+ * The tiled path gives fg8_linear's results bit for bit (and
+ * fg8_linear_run_chain's); the few-token kernel's sums may round differently
+ * within the stated tolerance. */
 FG8_API size_t fg8_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
 FG8_API fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K, int64_t ld_x,
                                     const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,

@@ -110,9 +110,32 @@ def test_fused_with_next_layer(fg8, orc, fmt, M, K1, N1, N2):
 
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("M,N,K", [(16, 4096, 1024), (1000, 512, 8192)])
+@pytest.mark.parametrize("M,N,K", [(1, 4104, 1024), (16, 4096, 1040), (9, 264, 4096)])
+def test_fused_entry_few_tokens_vs_oracle(fg8, orc, fmt, M, N, K):
+    """Up to 16 tokens: the few-token kernel with its own quantizer warps
+    (float and UE8M0), every element against the oracle."""
+    x = W.x_outliers(M, K, seed=M + K)
+    w = W.w_row_groups(N, K, 0.02, seed=N)
+    b = W.normal((N,), 0.1, seed=2)
+    wq, ws = fg8.quantize_weight(w.cuda(), fmt)
+    wsp = torch.zeros(fg8.fg8_linear_fused_workspace_bytes(M, N, K, fmt), dtype=torch.uint8, device="cuda")
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    xd, bd = x.cuda(), b.cuda()
+    for _ in range(2):
+        fg8.fg8_linear_fused(xd.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), bd.data_ptr(), y.data_ptr(), N,
+                             fmt, wsp.data_ptr(), wsp.numel(), stream=_s())
+    torch.cuda.synchronize()
+    assert fg8.fg8_check_device_status(wsp.data_ptr(), _s()) == 0
+    owq, ows = orc.quantize_weight(W.bf16_bits(w), fmt)
+    y64, bound, _ = orc.linear(W.bf16_bits(x), owq, ows, W.bf16_bits(b), fmt)
+    err = np.abs(_f64(y) - y64)
+    assert (err <= y_tolerance(bound)).all(), f"max err {np.nanmax(err)}"
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(40, 4096, 1024), (1000, 512, 8192)])
 def test_fused_entry_on_shapes_that_prepare_separately(fg8, fmt, M, N, K):
-    """Few tokens and long K take fg8_linear's own path through the same entry."""
+    """17 to 128 tokens and long K take fg8_linear's own path through the same entry."""
     x = W.x_normal(M, K, seed=M + K).cuda()
     wq, ws = fg8.quantize_weight(W.normal((N, K), 0.02, seed=N).cuda(), fmt)
     b = W.normal((N,), 0.1, seed=2).cuda()
