@@ -123,6 +123,30 @@ def test_dequantize_stays_in_bounds(fg8, fmt):
     assert cw.intact()
 
 
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M", [5, 300])   # few-token kernel quantizing x itself; tiled GEMM quantizing in-launch
+def test_fused_linear_stays_in_bounds(fg8, fmt, M):
+    N, K = 264, 400
+    ld_y = N + 8
+    x = W.x_outliers(M, K, seed=M + 3).cuda()
+    w = W.w_row_groups(N, K, 0.02, seed=M + 4).cuda()
+    b = W.normal((N,), 0.1, seed=M + 5).cuda()
+    wq, ws = fg8.quantize_weight(w, fmt)
+    cy = Canary(M * ld_y * 2, "cuda")
+    y = cy.matrix(BF16, M, N, ld_y)
+    need = fg8.fg8_linear_fused_workspace_bytes(M, N, K, fmt)
+    cw = Canary(need, "cuda")
+    cw.zeroed()
+    for _ in range(2):  # a second call on the same workspace: the flags' epoch has advanced
+        fg8.fg8_linear_fused(x.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), b.data_ptr(), cy.ptr(), ld_y,
+                             fmt, cw.ptr(), need, stream=_s())
+        assert fg8.fg8_check_device_status(cw.ptr(), _s()) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(y, fg8.linear(x, wq, ws, b, fmt))
+        assert cy.intact(), "y: a write outside [M, N] or into the row padding"
+        assert cw.intact(), "workspace: a write past fg8_linear_fused_workspace_bytes"
+
+
 @pytest.mark.parametrize("blk,sfmt", [(32, "ue8m0"), (64, "ue8m0"), (32, "float"), (64, "float")])
 def test_small_block_layer_stays_in_bounds(fg8, blk, sfmt):
     fmt = UE8M0 if sfmt == "ue8m0" else 0

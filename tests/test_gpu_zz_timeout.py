@@ -27,14 +27,20 @@ def _as_f64(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+@pytest.mark.parametrize("entry", ["linear", "fused"])  # fused: the kernels that quantize x in their launch
 @pytest.mark.parametrize("M", [16, 640])  # the few-token kernel and the tiled GEMM
 @pytest.mark.parametrize("fmt", [0, 1])
-def test_wait_limit_reports_timeout_and_context_survives(fg8, orc, M, fmt):
+def test_wait_limit_reports_timeout_and_context_survives(fg8, orc, M, fmt, entry):
     N, K = 512, 1024
     x = W.x_normal(M, K, seed=M + 1)
     w = W.normal((N, K), 0.02, seed=M + 2)
     wq, ws = fg8.quantize_weight(w.cuda(), fmt)
-    nb = fg8.fg8_linear_workspace_bytes(M, N, K, fmt)
+    if entry == "linear":
+        nb = fg8.fg8_linear_workspace_bytes(M, N, K, fmt)
+        call = fg8.fg8_linear
+    else:
+        nb = fg8.fg8_linear_fused_workspace_bytes(M, N, K, fmt)
+        call = fg8.fg8_linear_fused
     wsp = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream().cuda_stream
     xd = x.cuda()
@@ -42,16 +48,16 @@ def test_wait_limit_reports_timeout_and_context_survives(fg8, orc, M, fmt):
     try:
         fg8.fg8_set_wait_limit_ns(1_000_000)
         fg8.fg8_set_test_stall(True)
-        fg8.fg8_linear(xd.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), 0, y.data_ptr(), N, fmt,
-                       wsp.data_ptr(), nb, s)
+        call(xd.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), 0, y.data_ptr(), N, fmt, wsp.data_ptr(), nb,
+             stream=s)
         torch.cuda.synchronize()
         assert fg8.fg8_check_device_status(wsp.data_ptr(), s) == fg8.FG8_ERR_TIMEOUT
     finally:
         fg8.fg8_set_test_stall(False)
         fg8.fg8_set_wait_limit_ns(2_000_000_000)
     # the context is usable and the (re-zeroed) workspace gives correct results
-    fg8.fg8_linear(xd.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), 0, y.data_ptr(), N, fmt, wsp.data_ptr(),
-                   nb, s)
+    call(xd.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), 0, y.data_ptr(), N, fmt, wsp.data_ptr(), nb,
+         stream=s)
     torch.cuda.synchronize()
     assert fg8.fg8_check_device_status(wsp.data_ptr(), s) == fg8.FG8_OK
     owq, ows = orc.quantize_weight(W.bf16_bits(w), fmt)
