@@ -43,6 +43,7 @@ from ._capi import (  # noqa: F401  (re-exported C ABI)
     fg8_linear_run_chain,
     fg8_linear_static,
     fg8_linear_workspace_bytes,
+    fg8_linear_plan,
     fg8_quantize_act,
     fg8_quantize_act_block,
     fg8_quantize_act_static,

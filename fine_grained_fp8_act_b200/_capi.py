@@ -32,6 +32,7 @@ SIGNATURES = {
     "fg8_quantize_weight": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _INT, _VP]),
     "fg8_quantize_act": (_INT, [_VP, _I64, _I64, _I64, _VP, _VP, _INT, _VP]),
     "fg8_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _INT]),
+    "fg8_linear_plan": (_INT, [_I64, _I64, _I64, _INT, _VP]),
     "fg8_linear": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _I64, _INT, _VP, _SZ, _VP]),
     "fg8_linear_prepare": (_INT, [_VP, _I64, _I64, _I64, _I64, _VP, _INT, _VP, _SZ, _VP]),
     "fg8_grouped_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _INT]),
@@ -121,6 +122,14 @@ def fg8_quantize_act(x_bf16, M, K, ld_x, xq_e4m3, x_scale, fmt, stream):
 
 def fg8_linear_workspace_bytes(M, N, K, fmt) -> int:
     return int(lib().fg8_linear_workspace_bytes(M, N, K, fmt))
+
+
+def fg8_linear_plan(M, N, K, fmt):
+    """(kernel, tile width, split tiles, units per split tile): how fg8_linear runs
+    this shape on the current device; see include/fg8.h."""
+    out = (ctypes.c_int32 * 4)()
+    _check("fg8_linear_plan", lib().fg8_linear_plan(M, N, K, fmt, out))
+    return tuple(int(v) for v in out)
 
 
 def fg8_gemm_workspace_bytes(M, N, K, fmt) -> int:

@@ -145,12 +145,36 @@ size_t small_counter_bytes(int64_t N) {
   return nt > kHeaderCounters ? align_up(static_cast<size_t>(nt) * 4, kAlign) : 0;
 }
 
+// SM count the workspace sizes plan the tiled GEMM's split-K tail for: the
+// current device's (a B200's 148 when there is none to ask).
+int sizing_sms() {
+  DeviceInfo d;
+  if (current_device(&d) == FG8_OK && d.sms > 0) return d.sms;
+  return 148;
+}
+
 // fg8_linear's workspace: the prepare/run layout, then for few tokens the
-// small-M path's (counters beyond the header) and split-K partials.
+// small-M path's (counters beyond the header) and split-K partials, and for
+// the tiled GEMM the partials of its split-K tail (none for most shapes).
 size_t linear_workspace_need(int64_t M, int64_t N, int64_t K, int fmt) {
   size_t need = linear_ws_layout(M, N, K, fmt).total;
-  if (use_small_m(M, N)) need = align_up(need, kAlign) + small_counter_bytes(N) + small_m_partial_bytes(M, N, K);
-  return need;
+  if (use_small_m(M, N)) return align_up(need, kAlign) + small_counter_bytes(N) + small_m_partial_bytes(M, N, K);
+  const size_t area = gemm_split_area(M, N, K, fmt, sizing_sms());
+  return area > 0 ? align_up(need, kAlign) + area : need;
+}
+
+// fg8_gemm_prequant's workspace: its layout, then the split-K tail's partials.
+size_t gemm_workspace_need(int64_t M, int64_t N, int64_t K, int fmt) {
+  const size_t need = gemm_ws_layout(M, N, K, fmt).total;
+  const size_t area = gemm_split_area(M, N, K, fmt, sizing_sms());
+  return area > 0 ? align_up(need, kAlign) + area : need;
+}
+
+// The split-K tail's room inside a workspace whose own layout ends at `base`.
+void set_split_area(GemmArgs& g, void* workspace, size_t workspace_bytes, size_t base) {
+  const size_t off = align_up(base, kAlign);
+  g.split_ws = workspace_bytes > off ? static_cast<uint8_t*>(workspace) + off : nullptr;
+  g.split_bytes = workspace_bytes > off ? workspace_bytes - off : 0;
 }
 
 fg8_status check_workspace(void* ws, size_t bytes, size_t need) {
@@ -325,9 +349,33 @@ size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt
   return linear_workspace_need(M, N, K, fmt);
 }
 
+fg8_status fg8_linear_plan(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt, int32_t* plan) {
+  if (fg8_status st = check_gemm_shape(M, N, K, fmt); st != FG8_OK) return st;
+  if (plan == nullptr) return FG8_ERR_INVALID_ARG;
+  if (M > 0 && use_small_m(M, N)) {
+    plan[0] = use_fused_small_m(M, fmt) ? 2 : 1;
+    plan[1] = 0;
+    plan[2] = 0;
+    plan[3] = 1;
+    return FG8_OK;
+  }
+  const int sms = sizing_sms();
+  const int Kb = ceil_div(K, kGroup), align = fmt == FG8_SCALE_UE8M0 ? 4 : 1;
+  const int bn = choose_block_n(static_cast<int>(M), static_cast<int>(N), Kb, align, sms, true);
+  const int64_t tiles64 = static_cast<int64_t>(ceil_div(M, 128)) * ceil_div(N, bn);
+  const int tiles = static_cast<int>(tiles64 < (int64_t(1) << 30) ? tiles64 : (int64_t(1) << 30));
+  const SplitPlan pl = split_plan(tiles, ceil_div(M, 128), Kb, align, sms);
+  const bool split = pl.from < tiles && tiles - pl.from <= kHeaderCounters;
+  plan[0] = 0;
+  plan[1] = bn;
+  plan[2] = split ? tiles - pl.from : 0;
+  plan[3] = split ? pl.s : 1;
+  return FG8_OK;
+}
+
 size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt) {
   if (check_gemm_shape(M, N, K, fmt) != FG8_OK) return 0;
-  return gemm_ws_layout(M, N, K, fmt).total;
+  return gemm_workspace_need(M, N, K, fmt);
 }
 
 size_t fg8_grouped_linear_workspace_bytes(int64_t M, int64_t E, int64_t N, int64_t K, fg8_scale_fmt fmt) {
@@ -618,7 +666,8 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
                              workspace, stream);
   }
   const LinearWs L = linear_ws_layout(M, N, K, fmt);
-  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
+    return st;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -637,6 +686,7 @@ fg8_status fg8_linear_run(const void* wq_e4m3, const void* w_scale_inv, const vo
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
   g.test_stall = g_test_stall.load();
+  set_split_area(g, workspace, workspace_bytes, L.total);
   if (fmt == FG8_SCALE_FLOAT) {
     g.xs_t = reinterpret_cast<const float*>(ws + L.xs_off);
     g.ld_s = L.ld_s;
@@ -664,7 +714,8 @@ fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, co
     return FG8_ERR_ALIGNMENT;
   const LinearWs L = linear_ws_layout(M, N, K, fmt);
   const LinearWs Ln = linear_ws_layout(M, next_N, N, fmt);
-  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, linear_workspace_need(M, N, K, fmt)); st != FG8_OK)
+    return st;
   if (fg8_status st = check_workspace(next_workspace, next_workspace_bytes, Ln.total); st != FG8_OK) return st;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
@@ -700,6 +751,7 @@ fg8_status fg8_linear_run_chain(const void* wq_e4m3, const void* w_scale_inv, co
   g.nx_w_scale = next_w_scale_inv;
   g.nx_w_prep = wn + Ln.wsc_off;
   g.nx_N = static_cast<int>(next_N);
+  set_split_area(g, workspace, workspace_bytes, L.total);
   return cuda_status(launch_gemm(g, fmt, dev.sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -811,6 +863,9 @@ fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   g.qx = x_bf16;
   g.ld_qx = ld_x;
   g.qflags = reinterpret_cast<uint32_t*>(ws + fused_flags_off(M, N, K, fmt));
+  // the split-K tail as fg8_linear plans it (same tiles and sums, same bits);
+  // its partials end where the flags begin
+  set_split_area(g, workspace, fused_flags_off(M, N, K, fmt), L.total);
   g.qepoch = reinterpret_cast<uint32_t*>(ws + kHeaderEpochOffset);
   if (chain) {
     uint8_t* wn = static_cast<uint8_t*>(next_workspace);
@@ -837,7 +892,8 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
       (bias_bf16 != nullptr && !aligned16(bias_bf16)))
     return FG8_ERR_ALIGNMENT;
   const GemmWs L = gemm_ws_layout(M, N, K, fmt);
-  if (fg8_status st = check_workspace(workspace, workspace_bytes, L.total); st != FG8_OK) return st;
+  if (fg8_status st = check_workspace(workspace, workspace_bytes, gemm_workspace_need(M, N, K, fmt)); st != FG8_OK)
+    return st;
   DeviceInfo dev;
   if (fg8_status st = current_device(&dev); st != FG8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -858,6 +914,7 @@ fg8_status fg8_gemm_prequant(const void* xq_e4m3, const void* x_scale, const voi
   g.status = reinterpret_cast<uint32_t*>(ws);
   g.wait_limit_ns = g_wait_limit_ns.load();
   g.test_stall = g_test_stall.load();
+  set_split_area(g, workspace, workspace_bytes, L.total);
   if (fmt == FG8_SCALE_FLOAT) {
     if (fg8_status st = cuda_status(launch_xs_transpose(static_cast<const float*>(x_scale), static_cast<int>(M), Kb,
                                                         L.ld_s, reinterpret_cast<float*>(ws + L.xs_off), s));

@@ -119,7 +119,32 @@ struct GemmArgs {
   uint32_t* qflags;       // [ceil(M/128) * Kb]
   uint32_t* qepoch;       // the header's words: epoch, finished-CTA count, weight-packing CTA count
   const void* qwsc;       // UE8M0: this layer's weight scales [Nb][Kb], packed into sfb by phase one
+  // Optional: room for the split-K tail (split_plan below): the fp32 partial
+  // sums of the split tiles.  Used when split_bytes covers the plan's
+  // split_area_bytes; its arrival counters are the header's split-K counters
+  // (one per split tile, zero at rest).
+  uint8_t* split_ws;
+  size_t split_bytes;
 };
+
+// Split-K tail of the tiled GEMM.  With T tiles on `sms` persistent CTAs the
+// last wave holds T mod sms tiles and leaves the other SMs idle for a whole
+// tile's K loop.  The plan splits each of those tiles into S work units of
+// kbs consecutive K-blocks (one wave of at most `sms` units); each unit
+// writes its fp32 partial sum, and the tile's last unit to finish adds the S
+// partials in split order (so the result does not depend on which unit
+// finishes last) and stores the tile.  from == tiles: no split.
+struct SplitPlan {
+  int from = 0;  // first split tile (tiles before it run whole)
+  int s = 1;     // units per split tile
+  int kbs = 0;   // K-blocks per unit (the last unit may have fewer)
+};
+SplitPlan split_plan(int tiles, int m_blocks, int Kb, int kb_align, int sms);
+// Bytes of fp32 partials a plan needs with bn-wide tiles.
+size_t split_area_bytes(const SplitPlan& pl, int tiles, int bn);
+// The split-K area a tiled GEMM of this shape may use on a device with `sms`
+// SMs (the larger of the 128- and 256-wide tiles' plans).
+size_t gemm_split_area(int64_t M, int64_t N, int64_t K, int fmt, int sms);
 
 // Rows of the K-major float x-scale matrix: M rounded up to the tallest GEMM
 // tile (256 rows for a CTA pair), so every tile's 128-row slices are in range.
@@ -129,11 +154,13 @@ __host__ __device__ inline int64_t kmajor_ld(int64_t M) { return (M + 255) / 256
 cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, float* out, cudaStream_t s);
 
 // Workspace header: the sticky device status word at byte 0 and, from byte
-// kHeaderCounterOffset, the few-token path's split-K arrival counters (one
-// per 128-row weight tile, zero at rest: the last CTA of a tile resets its
-// counter).  Zeroed by the caller before first use.
+// kHeaderCounterOffset, split-K arrival counters: the few-token path's (one
+// per 128-row weight tile) or the tiled GEMM's split tail (one per split
+// tile); zero at rest, the last CTA of a tile resets its counter.  Zeroed by
+// the caller before first use.
 constexpr size_t kWorkspaceHeaderBytes = 1024;
 constexpr size_t kHeaderEpochOffset = 8;  // fused act-quant: epoch word, then the finished-CTA count
+constexpr size_t kHeaderSchedOffset = 24;  // tiled GEMM: work ticket counter, then the finished-CTA count
 constexpr size_t kHeaderCounterOffset = 64;
 constexpr int kHeaderCounters = static_cast<int>((kWorkspaceHeaderBytes - kHeaderCounterOffset) / 4);
 
@@ -191,7 +218,7 @@ cudaError_t launch_row_expert(const int32_t* counts, int E, int cap, int32_t* ro
                               cudaStream_t st);
 cudaError_t launch_scale_to_e8m0(const float* s, int64_t n, uint8_t* out, uint32_t* bad, int num_sms, cudaStream_t st);
 
-int choose_block_n(int M, int N, int num_sms);
+int choose_block_n(int M, int N, int Kb, int kb_align, int num_sms, bool split);
 
 // fg8_linear's host-side argument checks, workspace excepted (api.cu); an
 // fg8_status value.  Entry points built on fg8_linear run them before their

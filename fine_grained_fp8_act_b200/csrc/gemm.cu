@@ -33,6 +33,12 @@
 // equal ones per 128-block), accumulating the whole K range in TMEM.
 // Ragged edges: TMA zero-fills out-of-range rows/columns of A and B (they add
 // 0), and the bf16 TMA store clips rows >= M and columns >= N.
+// Split-K tail: when the tiles leave the last wave partly empty, each tile of
+// that wave is split over K into units that run on the otherwise idle SMs
+// (split_plan); the epilogues of a tile's first S-1 units write their fp32
+// partials to the workspace and count themselves in, and its last unit waits
+// for them, adds them in split order with its own last, and stores the tile
+// as usual.
 //
 // Every wait is bounded (global-timer limit and a shared abort flag); on
 // expiry the kernel records FG8_ERR_TIMEOUT in the status word, drains its
@@ -104,7 +110,42 @@ struct KParams {
   // one into the scale-factor tiles the producer reads (sfb_w = sfb)
   const uint8_t* wsc_src;
   uint8_t* sfb_w;
+  // split-K tail: work units 0 .. split_from-1 are whole tiles, then every
+  // tile from split_from on is split_s units of split_kbs K-blocks; partials
+  // of units s < split_s - 1: [(tile - split_from) * (split_s - 1) + s][BN * 128]
+  // fp32; split_cnt one arrival counter per split tile (zero at rest)
+  int split_from, split_s, split_kbs, num_work;
+  float* partials;
+  uint32_t* split_cnt;
+  // dynamic schedule: [0] the next work ticket, [1] CTAs finished (both zero
+  // at rest: the last CTA out resets them)
+  uint32_t* sched;
 };
+
+// One unit of a CTA's walk: a tile, the K-blocks [kb0, kb1) it computes, and
+// its split index (-1: the whole tile).
+struct Work {
+  int tile, kb0, kb1, s;
+};
+
+template <class C>
+__device__ __forceinline__ Work work_at(const KParams& p, int u) {
+  Work w;
+  if (!C::SPLIT || u < p.split_from) {
+    w.tile = u;
+    w.kb0 = 0;
+    w.kb1 = p.Kb;
+    w.s = -1;
+  } else {
+    const int j = u - p.split_from;
+    const int t = j / p.split_s;
+    w.tile = p.split_from + t;
+    w.s = j - t * p.split_s;
+    w.kb0 = w.s * p.split_kbs;
+    w.kb1 = min(p.Kb, w.kb0 + p.split_kbs);
+  }
+  return w;
+}
 
 constexpr uint32_t kStatusBadExpert = 1u;  // FG8_ERR_INVALID_ARG
 
@@ -120,9 +161,13 @@ __device__ __forceinline__ int tile_expert(const KParams& p, int m0, bool report
   return e;
 }
 
-template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false, bool SUBK_ = false, bool QIN_ = false>
+template <int BN_, int FMT_, int STAGES_, int OUTBUFS_, bool REQUANT_ = false, bool SUBK_ = false, bool QIN_ = false,
+          bool SPLIT_ = false>
 struct Cfg {
   static constexpr int BN = BN_, FMT = FMT_, STAGES = STAGES_;
+  // SPLIT: the launch has a split-K tail (work units past the whole tiles);
+  // the instance without it carries none of the hand-over code
+  static constexpr bool SPLIT = SPLIT_;
   // QIN: the kernel quantizes its own x (1 x 128 groups) before the tiles
   static constexpr bool QIN = QIN_;
   // REQUANT: the epilogue also quantizes its bf16 output rows, one 128-column
@@ -229,6 +274,38 @@ struct Ring {
     }
   }
 };
+
+// Work queue: the producer claims the CTA's work units -- first unit
+// blockIdx.x, then gridDim.x + a ticket from a global counter, so CTAs that
+// run ahead take more units -- and hands each index to the other roles
+// through kWorkSlots shared slots (an index >= num_work ends the walk).
+constexpr int kWorkSlots = 4;
+struct WorkQ {
+  volatile int* slot;
+  uint64_t* full;
+  uint64_t* empty;  // one arrival per consuming warp (MMA thread, scale warp, epilogue warps)
+};
+
+// The next unit index for a warp (every lane gets it; lane 0 releases the
+// slot), or -1 when the wait gave up.
+__device__ __forceinline__ int take_work_warp(const WorkQ& q, Ring& r, uint64_t limit, volatile int* abort_flag,
+                                              int lane) {
+  if (!mbar_wait_warp(q.full + r.slot, r.phase, limit, abort_flag)) return -1;
+  const int u = q.slot[r.slot];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(q.empty + r.slot);
+  r.template advance<kWorkSlots>();
+  return u;
+}
+
+// The same for a single thread.
+__device__ __forceinline__ int take_work(const WorkQ& q, Ring& r, uint64_t limit, volatile int* abort_flag) {
+  if (!mbar_wait(q.full + r.slot, r.phase, limit, abort_flag)) return -1;
+  const int u = q.slot[r.slot];
+  mbar_arrive(q.empty + r.slot);
+  r.template advance<kWorkSlots>();
+  return u;
+}
 
 // Quantize one output row's 128-column group (bf16-rounded values in `v`) as
 // the next layer's activation group: the same arithmetic, hence the same bits,
@@ -452,17 +529,29 @@ __device__ __forceinline__ bool unit_ready(const KParams& p, uint32_t epoch, int
 template <class C>
 __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
                                          uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* bfull,
-                                         uint64_t* bempty, volatile int* abort_flag, uint32_t epoch) {
+                                         uint64_t* bempty, const WorkQ& wq, volatile int* abort_flag,
+                                         uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring st, bi;
+  Ring st, bi, wr;
   // most recent issue phase per slot, for the drain at the end
   uint32_t st_issued = 0, bi_issued = 0;
   uint32_t st_par[C::STAGES], bi_par[2];
   bool ok = true;
   bool w_packed = false;
-  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
+  for (int u = static_cast<int>(blockIdx.x); ok;
+       u = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.sched, 1u))) {
+    // hand the unit (or the end of the walk) to the other roles
+    if (!mbar_wait(wq.empty + wr.slot, wr.phase ^ 1u, limit, abort_flag)) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    wq.slot[wr.slot] = u;
+    mbar_arrive(wq.full + wr.slot);
+    wr.template advance<kWorkSlots>();
+    if (u >= p.num_work) break;
+    const Work w = work_at<C>(p, u);
     int mb, nb;
-    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
     const int n0 = nb * C::BN;
     const int m0 = mb * kBlockM;
     const int e = tile_expert(p, m0, true);
@@ -484,7 +573,7 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
       bi_issued |= 1u << bi.slot;
       bi.template advance<2>();
     }
-    for (int kb = 0; kb < p.Kb; ++kb) {
+    for (int kb = w.kb0; kb < w.kb1; ++kb) {
       if (!mbar_wait(empty + st.slot, st.phase ^ 1u, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
         ok = false;
@@ -537,9 +626,9 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
 template <class C>
 __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint32_t tmem_base, uint64_t* full,
                                            uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* teardown,
-                                           uint64_t* stall, volatile int* abort_flag) {
+                                           uint64_t* stall, const WorkQ& wq, volatile int* abort_flag) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring st, ab;
+  Ring st, ab, wr;
   bool ok = true;
   // test hook: a barrier nothing arrives on, so the bounded wait runs out
   if (p.test_stall && !mbar_wait(stall, 0, limit, abort_flag)) {
@@ -549,13 +638,20 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   uint32_t sf_set = 1;  // the set the next copy goes to is sf_set ^ 1
   uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
-  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
+  while (ok) {
+    const int u = take_work(wq, wr, limit, abort_flag);
+    if (u < 0) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    if (u >= p.num_work) break;
+    const Work w = work_at<C>(p, u);
     if (p.row_expert != nullptr) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
       if (tile_expert(p, mb * kBlockM, false) < 0) continue;
     }
-    for (int kb = 0; kb < p.Kb; ++kb) {
+    for (int kb = w.kb0; kb < w.kb1; ++kb) {
       if (!mbar_wait(full + st.slot, st.phase, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
         ok = false;
@@ -607,7 +703,7 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
         }
         if (!ok) break;
       } else {
-        if (kb == 0) {
+        if (kb == w.kb0) {
           if (!mbar_wait(tempty + ab.slot, ab.phase ^ 1u, limit, abort_flag)) {
             raise_abort(abort_flag, p.status);
             ok = false;
@@ -636,9 +732,9 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
           // the byte of each row's scale word: the K-block's (1 x 128 groups) or the step's (1 x 32, 1 x 64)
           const uint32_t j = static_cast<uint32_t>(p.sf_shift == 0 ? k : (kb & 3));
           mma_mxf8f6f4(d, ad, bd, C::kIdesc | (j << 29) | (j << 4), sfa_t | (j << 30), sfb_t | (j << 30),
-                       (kb > 0 || k > 0) ? 1u : 0u);
+                       (kb > w.kb0 || k > 0) ? 1u : 0u);
         }
-        if (kb == p.Kb - 1) {
+        if (kb == w.kb1 - 1) {
           tc_commit(tfull + ab.slot);
           ab.template advance<C::kNumAcc>();
         }
@@ -662,12 +758,19 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
 // latency stays off the epilogue's path.  The epilogue warps release slots.
 template <class C>
 __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
-                                             volatile int* abort_flag, int lane, uint32_t epoch) {
+                                             const WorkQ& wq, volatile int* abort_flag, int lane, uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring sr;
-  for (int tile = static_cast<int>(blockIdx.x); tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
+  Ring sr, wr;
+  for (;;) {
+    const int u = take_work_warp(wq, wr, limit, abort_flag, lane);
+    if (u < 0) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    if (u >= p.num_work) break;
+    const Work w = work_at<C>(p, u);
     int mb, nb;
-    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
     const int e = tile_expert(p, mb * kBlockM, false);
     if (e < 0) continue;
     const float* xs = p.xs_t + mb * kBlockM + 4 * lane;
@@ -676,7 +779,8 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
     const int nwb = C::BN / p.wblk;
     const int wb = e * p.Nbs + min(nb * C::BN / p.wblk + (lane & 7), p.Nbs - 1);
     const float* ws = p.w_scale + static_cast<int64_t>(wb) * p.Kg;
-    for (int g = 0; g < p.Kg; ++g) {
+    const int g1 = min(p.Kg, w.kb1 * p.gsteps);
+    for (int g = w.kb0 * p.gsteps; g < g1; ++g) {
       if (!mbar_wait_warp(sempty + sr.slot, sr.phase ^ 1u, limit, abort_flag)) {
         raise_abort(abort_flag, p.status);
         cp_async_wait_all();
@@ -700,7 +804,8 @@ __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, ui
 template <class C>
 __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& p, uint8_t* smem, uint32_t tmem_base,
                                          uint64_t* tfull, uint64_t* tempty, uint64_t* bfull, uint64_t* bempty,
-                                         uint64_t* sfull, uint64_t* sempty, volatile int* abort_flag, int warp,
+                                         uint64_t* sfull, uint64_t* sempty, uint64_t* xbar, uint64_t* ybar,
+                                         volatile uint32_t* xlast, const WorkQ& wq, volatile int* abort_flag, int warp,
                                          int lane) {
   const uint64_t limit = p.wait_limit_ns;
   const int ew = warp - 4;
@@ -709,12 +814,20 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   const int col0 = wg * C::kCols;
   uint8_t* stg = smem + C::kOffStaging + ew * C::kOutBufs * C::kOutBuf;
   const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-  Ring ab, bi, sr;
+  Ring ab, bi, sr, wr;
   bool ok = true;
   const int sub_row = q * 32 + lane;  // this thread's row inside a tile
-  for (int tile = static_cast<int>(blockIdx.x); ok && tile < p.num_tiles; tile += static_cast<int>(gridDim.x)) {
+  uint32_t xph = 0;                   // parity of the split hand-over barriers
+  while (ok) {
+    const int u = take_work_warp(wq, wr, limit, abort_flag, lane);
+    if (u < 0) {
+      raise_abort(abort_flag, p.status);
+      break;
+    }
+    if (u >= p.num_work) break;
+    const Work w = work_at<C>(p, u);
     int mb, nb;
-    tile_coords(tile, p.num_m, p.num_n, mb, nb);
+    tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
     if (tile_expert(p, mb * kBlockM, false) < 0) continue;
     const int row0 = mb * kBlockM + q * 32;
     // the tile's bias (bias ring; zeros past N or without bias)
@@ -726,10 +839,11 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
     uint32_t acc[C::kCols];  // float bits
     if constexpr (C::FMT == 0) {
       // the promotion accumulates onto the bias: y = bias + sum_kb P_kb * s_kb
+      // (a split tile's first unit starts from the bias, the others from 0)
 #pragma unroll
       for (int i = 0; i < C::kCols / 8; ++i) {
         uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-        if (p.bias != nullptr && nb * C::BN + col0 + 8 * i < p.N)
+        if (p.bias != nullptr && w.s <= 0 && nb * C::BN + col0 + 8 * i < p.N)
           bv = *reinterpret_cast<const uint4*>(bias_s + (col0 + 8 * i) * 2);
         const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
@@ -741,7 +855,8 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       __syncwarp();
       if (lane == 0) mbar_arrive(bempty + bi.slot);
       bi.template advance<2>();
-      for (int g = 0; g < p.Kg; ++g) {
+      const int g1 = min(p.Kg, w.kb1 * p.gsteps);
+      for (int g = w.kb0 * p.gsteps; g < g1; ++g) {
         // sx(m, g) * sw(block of the chunk's columns, g) from the scale ring
         if (!mbar_wait_warp(sfull + sr.slot, sr.phase, limit, abort_flag)) {
           raise_abort(abort_flag, p.status);
@@ -825,6 +940,87 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
       ab.template advance<C::kNumAcc>();
     }
 
+    if (C::SPLIT && w.s >= 0) {
+      // A unit of a split tile.  Units 0 .. S-2 write their partial sums
+      // (fp32, each thread's columns as float4s, contiguous per warp) and
+      // count themselves in; unit S-1 waits for that count, adds the others'
+      // partials in split order and its own last, and goes on to store the
+      // tile.  All units of a split tile are in the last wave (one per CTA).
+      constexpr int kVec = C::kCols / 4;
+      const int j = w.tile - p.split_from;
+      const int et = ew * 32 + lane;
+      const bool reducer = w.s == p.split_s - 1;
+      const float4* part = reinterpret_cast<const float4*>(p.partials) +
+                           static_cast<int64_t>(j) * (p.split_s - 1) * (kVec * 256) + et;
+      if (!reducer) {
+        float4* mine = const_cast<float4*>(part) + static_cast<int64_t>(w.s) * (kVec * 256);
+#pragma unroll
+        for (int i = 0; i < kVec; ++i)
+          __stcg(mine + i * 256, make_float4(__uint_as_float(acc[4 * i]), __uint_as_float(acc[4 * i + 1]),
+                                             __uint_as_float(acc[4 * i + 2]), __uint_as_float(acc[4 * i + 3])));
+        __threadfence();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (ew == 0 && lane == 0) {
+        bool fine = mbar_wait(xbar, xph, limit, abort_flag);
+        if (fine && !reducer) {
+          __threadfence();
+          atomicAdd(p.split_cnt + j, 1u);
+        } else if (fine) {  // every other unit's partial is out; zero the counter for the next call
+          fine = flag_wait(p.split_cnt + j, static_cast<uint32_t>(p.split_s - 1), limit, abort_flag);
+          if (fine) {
+            __threadfence();
+            atomicExch(p.split_cnt + j, 0u);
+          }
+        }
+        *xlast = fine ? 1u : 2u;
+        mbar_arrive(ybar);
+      }
+      const bool got = mbar_wait_warp(ybar, xph, limit, abort_flag);
+      xph ^= 1u;
+      if (!got || *xlast == 2u) {
+        raise_abort(abort_flag, p.status);
+        break;
+      }
+      if (!reducer) {
+        if constexpr (C::FMT == 1) {  // the bias slot is not needed
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bempty + bi.slot);
+          bi.template advance<2>();
+        }
+        continue;
+      }
+      constexpr int kBatch = 4;  // float4s per thread in flight per partial
+#pragma unroll
+      for (int i0 = 0; i0 < kVec; i0 += kBatch) {
+        float4 t[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) t[i] = __ldcg(part + (i0 + i) * 256);
+        for (int sp = 1; sp < p.split_s - 1; ++sp) {
+          const float4* ps = part + static_cast<int64_t>(sp) * (kVec * 256);
+          float4 r[kBatch];
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) r[i] = __ldcg(ps + (i0 + i) * 256);
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) {
+            t[i].x = __fadd_rn(t[i].x, r[i].x);
+            t[i].y = __fadd_rn(t[i].y, r[i].y);
+            t[i].z = __fadd_rn(t[i].z, r[i].z);
+            t[i].w = __fadd_rn(t[i].w, r[i].w);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          uint32_t* a = acc + 4 * (i0 + i);
+          a[0] = __float_as_uint(__fadd_rn(t[i].x, __uint_as_float(a[0])));
+          a[1] = __float_as_uint(__fadd_rn(t[i].y, __uint_as_float(a[1])));
+          a[2] = __float_as_uint(__fadd_rn(t[i].z, __uint_as_float(a[2])));
+          a[3] = __float_as_uint(__fadd_rn(t[i].w, __uint_as_float(a[3])));
+        }
+      }
+    }
+
     // (UE8M0: + bias), round to bf16, stage 32 x 32 boxes (64-byte swizzle),
     // store them with TMA: one proxy fence and one bulk group per batch of
     // kOutBufs boxes.
@@ -904,9 +1100,18 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* sempty = sfull + C::kSRing;
   uint64_t* teardown = sempty + C::kSRing;
   uint64_t* stall = teardown + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall + 1);
+  uint64_t* xbar = stall + 1;  // split tiles: the epilogue warps' partials are out
+  uint64_t* ybar = xbar + 1;   // ... and the unit has been counted (verdict in xlast)
+  WorkQ wq;
+  wq.full = ybar + 1;
+  wq.empty = wq.full + kWorkSlots;
+  wq.slot = reinterpret_cast<volatile int*>(wq.empty + kWorkSlots);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wq.empty + kWorkSlots) + kWorkSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert(C::kOffBar + 8 * (2 * C::STAGES + 2 * C::kNumAcc + 4 + 2 * C::kSRing + 2) + 8 <= C::kOffBar + 512,
+  volatile uint32_t* xlast = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+  static_assert(C::kOffBar + 8 * (2 * C::STAGES + 2 * C::kNumAcc + 4 + 2 * C::kSRing + 4 + 2 * kWorkSlots) +
+                        4 * kWorkSlots + 16 <=
+                    C::kOffBar + 512,
                 "barrier block");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -933,6 +1138,12 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(teardown, 1);
     mbar_init(stall, 1);
+    mbar_init(xbar, C::kEpiWarps);
+    mbar_init(ybar, 1);
+    for (int s = 0; s < kWorkSlots; ++s) {
+      mbar_init(wq.full + s, 1);
+      mbar_init(wq.empty + s, 1 + (C::FMT == 0 ? 1 : 0) + C::kEpiWarps);  // MMA, scale warp, epilogue warps
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -957,11 +1168,11 @@ __global__ void __launch_bounds__(384, 1)
   if (warp < 4) {
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
-      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag, epoch);
+      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, wq, abort_flag, epoch);
     else if (warp == 1 && lane == 0)
-      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, abort_flag);
+      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, wq, abort_flag);
     if constexpr (C::FMT == 0) {
-      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, abort_flag, lane, epoch);
+      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, wq, abort_flag, lane, epoch);
     }
     if constexpr (C::REQUANT && C::FMT == 1) {
       if (warp == 2 || warp == 3)
@@ -970,13 +1181,24 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
-    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, sfull, sempty, abort_flag, warp, lane);
+    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, sfull, sempty, xbar, ybar, xlast, wq,
+                abort_flag, warp, lane);
   }
 
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
+  }
+  // the last CTA out puts the ticket counter back to zero (every CTA has
+  // taken its last ticket by now)
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      p.sched[0] = 0u;
+      p.sched[1] = 0u;
+      __threadfence();
+    }
   }
   if constexpr (C::QIN) {
     // the last CTA out advances the epoch: every CTA has read it and every
@@ -1075,11 +1297,32 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.qflags = g.qflags;
   p.qepoch = g.qepoch;
   p.xq_w = static_cast<uint8_t*>(const_cast<void*>(g.xq));
-  p.xs_w = C::FMT == 0 ? static_cast<void*>(const_cast<float*>(g.xs_t)) : static_cast<void*>(const_cast<uint8_t*>(g.sfa));
+  p.xs_w = C::FMT == 0 ? static_cast<void*>(const_cast<float*>(g.xs_t))
+                       : static_cast<void*>(const_cast<uint8_t*>(g.sfa));
   p.M_pad = (g.M + kBlockM - 1) / kBlockM * kBlockM;
   p.wsc_src = static_cast<const uint8_t*>(g.qwsc);
   p.sfb_w = const_cast<uint8_t*>(g.sfb);
   if (p.num_tiles == 0) return cudaSuccess;
+  // the split-K tail: tiled GEMMs with room for the partials (not the
+  // expert-grouped or sliced-promotion variants)
+  p.split_from = p.num_tiles;
+  p.split_s = 1;
+  p.split_kbs = p.Kb;
+  p.partials = nullptr;
+  p.split_cnt = nullptr;
+  if (C::SPLIT && g.row_expert == nullptr && g.split_ws != nullptr) {
+    const SplitPlan pl = split_plan(p.num_tiles, p.num_m, p.Kb, C::FMT == 1 && !g.sf32 ? 4 : 1, num_sms);
+    if (pl.from < p.num_tiles && split_area_bytes(pl, p.num_tiles, C::BN) <= g.split_bytes &&
+        p.num_tiles - pl.from <= kHeaderCounters) {
+      p.split_from = pl.from;
+      p.split_s = pl.s;
+      p.split_kbs = pl.kbs;
+      p.partials = reinterpret_cast<float*>(g.split_ws);
+      p.split_cnt = g.status + kHeaderCounterOffset / 4;
+    }
+  }
+  p.num_work = p.split_from + (p.num_tiles - p.split_from) * p.split_s;
+  p.sched = g.status + kHeaderSchedOffset / 4;
 
   // the shared-memory opt-in once per device: one bit per device; calls from
   // several host threads may repeat it, which is harmless
@@ -1103,26 +1346,97 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cfg.gridDim = dim3(p.num_tiles < num_sms ? p.num_tiles : num_sms);
+  cfg.gridDim = dim3(p.num_work < num_sms ? p.num_work : num_sms);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+template <class Plain, class Split>
+cudaError_t launch_either(bool split, const GemmArgs& g, int num_sms, cudaStream_t s) {
+  return split ? launch_cfg<Split>(g, num_sms, s) : launch_cfg<Plain>(g, num_sms, s);
+}
+
+// Estimated time of a split tail: units of k K-blocks, se of them per tile
+// (K-block periods; see split_plan).
+double split_cost(int k, int se) { return k + 4.0 + 3.0 * (se - 1); }
+
 }  // namespace
 
-int choose_block_n(int M, int N, int num_sms) {
-  // Per-CTA time ~ waves x (tile width / its throughput); the 256-wide tile
-  // moves ~1.6x more MMA work per operand byte and per epilogue instruction,
-  // so the 128-wide tile wins only when it cuts the wave count a lot.
+SplitPlan split_plan(int tiles, int m_blocks, int Kb, int kb_align, int sms) {
+  SplitPlan pl;
+  pl.from = tiles;
+  pl.kbs = Kb;
+  // Measured on the B200: with fewer than 64 K-blocks per tile, or more
+  // than 6 whole waves before the tail, the CTAs' spread in finishing their
+  // whole tiles eats the gain; with a single row block the tiles stream
+  // distinct weights and are bound by that, split or not.
+  if (tiles <= 0 || sms <= 0 || Kb < 64 || m_blocks < 2 || tiles / sms > 6) return pl;
+  const int rem = tiles % sms;
+  if (rem == 0) return pl;
+  // Cost of the tail in K-block periods: unsplit, a whole tile's K loop;
+  // split, a unit's K-blocks plus the write-back of the partials, the wait
+  // and the last unit's reading of the other S - 1 partials (128 KB each
+  // from L2 at ~0.1 TB/s per SM against ~0.6 us per 128 x 256 x 128
+  // K-block), fitted to timings of 2048- to 8192-token layers.
+  double best = Kb;
+  for (int S = 2; S <= Kb && rem * S <= sms; ++S) {
+    const int kbs = (Kb + S - 1) / S;
+    const int k = (kbs + kb_align - 1) / kb_align * kb_align;
+    const int se = (Kb + k - 1) / k;
+    if (se < 2 || rem * se > sms) continue;
+    const double cost = split_cost(k, se);
+    if (cost < best) {
+      best = cost;
+      pl.from = tiles - rem;
+      pl.s = se;
+      pl.kbs = k;
+    }
+  }
+  return pl;
+}
+
+size_t split_area_bytes(const SplitPlan& pl, int tiles, int bn) {
+  if (pl.from >= tiles) return 0;
+  // the last unit of a tile keeps its partial in registers
+  return static_cast<size_t>(tiles - pl.from) * (pl.s - 1) * bn * kBlockM * sizeof(float);
+}
+
+size_t gemm_split_area(int64_t M, int64_t N, int64_t K, int fmt, int sms) {
   const int64_t m_tiles = (M + kBlockM - 1) / kBlockM;
-  auto waves = [&](int bn) {
+  const int Kb = static_cast<int>((K + 127) / 128);
+  size_t area = 0;
+  for (int bn : {128, 256}) {
     const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
-    return (tiles + num_sms - 1) / num_sms;
+    if (tiles > (int64_t(1) << 30)) continue;
+    const int t = static_cast<int>(tiles);
+    const SplitPlan pl = split_plan(t, static_cast<int>(m_tiles), Kb, fmt == 1 ? 4 : 1, sms);
+    if (t - pl.from > kHeaderCounters) continue;
+    const size_t a = split_area_bytes(pl, t, bn);
+    if (a > area) area = a;
+  }
+  return area;
+}
+
+int choose_block_n(int M, int N, int Kb, int kb_align, int num_sms, bool split) {
+  const int m_blocks = static_cast<int>((M + kBlockM - 1) / kBlockM);
+  // Per-CTA time in K-block periods of the tile: the whole waves' K loops
+  // plus the tail (unsplit: one more K loop; split: the plan's estimate).
+  // The 256-wide tile moves ~1.6x more MMA work per operand byte and per
+  // epilogue instruction, so a 128-wide K-block costs ~0.6 / 0.5 of one.
+  const int64_t m_tiles = (M + kBlockM - 1) / kBlockM;
+  auto cost = [&](int bn) {
+    const int64_t tiles64 = m_tiles * ((N + bn - 1) / bn);
+    const int tiles = static_cast<int>(tiles64 < (int64_t(1) << 30) ? tiles64 : (int64_t(1) << 30));
+    double t = static_cast<double>((tiles + num_sms - 1) / num_sms) * Kb;
+    if (split) {
+      const SplitPlan pl = split_plan(tiles, m_blocks, Kb, kb_align, num_sms);
+      if (pl.from < tiles && tiles - pl.from <= kHeaderCounters)
+        t = static_cast<double>(pl.from / num_sms) * Kb + split_cost(pl.kbs, pl.s);
+    }
+    return t * (bn == 128 ? 128.0 / 0.6 : 256.0);
   };
-  const double cost128 = static_cast<double>(waves(128)) * 128.0 / 0.6;
-  const double cost256 = static_cast<double>(waves(256)) * 256.0;
-  return cost128 < cost256 ? 128 : 256;
+  return cost(128) < cost(256) ? 128 : 256;
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s) {
@@ -1131,47 +1445,77 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   // Long K: four stages (the float path's scale ring takes the shared memory
   // of the second staging box per warp).
   const bool short_k = g.Kb <= 32;
+  const int align = fmt == 1 ? 4 : 1;
+  // (the split-K tail only runs for block-128 scales with room for it)
+  const bool may_split = g.split_ws != nullptr && g.row_expert == nullptr && !g.sf32 && (g.wblk == 0 || g.wblk == 128);
+  // does the plan for bn-wide tiles split (and fit the room)?  Then the
+  // launch takes the instance with the hand-over code.
+  auto splits = [&](int bn) {
+    if (!may_split) return false;
+    const int m_tiles = (g.M + kBlockM - 1) / kBlockM;
+    const int tiles = m_tiles * ((g.N + bn - 1) / bn);
+    const SplitPlan pl = split_plan(tiles, m_tiles, g.Kb, align, num_sms);
+    return pl.from < tiles && tiles - pl.from <= kHeaderCounters && split_area_bytes(pl, tiles, bn) <= g.split_bytes;
+  };
   if (g.qx != nullptr) {  // x quantized inside the kernel: short K only (see can_quantize_in_gemm)
     if (!short_k || g.wblk > 0 && g.wblk != 128 || g.row_expert != nullptr) return cudaErrorInvalidValue;
     const bool requant = g.nx_xq != nullptr;
-    const int bnq = requant ? 256 : choose_block_n(g.M, g.N, num_sms);
+    // the tile width fg8_linear picks, so that both give the same bits
+    const int bnq = requant ? 256 : choose_block_n(g.M, g.N, g.Kb, align, num_sms, may_split);
+    const bool sp = splits(bnq);
     if (fmt == 0) {
-      if (requant) return launch_cfg<Cfg<256, 0, 3, 4, true, false, true>>(g, num_sms, s);
-      if (bnq == 256) return launch_cfg<Cfg<256, 0, 3, 4, false, false, true>>(g, num_sms, s);
-      return launch_cfg<Cfg<128, 0, 5, 2, false, false, true>>(g, num_sms, s);
+      if (requant)
+        return launch_either<Cfg<256, 0, 3, 4, true, false, true>, Cfg<256, 0, 3, 4, true, false, true, true>>(
+            sp, g, num_sms, s);
+      if (bnq == 256)
+        return launch_either<Cfg<256, 0, 3, 4, false, false, true>, Cfg<256, 0, 3, 4, false, false, true, true>>(
+            sp, g, num_sms, s);
+      return launch_either<Cfg<128, 0, 5, 2, false, false, true>, Cfg<128, 0, 5, 2, false, false, true, true>>(
+          sp, g, num_sms, s);
     }
-    if (requant) return launch_cfg<Cfg<256, 1, 3, 4, true, false, true>>(g, num_sms, s);
-    if (bnq == 256) return launch_cfg<Cfg<256, 1, 3, 4, false, false, true>>(g, num_sms, s);
-    return launch_cfg<Cfg<128, 1, 5, 2, false, false, true>>(g, num_sms, s);
+    if (requant)
+      return launch_either<Cfg<256, 1, 3, 4, true, false, true>, Cfg<256, 1, 3, 4, true, false, true, true>>(
+          sp, g, num_sms, s);
+    if (bnq == 256)
+      return launch_either<Cfg<256, 1, 3, 4, false, false, true>, Cfg<256, 1, 3, 4, false, false, true, true>>(
+          sp, g, num_sms, s);
+    return launch_either<Cfg<128, 1, 5, 2, false, false, true>, Cfg<128, 1, 5, 2, false, false, true, true>>(
+        sp, g, num_sms, s);
   }
   if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
+    const bool sp = splits(256);
     if (fmt == 0) {
-      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, true>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 1, true>>(g, num_sms, s);
+      if (short_k)
+        return launch_either<Cfg<256, 0, 3, 4, true>, Cfg<256, 0, 3, 4, true, false, false, true>>(sp, g, num_sms, s);
+      return launch_either<Cfg<256, 0, 4, 1, true>, Cfg<256, 0, 4, 1, true, false, false, true>>(sp, g, num_sms, s);
     }
-    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, true>>(g, num_sms, s);
-    return launch_cfg<Cfg<256, 1, 4, 1, true>>(g, num_sms, s);
+    if (short_k)
+      return launch_either<Cfg<256, 1, 3, 4, true>, Cfg<256, 1, 3, 4, true, false, false, true>>(sp, g, num_sms, s);
+    return launch_either<Cfg<256, 1, 4, 1, true>, Cfg<256, 1, 4, 1, true, false, false, true>>(sp, g, num_sms, s);
   }
-  const int bn = choose_block_n(g.M, g.N, num_sms);
-  if (fmt == 0 && g.wblk != 0 && g.wblk != 128) {  // float at block 64 / 32
+  const int bn = choose_block_n(g.M, g.N, g.Kb, align, num_sms, may_split);
+  if (fmt == 0 && g.wblk != 0 && g.wblk != 128) {  // float at block 64 / 32 (never split)
     if (bn == 256) {
       if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, false, true>>(g, num_sms, s);
       return launch_cfg<Cfg<256, 0, 4, 1, false, true>>(g, num_sms, s);
     }
     return launch_cfg<Cfg<128, 0, 5, 2, false, true>>(g, num_sms, s);
   }
+  const bool sp = splits(bn);
   if (fmt == 0) {
     if (bn == 256) {
-      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);
-      return launch_cfg<Cfg<256, 0, 4, 1>>(g, num_sms, s);
+      if (short_k)
+        return launch_either<Cfg<256, 0, 3, 4>, Cfg<256, 0, 3, 4, false, false, false, true>>(sp, g, num_sms, s);
+      return launch_either<Cfg<256, 0, 4, 1>, Cfg<256, 0, 4, 1, false, false, false, true>>(sp, g, num_sms, s);
     }
-    return launch_cfg<Cfg<128, 0, 5, 2>>(g, num_sms, s);
+    return launch_either<Cfg<128, 0, 5, 2>, Cfg<128, 0, 5, 2, false, false, false, true>>(sp, g, num_sms, s);
   }
   if (bn == 256) {
-    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4>>(g, num_sms, s);
-    return launch_cfg<Cfg<256, 1, 4, 1>>(g, num_sms, s);
+    if (short_k)
+      return launch_either<Cfg<256, 1, 3, 4>, Cfg<256, 1, 3, 4, false, false, false, true>>(sp, g, num_sms, s);
+    return launch_either<Cfg<256, 1, 4, 1>, Cfg<256, 1, 4, 1, false, false, false, true>>(sp, g, num_sms, s);
   }
-  return launch_cfg<Cfg<128, 1, 5, 2>>(g, num_sms, s);
+  return launch_either<Cfg<128, 1, 5, 2>, Cfg<128, 1, 5, 2, false, false, false, true>>(sp, g, num_sms, s);
 }
 
 }  // namespace fg8

@@ -19,10 +19,11 @@
 
 namespace {
 
-// 32 MiB: enough for, e.g., 8192 tokens x 3584 input channels, or the ESM-2
-// and Llama-3-8B shapes up to 2048 tokens (the workspace is M*K bytes of
-// quantized activations plus their scales and the weight scales).
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+// 64 MiB: enough for, e.g., 8192 tokens x 7168 input channels, or the ESM-2
+// and Llama-3-8B shapes up to 4096 tokens (the workspace is M*K bytes of
+// quantized activations plus their scales and the weight scales, and up to
+// 148 x 128 KiB of split-K partials for the tiled GEMM's last wave).
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 
 // The scratch.  In host code this name is only a stand-in for the device
 // symbol; the device address comes from cudaGetSymbolAddress below.

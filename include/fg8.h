@@ -93,8 +93,30 @@ FG8_API fg8_status fg8_quantize_act(const void* x_bf16, int64_t M, int64_t K, in
 
 /* Bytes of caller-owned device workspace fg8_linear needs for this shape
  * (quantized activations, their scales in the GEMM's layout, the scale-factor
- * tiles of the UE8M0 path and a device status word).  0 on bad arguments. */
+ * tiles of the UE8M0 path, a device status word, and the fp32 partial sums of
+ * the few-token kernel's split K or of the tiled GEMM's split-K tail, see
+ * fg8_linear_plan).  The tail is planned for the current device's SM count
+ * (148 when no device is visible); a workspace sized on a device with another
+ * count is still accepted, the tail then runs unsplit.  0 on bad arguments. */
 FG8_API size_t fg8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
+
+/* How fg8_linear runs this shape on the current device (148 SMs when none
+ * is visible), for callers that size launches or read profiles:
+ *   plan[0]  kernel: 0 the tiled GEMM, 1 the few-token split-K kernel on the
+ *            prepare step's activations, 2 the few-token kernel that also
+ *            quantizes x (no prepare launch)
+ *   plan[1]  tiled GEMM: tile width (128 or 256 output columns; 128 rows)
+ *   plan[2]  tiled GEMM: tiles of the last wave split over K (0: none)
+ *   plan[3]  tiled GEMM: work units per split tile (1: none).  The tiles of
+ *            the last, partial wave of persistent CTAs are each cut into
+ *            plan[3] runs of consecutive K-blocks on otherwise idle SMs; a
+ *            tile's last unit adds the fp32 partials in split order (the
+ *            same bits whichever unit finishes last), so these tiles' sums
+ *            round differently from a whole tile's, within the tolerance.
+ * fg8_linear_run_chain always uses 256-wide tiles (and its own tail plan);
+ * fg8_gemm_prequant, fg8_linear_static and fg8_linear_fused use fg8_linear's.
+ * Returns FG8_ERR_INVALID_ARG on bad arguments or a NULL plan. */
+FG8_API fg8_status fg8_linear_plan(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt, int32_t* plan);
 
 /* The layer ([zh] §八 step 6, FP8Linear.forward -> fp8_linear; [zh] §6.1 the
  * block (128,128) + dynamic-activation fast path):
@@ -207,11 +229,11 @@ FG8_API fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, in
  * can synchronize the device).  The pages have no counterpart of this entry
  * point; it computes exactly what fg8_linear computes, with the same
  * arguments minus the workspace.
- *   - Scratch: a fixed 32 MiB array in this library's device memory (a
+ *   - Scratch: a fixed 64 MiB array in this library's device memory (a
  *     file-scope __device__ array; every device that loads the library keeps
  *     it until the process exits).  No call allocates or frees anything.
  *   - Size limit: shapes whose fg8_linear_workspace_bytes(M, N, K, fmt)
- *     exceeds 32 MiB return FG8_ERR_WORKSPACE without launching.
+ *     exceeds 64 MiB return FG8_ERR_WORKSPACE without launching.
  *   - The first call on each device looks up the scratch's device address
  *     (this may load the library's device module); make that first call
  *     before any stream capture on that device.
@@ -226,7 +248,8 @@ FG8_API fg8_status fg8_linear_noalloc(const void* x_bf16, int64_t M, int64_t N, 
                                       const void* wq_e4m3, const void* w_scale_inv, const void* bias_bf16,
                                       void* y_bf16, int64_t ld_y, fg8_scale_fmt fmt, void* stream);
 
-/* Bytes of workspace fg8_gemm_prequant needs.  0 on bad arguments. */
+/* Bytes of workspace fg8_gemm_prequant needs (with room for the tiled GEMM's
+ * split-K tail, as fg8_linear_workspace_bytes).  0 on bad arguments. */
 FG8_API size_t fg8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, fg8_scale_fmt fmt);
 
 /* The GEMM alone on already-quantized activations (the layouts

@@ -189,6 +189,26 @@ def test_workspace_sizes(fg8):
     assert fg8.fg8_gemm_workspace_bytes(16, 256, 256, 1) >= 256 + 512 + 2 * 512
 
 
+def test_split_tail_workspace(fg8):
+    """The tiled GEMM's split-K tail: fg8_linear's workspace adds room for the
+    fp32 partials of the last wave's split tiles (128 x 128 or 128 x 256 per
+    unit, at most one wave of 148 units) on top of the layout that the
+    expert-grouped layer (which never splits) shares with it, and nothing
+    when both tile widths fill whole waves on 148 SMs."""
+    raw = _raw(fg8)
+    lin, grp = fg8.fg8_linear_workspace_bytes, raw.fg8_grouped_linear_workspace_bytes
+    M = 148 * 128  # 148 tiles of 128 x 256, 296 of 128 x 128, for N = 256
+    assert lin(M, 256, 4096, 0) == grp(M, 1, 256, 4096, 0)
+    for M, N, K in [(256, 2048, 8192), (2560, 2048, 8192), (2048, 12288, 12288), (4096, 4096, 14336)]:
+        extra = lin(M, N, K, 0) - grp(M, 1, N, K, 0)
+        assert extra > 0 and extra % (128 * 128 * 4) == 0 and extra <= 148 * 128 * 256 * 4 + 256, (M, N, K, extra)
+        assert fg8.fg8_linear_fused_workspace_bytes(M, N, K, 0) > lin(M, N, K, 0)
+    # too few K-blocks to pay for a split (the ESM-2 layer shapes), one row
+    # block, or many whole waves before the tail
+    for M, N, K in [(8176, 1920, 480), (64, 12288, 12288), (8192, 7168, 18432)]:
+        assert lin(M, N, K, 0) == grp(M, 1, N, K, 0), (M, N, K)
+
+
 def test_scale_fmt_validation(fg8):
     from fine_grained_fp8_act_b200 import scale_fmt_code
     assert scale_fmt_code("float") == 0 and scale_fmt_code("ue8m0") == 1

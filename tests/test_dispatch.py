@@ -1,8 +1,6 @@
 """The shape rule that picks the few-token kernel (C++) and its mirror in
-bench.py agree.  Without a GPU the library's choice shows in its workspace
-size: with float scales the prepare layout does not depend on N, so extra
-bytes are the few-token kernel's split-K partials (K = 8192 keeps the split
-count above 1 wherever that kernel runs with at most 74 weight tiles)."""
+bench.py agree (the library's choice read back through fg8_linear_plan), and
+the tiled GEMM's split-K tail plan behaves as documented."""
 import pytest
 
 import workloads as W
@@ -22,15 +20,9 @@ def fg8():
 def test_few_token_rule_matches_bench(fg8, M, N):
     import bench
     K = 8192
-    need = fg8.fg8_linear_workspace_bytes(M, N, K, 0)
-    tiled_need = fg8.fg8_linear_workspace_bytes(M, 1 << 20, K, 0)  # far past the rule: tiled
-    nt = -(-N // 128)
-    lib_small = need > tiled_need
+    lib_small = fg8.fg8_linear_plan(M, N, K, 0)[0] != 0
     bench_small = bench.layer_path(W.Gemm("t", M, K, N, 0)) != "tiled"
-    if 148 // nt >= 2:  # the few-token kernel would split K: its choice is visible
-        assert lib_small == bench_small, (M, N, lib_small, bench_small)
-    else:  # one split, no partials either way; the rule itself says tiled here
-        assert not lib_small and not bench_small
+    assert lib_small == bench_small, (M, N, lib_small, bench_small)
 
 
 def test_rule_boundaries(fg8):
@@ -40,3 +32,37 @@ def test_rule_boundaries(fg8):
     assert g(128, 9472) == "small" and g(128, 9480) == "tiled"           # ceil(N/256) <= 37
     assert g(129, 256) == "tiled"
     assert g(16, 4096, 1) == "fused" and g(17, 4096, 1) == "small" and g(16, 4096, 0) == "small"
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_rule_through_the_plan(fg8, fmt):
+    import bench
+    for M, N in [(1, 4096), (16, 4096), (17, 4096), (32, 1 << 16), (33, 1 << 16), (128, 9472), (128, 9480)]:
+        kind = fg8.fg8_linear_plan(M, N, 4096, fmt)[0]
+        path = bench.layer_path(W.Gemm("t", M, 4096, N, fmt))
+        assert kind == {"tiled": 0, "small": 1, "fused": 2}[path], (M, N, fmt, kind, path)
+
+
+def test_split_tail_plan(fg8):
+    """Whole waves on 148 SMs: no split.  Otherwise the last wave's tiles are
+    split so that all their units fit one wave, where a unit's K-blocks plus
+    the partials' write-back, wait and read-back beat a whole tile's K loop,
+    with at least 64 K-blocks, two row blocks and at most 6 whole waves."""
+    plan = fg8.fg8_linear_plan
+    # 16384 x 12288 x 12288: 6144 tiles of 128 x 256, 76 in the last wave
+    # (two units each would not fit one wave); 41 whole waves anyway
+    assert plan(16384, 12288, 12288, 0) == (0, 256, 0, 1)
+    # 2048 x 12288 x 12288: 768 tiles = 5 waves + 28; 5 units of 20 K-blocks
+    assert plan(2048, 12288, 12288, 0) == (0, 256, 28, 5)
+    assert plan(2048, 12288, 12288, 1) == (0, 256, 28, 5)
+    # 512 tokens: 192 tiles = 1 wave + 44; 3 units of 32 K-blocks
+    assert plan(512, 12288, 12288, 0) == (0, 256, 44, 3)
+    # one row block (streams the weights), too few K-blocks, too many waves
+    assert plan(64, 12288, 12288, 1) == (0, 128, 0, 1)
+    assert plan(8176, 1920, 480, 0)[2:] == (0, 1)
+    assert plan(4096, 14336, 4096, 0)[2:] == (0, 1)
+    assert plan(8192, 7168, 18432, 1)[2:] == (0, 1)
+    for M, N, K, fmt in [(4096, 4096, 14336, 0), (256, 2048, 8192, 0), (2560, 2048, 8192, 1), (2500, 2040, 8160, 0)]:
+        kind, bn, tiles, s = plan(M, N, K, fmt)
+        total = -(-M // 128) * -(-N // bn)
+        assert kind == 0 and tiles == total % 148 and s >= 2 and tiles * s <= 148, (M, N, K, fmt)

@@ -10,7 +10,7 @@ call after the first runs on a scratch that still holds the previous call's
 bytes.  Each result is checked against the CPU oracle within the tolerance
 every GPU test uses, and against fg8_linear on the same inputs bit for bit
 (the same kernels run on the same bytes).  It also checks that a shape beyond
-the scratch's 32 MiB and bad arguments are refused with their status.
+the scratch's 64 MiB and bad arguments are refused with their status.
 
 Kept in a file that pytest collects last, so that a stopping run has already
 run every other test; it passes alone in a fresh process too.
@@ -71,12 +71,14 @@ def test_noalloc_vs_oracle_calls_in_a_row(fg8, orc):
     _run_and_check(fg8, orc, 1, 4096, 1024, FLOAT, seed=44)
     _run_and_check(fg8, orc, 16, 1040, 2048, UE8M0, seed=45)   # fused few-token kernel (quantizes x itself)
     _run_and_check(fg8, orc, 1, 264, 4096, UE8M0, seed=46)
+    _run_and_check(fg8, orc, 200, 2048, 4096, FLOAT, seed=48)  # tiled GEMM split over K (partials in the scratch)
+    _run_and_check(fg8, orc, 256, 1024, 4096, UE8M0, seed=49)
     _run_and_check(fg8, orc, 300, 520, 1040, FLOAT, seed=47)   # back to the tiled GEMM
 
 
 def test_noalloc_refuses_shapes_beyond_its_scratch(fg8):
-    M, N, K = 8192, 1024, 8192  # needs > 64 MB of workspace
-    assert fg8.fg8_linear_workspace_bytes(M, N, K, FLOAT) > (32 << 20)
+    M, N, K = 8192, 1024, 8192  # needs > 64 MiB of workspace
+    assert fg8.fg8_linear_workspace_bytes(M, N, K, FLOAT) > (64 << 20)
     st = fg8.lib().fg8_linear_noalloc(16, M, N, K, K, 16, 16, None, 16, N, FLOAT, None)
     assert st == fg8.FG8_ERR_WORKSPACE
 
