@@ -160,7 +160,6 @@ cudaError_t launch_xs_transpose(const float* xs, int M, int Kb, int64_t ld_s, fl
 // the caller before first use.
 constexpr size_t kWorkspaceHeaderBytes = 1024;
 constexpr size_t kHeaderEpochOffset = 8;  // fused act-quant: epoch word, then the finished-CTA count
-constexpr size_t kHeaderSchedOffset = 24;  // tiled GEMM: work ticket counter, then the finished-CTA count
 constexpr size_t kHeaderCounterOffset = 64;
 constexpr int kHeaderCounters = static_cast<int>((kWorkspaceHeaderBytes - kHeaderCounterOffset) / 4);
 

@@ -117,9 +117,6 @@ struct KParams {
   int split_from, split_s, split_kbs, num_work;
   float* partials;
   uint32_t* split_cnt;
-  // dynamic schedule: [0] the next work ticket, [1] CTAs finished (both zero
-  // at rest: the last CTA out resets them)
-  uint32_t* sched;
 };
 
 // One unit of a CTA's walk: a tile, the K-blocks [kb0, kb1) it computes, and
@@ -274,38 +271,6 @@ struct Ring {
     }
   }
 };
-
-// Work queue: the producer claims the CTA's work units -- first unit
-// blockIdx.x, then gridDim.x + a ticket from a global counter, so CTAs that
-// run ahead take more units -- and hands each index to the other roles
-// through kWorkSlots shared slots (an index >= num_work ends the walk).
-constexpr int kWorkSlots = 4;
-struct WorkQ {
-  volatile int* slot;
-  uint64_t* full;
-  uint64_t* empty;  // one arrival per consuming warp (MMA thread, scale warp, epilogue warps)
-};
-
-// The next unit index for a warp (every lane gets it; lane 0 releases the
-// slot), or -1 when the wait gave up.
-__device__ __forceinline__ int take_work_warp(const WorkQ& q, Ring& r, uint64_t limit, volatile int* abort_flag,
-                                              int lane) {
-  if (!mbar_wait_warp(q.full + r.slot, r.phase, limit, abort_flag)) return -1;
-  const int u = q.slot[r.slot];
-  __syncwarp();
-  if (lane == 0) mbar_arrive(q.empty + r.slot);
-  r.template advance<kWorkSlots>();
-  return u;
-}
-
-// The same for a single thread.
-__device__ __forceinline__ int take_work(const WorkQ& q, Ring& r, uint64_t limit, volatile int* abort_flag) {
-  if (!mbar_wait(q.full + r.slot, r.phase, limit, abort_flag)) return -1;
-  const int u = q.slot[r.slot];
-  mbar_arrive(q.empty + r.slot);
-  r.template advance<kWorkSlots>();
-  return u;
-}
 
 // Quantize one output row's 128-column group (bf16-rounded values in `v`) as
 // the next layer's activation group: the same arithmetic, hence the same bits,
@@ -529,26 +494,15 @@ __device__ __forceinline__ bool unit_ready(const KParams& p, uint32_t epoch, int
 template <class C>
 __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
                                          uint8_t* smem, uint64_t* full, uint64_t* empty, uint64_t* bfull,
-                                         uint64_t* bempty, const WorkQ& wq, volatile int* abort_flag,
-                                         uint32_t epoch) {
+                                         uint64_t* bempty, volatile int* abort_flag, uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring st, bi, wr;
+  Ring st, bi;
   // most recent issue phase per slot, for the drain at the end
   uint32_t st_issued = 0, bi_issued = 0;
   uint32_t st_par[C::STAGES], bi_par[2];
   bool ok = true;
   bool w_packed = false;
-  for (int u = static_cast<int>(blockIdx.x); ok;
-       u = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.sched, 1u))) {
-    // hand the unit (or the end of the walk) to the other roles
-    if (!mbar_wait(wq.empty + wr.slot, wr.phase ^ 1u, limit, abort_flag)) {
-      raise_abort(abort_flag, p.status);
-      break;
-    }
-    wq.slot[wr.slot] = u;
-    mbar_arrive(wq.full + wr.slot);
-    wr.template advance<kWorkSlots>();
-    if (u >= p.num_work) break;
+  for (int u = static_cast<int>(blockIdx.x); ok && u < p.num_work; u += static_cast<int>(gridDim.x)) {
     const Work w = work_at<C>(p, u);
     int mb, nb;
     tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
@@ -626,9 +580,9 @@ __device__ __forceinline__ void producer(const CUtensorMap* tmA, const CUtensorM
 template <class C>
 __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint32_t tmem_base, uint64_t* full,
                                            uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* teardown,
-                                           uint64_t* stall, const WorkQ& wq, volatile int* abort_flag) {
+                                           uint64_t* stall, volatile int* abort_flag) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring st, ab, wr;
+  Ring st, ab;
   bool ok = true;
   // test hook: a barrier nothing arrives on, so the bounded wait runs out
   if (p.test_stall && !mbar_wait(stall, 0, limit, abort_flag)) {
@@ -638,13 +592,7 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
   uint32_t sf_set = 1;  // the set the next copy goes to is sf_set ^ 1
   uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::kSfaCol);
   uint32_t sfb_t = tmem_base + static_cast<uint32_t>(C::kSfbCol);
-  while (ok) {
-    const int u = take_work(wq, wr, limit, abort_flag);
-    if (u < 0) {
-      raise_abort(abort_flag, p.status);
-      break;
-    }
-    if (u >= p.num_work) break;
+  for (int u = static_cast<int>(blockIdx.x); ok && u < p.num_work; u += static_cast<int>(gridDim.x)) {
     const Work w = work_at<C>(p, u);
     if (p.row_expert != nullptr) {
       int mb, nb;
@@ -758,16 +706,10 @@ __device__ __forceinline__ void mma_issuer(const KParams& p, uint8_t* smem, uint
 // latency stays off the epilogue's path.  The epilogue warps release slots.
 template <class C>
 __device__ __forceinline__ void scale_loader(const KParams& p, uint8_t* smem, uint64_t* sfull, uint64_t* sempty,
-                                             const WorkQ& wq, volatile int* abort_flag, int lane, uint32_t epoch) {
+                                             volatile int* abort_flag, int lane, uint32_t epoch) {
   const uint64_t limit = p.wait_limit_ns;
-  Ring sr, wr;
-  for (;;) {
-    const int u = take_work_warp(wq, wr, limit, abort_flag, lane);
-    if (u < 0) {
-      raise_abort(abort_flag, p.status);
-      break;
-    }
-    if (u >= p.num_work) break;
+  Ring sr;
+  for (int u = static_cast<int>(blockIdx.x); u < p.num_work; u += static_cast<int>(gridDim.x)) {
     const Work w = work_at<C>(p, u);
     int mb, nb;
     tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
@@ -805,8 +747,7 @@ template <class C>
 __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& p, uint8_t* smem, uint32_t tmem_base,
                                          uint64_t* tfull, uint64_t* tempty, uint64_t* bfull, uint64_t* bempty,
                                          uint64_t* sfull, uint64_t* sempty, uint64_t* xbar, uint64_t* ybar,
-                                         volatile uint32_t* xlast, const WorkQ& wq, volatile int* abort_flag, int warp,
-                                         int lane) {
+                                         volatile uint32_t* xlast, volatile int* abort_flag, int warp, int lane) {
   const uint64_t limit = p.wait_limit_ns;
   const int ew = warp - 4;
   const int q = warp & 3;      // TMEM lane quadrant
@@ -814,17 +755,11 @@ __device__ __forceinline__ void epilogue(const CUtensorMap* tmY, const KParams& 
   const int col0 = wg * C::kCols;
   uint8_t* stg = smem + C::kOffStaging + ew * C::kOutBufs * C::kOutBuf;
   const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-  Ring ab, bi, sr, wr;
+  Ring ab, bi, sr;
   bool ok = true;
   const int sub_row = q * 32 + lane;  // this thread's row inside a tile
   uint32_t xph = 0;                   // parity of the split hand-over barriers
-  while (ok) {
-    const int u = take_work_warp(wq, wr, limit, abort_flag, lane);
-    if (u < 0) {
-      raise_abort(abort_flag, p.status);
-      break;
-    }
-    if (u >= p.num_work) break;
+  for (int u = static_cast<int>(blockIdx.x); ok && u < p.num_work; u += static_cast<int>(gridDim.x)) {
     const Work w = work_at<C>(p, u);
     int mb, nb;
     tile_coords(w.tile, p.num_m, p.num_n, mb, nb);
@@ -1102,16 +1037,10 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* stall = teardown + 1;
   uint64_t* xbar = stall + 1;  // split tiles: the epilogue warps' partials are out
   uint64_t* ybar = xbar + 1;   // ... and the unit has been counted (verdict in xlast)
-  WorkQ wq;
-  wq.full = ybar + 1;
-  wq.empty = wq.full + kWorkSlots;
-  wq.slot = reinterpret_cast<volatile int*>(wq.empty + kWorkSlots);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wq.empty + kWorkSlots) + kWorkSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ybar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile uint32_t* xlast = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
-  static_assert(C::kOffBar + 8 * (2 * C::STAGES + 2 * C::kNumAcc + 4 + 2 * C::kSRing + 4 + 2 * kWorkSlots) +
-                        4 * kWorkSlots + 16 <=
-                    C::kOffBar + 512,
+  static_assert(C::kOffBar + 8 * (2 * C::STAGES + 2 * C::kNumAcc + 4 + 2 * C::kSRing + 4) + 16 <= C::kOffBar + 512,
                 "barrier block");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1140,10 +1069,6 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(stall, 1);
     mbar_init(xbar, C::kEpiWarps);
     mbar_init(ybar, 1);
-    for (int s = 0; s < kWorkSlots; ++s) {
-      mbar_init(wq.full + s, 1);
-      mbar_init(wq.empty + s, 1 + (C::FMT == 0 ? 1 : 0) + C::kEpiWarps);  // MMA, scale warp, epilogue warps
-    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -1168,11 +1093,11 @@ __global__ void __launch_bounds__(384, 1)
   if (warp < 4) {
     setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0)
-      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, wq, abort_flag, epoch);
+      producer<C>(&tmA, &tmB, p, smem, full, empty, bfull, bempty, abort_flag, epoch);
     else if (warp == 1 && lane == 0)
-      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, wq, abort_flag);
+      mma_issuer<C>(p, smem, tmem_base, full, empty, tfull, tempty, teardown, stall, abort_flag);
     if constexpr (C::FMT == 0) {
-      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, wq, abort_flag, lane, epoch);
+      if (warp == 3) scale_loader<C>(p, smem, sfull, sempty, abort_flag, lane, epoch);
     }
     if constexpr (C::REQUANT && C::FMT == 1) {
       if (warp == 2 || warp == 3)
@@ -1181,8 +1106,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     setmaxnreg_inc<C::kRegsHigh>();
-    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, sfull, sempty, xbar, ybar, xlast, wq,
-                abort_flag, warp, lane);
+    epilogue<C>(&tmY, p, smem, tmem_base, tfull, tempty, bfull, bempty, sfull, sempty, xbar, ybar, xlast, abort_flag,
+                warp, lane);
   }
 
   __syncthreads();
@@ -1190,16 +1115,7 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
-  // the last CTA out puts the ticket counter back to zero (every CTA has
-  // taken its last ticket by now)
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-      p.sched[0] = 0u;
-      p.sched[1] = 0u;
-      __threadfence();
-    }
-  }
+
   if constexpr (C::QIN) {
     // the last CTA out advances the epoch: every CTA has read it and every
     // unit flag of this call holds epoch + 1, which no later call waits for
@@ -1322,7 +1238,6 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
     }
   }
   p.num_work = p.split_from + (p.num_tiles - p.split_from) * p.split_s;
-  p.sched = g.status + kHeaderSchedOffset / 4;
 
   // the shared-memory opt-in once per device: one bit per device; calls from
   // several host threads may repeat it, which is harmless
