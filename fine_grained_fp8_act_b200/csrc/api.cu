@@ -863,9 +863,7 @@ fg8_status fg8_linear_fused(const void* x_bf16, int64_t M, int64_t N, int64_t K,
   g.qx = x_bf16;
   g.ld_qx = ld_x;
   g.qflags = reinterpret_cast<uint32_t*>(ws + fused_flags_off(M, N, K, fmt));
-  // the split-K tail as fg8_linear plans it (same tiles and sums, same bits);
-  // its partials end where the flags begin
-  set_split_area(g, workspace, fused_flags_off(M, N, K, fmt), L.total);
+  // (no split-K tail: these short-K shapes never split, in fg8_linear either)
   g.qepoch = reinterpret_cast<uint32_t*>(ws + kHeaderEpochOffset);
   if (chain) {
     uint8_t* wn = static_cast<uint8_t*>(next_workspace);

@@ -1226,6 +1226,7 @@ cudaError_t launch_cfg(const GemmArgs& g, int num_sms, cudaStream_t s) {
   p.split_kbs = p.Kb;
   p.partials = nullptr;
   p.split_cnt = nullptr;
+  static_assert(!C::SPLIT || !C::QIN, "the in-launch quantization runs short K, which never splits");
   if (C::SPLIT && g.row_expert == nullptr && g.split_ws != nullptr) {
     const SplitPlan pl = split_plan(p.num_tiles, p.num_m, p.Kb, C::FMT == 1 && !g.sf32 ? 4 : 1, num_sms);
     if (pl.from < p.num_tiles && split_area_bytes(pl, p.num_tiles, C::BN) <= g.split_bytes &&
@@ -1375,38 +1376,27 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   if (g.qx != nullptr) {  // x quantized inside the kernel: short K only (see can_quantize_in_gemm)
     if (!short_k || g.wblk > 0 && g.wblk != 128 || g.row_expert != nullptr) return cudaErrorInvalidValue;
     const bool requant = g.nx_xq != nullptr;
-    // the tile width fg8_linear picks, so that both give the same bits
+    // the tile width fg8_linear picks, so that both give the same bits (short
+    // K never splits: the split-K tail needs at least 64 K-blocks)
     const int bnq = requant ? 256 : choose_block_n(g.M, g.N, g.Kb, align, num_sms, may_split);
-    const bool sp = splits(bnq);
     if (fmt == 0) {
-      if (requant)
-        return launch_either<Cfg<256, 0, 3, 4, true, false, true>, Cfg<256, 0, 3, 4, true, false, true, true>>(
-            sp, g, num_sms, s);
-      if (bnq == 256)
-        return launch_either<Cfg<256, 0, 3, 4, false, false, true>, Cfg<256, 0, 3, 4, false, false, true, true>>(
-            sp, g, num_sms, s);
-      return launch_either<Cfg<128, 0, 5, 2, false, false, true>, Cfg<128, 0, 5, 2, false, false, true, true>>(
-          sp, g, num_sms, s);
+      if (requant) return launch_cfg<Cfg<256, 0, 3, 4, true, false, true>>(g, num_sms, s);
+      if (bnq == 256) return launch_cfg<Cfg<256, 0, 3, 4, false, false, true>>(g, num_sms, s);
+      return launch_cfg<Cfg<128, 0, 5, 2, false, false, true>>(g, num_sms, s);
     }
-    if (requant)
-      return launch_either<Cfg<256, 1, 3, 4, true, false, true>, Cfg<256, 1, 3, 4, true, false, true, true>>(
-          sp, g, num_sms, s);
-    if (bnq == 256)
-      return launch_either<Cfg<256, 1, 3, 4, false, false, true>, Cfg<256, 1, 3, 4, false, false, true, true>>(
-          sp, g, num_sms, s);
-    return launch_either<Cfg<128, 1, 5, 2, false, false, true>, Cfg<128, 1, 5, 2, false, false, true, true>>(
-        sp, g, num_sms, s);
+    if (requant) return launch_cfg<Cfg<256, 1, 3, 4, true, false, true>>(g, num_sms, s);
+    if (bnq == 256) return launch_cfg<Cfg<256, 1, 3, 4, false, false, true>>(g, num_sms, s);
+    return launch_cfg<Cfg<128, 1, 5, 2, false, false, true>>(g, num_sms, s);
   }
   if (g.nx_xq != nullptr) {  // output re-quantization needs the 256-wide tile
-    const bool sp = splits(256);
     if (fmt == 0) {
-      if (short_k)
-        return launch_either<Cfg<256, 0, 3, 4, true>, Cfg<256, 0, 3, 4, true, false, false, true>>(sp, g, num_sms, s);
-      return launch_either<Cfg<256, 0, 4, 1, true>, Cfg<256, 0, 4, 1, true, false, false, true>>(sp, g, num_sms, s);
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4, true>>(g, num_sms, s);
+      return launch_either<Cfg<256, 0, 4, 1, true>, Cfg<256, 0, 4, 1, true, false, false, true>>(splits(256), g,
+                                                                                               num_sms, s);
     }
-    if (short_k)
-      return launch_either<Cfg<256, 1, 3, 4, true>, Cfg<256, 1, 3, 4, true, false, false, true>>(sp, g, num_sms, s);
-    return launch_either<Cfg<256, 1, 4, 1, true>, Cfg<256, 1, 4, 1, true, false, false, true>>(sp, g, num_sms, s);
+    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4, true>>(g, num_sms, s);
+    return launch_either<Cfg<256, 1, 4, 1, true>, Cfg<256, 1, 4, 1, true, false, false, true>>(splits(256), g,
+                                                                                             num_sms, s);
   }
   const int bn = choose_block_n(g.M, g.N, g.Kb, align, num_sms, may_split);
   if (fmt == 0 && g.wblk != 0 && g.wblk != 128) {  // float at block 64 / 32 (never split)
@@ -1419,15 +1409,13 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   const bool sp = splits(bn);
   if (fmt == 0) {
     if (bn == 256) {
-      if (short_k)
-        return launch_either<Cfg<256, 0, 3, 4>, Cfg<256, 0, 3, 4, false, false, false, true>>(sp, g, num_sms, s);
+      if (short_k) return launch_cfg<Cfg<256, 0, 3, 4>>(g, num_sms, s);
       return launch_either<Cfg<256, 0, 4, 1>, Cfg<256, 0, 4, 1, false, false, false, true>>(sp, g, num_sms, s);
     }
     return launch_either<Cfg<128, 0, 5, 2>, Cfg<128, 0, 5, 2, false, false, false, true>>(sp, g, num_sms, s);
   }
   if (bn == 256) {
-    if (short_k)
-      return launch_either<Cfg<256, 1, 3, 4>, Cfg<256, 1, 3, 4, false, false, false, true>>(sp, g, num_sms, s);
+    if (short_k) return launch_cfg<Cfg<256, 1, 3, 4>>(g, num_sms, s);
     return launch_either<Cfg<256, 1, 4, 1>, Cfg<256, 1, 4, 1, false, false, false, true>>(sp, g, num_sms, s);
   }
   return launch_either<Cfg<128, 1, 5, 2>, Cfg<128, 1, 5, 2, false, false, false, true>>(sp, g, num_sms, s);
