@@ -124,6 +124,31 @@ def test_dequantize_stays_in_bounds(fg8, fmt):
 
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(256, 2048, 8192), (300, 1032, 8192)])  # every tile split over K (ragged too)
+def test_split_tail_stays_in_bounds(fg8, fmt, M, N, K):
+    plan = fg8.fg8_linear_plan(M, N, K, fmt)
+    assert plan[2] > 0 and plan[3] >= 2, plan
+    ld_y = N + 8
+    x = W.x_outliers(M, K, seed=M + 11).cuda()
+    w = W.w_row_groups(N, K, 0.02, seed=M + 12).cuda()
+    b = W.normal((N,), 0.1, seed=M + 13).cuda()
+    wq, ws = fg8.quantize_weight(w, fmt)
+    cy = Canary(M * ld_y * 2, "cuda")
+    y = cy.matrix(BF16, M, N, ld_y)
+    need = fg8.fg8_linear_workspace_bytes(M, N, K, fmt)
+    cw = Canary(need, "cuda")
+    cw.zeroed()
+    for _ in range(2):  # the split counters are back at zero for the second call
+        fg8.fg8_linear(x.data_ptr(), M, N, K, K, wq.data_ptr(), ws.data_ptr(), b.data_ptr(), cy.ptr(), ld_y, fmt,
+                       cw.ptr(), need, _s())
+        assert fg8.fg8_check_device_status(cw.ptr(), _s()) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(y, fg8.linear(x, wq, ws, b, fmt))
+        assert cy.intact(), "y: a write outside [M, N] or into the row padding"
+        assert cw.intact(), "workspace: a write past fg8_linear_workspace_bytes (split-K partials included)"
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
 @pytest.mark.parametrize("M", [5, 300])   # few-token kernel quantizing x itself; tiled GEMM quantizing in-launch
 def test_fused_linear_stays_in_bounds(fg8, fmt, M):
     N, K = 264, 400
