@@ -72,6 +72,19 @@ def test_split_k_shapes(fg8, orc, fmt, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 2448), (16, 3000, 3200), (32, 9000, 1104), (5, 1032, 16384),
+                                   (17, 14336, 4096), (8, 4104, 14336)])
+def test_many_tiles_long_k(fg8, orc, fmt, M, N, K):
+    """Shapes with at least 4 x 148 (weight tile, K-block) pairs: many weight
+    tiles (ragged last tile, K-block and token batch) or few tiles with a
+    long K split over up to 16 CTAs.  Repeated calls give the same bits."""
+    x, w, b, wq, ws, y = _run(fg8, orc, M, N, K, fmt, seed=M + N + K)
+    y2 = fg8.linear(x, wq, ws, b, fmt)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+
+
+@pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
 def test_no_bias_and_zero_input(fg8, orc, fmt):
     _run(fg8, orc, 20, 264, 3072, fmt, seed=5, bias=False)
     x = torch.zeros(20, 3072, dtype=torch.bfloat16, device="cuda")

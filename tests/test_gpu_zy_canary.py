@@ -59,9 +59,10 @@ def test_quantizers_stay_in_bounds(fg8, fmt):
 
 
 @pytest.mark.parametrize("fmt", [FLOAT, UE8M0])
-@pytest.mark.parametrize("M", [3, 5, 40, 300])   # fused few-token (UE8M0), few-token, few-token, tiled
-def test_linear_stays_in_bounds(fg8, fmt, M):
-    N, K = 264, 400
+@pytest.mark.parametrize("M,N,K", [(3, 264, 400), (5, 264, 400), (40, 264, 400), (300, 264, 400),
+                                   (5, 1032, 16384), (24, 4104, 2432)])
+# fused few-token (UE8M0), few-token, few-token, tiled; few-token with long K / many tiles
+def test_linear_stays_in_bounds(fg8, fmt, M, N, K):
     ld_y = N + 8
     x = W.x_outliers(M, K, seed=M).cuda()
     w = W.w_row_groups(N, K, 0.02, seed=M + 1).cuda()
