@@ -1359,8 +1359,10 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
   // Short K: few K-blocks per tile, so the tile's output path dominates --
   // give every output chunk its own staging box and keep one stage fewer.
   // Long K: four stages (the float path's scale ring takes the shared memory
-  // of the second staging box per warp).
-  const bool short_k = g.Kb <= 32;
+  // of the second staging box per warp).  Measured crossover: float up to 32
+  // K-blocks per tile; UE8M0, whose MMAs run faster and want the deeper
+  // ring, up to 8 (12 to 32 K-blocks ran 7-18% faster with four stages).
+  const bool short_k = g.Kb <= (fmt == 1 ? 8 : 32);
   const int align = fmt == 1 ? 4 : 1;
   // (the split-K tail only runs for block-128 scales with room for it)
   const bool may_split = g.split_ws != nullptr && g.row_expert == nullptr && !g.sf32 && (g.wblk == 0 || g.wblk == 128);
@@ -1374,7 +1376,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int fmt, int num_sms, cudaStream_t s)
     return pl.from < tiles && tiles - pl.from <= kHeaderCounters && split_area_bytes(pl, tiles, bn) <= g.split_bytes;
   };
   if (g.qx != nullptr) {  // x quantized inside the kernel: short K only (see can_quantize_in_gemm)
-    if (!short_k || g.wblk > 0 && g.wblk != 128 || g.row_expert != nullptr) return cudaErrorInvalidValue;
+    if (g.Kb > 32 || g.wblk > 0 && g.wblk != 128 || g.row_expert != nullptr) return cudaErrorInvalidValue;
     const bool requant = g.nx_xq != nullptr;
     // the tile width fg8_linear picks, so that both give the same bits (short
     // K never splits: the split-K tail needs at least 64 K-blocks)
