@@ -553,6 +553,36 @@ def run_fg8(args, rank, world, local):
         torch.distributed.destroy_process_group()
 
 
+def host_link_ms(h2d_pairs, d2h_pairs, h2d, d2h, stream, steps, world, dev):
+    """Per-step time of an end-to-end leg's host copies alone, with no kernels:
+    the same buffers and bytes each way, both directions at once on their own
+    streams.  This is the host link's bound for the end-to-end number (on the
+    B200 boxes the two directions share the link: about 55 GB/s one way
+    alone, 47 GB/s each way together)."""
+    def copies():
+        with torch.cuda.stream(h2d):
+            for src, dst in h2d_pairs:
+                dst.copy_(src, non_blocking=True)
+        with torch.cuda.stream(d2h):
+            for src, dst in d2h_pairs:
+                dst.copy_(src, non_blocking=True)
+
+    copies()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h2d.wait_event(e0)
+    d2h.wait_event(e0)
+    for _ in range(steps):
+        copies()
+    stream.wait_stream(h2d)
+    stream.wait_stream(d2h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+
+
 def run_e2e(fg8, plan, args, stream, dev, world, chain, paths):
     """Same metric through the public calls with host buffers, as a serving
     loop runs it: every step copies its input from pinned host memory to the
@@ -647,9 +677,11 @@ def run_e2e(fg8, plan, args, stream, dev, world, chain, paths):
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     flops = sum_over_ranks(sum(gemm_flops(L["g"]) for L in plan) * steps, world, dev)
+    link = host_link_ms([(x_host, x_dev[0])], [(y_dev[0], y_host[0])], h2d, d2h, stream, steps, world, dev)
     return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host[0].numel() * 2,
             "steps": steps, "ms_per_step": ms / steps,
+            "host_link_ms_per_step": link, "frac_of_host_link": link / (ms / steps),
             "overlap": "input and output copies on their own streams, overlapping the neighbouring steps' kernels"}
 
 
@@ -873,9 +905,12 @@ def run_moe(args, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize()
     ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    link = host_link_ms(list(zip(xh + [reh], xd[0] + [red[0]])), [(yd[0], yh[0])], h2d, d2h, stream, e2e_steps,
+                        world, dev)
     e2e = {"value": sum_over_ranks(flops_step * e2e_steps, world, dev) / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": sum(a.numel() * 2 for a in xh) + reh.numel() * 4,
            "d2h_bytes_per_step": yh[0].numel() * 2, "steps": e2e_steps, "ms_per_step": ems / e2e_steps,
+           "host_link_ms_per_step": link, "frac_of_host_link": link / (ems / e2e_steps),
            "overlap": "input and output copies on their own streams, overlapping the neighbouring steps' kernels"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
