@@ -1,0 +1,133 @@
+"""A seeded sweep of random layer shapes through fg8.linear vs the CPU oracle.
+
+The fixed-shape tests pin each kernel path on hand-picked sizes; this sweep
+draws M, N and K at random inside each path's range, in both scale formats and
+at weight blocks 128, 64 and 32, so that the dispatch rule, the tile and
+K-block edges, the split-K tail plans and the few-token split counts meet
+shapes nobody chose.  Each case is checked within the y tolerance on every row
+(small M) or on sampled rows that always include the first and last row and
+the 128-row tile boundaries, the weight codes are compared with the oracle's
+bit for bit, and a second call must give the same bits.  A CPU test checks
+that the drawn shapes really reach every path fg8_linear_plan reports
+(tiled with and without a split tail, the few-token kernel, the fused
+few-token kernel).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from conftest import y_tolerance
+
+FLOAT, UE8M0 = 0, 1
+
+
+def _cases():
+    """(name, M, N, K, fmt, block, bias): N a multiple of 8 and K of 16 (the
+    rows' 16-byte alignment the boundary asks for), everything else free."""
+    rng = np.random.default_rng(20261203)
+    out = []
+
+    def draw(kind, n, m_lo, m_hi, n_lo, n_hi, k_lo, k_hi, block=128):
+        for i in range(n):
+            M = int(rng.integers(m_lo, m_hi + 1))
+            N = 8 * int(rng.integers(n_lo // 8, n_hi // 8 + 1))
+            K = 16 * int(rng.integers(k_lo // 16, k_hi // 16 + 1))
+            fmt = len(out) % 2
+            bias = bool(rng.integers(0, 4))  # three in four with a bias
+            out.append((f"{kind}{i}", M, N, K, fmt, block, bias))
+
+    draw("few", 32, 1, 32, 8, 3072, 16, 4096)             # few-token kernel (fused for UE8M0 and M <= 16)
+    draw("mid", 24, 33, 128, 8, 12288, 16, 2048)           # few-token below the tiled rule, tiled above
+    draw("tiled", 32, 129, 1100, 128, 2400, 16, 2560)     # whole tiles, short and long K
+    draw("split", 20, 129, 640, 256, 2560, 8192, 10240)    # >= 64 K-blocks: split-K tails
+    draw("b64_", 12, 1, 700, 8, 1536, 16, 2048, block=64)
+    draw("b32_", 12, 1, 700, 8, 1536, 16, 2048, block=32)
+    return out
+
+
+CASES = _cases()
+
+
+def test_sweep_reaches_every_path():
+    """The drawn shapes reach each kernel fg8_linear_plan can report, in both
+    formats (block-128 cases), including split-K tails."""
+    from fine_grained_fp8_act_b200 import build
+    build.build()
+    import fine_grained_fp8_act_b200 as fg8
+    seen = set()
+    for _, M, N, K, fmt, block, _ in CASES:
+        if block != 128:
+            continue
+        kernel, _, split_tiles, _ = fg8.fg8_linear_plan(M, N, K, fmt)
+        seen.add((fmt, kernel, kernel == 0 and split_tiles > 0))
+    want = {(FLOAT, 0, False), (FLOAT, 0, True), (FLOAT, 1, False),
+            (UE8M0, 0, False), (UE8M0, 0, True), (UE8M0, 2, False)}
+    assert want <= seen, sorted(want - seen)
+
+
+def test_tolerance_admits_the_rounded_output(orc):
+    """A bias-dominated layer with few K-elements (shapes the sweep draws):
+    the oracle's own correctly rounded bf16 y misses the bound 8e-3 * sum |xhat
+    * what| + 1e-6 on some element, and is within it once half a bf16 ulp of y
+    (the output format's rounding) is added, which the sweep therefore uses."""
+    M, N, K, fmt, block = 309, 1304, 48, UE8M0, 64
+    seed = M * 7919 + N * 31 + K
+    x = W.x_outliers(M, K, seed=seed)
+    w = W.w_row_groups(N, K, 0.02, seed=seed + 1, rows_per_group=block)
+    b = W.normal((N,), 0.1, seed=seed + 2)
+    owq, ows = orc.quantize_weight(W.bf16_bits(w), fmt, block)
+    y64, bound, ybf = orc.linear(W.bf16_bits(x), owq, ows, W.bf16_bits(b), fmt, block=block)
+    rounded = (ybf.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    err = np.abs(rounded - y64)
+    assert (err > y_tolerance(bound)).any()
+    assert (err <= y_tolerance(bound, y64, rounded)).all()
+
+
+@pytest.fixture(scope="module")
+def fg8():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import fine_grained_fp8_act_b200 as m
+    m.lib()
+    return m
+
+
+def _f64(t):
+    return (W.bf16_bits(t.cpu()).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _rows(M, seed):
+    if M <= 48:
+        return None
+    rng = np.random.default_rng(seed)
+    r = {0, M - 1, M // 2} | {b + d for b in range(128, M, 128) for d in (-1, 0) if b + d < M}
+    r |= set(int(v) for v in rng.integers(0, M, 16))
+    return np.array(sorted(r), dtype=np.int64)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,N,K,fmt,block,bias", CASES, ids=[c[0] for c in CASES])
+def test_random_shape_vs_oracle(fg8, orc, name, M, N, K, fmt, block, bias):
+    seed = M * 7919 + N * 31 + K
+    x = W.x_outliers(M, K, seed=seed)
+    w = W.w_row_groups(N, K, 0.02, seed=seed + 1, rows_per_group=block)
+    b = W.normal((N,), 0.1, seed=seed + 2) if bias else None
+    xd, wd = x.cuda(), w.cuda()
+    bd = None if b is None else b.cuda()
+    wq, ws = fg8.quantize_weight(wd, fmt, block=block)
+    y = fg8.linear(xd, wq, ws, bd, fmt, block=block)
+    y_again = fg8.linear(xd, wq, ws, bd, fmt, block=block)
+    torch.cuda.synchronize()
+    owq, ows = orc.quantize_weight(W.bf16_bits(w), fmt, block)
+    assert np.array_equal(wq.view(torch.uint8).cpu().numpy(), owq), f"{name}: weight codes"
+    r = _rows(M, seed)
+    y64, bound, _ = orc.linear(W.bf16_bits(x), owq, ows, None if b is None else W.bf16_bits(b), fmt, rows=r,
+                               block=block)
+    got = _f64(y if r is None else y[torch.from_numpy(r).cuda()])
+    err = np.abs(got - y64)
+    bad = ~(err <= y_tolerance(bound, y64, got))
+    plan = fg8.fg8_linear_plan(M, N, K, fmt) if block == 128 else None
+    assert not bad.any(), (f"{name} M={M} N={N} K={K} fmt={fmt} block={block} plan={plan}: "
+                           f"{int(bad.sum())} elements out of tolerance, max err {np.nanmax(err)}")
+    assert torch.equal(y, y_again), f"{name}: a second call gave other bits"
