@@ -17,6 +17,7 @@ import pytest
 import torch
 
 import workloads as W
+from _ws_layout import decode
 from conftest import y_tolerance
 
 FLOAT, UE8M0 = 0, 1
@@ -131,3 +132,149 @@ def test_random_shape_vs_oracle(fg8, orc, name, M, N, K, fmt, block, bias):
     assert not bad.any(), (f"{name} M={M} N={N} K={K} fmt={fmt} block={block} plan={plan}: "
                            f"{int(bad.sum())} elements out of tolerance, max err {np.nanmax(err)}")
     assert torch.equal(y, y_again), f"{name}: a second call gave other bits"
+
+
+# ------------------------------------------- chained, fused and static ----
+def _entry_cases():
+    """Random shapes for the entry points beside fg8_linear: (name, M, K1, N1,
+    N2, fmt, bias).  N1 is the next layer's K, so a multiple of 16."""
+    rng = np.random.default_rng(4417)
+    out = []
+    for i in range(24):
+        M = int(rng.integers(1, 1101)) if i % 3 else int(rng.integers(1, 40))
+        K1 = 16 * int(rng.integers(1, 257))
+        N1 = 16 * int(rng.integers(1, 161))
+        N2 = 8 * int(rng.integers(1, 241))
+        out.append((f"e{i}", M, K1, N1, N2, i % 2, bool(rng.integers(0, 4))))
+    return out
+
+
+ENTRY_CASES = _entry_cases()
+
+
+def _same(got, want, what):
+    got, want = np.ascontiguousarray(got), np.ascontiguousarray(want)
+    if not np.array_equal(got, want):
+        bad = np.argwhere(got != want)
+        raise AssertionError(f"{what}: {len(bad)} mismatches, first at {tuple(bad[0])}")
+
+
+def _check_y(y, y64, bound, what):
+    got = _f64(y)
+    err = np.abs(got - y64)
+    bad = ~(err <= y_tolerance(bound, y64, got))
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements out of tolerance, max err {np.nanmax(err)}"
+
+
+def _layers(fg8, orc, M, K1, N1, N2, fmt, bias):
+    seed = M * 131 + K1 * 7 + N1 * 3 + N2
+    x = W.x_outliers(M, K1, seed=seed)
+    w1 = W.w_row_groups(N1, K1, 0.02, seed=seed + 1)
+    w2 = W.normal((N2, N1), 0.02, seed=seed + 2)
+    b1 = W.normal((N1,), 0.1, seed=seed + 3) if bias else None
+    wq1, ws1 = fg8.quantize_weight(w1.cuda(), fmt)
+    wq2, ws2 = fg8.quantize_weight(w2.cuda(), fmt)
+    owq1, ows1 = orc.quantize_weight(W.bf16_bits(w1), fmt)
+    owq2, ows2 = orc.quantize_weight(W.bf16_bits(w2), fmt)
+    return x, b1, (wq1, ws1, owq1, ows1), (wq2, ws2, owq2, ows2)
+
+
+def _check_chain(fg8, orc, name, M, N1, N2, fmt, x, b1, y1, wsn, second, rows):
+    """y1 vs the oracle; the next layer's codes and scales decoded from its
+    workspace vs the oracle's quantization of the stored y1, bit for bit; y2
+    (fg8_linear_run from that workspace) vs the oracle on those codes."""
+    wq2, ws2, owq2, ows2 = second
+    y2 = torch.full((M, N2), float("nan"), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    fg8.fg8_linear_run(wq2.data_ptr(), ws2.data_ptr(), 0, y2.data_ptr(), M, N2, N1, N2, fmt, wsn.data_ptr(),
+                       wsn.numel(), s)
+    torch.cuda.synchronize()
+    assert fg8.fg8_check_device_status(wsn.data_ptr(), s) == 0
+    nxq, nxs = decode(wsn.cpu().numpy(), M, N1, fmt)
+    oxq, oxs = orc.quantize_act(W.bf16_bits(y1.cpu()), fmt)
+    _same(nxq, oxq, f"{name}: requantized codes of y1")
+    _same(nxs, oxs.view(np.uint32) if fmt == FLOAT else oxs, f"{name}: requantized scales of y1")
+    y2_64, bound2, _ = orc.linear_dequant(oxq, oxs, owq2, ows2, None, fmt, rows=rows)
+    _check_y(y2 if rows is None else y2[torch.from_numpy(rows).cuda()], y2_64, bound2, f"{name}: y2")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,K1,N1,N2,fmt,bias", ENTRY_CASES, ids=[c[0] for c in ENTRY_CASES])
+def test_random_chain_vs_oracle(fg8, orc, name, M, K1, N1, N2, fmt, bias):
+    """fg8_linear_prepare + fg8_linear_run_chain (the epilogue quantizes y1 for
+    the next layer) + fg8_linear_run of the next layer."""
+    x, b1, first, second = _layers(fg8, orc, M, K1, N1, N2, fmt, bias)
+    wq1, ws1, owq1, ows1 = first
+    s = torch.cuda.current_stream().cuda_stream
+    wsa = torch.zeros(fg8.fg8_linear_workspace_bytes(M, N1, K1, fmt), dtype=torch.uint8, device="cuda")
+    wsb = torch.zeros(fg8.fg8_linear_workspace_bytes(M, N2, N1, fmt), dtype=torch.uint8, device="cuda")
+    y1 = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+    xd = x.cuda()
+    b1d = None if b1 is None else b1.cuda()
+    fg8.fg8_linear_prepare(xd.data_ptr(), M, N1, K1, K1, ws1.data_ptr(), fmt, wsa.data_ptr(), wsa.numel(), s)
+    fg8.fg8_linear_run_chain(wq1.data_ptr(), ws1.data_ptr(), 0 if b1d is None else b1d.data_ptr(), y1.data_ptr(),
+                             M, N1, K1, N1, fmt, wsa.data_ptr(), wsa.numel(), N2, ws2_ptr(second), wsb.data_ptr(),
+                             wsb.numel(), s)
+    torch.cuda.synchronize()
+    assert fg8.fg8_check_device_status(wsa.data_ptr(), s) == 0
+    rows = _rows(M, M + K1)
+    y1_64, bound1, _ = orc.linear(W.bf16_bits(x), owq1, ows1, None if b1 is None else W.bf16_bits(b1), fmt,
+                                  rows=rows)
+    _check_y(y1 if rows is None else y1[torch.from_numpy(rows).cuda()], y1_64, bound1, f"{name}: y1")
+    _check_chain(fg8, orc, name, M, N1, N2, fmt, x, b1, y1, wsb, second, rows)
+
+
+def ws2_ptr(second):
+    return second[1].data_ptr()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,K1,N1,N2,fmt,bias", ENTRY_CASES, ids=[c[0] for c in ENTRY_CASES])
+def test_random_fused_vs_oracle(fg8, orc, name, M, K1, N1, N2, fmt, bias):
+    """fg8_linear_fused (x quantized inside the GEMM's launch where the shape
+    allows it), with the next layer's quantization on every other case; two
+    calls on one workspace give the same bits."""
+    x, b1, first, second = _layers(fg8, orc, M, K1, N1, N2, fmt, bias)
+    wq1, ws1, owq1, ows1 = first
+    s = torch.cuda.current_stream().cuda_stream
+    chain = int(name[1:]) % 4 < 2
+    wsa = torch.zeros(fg8.fg8_linear_fused_workspace_bytes(M, N1, K1, fmt), dtype=torch.uint8, device="cuda")
+    wsb = torch.zeros(fg8.fg8_linear_workspace_bytes(M, N2, N1, fmt), dtype=torch.uint8, device="cuda")
+    xd = x.cuda()
+    b1d = None if b1 is None else b1.cuda()
+    ys = []
+    for _ in range(2):
+        y1 = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+        fg8.fg8_linear_fused(xd.data_ptr(), M, N1, K1, K1, wq1.data_ptr(), ws1.data_ptr(),
+                             0 if b1d is None else b1d.data_ptr(), y1.data_ptr(), N1, fmt, wsa.data_ptr(),
+                             wsa.numel(), N2 if chain else 0, ws2_ptr(second) if chain else None,
+                             wsb.data_ptr() if chain else None, wsb.numel() if chain else 0, stream=s)
+        torch.cuda.synchronize()
+        assert fg8.fg8_check_device_status(wsa.data_ptr(), s) == 0
+        ys.append(y1)
+    assert torch.equal(ys[0], ys[1]), f"{name}: a second call gave other bits"
+    y1 = ys[1]
+    rows = _rows(M, M + K1)
+    y1_64, bound1, _ = orc.linear(W.bf16_bits(x), owq1, ows1, None if b1 is None else W.bf16_bits(b1), fmt,
+                                  rows=rows)
+    _check_y(y1 if rows is None else y1[torch.from_numpy(rows).cuda()], y1_64, bound1, f"{name}: y1")
+    if chain:
+        _check_chain(fg8, orc, name, M, N1, N2, fmt, x, b1, y1, wsb, second, rows)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,K1,N1,N2,fmt,bias", ENTRY_CASES[::2], ids=[c[0] for c in ENTRY_CASES[::2]])
+def test_random_static_vs_oracle(fg8, orc, name, M, K1, N1, N2, fmt, bias):
+    """fg8_linear_static (one precomputed activation scale, float weight
+    scales) on the same random shapes."""
+    x, b1, first, _ = _layers(fg8, orc, M, K1, N1, N2, FLOAT, bias)
+    wq1, ws1, owq1, ows1 = first
+    scale = float(np.float32(3.0 / 448.0))  # the 20x outlier channels saturate
+    st = torch.tensor([scale], dtype=torch.float32, device="cuda")
+    y1 = fg8.linear_static(x.cuda(), st, wq1, ws1, None if b1 is None else b1.cuda())
+    torch.cuda.synchronize()
+    oq, oxs = orc.quantize_act_static(W.bf16_bits(x), scale)
+    rows = _rows(M, M + K1)
+    y64, bound, _ = orc.linear_dequant(oq, oxs, owq1, ows1, None if b1 is None else W.bf16_bits(b1), FLOAT,
+                                       rows=rows)
+    _check_y(y1 if rows is None else y1[torch.from_numpy(rows).cuda()], y64, bound, f"{name}: y")
