@@ -1,4 +1,4 @@
-"""A seeded sweep of random layer shapes through fg8.linear vs the CPU oracle.
+"""Seeded sweeps of random layer shapes through every entry point vs the CPU oracle.
 
 The fixed-shape tests pin each kernel path on hand-picked sizes; this sweep
 draws M, N and K at random inside each path's range, in both scale formats and
@@ -10,7 +10,10 @@ the 128-row tile boundaries, the weight codes are compared with the oracle's
 bit for bit, and a second call must give the same bits.  A CPU test checks
 that the drawn shapes really reach every path fg8_linear_plan reports
 (tiled with and without a split tail, the few-token kernel, the fused
-few-token kernel).
+few-token kernel).  The same kind of draw runs the two-layer chain (the
+epilogue's requantized codes and scales bit-exact against the oracle's
+quantization of the stored output), the in-launch quantization, the static
+activation scale and the MoE expert GEMM on random routing.
 """
 import numpy as np
 import pytest
@@ -278,3 +281,54 @@ def test_random_static_vs_oracle(fg8, orc, name, M, K1, N1, N2, fmt, bias):
     y64, bound, _ = orc.linear_dequant(oq, oxs, owq1, ows1, None if b1 is None else W.bf16_bits(b1), FLOAT,
                                        rows=rows)
     _check_y(y1 if rows is None else y1[torch.from_numpy(rows).cuda()], y64, bound, f"{name}: y")
+
+
+# ----------------------------------------------------------- MoE experts ----
+def _grouped_cases():
+    """(name, T tokens, E experts, topk, K, N, fmt, skew, bias)."""
+    rng = np.random.default_rng(977)
+    out = []
+    for i in range(12):
+        E = int(rng.integers(1, 13))
+        out.append((f"g{i}", int(rng.integers(1, 257)), E, int(rng.integers(1, min(E, 4) + 1)),
+                    16 * int(rng.integers(1, 65)), 8 * int(rng.integers(1, 65)), i % 2,
+                    float(rng.uniform(0.3, 2.0)), bool(rng.integers(0, 4))))
+    return out
+
+
+GROUPED_CASES = _grouped_cases()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,T,E,topk,K,N,fmt,skew,bias", GROUPED_CASES, ids=[c[0] for c in GROUPED_CASES])
+def test_random_grouped_vs_oracle(fg8, orc, name, T, E, topk, K, N, fmt, skew, bias):
+    """fg8_grouped_linear on random routing (log-normal expert popularity,
+    padded expert runs) and random shapes: every written row vs the oracle,
+    the padding blocks' rows left untouched."""
+    seed = T * 17 + E * 5 + K + N
+    rt, re = W.moe_routing(T, E, topk, seed=seed, skew=skew)
+    x = W.gather_rows(W.x_outliers(T, K, seed=seed + 1), rt)
+    M = x.shape[0]
+    ws_bf16 = [W.w_row_groups(N, K, 0.02, seed=seed + 10 + e) for e in range(E)]
+    qs = [fg8.quantize_weight(w.cuda(), fmt) for w in ws_bf16]
+    wq = torch.stack([q.view(torch.uint8) for q, _ in qs])
+    ws = torch.stack([s if s.element_size() != 1 else s.view(torch.uint8) for _, s in qs])
+    b = W.normal((E, N), 0.1, seed=seed + 2) if bias else None
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nb = fg8.fg8_grouped_linear_workspace_bytes(M, E, N, K, fmt)
+    wsp = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    xd, red = x.cuda(), re.cuda()
+    bd = None if b is None else b.cuda()
+    fg8.fg8_grouped_linear(xd.data_ptr(), M, K, K, red.data_ptr(), E, N, wq.data_ptr(), ws.data_ptr(),
+                           0 if bd is None else bd.data_ptr(), y.data_ptr(), N, fmt, wsp.data_ptr(), nb, s)
+    torch.cuda.synchronize()
+    assert fg8.fg8_check_device_status(wsp.data_ptr(), s) == 0
+    y64, bound, _, written = orc.grouped_linear(W.bf16_bits(x), re.numpy(), wq.cpu().numpy(), ws.cpu().numpy(),
+                                                None if b is None else W.bf16_bits(b), fmt)
+    got = _f64(y)
+    assert np.isnan(got[~written]).all(), f"{name}: rows of skipped blocks were written"
+    assert written[re.numpy() >= 0].all()
+    err = np.abs(got[written] - y64[written])
+    bad = ~(err <= y_tolerance(bound[written], y64[written], got[written]))
+    assert not bad.any(), f"{name} M={M} E={E} K={K} N={N} fmt={fmt}: {int(bad.sum())} out of tolerance"
