@@ -13,7 +13,9 @@ that the drawn shapes really reach every path fg8_linear_plan reports
 few-token kernel).  The same kind of draw runs the two-layer chain (the
 epilogue's requantized codes and scales bit-exact against the oracle's
 quantization of the stored output), the in-launch quantization, the static
-activation scale and the MoE expert GEMM on random routing.
+activation scale, the MoE expert GEMM on random routing, and the
+quantizers themselves (strided rows, blocks 128/64/32, codes and scales bit
+for bit, and Fp8Dequantize back).
 """
 import numpy as np
 import pytest
@@ -332,3 +334,46 @@ def test_random_grouped_vs_oracle(fg8, orc, name, T, E, topk, K, N, fmt, skew, b
     err = np.abs(got[written] - y64[written])
     bad = ~(err <= y_tolerance(bound[written], y64[written], got[written]))
     assert not bad.any(), f"{name} M={M} E={E} K={K} N={N} fmt={fmt}: {int(bad.sum())} out of tolerance"
+
+
+# ----------------------------------------------------------- quantizers ----
+def _quant_cases():
+    """(name, rows, cols, pad, fmt, block): pad extra bf16 columns per row of
+    the input's allocation (a strided view), a multiple of 8."""
+    rng = np.random.default_rng(5311)
+    return [(f"q{i}", int(rng.integers(1, 3000)), 16 * int(rng.integers(1, 400)), 8 * int(rng.integers(0, 3)),
+             i % 2, (128, 64, 32)[i % 3]) for i in range(18)]
+
+
+QUANT_CASES = _quant_cases()
+
+
+def _scale_bits(s):
+    """Scales as bit patterns: float32 as uint32, UE8M0 bytes as they are."""
+    if isinstance(s, torch.Tensor):
+        s = (s.view(torch.uint8) if s.element_size() == 1 else s).cpu().numpy()
+    return s.view(np.uint32) if s.dtype == np.float32 else s
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,K,pad,fmt,block", QUANT_CASES, ids=[c[0] for c in QUANT_CASES])
+def test_random_quantizers_bits(fg8, orc, name, M, K, pad, fmt, block):
+    """Activation and weight quantization of random shapes (strided rows for
+    x), codes and scales bit for bit against the oracle; block 128 weights
+    also back through Fp8Dequantize, bit for bit."""
+    wide = W.x_outliers(M, K + pad, seed=M + K + pad)
+    x = wide.cuda()[:, :K]
+    xq, xs = fg8.quantize_act(x, fmt, block=block)
+    wq, ws = fg8.quantize_weight(x, fmt, block=block)  # the same matrix as a weight [N = M, K]
+    torch.cuda.synchronize()
+    bits = W.bf16_bits(wide[:, :K].contiguous())
+    oq, oxs = orc.quantize_act(bits, fmt, block)
+    owq, ows = orc.quantize_weight(bits, fmt, block)
+    _same(xq.view(torch.uint8).cpu().numpy(), oq, f"{name}: activation codes")
+    _same(_scale_bits(xs), _scale_bits(oxs), f"{name}: activation scales")
+    _same(wq.view(torch.uint8).cpu().numpy(), owq, f"{name}: weight codes")
+    _same(_scale_bits(ws), _scale_bits(ows), f"{name}: weight scales")
+    if block == 128:
+        wd = fg8.dequantize_weight(wq, ws, fmt)
+        torch.cuda.synchronize()
+        _same(W.bf16_bits(wd.cpu()), orc.dequantize_weight(owq, ows, fmt), f"{name}: dequantized weight")
