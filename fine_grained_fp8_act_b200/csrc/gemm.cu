@@ -1283,11 +1283,15 @@ SplitPlan split_plan(int tiles, int m_blocks, int Kb, int kb_align, int sms) {
   SplitPlan pl;
   pl.from = tiles;
   pl.kbs = Kb;
-  // Measured on the B200: with fewer than 64 K-blocks per tile, or more
-  // than 6 whole waves before the tail, the CTAs' spread in finishing their
-  // whole tiles eats the gain; with a single row block the tiles stream
-  // distinct weights and are bound by that, split or not.
-  if (tiles <= 0 || sms <= 0 || Kb < 64 || m_blocks < 2 || tiles / sms > 6) return pl;
+  // Measured on the B200: with fewer than 64 K-blocks per tile the CTAs'
+  // spread in finishing their whole tiles eats the gain; with a single row
+  // block the tiles stream distinct weights and are bound by that, split or
+  // not.  The spread grows with the whole waves before the tail: past 6 of
+  // them a split has to save 60 K-block periods (it then gained 1-3% on
+  // 3584- to 8192-token layers of 96 and 144 K-blocks with a nearly empty
+  // last wave, and lost ~0.5% where it saved 41), past 16 none is tried.
+  const int waves = sms > 0 ? tiles / sms : 0;
+  if (tiles <= 0 || sms <= 0 || Kb < 64 || m_blocks < 2 || waves > 16) return pl;
   const int rem = tiles % sms;
   if (rem == 0) return pl;
   // Cost of the tail in K-block periods: unsplit, a whole tile's K loop;
@@ -1295,7 +1299,7 @@ SplitPlan split_plan(int tiles, int m_blocks, int Kb, int kb_align, int sms) {
   // and the last unit's reading of the other S - 1 partials (128 KB each
   // from L2 at ~0.1 TB/s per SM against ~0.6 us per 128 x 256 x 128
   // K-block), fitted to timings of 2048- to 8192-token layers.
-  double best = Kb;
+  double best = waves > 6 ? Kb - 60 : Kb;
   for (int S = 2; S <= Kb && rem * S <= sms; ++S) {
     const int kbs = (Kb + S - 1) / S;
     const int k = (kbs + kb_align - 1) / kb_align * kb_align;

@@ -47,7 +47,8 @@ def test_split_tail_plan(fg8):
     """Whole waves on 148 SMs: no split.  Otherwise the last wave's tiles are
     split so that all their units fit one wave, where a unit's K-blocks plus
     the partials' write-back, wait and read-back beat a whole tile's K loop,
-    with at least 64 K-blocks, two row blocks and at most 6 whole waves."""
+    with at least 64 K-blocks and two row blocks; after more than 6 whole
+    waves only a split that saves over 60 K-block periods, after 16 none."""
     plan = fg8.fg8_linear_plan
     # 16384 x 12288 x 12288: 6144 tiles of 128 x 256, 76 in the last wave
     # (two units each would not fit one wave); 41 whole waves anyway
@@ -61,7 +62,13 @@ def test_split_tail_plan(fg8):
     assert plan(64, 12288, 12288, 1) == (0, 128, 0, 1)
     assert plan(8176, 1920, 480, 0)[2:] == (0, 1)
     assert plan(4096, 14336, 4096, 0)[2:] == (0, 1)
-    assert plan(8192, 7168, 18432, 1)[2:] == (0, 1)
+    # 4096 x 12288 x 12288: 10 waves + 56 tiles; 2 units would save 41 periods
+    assert plan(4096, 12288, 12288, 0)[2:] == (0, 1)
+    # many waves, a nearly empty last wave, long K: 6 units of 24 K-blocks
+    assert plan(8192, 7168, 18432, 1) == (0, 256, 16, 6)
+    assert plan(6144, 7168, 18432, 0) == (0, 256, 12, 6)
+    # 20480 x 4096: 2560 tiles = 17 whole waves + 44: never
+    assert plan(20480, 4096, 18432, 0)[2:] == (0, 1)
     for M, N, K, fmt in [(4096, 4096, 14336, 0), (256, 2048, 8192, 0), (2560, 2048, 8192, 1), (2500, 2040, 8160, 0)]:
         kind, bn, tiles, s = plan(M, N, K, fmt)
         total = -(-M // 128) * -(-N // bn)
