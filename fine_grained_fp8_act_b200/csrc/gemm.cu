@@ -280,10 +280,17 @@ __device__ __forceinline__ void requant_group(const KParams& p, const uint32_t (
   static_assert(C::kCols == 128, "one group per thread");
   const int valid = p.N - n_first;  // real columns of this group (may be <= 0 past N)
   const int g = n_first / 128;      // the next layer's K-block
-  float amax = 0.0f;
+  // four independent max chains (max is exact in any order)
+  float m4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (valid >= 128) {
 #pragma unroll
-  for (int j = 0; j < 128; ++j)
-    if (j < valid) amax = fmaxf(amax, fabsf(__uint_as_float(v[j])));
+    for (int j = 0; j < 128; ++j) m4[j & 3] = fmaxf(m4[j & 3], fabsf(__uint_as_float(v[j])));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 128; ++j)
+      if (j < valid) m4[j & 3] = fmaxf(m4[j & 3], fabsf(__uint_as_float(v[j])));
+  }
+  const float amax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   const float s = qm::group_scale(amax);
   const uint32_t sbyte = C::FMT == 1 ? qm::e8m0_ceil_byte(s) : 0u;
   const bool store = row < p.M && valid > 0;
