@@ -199,13 +199,15 @@ def test_split_tail_workspace(fg8):
     lin, grp = fg8.fg8_linear_workspace_bytes, raw.fg8_grouped_linear_workspace_bytes
     M = 148 * 128  # 148 tiles of 128 x 256, 296 of 128 x 128, for N = 256
     assert lin(M, 256, 4096, 0) == grp(M, 1, 256, 4096, 0)
-    for M, N, K in [(256, 2048, 8192), (2560, 2048, 8192), (2048, 12288, 12288), (4096, 4096, 14336)]:
+    for M, N, K in [(256, 2048, 8192), (2560, 2048, 8192), (2048, 12288, 12288), (4096, 4096, 14336),
+                    (8192, 7168, 18432)]:
         extra = lin(M, N, K, 0) - grp(M, 1, N, K, 0)
         assert extra > 0 and extra % (128 * 128 * 4) == 0 and extra <= 148 * 128 * 256 * 4 + 256, (M, N, K, extra)
         assert fg8.fg8_linear_fused_workspace_bytes(M, N, K, 0) > lin(M, N, K, 0)
     # too few K-blocks to pay for a split (the ESM-2 layer shapes), one row
-    # block, or many whole waves before the tail
-    for M, N, K in [(8176, 1920, 480), (64, 12288, 12288), (8192, 7168, 18432)]:
+    # block, many whole waves before a tail that a split would shorten too
+    # little, or more than 16 whole waves
+    for M, N, K in [(8176, 1920, 480), (64, 12288, 12288), (4096, 12288, 12288), (20480, 4096, 18432)]:
         assert lin(M, N, K, 0) == grp(M, 1, N, K, 0), (M, N, K)
 
 
