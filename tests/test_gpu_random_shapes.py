@@ -15,7 +15,8 @@ epilogue's requantized codes and scales bit-exact against the oracle's
 quantization of the stored output), the in-launch quantization, the static
 activation scale, the MoE expert GEMM on random routing, and the
 quantizers themselves (strided rows, blocks 128/64/32, codes and scales bit
-for bit, and Fp8Dequantize back).
+for bit, and Fp8Dequantize back).  A last set takes M, N and K on and next
+to the tile, block and path boundaries and checks every element.
 """
 import numpy as np
 import pytest
@@ -377,3 +378,38 @@ def test_random_quantizers_bits(fg8, orc, name, M, K, pad, fmt, block):
         wd = fg8.dequantize_weight(wq, ws, fmt)
         torch.cuda.synchronize()
         _same(W.bf16_bits(wd.cpu()), orc.dequantize_weight(owq, ows, fmt), f"{name}: dequantized weight")
+
+
+# ----------------------------------------------------- boundary values ----
+def _edge_cases():
+    """Shapes whose M, N and K sit on or next to a tile, block or path
+    boundary (the few-token limits 16 / 32 / 128, the 128-row tile, the
+    128- and 256-column tiles, the 128-channel group), a seeded subset of
+    their product, both formats."""
+    Ms = [1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 257, 383]
+    Ns = [8, 120, 128, 136, 248, 256, 264, 1016, 1024, 1032]
+    Ks = [16, 112, 128, 144, 240, 256, 272, 1024, 4080, 4112]
+    rng = np.random.default_rng(8128)
+    combos = [(m, n, k) for m in Ms for n in Ns for k in Ks]
+    pick = rng.choice(len(combos), size=64, replace=False)
+    return [(f"edge{i}", *combos[j], i % 2) for i, j in enumerate(sorted(pick))]
+
+
+EDGE_CASES = _edge_cases()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,N,K,fmt", EDGE_CASES, ids=[c[0] for c in EDGE_CASES])
+def test_edge_shape_vs_oracle(fg8, orc, name, M, N, K, fmt):
+    """Every element against the oracle (these shapes are small)."""
+    seed = M * 977 + N * 13 + K
+    x = W.x_outliers(M, K, seed=seed)
+    w = W.w_row_groups(N, K, 0.02, seed=seed + 1)
+    b = W.normal((N,), 0.1, seed=seed + 2)
+    wq, ws = fg8.quantize_weight(w.cuda(), fmt)
+    y = fg8.linear(x.cuda(), wq, ws, b.cuda(), fmt)
+    torch.cuda.synchronize()
+    owq, ows = orc.quantize_weight(W.bf16_bits(w), fmt)
+    assert np.array_equal(wq.view(torch.uint8).cpu().numpy(), owq), f"{name}: weight codes"
+    y64, bound, _ = orc.linear(W.bf16_bits(x), owq, ows, W.bf16_bits(b), fmt)
+    _check_y(y, y64, bound, f"{name} M={M} N={N} K={K} fmt={fmt} plan={fg8.fg8_linear_plan(M, N, K, fmt)}")
